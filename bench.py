@@ -1,0 +1,481 @@
+"""Benchmark: retained-mass block-sparse attention on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+A step is one calibrate-then-reuse cycle of the 720p workload (the default config,
+Wan-14B-like: B=1, 40 heads, D=128, 21x45x80 tokens padded to 24x48x80, 64-token blocks):
+    calibration  tile_permute(Q, K) -> block_mass -> topp_select(0.99)
+    10 x reuse   tile_permute(Q_r, K_r, V_r) -> bsattn_fwd(frozen lists) -> inverse permute
+on seeded synthetic inputs already resident in HBM (Q/K/V of 774 MB each, far above L2).
+
+value  = executed attention TFLOP/s of the whole step: FLOPs of the kept blocks of the 10
+         reuse calls (4 * 64 * 64 * D per kept (query block, kv block) pair) divided by
+         the device time of the whole cycle, max over ranks.
+fwd    = the same FLOPs over the bsattn_fwd launches alone (CUDA events on the launch
+         stream) -> roofline of the dominant kernel.
+e2e    = the same metric through the public API with inputs copied from pinned host
+         memory and outputs copied back inside the timed region.
+--impl reference times the CPU oracle (the only other implementation of the method) on
+a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="wan14b_720p")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--reuse", type=int, default=None, help="reuse calls per step (default: the workload's)")
+    ap.add_argument("--tau", type=float, default=0.99)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-sample-rows", type=int, default=256)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    def __init__(self, gpu_index: int, path: str):
+        self.path = path
+        self.proc = None
+        try:
+            self.f = open(path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={CLOCK_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 active=parts[4], hw=parts[5], hwt=parts[6], swt=parts[7],
+                                 pcap=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 300] or rows
+        sms = sorted(r["sm"] for r in load)
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": sms[len(sms) // 2], "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=600))
+        pg = dist
+    return world, rank, local, pg
+
+
+def max_over_ranks(x: float, pg) -> float:
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+# ============================================================================ ours
+def run_ours(args, world, rank, local, pg):
+    import torch
+
+    import block_sparse_attention_25_b200 as bsa
+    from block_sparse_attention_25_b200 import build, synth
+
+    build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = synth.WORKLOADS[args.config]
+    n_reuse = args.reuse if args.reuse is not None else max(wl.redraws, 1)
+    s = bsa.Shape.of(wl)
+    fp8 = wl.fp8
+    seed_wl = wl.scaled(seed=wl.seed + 7919 * rank)  # independent problem per rank
+
+    # ---- inputs resident in HBM: the calibration draw and n_reuse correlated re-draws
+    draws = [synth.draw_qkv(seed_wl, device=dev)]
+    for r in range(1, n_reuse + 1):
+        draws.append(synth.redraw_qkv(seed_wl, r, device=dev))
+    torch.cuda.synchronize()
+
+    tiled = (s.batch, s.heads, s.Np, s.head_dim)
+    qt = torch.empty(tiled, dtype=torch.bfloat16, device=dev)
+    kt = torch.empty_like(qt)
+    vt = torch.empty_like(qt)
+    if fp8:
+        q8 = torch.empty(tiled, dtype=torch.uint8, device=dev)
+        k8, v8 = torch.empty_like(q8), torch.empty_like(q8)
+        sc = [torch.empty((s.batch, s.heads, s.Np // 64), dtype=torch.float32, device=dev)
+              for _ in range(3)]
+    out_t = torch.empty_like(qt)
+    out_r = [torch.empty((s.batch, s.S, s.heads, s.head_dim), dtype=torch.bfloat16, device=dev)
+             for _ in range(n_reuse)]
+    mass = torch.empty((s.batch, s.heads, s.n_qb, s.n_kb), dtype=torch.float32, device=dev)
+    row_ptr = torch.empty(s.rows + 1, dtype=torch.int32, device=dev)
+    col_idx = torch.empty(s.rows * s.n_kb, dtype=torch.int32, device=dev)
+    ws_m = bsa.new_workspace(s, bsa.OP_BLOCK_MASS, dev)
+    ws_t = bsa.new_workspace(s, bsa.OP_TOPP_SELECT, dev)
+    ws_f = bsa.new_workspace(s, bsa.OP_FWD, dev)
+    stream = torch.cuda.current_stream()
+    fwd_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_reuse)] for _ in range(args.steps)]
+    cur = {"step": 0}
+    cal_ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    launches_per_step = 0
+
+    def step(time_fwd: bool):
+        nonlocal launches_per_step
+        n = 0
+        q0, k0, _ = draws[0]
+        cal_ev[0].record(stream)
+        bsa.tile_permute(q0, s, out=qt)
+        bsa.tile_permute(k0, s, out=kt)
+        bsa.block_mass(qt, kt, s, out=mass, ws=ws_m)
+        bsa.topp_select(mass, s, args.tau, ws=ws_t, row_ptr=row_ptr, col_idx=col_idx)
+        cal_ev[1].record(stream)
+        n += 2 + 1 + 3
+        for r in range(n_reuse):
+            q, k, v = draws[r + 1]
+            if fp8:
+                bsa.tile_permute_quant_e4m3(q, s, out=q8, scales=sc[0])
+                bsa.tile_permute_quant_e4m3(k, s, out=k8, scales=sc[1])
+                bsa.tile_permute_quant_e4m3(v, s, out=v8, scales=sc[2])
+                if time_fwd:
+                    fwd_ev[cur["step"]][r][0].record(stream)
+                bsa.bsattn_fwd(q8, k8, v8, row_ptr, col_idx, s, scales=sc, out=out_t, ws=ws_f)
+            else:
+                bsa.tile_permute(q, s, out=qt)
+                bsa.tile_permute(k, s, out=kt)
+                bsa.tile_permute(v, s, out=vt)
+                if time_fwd:
+                    fwd_ev[cur["step"]][r][0].record(stream)
+                bsa.bsattn_fwd(qt, kt, vt, row_ptr, col_idx, s, out=out_t, ws=ws_f)
+            if time_fwd:
+                fwd_ev[cur["step"]][r][1].record(stream)
+            bsa.tile_permute(out_t, s, inverse=True, out=out_r[r])
+            n += 3 + 2 + 1
+        launches_per_step = n
+
+    # warm-up
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    for w in (ws_m, ws_t, ws_f):
+        st = bsa.device_status(w)
+        if st != 0:
+            raise RuntimeError(f"device status {st} after warm-up: {bsa.device_status_words(w)}")
+
+    # executed FLOPs of one reuse call: kept pairs * 4 * q_block * 64 * D
+    nnz = int(row_ptr[-1].item())
+    kept_frac = nnz / float(s.rows * s.n_kb)
+    flops_call = 4.0 * nnz * s.q_block * 64 * s.head_dim
+    dense_flops_call = 4.0 * s.rows * s.n_kb * s.q_block * 64 * s.head_dim
+
+    # timed region
+    clk = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")) \
+        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ClockSampler(local, f"/tmp/bsa_clocks_{rank}.csv")
+    barrier(pg)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        cur["step"] = i
+        step(True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(pg)
+    clocks = clk.stop()
+    # every bsattn_fwd launch of the timed region (CUDA events on the launch stream)
+    fwd_ms = [a.elapsed_time(b) for evs in fwd_ev for a, b in evs]
+    cal_ms = cal_ev[0].elapsed_time(cal_ev[1])
+    elapsed_ms = t0.elapsed_time(t1)
+    elapsed_ms = max_over_ranks(elapsed_ms, pg)
+    for w in (ws_m, ws_t, ws_f):
+        st = bsa.device_status(w)
+        if st != 0:
+            raise RuntimeError(f"device status {st} after timing: {bsa.device_status_words(w)}")
+
+    ms_step = elapsed_ms / args.steps
+    total_flops = flops_call * n_reuse * args.steps * world
+    value = total_flops / (elapsed_ms * 1e-3) / 1e12
+    fwd_avg_ms = sum(fwd_ms) / len(fwd_ms)
+    fwd_tflops = flops_call / (fwd_avg_ms * 1e-3) / 1e12
+    pk = peaks()
+    peak = pk["bf16_sus"] * (2.0 if fp8 else 1.0)
+    peak_note = ("sustained bf16 of " + pk["source"]) + (" x2 (fp8 nominal ratio)" if fp8 else "")
+
+    # ---- end to end through the public API, host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, bsa, s, draws, n_reuse, row_ptr, col_idx, flops_call, dev, stream,
+                      fp8, pg, world)
+
+    result = {
+        "metric": "bsattn_fwd ms/call & executed TFLOPS at 99% retained mass, % of bf16 peak",
+        "value": round(value, 2),
+        "unit": "TFLOP/s (executed, kept blocks)",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3" if fp8 else "bf16",
+        "data": "synthetic (seeded 3D random-Fourier-feature Q/K/V + noise, correlated re-draws)",
+        "config": {
+            "workload": wl.name,
+            "grid": f"{wl.T}x{wl.H}x{wl.W} padded {wl.Tp}x{wl.Hp}x{wl.Wp}",
+            "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
+            "q_block": wl.q_block, "kv_block": 64, "tokens": wl.S, "slots": wl.Np,
+            "threshold": args.tau, "reuse_calls_per_step": n_reuse,
+            "kept_fraction": round(kept_frac, 5),
+            "bsattn_fwd_ms_per_call": round(fwd_avg_ms, 3),
+            "bsattn_fwd_tflops": round(fwd_tflops, 2),
+            "bsattn_fwd_pct_of_peak": round(100.0 * fwd_tflops / peak, 2),
+            "dense_equivalent_tflops": round(dense_flops_call / (fwd_avg_ms * 1e-3) / 1e12, 2),
+            "calibration_ms": round(cal_ms, 3),
+            "executed_tflop_per_call": round(flops_call / 1e12, 3),
+            "l2": "inputs larger than L2 (774 MB per tensor); no flush needed",
+            "parallelism": f"independent problem per GPU x{world}",
+        },
+        "roofline": {
+            "bound": "tensor", "achieved": round(fwd_tflops, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(fwd_tflops / peak, 4), "traffic": None,
+            "kernel": "bsattn_fwd_bf16_kernel<128>" if not fp8 else "bsattn_fwd_e4m3_kernel",
+            "peak_source": peak_note,
+        },
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        result["e2e"] = e2e
+    return result
+
+
+def run_e2e(args, bsa, s, draws, n_reuse, row_ptr, col_idx, flops_call, dev, stream, fp8, pg,
+            world):
+    """Same cycle through the public API, every input copied in from pinned host memory and
+    every output copied back, inside the timed region."""
+    import torch
+    host = [tuple(x.to("cpu").pin_memory() for x in d) for d in draws]
+    out_host = [torch.empty((s.batch, s.S, s.heads, s.head_dim), dtype=torch.bfloat16).pin_memory()
+                for _ in range(n_reuse)]
+    dq = torch.empty_like(draws[0][0])
+    dk = torch.empty_like(dq)
+    dv = torch.empty_like(dq)
+    tiled = (s.batch, s.heads, s.Np, s.head_dim)
+    qt = torch.empty(tiled, dtype=torch.bfloat16, device=dev)
+    kt, vt, ot = torch.empty_like(qt), torch.empty_like(qt), torch.empty_like(qt)
+    o_r = torch.empty_like(dq)
+    mass = torch.empty((s.batch, s.heads, s.n_qb, s.n_kb), dtype=torch.float32, device=dev)
+    rp = torch.empty_like(row_ptr)
+    ci = torch.empty_like(col_idx)
+    ws_m = bsa.new_workspace(s, bsa.OP_BLOCK_MASS, dev)
+    ws_t = bsa.new_workspace(s, bsa.OP_TOPP_SELECT, dev)
+    ws_f = bsa.new_workspace(s, bsa.OP_FWD, dev)
+    if fp8:
+        q8 = torch.empty(tiled, dtype=torch.uint8, device=dev)
+        k8, v8 = torch.empty_like(q8), torch.empty_like(q8)
+        sc = [torch.empty((s.batch, s.heads, s.Np // 64), dtype=torch.float32, device=dev)
+              for _ in range(3)]
+    h2d = d2h = 0
+
+    def cycle():
+        nonlocal h2d, d2h
+        h2d = d2h = 0
+        dq.copy_(host[0][0], non_blocking=True)
+        dk.copy_(host[0][1], non_blocking=True)
+        h2d += 2 * dq.numel() * 2
+        bsa.tile_permute(dq, s, out=qt)
+        bsa.tile_permute(dk, s, out=kt)
+        bsa.block_mass(qt, kt, s, out=mass, ws=ws_m)
+        bsa.topp_select(mass, s, args.tau, ws=ws_t, row_ptr=rp, col_idx=ci)
+        for r in range(n_reuse):
+            for dst, src in zip((dq, dk, dv), host[r + 1]):
+                dst.copy_(src, non_blocking=True)
+            h2d += 3 * dq.numel() * 2
+            if fp8:
+                bsa.tile_permute_quant_e4m3(dq, s, out=q8, scales=sc[0])
+                bsa.tile_permute_quant_e4m3(dk, s, out=k8, scales=sc[1])
+                bsa.tile_permute_quant_e4m3(dv, s, out=v8, scales=sc[2])
+                bsa.bsattn_fwd(q8, k8, v8, rp, ci, s, scales=sc, out=ot, ws=ws_f)
+            else:
+                bsa.tile_permute(dq, s, out=qt)
+                bsa.tile_permute(dk, s, out=kt)
+                bsa.tile_permute(dv, s, out=vt)
+                bsa.bsattn_fwd(qt, kt, vt, rp, ci, s, out=ot, ws=ws_f)
+            bsa.tile_permute(ot, s, inverse=True, out=o_r)
+            out_host[r].copy_(o_r, non_blocking=True)
+            d2h += o_r.numel() * 2
+
+    cycle()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 2))
+    barrier(pg)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        cycle()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), pg)
+    val = flops_call * n_reuse * steps * world / (ms * 1e-3) / 1e12
+    return {"value": round(val, 2), "unit": "TFLOP/s (executed, kept blocks)",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 3)}
+
+
+# ============================================================================ CPU oracle
+def oracle_sample(wl, n_rows: int, seed: int = 0):
+    """Time the oracle's masked attention on n_rows sampled query rows of the workload
+    (seeded synthetic inputs on the host, a seeded CSR at the workload's kept fraction).
+    Returns (executed FLOPs, seconds, description)."""
+    import numpy as np
+    import torch
+    from threadpoolctl import threadpool_limits
+
+    from block_sparse_attention_25_b200 import synth
+    from oracle import bsa_oracle as O
+
+    g = O.Grid(wl.T, wl.H, wl.W, wl.Tp, wl.Hp, wl.Wp)
+    heads = 2
+    small = wl.scaled(heads=heads)
+    q, k, v = synth.draw_qkv(small, device="cpu")
+    qt, kt, vt = (O.permute_forward(x.to(torch.float64).numpy(), g) for x in (q, k, v))
+    n_qb, n_kb = wl.Np // wl.q_block, wl.Np // 64
+    rp, ci = synth.draw_keep_csr(heads * n_qb, n_kb, 0.957, seed=seed)
+    rp, ci = rp.numpy(), ci.numpy()
+    valid = O.valid_slots(g)
+    rng = np.random.default_rng(seed)
+    cand = np.nonzero(valid)[0]
+    rows = [(0, int(rng.integers(0, heads)), int(p)) for p in rng.choice(cand, n_rows, replace=False)]
+    flops = 0.0
+    with threadpool_limits(limits=1):
+        t = time.perf_counter()
+        for (b, h, p) in rows:
+            O.masked_attention_query(qt, kt, vt, g, b, h, p, wl.q_block, 64, rp, ci,
+                                     1.0 / math.sqrt(wl.head_dim))
+            r = h * n_qb + p // wl.q_block
+            blocks = ci[rp[r]:rp[r + 1]]
+            nk = int(sum(valid[j * 64:(j + 1) * 64].sum() for j in blocks))
+            flops += 4.0 * wl.head_dim * nk
+        dt = time.perf_counter() - t
+    desc = (f"oracle masked attention (numpy fp64, 1 thread) on {n_rows} sampled query rows of "
+            f"{wl.name} with a seeded CSR at 0.957 kept; TFLOP/s = executed FLOPs of those rows / time")
+    return flops, dt, desc
+
+
+def run_reference(args, world, rank, pg):
+    from block_sparse_attention_25_b200 import synth
+    wl = synth.WORKLOADS[args.config]
+    if rank != 0:
+        return None
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_sample(wl, 4)
+    tot_f = tot_t = 0.0
+    desc = ""
+    for i in range(args.steps):
+        f, t, desc = oracle_sample(wl, args.cpu_sample_rows, seed=i)
+        tot_f += f
+        tot_t += t
+    val = tot_f / tot_t / 1e12
+    return {
+        "impl": "reference",
+        "metric": "bsattn_fwd ms/call & executed TFLOPS at 99% retained mass, % of bf16 peak",
+        "value": val, "unit": "TFLOP/s (executed, kept blocks)", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": wl.name},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s (executed, kept blocks)", "cores": 1,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": val, "unit": "TFLOP/s (executed, kept blocks)", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    world, rank, local, pg = dist_setup(args)
+    if args.impl == "reference":
+        res = run_reference(args, world, rank, pg)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return
+    res = run_ours(args, world, rank, local, pg)
+    if rank == 0:
+        from block_sparse_attention_25_b200 import synth
+        wl = synth.WORKLOADS[args.config]
+        f, t, desc = oracle_sample(wl, args.cpu_sample_rows)
+        res["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s (executed, kept blocks)",
+                               "cores": 1, "kind": "oracle", "sample": desc,
+                               "seconds": round(t, 2)}
+        print(json.dumps(res), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,16 @@
+"""Retained-mass block-sparse attention for long 3D video token sequences on B200.
+
+The compute path is libbsattn.so (hand-written sm_100a CUDA behind a C ABI, declared in
+include/bsattn.h); this package is its thin binding plus the seeded input generator.
+"""
+from .bsattn import (  # noqa: F401
+    BsaError, Shape, bsattn_fwd, block_mass, clear_status, default_scale, device_status,
+    device_status_words, lib, new_workspace, tile_permute, tile_permute_quant_e4m3, topp_select,
+    workspace_bytes, OP_BLOCK_MASS, OP_FWD, OP_TOPP_SELECT,
+)
+
+__all__ = [
+    "BsaError", "Shape", "bsattn_fwd", "block_mass", "clear_status", "default_scale",
+    "device_status", "device_status_words", "lib", "new_workspace", "tile_permute",
+    "tile_permute_quant_e4m3", "topp_select", "workspace_bytes",
+]

@@ -1,0 +1,279 @@
+"""Thin Python binding of libbsattn.so (ctypes).
+
+Argument marshalling only: every step of the path runs in the library's CUDA kernels.
+PyTorch provides device memory and the current CUDA stream.  There is no fallback: if
+the library cannot be loaded every call raises.
+
+Names follow the C ABI in include/bsattn.h:
+    tile_permute, tile_permute_quant_e4m3, block_mass, topp_select, bsattn_fwd
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libbsattn.so")
+
+BSA_OK = 0
+STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "capacity too small",
+                4: "CUDA error", 5: "device wait timed out", 6: "device-side input check failed"}
+BSA_BF16, BSA_FP32, BSA_E4M3 = 0, 1, 2
+OP_BLOCK_MASS, OP_TOPP_SELECT, OP_FWD = 0, 1, 2
+
+
+class BsaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} (status {status})")
+        self.status = status
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("batch", "heads", "head_dim", "T", "H", "W", "Tp", "Hp", "Wp", "q_block", "kv_block")]
+
+
+@dataclass(frozen=True)
+class Shape:
+    """Problem shape; mirrors bsa_shape."""
+    batch: int
+    heads: int
+    head_dim: int
+    T: int
+    H: int
+    W: int
+    Tp: int
+    Hp: int
+    Wp: int
+    q_block: int = 64
+    kv_block: int = 64
+
+    @classmethod
+    def of(cls, wl) -> "Shape":
+        return cls(*wl.shape_tuple()) if hasattr(wl, "shape_tuple") else cls(*wl)
+
+    @property
+    def S(self):
+        return self.T * self.H * self.W
+
+    @property
+    def Np(self):
+        return self.Tp * self.Hp * self.Wp
+
+    @property
+    def n_qb(self):
+        return self.Np // self.q_block
+
+    @property
+    def n_kb(self):
+        return self.Np // self.kv_block
+
+    @property
+    def rows(self):
+        return self.batch * self.heads * self.n_qb
+
+    def c(self) -> _Shape:
+        return _Shape(self.batch, self.heads, self.head_dim, self.T, self.H, self.W,
+                      self.Tp, self.Hp, self.Wp, self.q_block, self.kv_block)
+
+
+_lib_handle = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbsattn.so (raises if it has not been built)."""
+    global _lib_handle
+    if _lib_handle is not None:
+        return _lib_handle
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                           "`python -m block_sparse_attention_25_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, S, F, L64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float, ctypes.c_int64
+    SP = ctypes.POINTER(_Shape)
+    sig = {
+        "bsa_workspace_bytes": (S, [SP, I]),
+        "bsa_clear_status": (I, [P, P]),
+        "bsa_device_status": (I, [P, P]),
+        "bsa_device_status_words": (I, [P, ctypes.POINTER(ctypes.c_uint32), P]),
+        "bsa_status_string": (ctypes.c_char_p, [I]),
+        "bsa_tile_permute": (I, [SP, I, I, P, P, P]),
+        "bsa_tile_permute_quant_e4m3": (I, [SP, P, P, P, P]),
+        "bsa_block_mass": (I, [SP, P, P, F, P, P, S, P]),
+        "bsa_topp_select": (I, [SP, P, F, P, P, L64, P, S, P]),
+        "bsa_fwd": (I, [SP, I, P, P, P, P, P, P, P, P, F, P, P, P, S, P]),
+        "bsa_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib_handle = L
+    return L
+
+
+EXPORTED_SYMBOLS = ("bsa_workspace_bytes", "bsa_clear_status", "bsa_device_status",
+                    "bsa_device_status_words", "bsa_status_string", "bsa_tile_permute",
+                    "bsa_tile_permute_quant_e4m3", "bsa_block_mass", "bsa_topp_select", "bsa_fwd",
+                    "bsa_version")
+
+
+def _check(status: int, what: str):
+    if status != BSA_OK:
+        raise BsaError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, shape, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name}: must be a contiguous CUDA tensor")
+
+
+def workspace_bytes(shape: Shape, op: int) -> int:
+    return int(lib().bsa_workspace_bytes(ctypes.byref(shape.c()), op))
+
+
+def new_workspace(shape: Shape, op: int, device="cuda") -> torch.Tensor:
+    """Allocate a workspace for `op` and clear its status header."""
+    n = workspace_bytes(shape, op)
+    if n == 0:
+        raise BsaError(1, "workspace size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _check(lib().bsa_clear_status(_ptr(ws), _stream()), "bsa_clear_status")
+    return ws
+
+
+def clear_status(ws: torch.Tensor, stream=None):
+    _check(lib().bsa_clear_status(_ptr(ws), _stream(stream)), "bsa_clear_status")
+
+
+def device_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronise and return the workspace's device status code (0 = ok)."""
+    return int(lib().bsa_device_status(_ptr(ws), _stream(stream)))
+
+
+def device_status_words(ws: torch.Tensor, stream=None):
+    w = (ctypes.c_uint32 * 4)()
+    _check(lib().bsa_device_status_words(_ptr(ws), w, _stream(stream)), "bsa_device_status_words")
+    return list(w)
+
+
+def tile_permute(x: torch.Tensor, shape: Shape, inverse: bool = False, out=None, stream=None):
+    """Raster [B,S,Hh,D] -> tile-major [B,Hh,Np,D] (inverse=False) or back."""
+    dt = {torch.bfloat16: BSA_BF16, torch.float32: BSA_FP32}.get(x.dtype)
+    if dt is None:
+        raise TypeError("tile_permute: bf16 or fp32")
+    raster = (shape.batch, shape.S, shape.heads, shape.head_dim)
+    tiled = (shape.batch, shape.heads, shape.Np, shape.head_dim)
+    src_shape, dst_shape = (tiled, raster) if inverse else (raster, tiled)
+    _need(x, x.dtype, src_shape, "src")
+    if out is None:
+        out = torch.empty(dst_shape, dtype=x.dtype, device=x.device)
+    _need(out, x.dtype, dst_shape, "dst")
+    _check(lib().bsa_tile_permute(ctypes.byref(shape.c()), dt, int(bool(inverse)), _ptr(x),
+                                  _ptr(out), _stream(stream)), "bsa_tile_permute")
+    return out
+
+
+def tile_permute_quant_e4m3(x: torch.Tensor, shape: Shape, out=None, scales=None, stream=None):
+    """Raster bf16 -> (tile-major e4m3 codes uint8 [B,Hh,Np,D], fp32 scales [B,Hh,Np/64])."""
+    _need(x, torch.bfloat16, (shape.batch, shape.S, shape.heads, shape.head_dim), "src")
+    if out is None:
+        out = torch.empty((shape.batch, shape.heads, shape.Np, shape.head_dim), dtype=torch.uint8,
+                          device=x.device)
+    if scales is None:
+        scales = torch.empty((shape.batch, shape.heads, shape.Np // 64), dtype=torch.float32,
+                             device=x.device)
+    _check(lib().bsa_tile_permute_quant_e4m3(ctypes.byref(shape.c()), _ptr(x), _ptr(out),
+                                             _ptr(scales), _stream(stream)),
+           "bsa_tile_permute_quant_e4m3")
+    return out, scales
+
+
+def default_scale(shape: Shape) -> float:
+    return 1.0 / math.sqrt(shape.head_dim)
+
+
+def block_mass(q, k, shape: Shape, softmax_scale=None, out=None, ws=None, stream=None):
+    """Exact block masses fp32 [B,Hh,Np/q_block,Np/64] of tile-major bf16 q, k."""
+    tiled = (shape.batch, shape.heads, shape.Np, shape.head_dim)
+    _need(q, torch.bfloat16, tiled, "q")
+    _need(k, torch.bfloat16, tiled, "k")
+    if out is None:
+        out = torch.empty((shape.batch, shape.heads, shape.n_qb, shape.n_kb), dtype=torch.float32,
+                          device=q.device)
+    if ws is None:
+        ws = new_workspace(shape, OP_BLOCK_MASS, q.device)
+    scale = default_scale(shape) if softmax_scale is None else float(softmax_scale)
+    _check(lib().bsa_block_mass(ctypes.byref(shape.c()), _ptr(q), _ptr(k), scale, _ptr(out),
+                                _ptr(ws), ws.numel(), _stream(stream)), "bsa_block_mass")
+    return out
+
+
+def topp_select(mass, shape: Shape, threshold: float = 0.99, col_capacity=None, ws=None,
+                row_ptr=None, col_idx=None, stream=None):
+    """CSR (row_ptr int32 [R+1], col_idx int32 [capacity]) of the kept kv blocks.
+
+    col_idx is returned at full capacity (R * n_kb entries by default); the valid prefix
+    is row_ptr[-1] entries long.
+    """
+    R = shape.rows
+    _need(mass, torch.float32, (shape.batch, shape.heads, shape.n_qb, shape.n_kb), "mass")
+    cap = R * shape.n_kb if col_capacity is None else int(col_capacity)
+    if row_ptr is None:
+        row_ptr = torch.empty(R + 1, dtype=torch.int32, device=mass.device)
+    if col_idx is None:
+        col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=mass.device)
+    if ws is None:
+        ws = new_workspace(shape, OP_TOPP_SELECT, mass.device)
+    _check(lib().bsa_topp_select(ctypes.byref(shape.c()), _ptr(mass), float(threshold),
+                                 _ptr(row_ptr), _ptr(col_idx), cap, _ptr(ws), ws.numel(),
+                                 _stream(stream)), "bsa_topp_select")
+    return row_ptr, col_idx
+
+
+def bsattn_fwd(q, k, v, row_ptr, col_idx, shape: Shape, softmax_scale=None, scales=None,
+               want_lse=False, out=None, lse=None, ws=None, stream=None):
+    """Block-sparse attention over CSR lists.  bf16 q/k/v, or e4m3 codes (uint8) with
+    scales=(q_scales, k_scales, v_scales).  Returns out (bf16 tile-major) or (out, lse)."""
+    tiled = (shape.batch, shape.heads, shape.Np, shape.head_dim)
+    fp8 = q.dtype == torch.uint8
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.uint8 if fp8 else torch.bfloat16, tiled, n)
+    _need(row_ptr, torch.int32, (shape.rows + 1,), "row_ptr")
+    if col_idx.dtype != torch.int32 or not col_idx.is_cuda:
+        raise TypeError("col_idx: int32 CUDA tensor")
+    sq = sk = sv = None
+    if fp8:
+        if scales is None:
+            raise ValueError("e4m3 inputs need per-tile scales")
+        sq, sk, sv = scales
+        for t, n in ((sq, "q_scales"), (sk, "k_scales"), (sv, "v_scales")):
+            _need(t, torch.float32, (shape.batch, shape.heads, shape.Np // 64), n)
+    if out is None:
+        out = torch.empty(tiled, dtype=torch.bfloat16, device=q.device)
+    if want_lse and lse is None:
+        lse = torch.empty((shape.batch, shape.heads, shape.Np), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = new_workspace(shape, OP_FWD, q.device)
+    scale = default_scale(shape) if softmax_scale is None else float(softmax_scale)
+    _check(lib().bsa_fwd(ctypes.byref(shape.c()), BSA_E4M3 if fp8 else BSA_BF16, _ptr(q), _ptr(k),
+                         _ptr(v), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(row_ptr), _ptr(col_idx), scale,
+                         _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)), "bsa_fwd")
+    return (out, lse) if want_lse else out

@@ -1,0 +1,260 @@
+// C ABI of libbsattn.so: argument checks, workspace layout, tensor-map encoding and
+// kernel launches.  See include/bsattn.h for the contract of every entry point.
+#include <cstring>
+#include <mutex>
+
+#include "../../include/bsattn.h"
+#include "bsa_kernels.cuh"
+
+namespace bsa {
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+cudaError_t encode_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                           int elem_bytes, int D, int Np, int bh, int box_d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorInitializationError;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Np),
+                              static_cast<cuuint64_t>(bh)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * elem_bytes,
+                                 static_cast<cuuint64_t>(Np) * D * elem_bytes};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_d), static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = fn(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace bsa
+
+using bsa::AttnDims;
+using bsa::GridDims;
+
+namespace {
+
+// Host-side shape checks shared by every entry point.
+bsa_status check_shape(const bsa_shape* s, bool attention) {
+  if (s == nullptr) return BSA_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->heads < 1 || s->head_dim < 1) return BSA_ERR_INVALID_ARG;
+  if (s->T < 1 || s->H < 1 || s->W < 1) return BSA_ERR_INVALID_ARG;
+  if (s->Tp < s->T || s->Hp < s->H || s->Wp < s->W) return BSA_ERR_INVALID_ARG;
+  if ((s->Tp & 3) || (s->Hp & 3) || (s->Wp & 3)) return BSA_ERR_INVALID_ARG;
+  const long long np = 1LL * s->Tp * s->Hp * s->Wp;
+  if (np >= (1LL << 30)) return BSA_ERR_UNSUPPORTED;
+  if (s->head_dim != 64 && s->head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (attention) {
+    if (s->kv_block != 64) return BSA_ERR_UNSUPPORTED;
+    if (s->q_block != 64 && s->q_block != 128) return BSA_ERR_UNSUPPORTED;
+    if (np % s->q_block) return BSA_ERR_INVALID_ARG;
+    const long long rows = 1LL * s->batch * s->heads * (np / s->q_block);
+    if (rows >= (1LL << 31)) return BSA_ERR_UNSUPPORTED;
+    if (np / 64 > 4096) return BSA_ERR_UNSUPPORTED;  // selection and schedule bitmaps
+    // CSR offsets are int32
+    if (rows * (np / 64) >= (1LL << 31)) return BSA_ERR_UNSUPPORTED;
+  }
+  return BSA_OK;
+}
+
+GridDims make_grid(const bsa_shape* s) {
+  GridDims g;
+  g.T = s->T;
+  g.H = s->H;
+  g.W = s->W;
+  g.Tp = s->Tp;
+  g.Hp = s->Hp;
+  g.Wp = s->Wp;
+  g.nth = s->Hp / 4;
+  g.ntw = s->Wp / 4;
+  g.S = s->T * s->H * s->W;
+  g.Np = s->Tp * s->Hp * s->Wp;
+  return g;
+}
+
+AttnDims make_attn(const bsa_shape* s) {
+  AttnDims a;
+  a.g = make_grid(s);
+  a.batch = s->batch;
+  a.heads = s->heads;
+  a.head_dim = s->head_dim;
+  a.q_block = s->q_block;
+  a.n_qb = a.g.Np / s->q_block;
+  a.n_kb = a.g.Np / 64;
+  a.n_cta_per_head = (a.g.Np + 255) / 256;
+  return a;
+}
+
+bsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
+
+size_t workspace_bytes(const bsa_shape* s, int op) {
+  if (check_shape(s, true) != BSA_OK) return 0;
+  const AttnDims a = make_attn(s);
+  switch (op) {
+    case BSA_OP_BLOCK_MASS:
+      return bsa::kStatusBytes + bsa::mass_scratch_bytes(a);
+    case BSA_OP_TOPP_SELECT:
+      return bsa::kStatusBytes +
+             bsa::topp_scratch_bytes(1LL * a.batch * a.heads * a.n_qb, a.n_kb);
+    case BSA_OP_FWD:
+      return bsa::kStatusBytes + bsa::fwd_scratch_bytes(a);
+    default:
+      return 0;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bsa_version(void) { return "bsattn 0.1 sm_100a"; }
+
+const char* bsa_status_string(bsa_status st) {
+  switch (st) {
+    case BSA_OK: return "ok";
+    case BSA_ERR_INVALID_ARG: return "invalid argument";
+    case BSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case BSA_ERR_CAPACITY: return "capacity too small";
+    case BSA_ERR_CUDA: return "CUDA error";
+    case BSA_ERR_TIMEOUT: return "device wait timed out";
+    case BSA_ERR_DEVICE_INPUT: return "device-side input check failed";
+  }
+  return "unknown status";
+}
+
+size_t bsa_workspace_bytes(const bsa_shape* shape, int op) { return workspace_bytes(shape, op); }
+
+bsa_status bsa_clear_status(void* ws, bsa_stream_t stream) {
+  if (ws == nullptr) return BSA_ERR_INVALID_ARG;
+  return from_cuda(cudaMemsetAsync(ws, 0, bsa::kStatusBytes, stream));
+}
+
+bsa_status bsa_device_status_words(const void* ws, uint32_t out_words[4], bsa_stream_t stream) {
+  if (ws == nullptr || out_words == nullptr) return BSA_ERR_INVALID_ARG;
+  cudaError_t e = cudaMemcpyAsync(out_words, ws, 4 * sizeof(uint32_t), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  return from_cuda(e);
+}
+
+bsa_status bsa_device_status(const void* ws, bsa_stream_t stream) {
+  uint32_t w[4] = {0, 0, 0, 0};
+  const bsa_status st = bsa_device_status_words(ws, w, stream);
+  if (st != BSA_OK) return st;
+  if (w[0] & bsa::FLAG_TIMEOUT) return BSA_ERR_TIMEOUT;
+  if (w[0] & bsa::FLAG_DEVICE_INPUT) return BSA_ERR_DEVICE_INPUT;
+  if (w[0] & bsa::FLAG_CAPACITY) return BSA_ERR_CAPACITY;
+  return BSA_OK;
+}
+
+bsa_status bsa_tile_permute(const bsa_shape* shape, bsa_dtype dtype, int inverse, const void* src,
+                            void* dst, bsa_stream_t stream) {
+  bsa_status st = check_shape(shape, false);
+  if (st != BSA_OK) return st;
+  if (src == nullptr || dst == nullptr || !bsa::aligned16(src) || !bsa::aligned16(dst))
+    return BSA_ERR_INVALID_ARG;
+  if (dtype != BSA_BF16 && dtype != BSA_FP32) return BSA_ERR_UNSUPPORTED;
+  if (inverse != 0 && inverse != 1) return BSA_ERR_INVALID_ARG;
+  const GridDims g = make_grid(shape);
+  const int row_bytes = shape->head_dim * (dtype == BSA_BF16 ? 2 : 4);
+  return from_cuda(bsa::launch_tile_permute(g, shape->batch, shape->heads, row_bytes, inverse, src,
+                                            dst, stream));
+}
+
+bsa_status bsa_tile_permute_quant_e4m3(const bsa_shape* shape, const void* src_bf16, uint8_t* dst,
+                                       float* tile_scales, bsa_stream_t stream) {
+  bsa_status st = check_shape(shape, false);
+  if (st != BSA_OK) return st;
+  if (src_bf16 == nullptr || dst == nullptr || tile_scales == nullptr ||
+      !bsa::aligned16(src_bf16) || !bsa::aligned16(dst) ||
+      (reinterpret_cast<uintptr_t>(tile_scales) & 3u))
+    return BSA_ERR_INVALID_ARG;
+  const long long ntiles = 1LL * shape->batch * shape->heads * (1LL * shape->Tp * shape->Hp * shape->Wp / 64);
+  if (ntiles >= (1LL << 31)) return BSA_ERR_UNSUPPORTED;
+  const GridDims g = make_grid(shape);
+  return from_cuda(bsa::launch_tile_permute_quant_e4m3(g, shape->batch, shape->heads,
+                                                       shape->head_dim, src_bf16, dst,
+                                                       tile_scales, stream));
+}
+
+bsa_status bsa_block_mass(const bsa_shape* shape, const void* q, const void* k, float softmax_scale,
+                          float* mass, void* ws, size_t ws_bytes, bsa_stream_t stream) {
+  bsa_status st = check_shape(shape, true);
+  if (st != BSA_OK) return st;
+  if (q == nullptr || k == nullptr || mass == nullptr || ws == nullptr || !bsa::aligned16(q) ||
+      !bsa::aligned16(k) || !bsa::aligned16(ws) || (reinterpret_cast<uintptr_t>(mass) & 3u))
+    return BSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f)) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(shape, BSA_OP_BLOCK_MASS)) return BSA_ERR_CAPACITY;
+  const AttnDims a = make_attn(shape);
+  return from_cuda(bsa::launch_block_mass(a, q, k, softmax_scale, mass, ws, stream));
+}
+
+bsa_status bsa_topp_select(const bsa_shape* shape, const float* mass, float threshold,
+                           int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, void* ws,
+                           size_t ws_bytes, bsa_stream_t stream) {
+  bsa_status st = check_shape(shape, true);
+  if (st != BSA_OK) return st;
+  if (mass == nullptr || row_ptr == nullptr || ws == nullptr || !bsa::aligned16(ws) ||
+      (reinterpret_cast<uintptr_t>(mass) & 3u))
+    return BSA_ERR_INVALID_ARG;
+  if (col_capacity < 0 || (col_capacity > 0 && col_idx == nullptr)) return BSA_ERR_INVALID_ARG;
+  if (!(threshold > 0.f && threshold <= 1.f)) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(shape, BSA_OP_TOPP_SELECT)) return BSA_ERR_CAPACITY;
+  const AttnDims a = make_attn(shape);
+  const long long rows = 1LL * a.batch * a.heads * a.n_qb;
+  return from_cuda(bsa::launch_topp_select(mass, rows, a.n_kb, threshold, row_ptr, col_idx,
+                                           col_capacity, ws, stream));
+}
+
+bsa_status bsa_fwd(const bsa_shape* shape, bsa_dtype dtype, const void* q, const void* k,
+                   const void* v, const float* q_scales, const float* k_scales,
+                   const float* v_scales, const int32_t* row_ptr, const int32_t* col_idx,
+                   float softmax_scale, void* out, float* lse, void* ws, size_t ws_bytes,
+                   bsa_stream_t stream) {
+  bsa_status st = check_shape(shape, true);
+  if (st != BSA_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || row_ptr == nullptr || col_idx == nullptr ||
+      out == nullptr || ws == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (!bsa::aligned16(q) || !bsa::aligned16(k) || !bsa::aligned16(v) || !bsa::aligned16(out) ||
+      !bsa::aligned16(ws) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return BSA_ERR_INVALID_ARG;
+  if (dtype == BSA_E4M3) {
+    if (q_scales == nullptr || k_scales == nullptr || v_scales == nullptr) return BSA_ERR_INVALID_ARG;
+    if (shape->head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  } else if (dtype != BSA_BF16) {
+    return BSA_ERR_UNSUPPORTED;
+  }
+  if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f)) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(shape, BSA_OP_FWD)) return BSA_ERR_CAPACITY;
+  const AttnDims a = make_attn(shape);
+  const cudaError_t e =
+      bsa::launch_bsattn_fwd(a, dtype == BSA_E4M3 ? 1 : 0, q, k, v, q_scales, k_scales, v_scales,
+                             row_ptr, col_idx, softmax_scale, out, lse, ws, stream);
+  if (e == cudaErrorNotSupported) return BSA_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,526 @@
+// Block-sparse flash-attention forward over frozen CSR kv-block lists, sm_100a.
+//
+// "LoSA: Near-Lossless Sparse Attention for Training-Free Video Diffusion Acceleration",
+// Abstract: the block indices selected at the calibration step are frozen and reused by
+// the attention of all remaining steps; softmax runs over the kept blocks only.
+// "FPSAttention", Abstract: FP8 e4m3 operands with one scale per 3D tile.
+//
+// Work decomposition
+//   One CTA owns 256 consecutive query slots of one (batch, head): two M=128 tiles, so
+//   every K/V tile fetched into shared memory feeds two tensor-core tiles.  The CTA walks
+//   the sorted union of its query blocks' kv lists (built by bsattn_schedule_kernel) two
+//   kv blocks (N = 128 keys) per step; keys of a block that a query block did not keep
+//   are masked to -inf for that block's rows.
+//
+// Warp roles (320 threads)
+//   warps 0-3  softmax for Q tile 0, one thread per query row (TMEM lanes 0..127)
+//   warps 4-7  softmax for Q tile 1
+//   warp 8     TMA producer: Q once, then K and V of every step into rings
+//   warp 9     tcgen05.mma issuer (one thread) and TMEM owner
+//
+// Tensor memory (512 columns x 128 lanes x 32 bit)
+//   S0 [0,128)  S1 [128,256)  O0 [256,256+D)  O1 [256+D,256+2D)
+//   P_t (bf16 pairs) overwrites the first 64 columns of S_t once S_t has been read.
+//
+// Per step s, the MMA thread issues for t = 0, 1:  O_t += P_t(s-1) V(s-1);  S_t(s) = Q_t K(s)^T
+// and commits S_full[t] after both, so when softmax t sees S_t(s) the previous PV into O_t
+// has completed and O_t may be rescaled in place.  Rescaling is lazy: the running max used
+// for exponentiation moves only when a row's max grows by more than 8 (log2 units), so
+// P <= 256 and, for smooth attention, O is almost never touched.
+#include "bsa_kernels.cuh"
+
+namespace bsa {
+
+namespace fwd {
+
+constexpr int kThreads = 320;
+constexpr int kRowsPerCta = 256;
+constexpr float kRescaleLog2 = 8.0f;
+
+// Schedule entry: (j << 5) | (has_pad_keys << 4) | keep bits for the CTA's <= 4 query blocks.
+__device__ __forceinline__ int entry_block(uint32_t e) { return static_cast<int>(e >> 5); }
+
+}  // namespace fwd
+
+// Build, per CTA, the ascending union of its query blocks' kv lists with keep bits.
+// One 256-thread CTA per attention CTA.  Validates the CSR rows it reads.
+__global__ void __launch_bounds__(256) bsattn_schedule_kernel(AttnDims a,
+                                                              const int32_t* __restrict__ row_ptr,
+                                                              const int32_t* __restrict__ col_idx,
+                                                              int32_t* __restrict__ counts,
+                                                              uint32_t* __restrict__ entries,
+                                                              uint32_t* status) {
+  __shared__ uint32_t bm[4][128];  // up to 4096 kv blocks per query block
+  __shared__ int warp_tot[8];
+  const int cta = blockIdx.x;
+  const int bh = cta / a.n_cta_per_head;
+  const int c = cta - bh * a.n_cta_per_head;
+  const int nq = fwd::kRowsPerCta / a.q_block;
+  const int tid = threadIdx.x;
+  for (int i = tid; i < 4 * 128; i += 256) (&bm[0][0])[i] = 0u;
+  __syncthreads();
+  for (int slot = 0; slot < nq; ++slot) {
+    const int qb = c * nq + slot;
+    if (qb >= a.n_qb) break;
+    const long long r = static_cast<long long>(bh) * a.n_qb + qb;
+    const int beg = row_ptr[r], end = row_ptr[r + 1];
+    if (beg < 0 || end < beg || end - beg > a.n_kb) {
+      if (tid == 0) record_status(status, FLAG_DEVICE_INPUT, DETAIL_CSR_ROWPTR, static_cast<uint32_t>(r), 0u);
+      continue;
+    }
+    for (int e = beg + tid; e < end; e += 256) {
+      const int j = col_idx[e];
+      if (j < 0 || j >= a.n_kb) {
+        record_status(status, FLAG_DEVICE_INPUT, DETAIL_CSR_RANGE, static_cast<uint32_t>(r), static_cast<uint32_t>(e));
+        continue;
+      }
+      if (e > beg && col_idx[e - 1] >= j)
+        record_status(status, FLAG_DEVICE_INPUT, DETAIL_CSR_ORDER, static_cast<uint32_t>(r), static_cast<uint32_t>(e));
+      atomicOr(&bm[slot][j >> 5], 1u << (j & 31));
+    }
+  }
+  __syncthreads();
+  uint32_t* out = entries + static_cast<long long>(cta) * a.n_kb;
+  int base = 0;
+  for (int j0 = 0; j0 < a.n_kb; j0 += 256) {
+    const int j = j0 + tid;
+    uint32_t keep = 0;
+    if (j < a.n_kb) {
+#pragma unroll
+      for (int s = 0; s < 4; ++s) keep |= ((bm[s][j >> 5] >> (j & 31)) & 1u) << s;
+    }
+    const bool any = keep != 0;
+    const uint32_t bal = __ballot_sync(0xffffffffu, any);
+    const int wpos = __popc(bal & ((1u << lane_id()) - 1u));
+    if (lane_id() == 0) warp_tot[tid >> 5] = __popc(bal);
+    __syncthreads();
+    int before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      if (w < (tid >> 5)) before += warp_tot[w];
+      tot += warp_tot[w];
+    }
+    if (any) {
+      const uint32_t pad = tile_has_pad(a.g, j) ? 1u : 0u;
+      out[base + before + wpos] = (static_cast<uint32_t>(j) << 5) | (pad << 4) | keep;
+    }
+    base += tot;
+    __syncthreads();
+  }
+  if (tid == 0) counts[cta] = base;
+}
+
+struct FwdParams {
+  AttnDims a;
+  const int32_t* counts;
+  const uint32_t* entries;
+  __nv_bfloat16* out;
+  float* lse;
+  uint32_t* status;
+  float scale_log2;  // softmax_scale * log2(e)
+};
+
+template <int D>
+struct FwdSmem {
+  static constexpr int kChunks = D / 64;             // 128-byte swizzle chunks per row
+  static constexpr int kQTile = 128 * D * 2;         // one 128-row Q tile
+  static constexpr int kKVStage = 128 * D * 2;       // two 64-row kv blocks
+  static constexpr int kKStages = (D == 128) ? 3 : 4;
+  static constexpr int kVStages = (D == 128) ? 2 : 4;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + 2 * kQTile;
+  static constexpr int kVOff = kKOff + kKStages * kKVStage;
+  static constexpr int kBarOff = kVOff + kVStages * kKVStage;
+  static constexpr int kBytes = kBarOff + 256;
+  static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+};
+
+template <int D>
+__global__ void __launch_bounds__(fwd::kThreads, 1)
+    bsattn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
+                           const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdSmem<D>;
+  constexpr int KS = L::kKStages, VS = L::kVStages;
+  extern __shared__ uint8_t smem_raw[];
+  // 128-byte-swizzled operand tiles need 1024-byte alignment in the shared window.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* bar_q = bars + 0;
+  uint64_t* bar_kfull = bars + 1;
+  uint64_t* bar_kempty = bar_kfull + KS;
+  uint64_t* bar_vfull = bar_kempty + KS;
+  uint64_t* bar_vempty = bar_vfull + VS;
+  uint64_t* bar_sfull = bar_vempty + VS;  // [2]
+  uint64_t* bar_pfull = bar_sfull + 2;    // [2]
+  uint64_t* bar_ofull = bar_pfull + 2;
+  uint64_t* bar_drain = bar_ofull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const AttnDims& a = p.a;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int cta = blockIdx.x;
+  const int bh = cta / a.n_cta_per_head;
+  const int row0 = (cta - bh * a.n_cta_per_head) * fwd::kRowsPerCta;
+  const int n_ent = p.counts[cta];
+  const int nsteps = (n_ent + 1) >> 1;
+  const uint32_t* ent = p.entries + static_cast<long long>(cta) * a.n_kb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < KS; ++i) {
+      mbar_init(bar_kfull + i, 1);
+      mbar_init(bar_kempty + i, 1);
+    }
+    for (int i = 0; i < VS; ++i) {
+      mbar_init(bar_vfull + i, 1);
+      mbar_init(bar_vempty + i, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_sfull + t, 1);
+      mbar_init(bar_pfull + t, 128);
+    }
+    mbar_init(bar_ofull, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && nsteps > 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      mbar_arrive_expect_tx(bar_q, 2 * L::kQTile);
+      for (int t = 0; t < 2; ++t)
+        for (int ch = 0; ch < L::kChunks; ++ch)
+          tma_load_3d(smem + L::kQOff + t * L::kQTile + ch * (128 * 128), &tm_q, bar_q, ch * 64,
+                      row0 + t * 128, bh);
+      for (int s = 0; s < nsteps; ++s) {
+        const int nb = (2 * s + 1 < n_ent) ? 2 : 1;
+        const int j0 = fwd::entry_block(ent[2 * s]);
+        const int j1 = nb == 2 ? fwd::entry_block(ent[2 * s + 1]) : 0;
+        const int ks = s % KS;
+        if (s >= KS && !mbar_wait(bar_kempty + ks, ((s / KS) - 1) & 1, abort_flag, p.status,
+                                  DETAIL_WAIT_K_EMPTY))
+          break;
+        mbar_arrive_expect_tx(bar_kfull + ks, nb * 64 * D * 2);
+        uint8_t* kst = smem + L::kKOff + ks * L::kKVStage;
+        for (int ch = 0; ch < L::kChunks; ++ch) {
+          tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * 64, j0 * 64, bh);
+          if (nb == 2)
+            tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * 64,
+                        j1 * 64, bh);
+        }
+        const int vs = s % VS;
+        if (s >= VS && !mbar_wait(bar_vempty + vs, ((s / VS) - 1) & 1, abort_flag, p.status,
+                                  DETAIL_WAIT_V_EMPTY))
+          break;
+        mbar_arrive_expect_tx(bar_vfull + vs, nb * 64 * D * 2);
+        uint8_t* vst = smem + L::kVOff + vs * L::kKVStage;
+        for (int ch = 0; ch < L::kChunks; ++ch) {
+          tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * 64, j0 * 64, bh);
+          if (nb == 2)
+            tma_load_3d(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch * 64,
+                        j1 * 64, bh);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nsteps > 0) {
+      const uint32_t q_base = smem_u32(smem + L::kQOff);
+      const uint32_t k_base = smem_u32(smem + L::kKOff);
+      const uint32_t v_base = smem_u32(smem + L::kVOff);
+      const uint32_t idesc_pv = make_idesc(1u, 1u, 128u, static_cast<uint32_t>(D));
+      bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, DETAIL_WAIT_Q);
+      auto issue_pv = [&](int t, int sp) {
+        // O_t (+)= P_t(sp) V(sp); K dimension = keys of step sp (64 or 128).
+        const int nbp = (2 * sp + 1 < n_ent) ? 2 : 1;
+        const uint32_t vb = v_base + (sp % VS) * L::kKVStage;
+        const uint32_t p_tmem = tmem + t * 128;
+        const uint32_t o_tmem = tmem + 256 + t * D;
+        for (int kk = 0; kk < nbp * 4; ++kk) {
+          const uint64_t bdesc = make_sdesc_sw128(vb + kk * 2048, 128 * 128, 1024);
+          mma_f16_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (sp > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      for (int s = 0; s < nsteps && ok; ++s) {
+        const int ks = s % KS;
+        const int nb = (2 * s + 1 < n_ent) ? 2 : 1;
+        const uint32_t idesc_qk = make_idesc(1u, 0u, 128u, static_cast<uint32_t>(nb * 64));
+        if (!mbar_wait(bar_kfull + ks, (s / KS) & 1, abort_flag, p.status, DETAIL_WAIT_K_FULL)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t kb = k_base + ks * L::kKVStage;
+        for (int t = 0; t < 2; ++t) {
+          if (s > 0) {
+            if (!mbar_wait(bar_pfull + t, (s - 1) & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL)) {
+              ok = false;
+              break;
+            }
+            if (t == 0 && !mbar_wait(bar_vfull + ((s - 1) % VS), ((s - 1) / VS) & 1, abort_flag,
+                                     p.status, DETAIL_WAIT_V_FULL)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(t, s - 1);
+            if (t == 1) mma_commit(bar_vempty + ((s - 1) % VS));
+          }
+          const uint32_t qb = q_base + t * L::kQTile;
+          const uint32_t s_tmem = tmem + t * 128;
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            const uint64_t adesc = make_sdesc_sw128(qb + off, 16, 1024);
+            const uint64_t bdesc = make_sdesc_sw128(kb + off, 16, 1024);
+            mma_f16_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_sfull + t);
+        }
+        if (!ok) break;
+        mma_commit(bar_kempty + ks);
+      }
+      if (ok) {
+        const int sl = nsteps - 1;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!mbar_wait(bar_pfull + t, sl & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL)) {
+            ok = false;
+            break;
+          }
+          if (t == 0 && !mbar_wait(bar_vfull + (sl % VS), (sl / VS) & 1, abort_flag, p.status,
+                                   DETAIL_WAIT_V_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(t, sl);
+        }
+        if (ok) mma_commit(bar_ofull);
+      }
+      // Whatever happened, let every issued MMA finish before TMEM is released.
+      mma_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0, p.status, DETAIL_WAIT_O_FULL);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    const int t = warp >> 2;           // Q tile
+    const int wq = warp & 3;           // TMEM lane quarter
+    const int row = wq * 32 + lane;    // row inside the tile
+    const int local = t * 128 + row;   // row inside the CTA
+    const int slot = row0 + local;     // query slot inside the head
+    const int qsel = local / a.q_block;
+    const bool in_range = slot < a.g.Np;
+    const bool q_valid = in_range && slot_valid(a.g, slot);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t s_addr = lane_base + t * 128;
+    const uint32_t o_addr = lane_base + 256 + t * D;
+    const float c = p.scale_log2;
+    float m_run = -INFINITY;  // running max, scaled log2 units
+    float l_run = 0.f;
+    bool ok = true;
+
+    uint32_t e0n = nsteps > 0 ? ent[0] : 0u;
+    uint32_t e1n = n_ent > 1 ? ent[1] : 0u;
+    for (int s = 0; s < nsteps; ++s) {
+      const int nb = (2 * s + 1 < n_ent) ? 2 : 1;
+      const uint32_t e0 = e0n, e1 = e1n;
+      if (s + 1 < nsteps) {
+        e0n = ent[2 * s + 2];
+        e1n = (2 * s + 3 < n_ent) ? ent[2 * s + 3] : 0u;
+      }
+      const bool got = __all_sync(
+          0xffffffffu, mbar_wait(bar_sfull + t, s & 1, abort_flag, p.status, DETAIL_WAIT_S_FULL));
+      if (!got) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sv[128];
+      tmem_ld32(s_addr + 0, sv + 0);
+      tmem_ld32(s_addr + 32, sv + 32);
+      if (nb == 2) {
+        tmem_ld32(s_addr + 64, sv + 64);
+        tmem_ld32(s_addr + 96, sv + 96);
+      }
+      tmem_ld_wait();
+      // Column masks (warp-uniform: a warp's rows share one query block).  A block this
+      // query block did not keep, or a pad key, or the absent half of a 1-block step -> -inf.
+      uint64_t mk0 = 0ull, mk1 = 0ull;
+      if ((e0 >> qsel) & 1u) mk0 = ((e0 >> 4) & 1u) ? tile_valid_mask(a.g, fwd::entry_block(e0)) : ~0ull;
+      if (nb == 2 && ((e1 >> qsel) & 1u))
+        mk1 = ((e1 >> 4) & 1u) ? tile_valid_mask(a.g, fwd::entry_block(e1)) : ~0ull;
+      if ((mk0 & mk1) != ~0ull) {
+        const uint32_t mw[4] = {static_cast<uint32_t>(mk0), static_cast<uint32_t>(mk0 >> 32),
+                                static_cast<uint32_t>(mk1), static_cast<uint32_t>(mk1 >> 32)};
+#pragma unroll
+        for (int i = 0; i < 128; ++i) sv[i] = ((mw[i >> 5] >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
+      }
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+#pragma unroll
+      for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
+      float mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float m_new = mrow * c;
+      float factor = 1.f;
+      bool resc = false;
+      if (m_new > m_run + fwd::kRescaleLog2 || (m_run == -INFINITY && m_new != -INFINITY)) {
+        if (m_run != -INFINITY) {
+          factor = fast_exp2(m_run - m_new);
+          resc = true;
+        }
+        m_run = m_new;
+      }
+      // P = exp2(S*c - m), packed to bf16 pairs and stored over S_t 16 columns at a time.
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        if (ch >= 2 && nb == 1) break;
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(fmaf(sv[32 * ch + 2 * i], c, -m_use));
+          const float p1 = fast_exp2(fmaf(sv[32 * ch + 2 * i + 1], c, -m_use));
+          ls[i & 3] += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        BSA_TMEM_ST_X16(s_addr + 16 * ch, pk);
+      }
+      // factor is 1 unless this row's reference max moved; it scales only the old sum.
+      l_run = fmaf(l_run, factor, (ls[0] + ls[1]) + (ls[2] + ls[3]));
+      if (__any_sync(0xffffffffu, resc)) {
+        // O_t is quiescent: the PV of the previous step completed before S_full fired.
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float ov[32];
+          tmem_ld32(o_addr + c0, ov);
+          tmem_ld_wait();
+          uint32_t r[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(ov[i] * factor);
+          BSA_TMEM_ST_X16(o_addr + c0, r);
+          BSA_TMEM_ST_X16(o_addr + c0 + 16, (r + 16));
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_pfull + t);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    const float inv_l = (l_run > 0.f && q_valid) ? 1.f / l_run : 0.f;
+    bool have_o = ok && nsteps > 0;
+    if (have_o) {
+      have_o = __all_sync(0xffffffffu,
+                          mbar_wait(bar_ofull, 0, abort_flag, p.status, DETAIL_WAIT_O_FULL));
+      tc_fence_after();
+    }
+    __nv_bfloat16* orow = p.out + (static_cast<long long>(bh) * a.g.Np + slot) * D;
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      float ov[32];
+      if (have_o) {
+        tmem_ld32(o_addr + c0, ov);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] = 0.f;
+      }
+      if (in_range) {
+        uint4 w[4];
+        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) wp[i] = pack_bf16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l);
+        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = w[i];
+      }
+    }
+    if (p.lse != nullptr && in_range) {
+      const float lse = (l_run > 0.f && q_valid) ? (m_run + __log2f(l_run)) * 0.6931471805599453f
+                                                 : -INFINITY;
+      p.lse[static_cast<long long>(bh) * a.g.Np + slot] = lse;
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+size_t fwd_scratch_bytes(const AttnDims& a) {
+  const long long ctas = static_cast<long long>(a.batch) * a.heads * a.n_cta_per_head;
+  const size_t counts = (static_cast<size_t>(ctas) * 4 + 255) & ~static_cast<size_t>(255);
+  return counts + static_cast<size_t>(ctas) * a.n_kb * 4;
+}
+
+template <int D>
+static cudaError_t launch_fwd_bf16(const AttnDims& a, const void* q, const void* k, const void* v,
+                                   const FwdParams& prm, long long ctas, cudaStream_t stream) {
+  using L = FwdSmem<D>;
+  CUtensorMap tq, tk, tv;
+  const int bh = a.batch * a.heads;
+  cudaError_t e = encode_tmap_3d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.g.Np, bh, 64, 128);
+  if (e != cudaSuccess) return e;
+  e = encode_tmap_3d(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.g.Np, bh, 64, 64);
+  if (e != cudaSuccess) return e;
+  e = encode_tmap_3d(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.g.Np, bh, 64, 64);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bsattn_fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           L::kAlloc);
+  if (e != cudaSuccess) return e;
+  bsattn_fwd_bf16_kernel<D><<<static_cast<unsigned>(ctas), fwd::kThreads, L::kAlloc, stream>>>(
+      tq, tk, tv, prm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bsattn_fwd(const AttnDims& a, int fp8, const void* q, const void* k,
+                              const void* v, const float* q_scales, const float* k_scales,
+                              const float* v_scales, const int32_t* row_ptr,
+                              const int32_t* col_idx, float softmax_scale, void* out, float* lse,
+                              void* ws, cudaStream_t stream) {
+  (void)q_scales;
+  (void)k_scales;
+  (void)v_scales;
+  if (fp8) return cudaErrorNotSupported;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base);
+  const long long ctas = static_cast<long long>(a.batch) * a.heads * a.n_cta_per_head;
+  if (ctas == 0) return cudaSuccess;
+  const size_t counts_bytes = (static_cast<size_t>(ctas) * 4 + 255) & ~static_cast<size_t>(255);
+  int32_t* counts = reinterpret_cast<int32_t*>(base + kStatusBytes);
+  uint32_t* entries = reinterpret_cast<uint32_t*>(base + kStatusBytes + counts_bytes);
+  bsattn_schedule_kernel<<<static_cast<unsigned>(ctas), 256, 0, stream>>>(a, row_ptr, col_idx,
+                                                                         counts, entries, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  FwdParams prm;
+  prm.a = a;
+  prm.counts = counts;
+  prm.entries = entries;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.status = status;
+  prm.scale_log2 = softmax_scale * 1.4426950408889634f;
+  if (a.head_dim == 128) return launch_fwd_bf16<128>(a, q, k, v, prm, ctas, stream);
+  return launch_fwd_bf16<64>(a, q, k, v, prm, ctas, stream);
+}
+
+}  // namespace bsa

@@ -1,0 +1,316 @@
+// Dense calibration pass: exact softmax attention mass of every (query block, kv block)
+// pair, sm_100a.
+//
+// "LoSA: Near-Lossless Sparse Attention for Training-Free Video Diffusion Acceleration",
+// Abstract: the method measures exact block attention masses at one early dense step.
+//
+// mass[b,h,i,j] = mean over the valid queries q of block i of
+//                 sum over the valid keys k of block j of softmax_k(scale * q.k).
+//
+// One CTA owns 256 query slots (two M=128 tiles) and walks every kv block twice, two
+// blocks (N = 128 keys) per step:
+//   pass 1: S = Q K^T on the tensor cores, online row max and sum -> exact log-sum-exp;
+//   pass 2: S again, p = exp2(S*c - lse2), per-block row sums, then a sum over the rows
+//           of each query block (warp shuffles + shared memory, fixed order, so the result
+//           is deterministic).
+// Warp roles (320 threads): warps 0-3 / 4-7 row owners of tile 0 / 1, warp 8 TMA
+// producer (K only), warp 9 MMA issuer and TMEM owner.  TMEM holds two S buffers per
+// tile (4 x 128 columns), so the tensor core computes step s+1 while step s is reduced.
+#include "bsa_kernels.cuh"
+
+namespace bsa {
+
+namespace mass {
+constexpr int kThreads = 320;
+constexpr int kRowsPerCta = 256;
+}  // namespace mass
+
+struct MassParams {
+  AttnDims a;
+  float* mass;
+  uint32_t* status;
+  float scale_log2;
+};
+
+template <int D>
+struct MassSmem {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kQTile = 128 * D * 2;
+  static constexpr int kKStage = 128 * D * 2;
+  static constexpr int kKStages = (D == 128) ? 4 : 6;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = 2 * kQTile;
+  static constexpr int kRedOff = kKOff + kKStages * kKStage;   // float [2 parity][2 tile][4 warp][2 blk]
+  static constexpr int kBarOff = kRedOff + 2 * 2 * 4 * 2 * 4;
+  static constexpr int kBytes = kBarOff + 256;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(mass::kThreads, 1)
+    block_mass_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k, const MassParams p) {
+  using L = MassSmem<D>;
+  constexpr int KS = L::kKStages;
+  extern __shared__ uint8_t smem_raw[];
+  // 128-byte-swizzled operand tiles need 1024-byte alignment in the shared window.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_kfull = bars + 1;
+  uint64_t* bar_kempty = bar_kfull + KS;
+  uint64_t* bar_sfull = bar_kempty + KS;  // [tile][buf] = 4
+  uint64_t* bar_sempty = bar_sfull + 4;   // [tile][buf] = 4
+  uint64_t* bar_drain = bar_sempty + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* nvalid_sm = reinterpret_cast<int*>(tmem_slot + 2);  // [2 tile][4 warp]
+  float* red = reinterpret_cast<float*>(smem + L::kRedOff);
+
+  const AttnDims& a = p.a;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int cta = blockIdx.x;
+  const int bh = cta / a.n_cta_per_head;
+  const int row0 = (cta - bh * a.n_cta_per_head) * mass::kRowsPerCta;
+  const int npass = (a.n_kb + 1) >> 1;  // steps per pass
+  const int nsteps = 2 * npass;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < KS; ++i) {
+      mbar_init(bar_kfull + i, 1);
+      mbar_init(bar_kempty + i, 1);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(bar_sfull + i, 1);
+      mbar_init(bar_sempty + i, 128);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      mbar_arrive_expect_tx(bar_q, 2 * L::kQTile);
+      for (int t = 0; t < 2; ++t)
+        for (int ch = 0; ch < L::kChunks; ++ch)
+          tma_load_3d(smem + L::kQOff + t * L::kQTile + ch * (128 * 128), &tm_q, bar_q, ch * 64,
+                      row0 + t * 128, bh);
+      for (int s = 0; s < nsteps; ++s) {
+        const int st = s % npass;
+        const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+        const int ks = s % KS;
+        if (s >= KS && !mbar_wait(bar_kempty + ks, ((s / KS) - 1) & 1, abort_flag, p.status,
+                                  DETAIL_WAIT_K_EMPTY))
+          break;
+        mbar_arrive_expect_tx(bar_kfull + ks, nb * 64 * D * 2);
+        uint8_t* kst = smem + L::kKOff + ks * L::kKStage;
+        for (int ch = 0; ch < L::kChunks; ++ch) {
+          tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * 64, 2 * st * 64, bh);
+          if (nb == 2)
+            tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * 64,
+                        (2 * st + 1) * 64, bh);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {
+      const uint32_t q_base = smem_u32(smem + L::kQOff);
+      const uint32_t k_base = smem_u32(smem + L::kKOff);
+      bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, DETAIL_WAIT_Q);
+      for (int s = 0; s < nsteps && ok; ++s) {
+        const int st = s % npass;
+        const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+        const int ks = s % KS;
+        const int buf = s & 1;
+        const uint32_t idesc = make_idesc(1u, 0u, 128u, static_cast<uint32_t>(nb * 64));
+        if (!mbar_wait(bar_kfull + ks, (s / KS) & 1, abort_flag, p.status, DETAIL_WAIT_K_FULL)) {
+          ok = false;
+          break;
+        }
+        const uint32_t kb = k_base + ks * L::kKStage;
+        for (int t = 0; t < 2; ++t) {
+          if (s >= 2 && !mbar_wait(bar_sempty + 2 * t + buf, ((s >> 1) - 1) & 1, abort_flag,
+                                   p.status, DETAIL_WAIT_P_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t qb = q_base + t * L::kQTile;
+          const uint32_t s_tmem = tmem + (2 * t + buf) * 128;
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            mma_f16_ss(s_tmem, make_sdesc_sw128(qb + off, 16, 1024),
+                       make_sdesc_sw128(kb + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_sfull + 2 * t + buf);
+        }
+        if (!ok) break;
+        mma_commit(bar_kempty + ks);
+      }
+      mma_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0, p.status, DETAIL_WAIT_O_FULL);
+    }
+  } else {
+    const int t = warp >> 2;
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const int local = t * 128 + row;
+    const int slot = row0 + local;
+    const bool q_valid = slot < a.g.Np && slot_valid(a.g, slot);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const float c = p.scale_log2;
+    // valid queries per warp, then per query block
+    const int wcount = __popc(__ballot_sync(0xffffffffu, q_valid));
+    if (lane == 0) nvalid_sm[t * 4 + wq] = wcount;
+    named_bar_sync(1 + t, 128);
+    const int warps_per_qb = a.q_block / 32;  // 2 or 4
+    const int qb_first_warp = (wq / warps_per_qb) * warps_per_qb;
+    int nvq = 0;
+    for (int i = 0; i < warps_per_qb; ++i) nvq += nvalid_sm[t * 4 + qb_first_warp + i];
+    const int qb_global = (row0 + t * 128 + qb_first_warp * 32) / a.q_block;
+    const bool writer = (wq == qb_first_warp) && lane < 2 && qb_global < a.n_qb;
+    float* mass_row = p.mass + (static_cast<long long>(bh) * a.n_qb + qb_global) * a.n_kb;
+    const float inv_nvq = nvq > 0 ? 1.f / static_cast<float>(nvq) : 0.f;
+
+    float m_run = -INFINITY, l_run = 0.f, lse2 = 0.f;
+    bool ok = true;
+    for (int s = 0; s < nsteps; ++s) {
+      const int st = s % npass;
+      const bool pass2 = s >= npass;
+      const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+      const int buf = s & 1;
+      if (s == npass) lse2 = (l_run > 0.f) ? m_run + log2f(l_run) : INFINITY;
+      // A warp that gives up keeps stepping (without touching TMEM) so that every warp of
+      // the group passes the same named barriers.
+      bool got = ok ? mbar_wait(bar_sfull + 2 * t + buf, (s >> 1) & 1, abort_flag, p.status,
+                                DETAIL_WAIT_S_FULL)
+                    : false;
+      got = __all_sync(0xffffffffu, got);
+      ok = got;
+      float rs[2] = {0.f, 0.f};
+      if (got) {
+        float sv[128];
+        tc_fence_after();
+        const uint32_t s_addr = lane_base + (2 * t + buf) * 128;
+        tmem_ld32(s_addr + 0, sv + 0);
+        tmem_ld32(s_addr + 32, sv + 32);
+        if (nb == 2) {
+          tmem_ld32(s_addr + 64, sv + 64);
+          tmem_ld32(s_addr + 96, sv + 96);
+        }
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(bar_sempty + 2 * t + buf);
+        // Pad keys and the absent half of a 1-block step -> -inf (same for every row).
+        const int j0 = 2 * st;
+        const uint64_t mk0 = tile_has_pad(a.g, j0) ? tile_valid_mask(a.g, j0) : ~0ull;
+        const uint64_t mk1 =
+            nb == 2 ? (tile_has_pad(a.g, j0 + 1) ? tile_valid_mask(a.g, j0 + 1) : ~0ull) : 0ull;
+        if ((mk0 & mk1) != ~0ull) {
+          const uint32_t mw[4] = {static_cast<uint32_t>(mk0), static_cast<uint32_t>(mk0 >> 32),
+                                  static_cast<uint32_t>(mk1), static_cast<uint32_t>(mk1 >> 32)};
+#pragma unroll
+          for (int i = 0; i < 128; ++i) sv[i] = ((mw[i >> 5] >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
+        }
+        if (!pass2) {
+          float mx[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+#pragma unroll
+          for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
+          const float mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+          const float m_new = fmaxf(m_run, mrow * c);
+          if (m_new != -INFINITY) {
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 128; ++i) ls[i & 3] += fast_exp2(fmaf(sv[i], c, -m_new));
+            l_run = l_run * fast_exp2(m_run - m_new) + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+            m_run = m_new;
+          }
+        } else if (q_valid) {
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 64; ++i) acc[i & 3] += fast_exp2(fmaf(sv[64 * b + i], c, -lse2));
+            rs[b] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+          }
+        }
+      }
+      if (pass2) {
+        // Sum the per-row block masses over the rows of each query block: warp shuffles,
+        // then the 2 or 4 warps of the block through shared memory in a fixed order.
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          rs[0] += __shfl_xor_sync(0xffffffffu, rs[0], o);
+          rs[1] += __shfl_xor_sync(0xffffffffu, rs[1], o);
+        }
+        float* rbuf = red + ((s & 1) * 2 + t) * 8;
+        if (lane < 2) rbuf[wq * 2 + lane] = lane == 0 ? rs[0] : rs[1];
+        named_bar_sync(1 + t, 128);
+        if (writer && (lane < nb)) {
+          float tot = 0.f;
+          for (int i = 0; i < warps_per_qb; ++i) tot += rbuf[(qb_first_warp + i) * 2 + lane];
+          mass_row[2 * st + lane] = tot * inv_nvq;
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+size_t mass_scratch_bytes(const AttnDims& a) {
+  (void)a;
+  return 0;
+}
+
+template <int D>
+static cudaError_t launch_mass(const AttnDims& a, const void* q, const void* k,
+                               const MassParams& prm, long long ctas, cudaStream_t stream) {
+  using L = MassSmem<D>;
+  CUtensorMap tq, tk;
+  const int bh = a.batch * a.heads;
+  cudaError_t e = encode_tmap_3d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.g.Np, bh, 64, 128);
+  if (e != cudaSuccess) return e;
+  e = encode_tmap_3d(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.g.Np, bh, 64, 64);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(block_mass_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           L::kAlloc);
+  if (e != cudaSuccess) return e;
+  block_mass_kernel<D><<<static_cast<unsigned>(ctas), mass::kThreads, L::kAlloc, stream>>>(tq, tk,
+                                                                                          prm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_block_mass(const AttnDims& a, const void* q, const void* k, float softmax_scale,
+                              float* mass_out, void* ws, cudaStream_t stream) {
+  const long long ctas = static_cast<long long>(a.batch) * a.heads * a.n_cta_per_head;
+  if (ctas == 0) return cudaSuccess;
+  MassParams prm;
+  prm.a = a;
+  prm.mass = mass_out;
+  prm.status = static_cast<uint32_t*>(ws);
+  prm.scale_log2 = softmax_scale * 1.4426950408889634f;
+  if (a.head_dim == 128) return launch_mass<128>(a, q, k, prm, ctas, stream);
+  return launch_mass<64>(a, q, k, prm, ctas, stream);
+}
+
+}  // namespace bsa

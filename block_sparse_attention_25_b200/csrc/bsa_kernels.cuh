@@ -1,0 +1,117 @@
+// Internal interface between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include "bsa_common.cuh"
+
+namespace bsa {
+
+// Token grid of one (batch, head) slice.
+struct GridDims {
+  int T, H, W;     // valid grid
+  int Tp, Hp, Wp;  // padded grid (multiples of 4)
+  int nth, ntw;    // tiles along h and w (Hp/4, Wp/4)
+  int S, Np;       // valid tokens, padded slots
+};
+
+// Attention problem in tile-major layout.
+struct AttnDims {
+  GridDims g;
+  int batch, heads, head_dim;
+  int q_block;     // 64 or 128
+  int n_qb, n_kb;  // query blocks, kv blocks (64 slots each) per head
+  int n_cta_per_head;  // ceil(Np / 256): CTAs covering one head's query slots
+};
+
+// ---------------------------------------------------------------- grid geometry
+// Slot p of the tile-major order: tile = p / 64, inner = p % 64; tiles run row-major over
+// (t/4, h/4, w/4), inner slots row-major over (t%4, h%4, w%4).
+
+// Raster token index held by slot p, or -1 for a pad slot.
+__device__ __forceinline__ int slot_to_token(const GridDims& g, int p) {
+  const int tile = p >> 6, inner = p & 63;
+  const int tw = tile % g.ntw;
+  const int rest = tile / g.ntw;
+  const int th = rest % g.nth;
+  const int tt = rest / g.nth;
+  const int t = tt * 4 + (inner >> 4);
+  const int h = th * 4 + ((inner >> 2) & 3);
+  const int w = tw * 4 + (inner & 3);
+  if (t >= g.T || h >= g.H || w >= g.W) return -1;
+  return (t * g.H + h) * g.W + w;
+}
+
+__device__ __forceinline__ int token_to_slot(const GridDims& g, int s) {
+  const int w = s % g.W;
+  const int rest = s / g.W;
+  const int h = rest % g.H;
+  const int t = rest / g.H;
+  const int tile = ((t >> 2) * g.nth + (h >> 2)) * g.ntw + (w >> 2);
+  return tile * 64 + (((t & 3) * 4 + (h & 3)) * 4 + (w & 3));
+}
+
+__device__ __forceinline__ bool slot_valid(const GridDims& g, int p) {
+  return slot_to_token(g, p) >= 0;
+}
+
+// Valid-slot mask of tile j: bit i set when slot i of the tile lies inside the grid.
+__device__ __forceinline__ uint64_t tile_valid_mask(const GridDims& g, int j) {
+  const int tw = j % g.ntw;
+  const int rest = j / g.ntw;
+  const int th = rest % g.nth;
+  const int tt = rest / g.nth;
+  const int vt = min(4, max(0, g.T - 4 * tt));
+  const int vh = min(4, max(0, g.H - 4 * th));
+  const int vw = min(4, max(0, g.W - 4 * tw));
+  const uint64_t row4 = (1ull << vw) - 1ull;
+  uint64_t m16 = 0;
+  for (int i = 0; i < vh; ++i) m16 |= row4 << (4 * i);
+  uint64_t m64 = 0;
+  for (int i = 0; i < vt; ++i) m64 |= m16 << (16 * i);
+  return m64;
+}
+
+__device__ __forceinline__ bool tile_has_pad(const GridDims& g, int j) {
+  const int tw = j % g.ntw;
+  const int rest = j / g.ntw;
+  const int th = rest % g.nth;
+  const int tt = rest / g.nth;
+  return 4 * tt + 4 > g.T || 4 * th + 4 > g.H || 4 * tw + 4 > g.W;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+cudaError_t launch_tile_permute(const GridDims& g, int batch, int heads, int row_bytes,
+                                int inverse, const void* src, void* dst, cudaStream_t stream);
+
+cudaError_t launch_tile_permute_quant_e4m3(const GridDims& g, int batch, int heads, int head_dim,
+                                           const void* src, uint8_t* dst, float* scales,
+                                           cudaStream_t stream);
+
+// Top-p selection.  Workspace layout after the status header: counts int32 [R],
+// bitmaps uint32 [R][words].
+size_t topp_scratch_bytes(long long rows, int n_kb);
+cudaError_t launch_topp_select(const float* mass, long long rows, int n_kb, float threshold,
+                               int32_t* row_ptr, int32_t* col_idx, long long col_capacity,
+                               void* ws, cudaStream_t stream);
+
+// Block-sparse forward.  Scratch after the status header: per-CTA schedule.
+size_t fwd_scratch_bytes(const AttnDims& a);
+cudaError_t launch_bsattn_fwd(const AttnDims& a, int fp8, const void* q, const void* k,
+                              const void* v, const float* q_scales, const float* k_scales,
+                              const float* v_scales, const int32_t* row_ptr,
+                              const int32_t* col_idx, float softmax_scale, void* out, float* lse,
+                              void* ws, cudaStream_t stream);
+
+// Dense calibration pass.
+size_t mass_scratch_bytes(const AttnDims& a);
+cudaError_t launch_block_mass(const AttnDims& a, const void* q, const void* k, float softmax_scale,
+                              float* mass, void* ws, cudaStream_t stream);
+
+// Encode a rank-3 bf16/e4m3 tensor map over [bh][Np][D] with a (box_d x box_rows x 1) box
+// and 128-byte swizzle.
+cudaError_t encode_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                           int elem_bytes, int D, int Np, int bh, int box_d, int box_rows);
+
+}  // namespace bsa

@@ -1,0 +1,162 @@
+/*
+ * bsattn.h -- C ABI of libbsattn.so: retained-mass block-sparse self-attention over a
+ * long 3D video token sequence, written for NVIDIA B200 (sm_100a).
+ *
+ * The method: one dense calibration call measures the exact softmax attention mass of
+ * every (head, query block, key/value block) pair; for each head and query block the
+ * smallest key/value block set whose mass reaches a threshold (99% by default) is kept;
+ * later calls attend only over those frozen block lists.
+ *   - "LoSA: Near-Lossless Sparse Attention for Training-Free Video Diffusion
+ *     Acceleration", Abstract (masses, threshold, frozen lists).
+ *   - "FPSAttention: Training-Aware FP8 and Sparsity Co-Design for Fast Video
+ *     Diffusion", Abstract, innovation 1 (the 3D tile as the unit of sparsity and of
+ *     the FP8 scale).
+ *   - "Sparse VideoGen2: Accelerate Video Generation with Sparse Attention via
+ *     Semantic-Aware Permutation", Abstract (top-p dynamic budget control).
+ *
+ * Conventions shared by every call
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The library
+ *     allocates no memory and keeps no global state; scratch space is the caller's
+ *     workspace (`ws`), sized by bsa_workspace_bytes().
+ *   - Every call is asynchronous and ordered on `stream` (NULL = legacy default
+ *     stream).  A call returns after launching; results are ready when the stream is.
+ *   - Arguments are checked on the host before anything is launched.  A bad argument
+ *     returns a non-zero status and launches nothing.  Checks that need device data
+ *     (CSR contents, mass values, pipeline time limits) set bits in the status word at
+ *     the head of the workspace; read them with bsa_device_status().
+ *   - Errors cross the ABI only as bsa_status codes: no exceptions, no printing, no
+ *     exit, no trap.
+ *   - Layouts.  raster: [B, S, Hh, D] with S = T*H*W and token s = (t*H + h)*W + w.
+ *     tile-major: [B, Hh, Np, D] with Np = Tp*Hp*Wp; slot p = tile*64 + inner, where
+ *     tile = ((t/4)*(Hp/4) + h/4)*(Wp/4) + w/4 and inner = ((t%4)*4 + h%4)*4 + w%4.
+ *     Slots outside the valid T x H x W grid are pad slots.  Query block i is slots
+ *     [i*q_block, (i+1)*q_block); kv block j is slots [j*64, (j+1)*64), one tile.
+ *   - Sizes: head_dim in {64, 128}; q_block in {64, 128}; kv_block = 64; Tp, Hp, Wp
+ *     multiples of 4 covering T, H, W; B*Hh*Np*D < 2^31 elements per tensor is not
+ *     required (64-bit offsets are used), but B*Hh*(Np/q_block) rows must fit int32.
+ *   - Pointers to bf16 / fp32 / e4m3 tensors must be 16-byte aligned.
+ */
+#ifndef BSATTN_H
+#define BSATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BSA_API __attribute__((visibility("default")))
+#else
+#define BSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* bsa_stream_t;
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad alignment, bad threshold */
+  BSA_ERR_UNSUPPORTED = 2,   /* shape outside the supported set (head_dim, block sizes) */
+  BSA_ERR_CAPACITY = 3,      /* workspace or col_idx capacity too small */
+  BSA_ERR_CUDA = 4,          /* a CUDA runtime / driver call failed */
+  BSA_ERR_TIMEOUT = 5,       /* a device pipeline wait hit its time limit and gave up */
+  BSA_ERR_DEVICE_INPUT = 6   /* device data failed a check (CSR order/range, mass values) */
+} bsa_status;
+
+typedef enum { BSA_BF16 = 0, BSA_FP32 = 1, BSA_E4M3 = 2 } bsa_dtype;
+
+typedef enum { BSA_OP_BLOCK_MASS = 0, BSA_OP_TOPP_SELECT = 1, BSA_OP_FWD = 2 } bsa_op;
+
+typedef struct {
+  int32_t batch, heads, head_dim; /* B, Hh, D */
+  int32_t T, H, W;                /* valid token grid */
+  int32_t Tp, Hp, Wp;             /* padded grid, multiples of 4 */
+  int32_t q_block, kv_block;      /* tokens per query block (64 | 128), per kv block (64) */
+} bsa_shape;
+
+/* Bytes of workspace that `op` needs for `shape` (0 on an invalid shape).  Every
+ * workspace starts with a 256-byte status header; the rest is scratch whose contents
+ * do not persist meaningfully between calls. */
+BSA_API size_t bsa_workspace_bytes(const bsa_shape* shape, int op);
+
+/* Zero the status header of a workspace (stream-ordered).  Call once before the first
+ * use of a workspace and after reading an error. */
+BSA_API bsa_status bsa_clear_status(void* ws, bsa_stream_t stream);
+
+/* Synchronise `stream`, then report the status header of `ws`: BSA_OK, or the first
+ * error class recorded by a device-side check (TIMEOUT before DEVICE_INPUT before
+ * CAPACITY).  The header is left as it is. */
+BSA_API bsa_status bsa_device_status(const void* ws, bsa_stream_t stream);
+
+/* Raw status header words (flags, detail) for diagnostics; synchronises `stream`. */
+BSA_API bsa_status bsa_device_status_words(const void* ws, uint32_t out_words[4], bsa_stream_t stream);
+
+BSA_API const char* bsa_status_string(bsa_status status);
+
+/* 3D tile permutation ("FPSAttention", Abstract, innovation 1: unified 3D tile-wise
+ * granularity).  inverse = 0: raster src [B,S,Hh,D] -> tile-major dst [B,Hh,Np,D],
+ * pad slots written as zero.  inverse = 1: tile-major src -> raster dst, pad slots
+ * dropped.  dtype BSA_BF16 or BSA_FP32 (elements copied bit for bit).  src and dst
+ * must not overlap. */
+BSA_API bsa_status bsa_tile_permute(const bsa_shape* shape, bsa_dtype dtype, int inverse,
+                            const void* src, void* dst, bsa_stream_t stream);
+
+/* Permutation fused with per-tile FP8 quantisation ("FPSAttention", Abstract: FP8
+ * quantisation at the 3D tile granularity).  src: raster bf16 [B,S,Hh,D].  dst:
+ * tile-major e4m3 codes [B,Hh,Np,D].  tile_scales: fp32 [B,Hh,Np/64], one per
+ * (batch, head, 64-token tile): s = absmax/448 in fp32 (1 when the tile is all zero);
+ * code = e4m3 round-to-nearest-even, saturating, of x/s computed in fp32. */
+BSA_API bsa_status bsa_tile_permute_quant_e4m3(const bsa_shape* shape, const void* src_bf16,
+                                       uint8_t* dst, float* tile_scales, bsa_stream_t stream);
+
+/* Exact block attention masses at a dense step ("LoSA", Abstract: the masses of all
+ * block pairs are measured exactly on one early step that runs dense attention).  q, k: tile-major bf16 [B,Hh,Np,D] with
+ * zero pad slots.  mass: fp32 [B,Hh,Np/q_block,Np/64]; mass[b,h,i,j] is the mean over
+ * the valid queries of block i of the softmax(softmax_scale * q.k) probability on the
+ * valid keys of block j (pad keys excluded).  Rows of a block with no valid query are
+ * zero.  Two dense passes on tcgen05 tensor cores (log-sum-exp, then mass). */
+BSA_API bsa_status bsa_block_mass(const bsa_shape* shape, const void* q, const void* k,
+                          float softmax_scale, float* mass, void* ws, size_t ws_bytes,
+                          bsa_stream_t stream);
+
+/* Retained-mass (top-p) block selection ("LoSA", Abstract: per head and query block,
+ * the fewest kv blocks whose mass reaches the threshold are kept; "Sparse VideoGen2",
+ * Abstract: top-p dynamic budget control).  mass: fp32 [R, Np/64] with
+ * R = B*Hh*(Np/q_block), values finite in [0, 4096].  Per row, masses become integers
+ * q = rint(m * 2^40); target = ceil(threshold * sum q) (one fp64 multiply); blocks are
+ * ranked by (q desc, index asc) and the shortest prefix reaching the target is kept.
+ * Output CSR: row_ptr int32 [R+1] (row_ptr[0] = 0), col_idx int32 ascending within a
+ * row.  threshold in (0, 1].  col_capacity = entries available at col_idx; R*(Np/64)
+ * always suffices.  If the selection needs more, row_ptr is still complete, col_idx
+ * holds what fits and the status header records CAPACITY. */
+BSA_API bsa_status bsa_topp_select(const bsa_shape* shape, const float* mass, float threshold,
+                           int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                           void* ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* Block-sparse attention forward over frozen CSR block lists ("LoSA", Abstract: the
+ * frozen block indices are reused for all remaining steps).  For each query slot of
+ * row r = (b*Hh + h)*(Np/q_block) + p/q_block: softmax(softmax_scale * q.k) over the
+ * valid keys of the kv blocks col_idx[row_ptr[r] .. row_ptr[r+1]) only, times v.
+ * q, k, v: tile-major [B,Hh,Np,D]; dtype BSA_BF16 (q_scales etc. NULL) or BSA_E4M3
+ * (codes plus fp32 per-tile scales [B,Hh,Np/64] from bsa_tile_permute_quant_e4m3).
+ * col_idx must be strictly ascending within each row and < Np/64 (checked on the
+ * device; violations set DEVICE_INPUT and the row attends to the set of its indices).
+ * out: bf16 tile-major [B,Hh,Np,D]; pad query slots and rows with no kept valid key
+ * are written as zero.  lse (nullable): fp32 [B,Hh,Np], natural-log log-sum-exp of
+ * the kept logits (-inf where out is zero). */
+BSA_API bsa_status bsa_fwd(const bsa_shape* shape, bsa_dtype dtype,
+                   const void* q, const void* k, const void* v,
+                   const float* q_scales, const float* k_scales, const float* v_scales,
+                   const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale,
+                   void* out, float* lse, void* ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* Library build identification (static string). */
+BSA_API const char* bsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSATTN_H */

@@ -149,7 +149,8 @@ def block_mass_row(qt, kt, g: Grid, b: int, h: int, i: int, q_block: int, kv_blo
                    scale: float) -> np.ndarray:
     """Mass of query block i of head (b, h) over every kv block: float64 [Np // kv_block].
 
-    [LoSA] "exact block attention masses" at a dense step; definition per reading R2.
+    [LoSA] the block masses are measured exactly on one dense step; definition per
+    reading R2.
     qt, kt: tile-major [B, Hh, Np, D] arrays (any float dtype; widened to float64).
     """
     valid = valid_slots(g)
@@ -197,7 +198,8 @@ def topp_target(total: int, tau) -> int:
 def topp_select_row(m_row, tau) -> np.ndarray:
     """Smallest kv-block set whose mass reaches tau of the row's total.
 
-    [LoSA] "the smallest key/value block set meeting the threshold"; [SVG2] top-p.
+    [LoSA] per head and query block, the fewest kv blocks whose mass reaches the
+    threshold; [SVG2] top-p budget control.
     Greedy on the descending order is minimal: any k blocks hold at most the k largest
     masses.  Ties between equal masses go to the lower block index (reading R3).
     Returns the kept block indices ascending (int64).

@@ -1,0 +1,76 @@
+"""Shared helpers for the GPU parity tests: seeded inputs, oracle calls, comparisons."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from block_sparse_attention_25_b200 import synth
+from oracle import bsa_oracle as O
+
+# Tolerances (bf16 attention output against fp64; masses; FP8 output).
+ATTN_MAX_ABS = 2e-2
+ATTN_MEAN_ABS = 2e-3
+MASS_ABS = 1e-4
+FP8_MAX_ABS = 6e-2
+
+
+def grid_of(wl) -> O.Grid:
+    return O.Grid(wl.T, wl.H, wl.W, wl.Tp, wl.Hp, wl.Wp)
+
+
+def small_workloads():
+    """Shapes the oracle finishes in seconds that span several CTAs and ragged tails."""
+    W = synth.Workload
+    return [
+        # ragged pads in t, h, w; Np = 1152 -> 4.5 CTAs of 256 rows; 18 kv blocks
+        W("ragged-6x10x11-h3-d128-bq64", 1, 3, 128, 6, 10, 11, 8, 12, 12, 64, 64, seed=11),
+        # odd kv-block count (9), partial last Q tile, q_block 128 needs Np % 128 == 0
+        W("odd-3x9x10-h2-d128-bq64", 1, 2, 128, 3, 9, 10, 4, 12, 12, 64, 64, seed=12),
+        W("ragged-6x10x11-h2-d128-bq128", 1, 2, 128, 6, 10, 11, 8, 12, 12, 128, 64, seed=13),
+        W("ragged-5x7x9-h2-d64-bq64", 2, 2, 64, 5, 7, 9, 8, 8, 12, 64, 64, seed=14),
+        W("whole-pad-tiles-3x4x9-h2-d64-bq128", 1, 2, 64, 3, 4, 9, 8, 4, 12, 128, 64, seed=15),
+    ]
+
+
+def draw(wl, device="cpu", sharp=1.0, value_scale=None):
+    """bf16 raster q, k, v (CPU) for a workload; value_scale overrides the recipe's."""
+    if value_scale is not None:
+        wl = wl.scaled(value_scale=value_scale)
+    wl = wl.scaled(storage="bf16")
+    return synth.draw_qkv(wl, device=device, sharpness=sharp)
+
+
+def to_np64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def oracle_tiled(x_raster_bf16: torch.Tensor, g: O.Grid) -> np.ndarray:
+    """Oracle permutation of a bf16 raster tensor, as float64."""
+    return O.permute_forward(to_np64(x_raster_bf16), g)
+
+
+def attn_errors(got: np.ndarray, ref: np.ndarray):
+    err = np.abs(got - ref)
+    scale = max(np.abs(ref).max(), 1e-30)
+    return dict(max_abs=float(err.max()), mean_abs=float(err.mean()),
+                max_rel_to_max=float(err.max() / scale),
+                rms_rel=float(np.sqrt((err ** 2).mean()) / max(np.sqrt((ref ** 2).mean()), 1e-30)))
+
+
+def csr_from_oracle(mass64: np.ndarray, tau: float):
+    rp, ci = O.topp_select(mass64.astype(np.float32).reshape(-1, mass64.shape[-1]), tau)
+    return rp, ci
+
+
+def csr_to_device(rp, ci, device):
+    rp_t = torch.as_tensor(np.asarray(rp, dtype=np.int32), device=device)
+    ci_np = np.asarray(ci, dtype=np.int32)
+    if ci_np.size == 0:
+        ci_np = np.zeros(1, dtype=np.int32)
+    return rp_t, torch.as_tensor(ci_np, device=device)
+
+
+def scale_of(wl) -> float:
+    return 1.0 / math.sqrt(wl.head_dim)

@@ -1,0 +1,142 @@
+"""Host-only checks of the C ABI: the library loads, exports every declared symbol, sizes
+workspaces, and rejects bad arguments before launching anything.
+
+Every call here that passes pointers fails host-side validation by construction (bad
+shape, null or misaligned pointer, bad threshold, short workspace), so nothing is ever
+launched -- these tests are safe with or without a GPU.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bsattn.h")
+
+
+@pytest.fixture(scope="module")
+def B():
+    from block_sparse_attention_25_b200 import build
+    build.build()
+    import block_sparse_attention_25_b200 as b
+    b.lib()
+    return b
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"BSA_API\s+[\w\s\*]+?\b(bsa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_symbols()
+    for n in ("bsa_tile_permute", "bsa_block_mass", "bsa_topp_select", "bsa_fwd",
+              "bsa_tile_permute_quant_e4m3", "bsa_workspace_bytes", "bsa_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(B):
+    out = subprocess.run(["nm", "-D", "--defined-only", B.bsattn.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (bsa_\w+)", out))
+    missing = [n for n in declared_symbols() if n not in exported]
+    assert not missing, missing
+    for n in declared_symbols():
+        assert hasattr(B.lib(), n)
+
+
+def test_library_is_built_for_sm100a(B):
+    out = subprocess.run(["cuobjdump", "--list-elf", B.bsattn.LIB_PATH], capture_output=True,
+                         text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    assert "sm_100a" in out.stdout
+
+
+WL = dict(batch=1, heads=40, head_dim=128, T=21, H=45, W=80, Tp=24, Hp=48, Wp=80)
+
+
+def test_workspace_sizes(B):
+    s = B.Shape(**WL, q_block=64, kv_block=64)
+    R, nkb = s.rows, s.n_kb
+    assert B.workspace_bytes(s, B.OP_BLOCK_MASS) >= 256
+    assert B.workspace_bytes(s, B.OP_TOPP_SELECT) >= 256 + 4 * R + R * ((nkb + 31) // 32) * 4
+    ctas = s.batch * s.heads * ((s.Np + 255) // 256)
+    assert B.workspace_bytes(s, B.OP_FWD) >= 256 + 4 * ctas + ctas * nkb * 4
+    assert B.workspace_bytes(s, 99) == 0
+
+
+@pytest.mark.parametrize("bad", [
+    dict(head_dim=96), dict(q_block=96), dict(kv_block=128), dict(Tp=22), dict(Tp=20),
+    dict(heads=0), dict(W=0),
+])
+def test_invalid_shapes_have_no_workspace(B, bad):
+    kw = dict(WL, q_block=64, kv_block=64)
+    kw.update(bad)
+    assert B.workspace_bytes(B.Shape(**kw), B.OP_FWD) == 0
+
+
+def _c(B, **kw):
+    d = dict(WL, q_block=64, kv_block=64)
+    d.update(kw)
+    return ctypes.byref(B.Shape(**d).c())
+
+
+FAKE = ctypes.c_void_p(0x10000)       # aligned, never dereferenced: every call below fails validation
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def test_rejections_before_launch(B):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("fake-pointer validation checks run on hosts without a GPU only")
+    L = B.lib()
+    n = None
+    assert L.bsa_clear_status(n, n) == 1
+    assert L.bsa_tile_permute(None, 0, 0, FAKE, FAKE, n) == 1
+    assert L.bsa_tile_permute(_c(B), 0, 0, n, FAKE, n) == 1
+    assert L.bsa_tile_permute(_c(B), 0, 0, MISALIGNED, FAKE, n) == 1
+    assert L.bsa_tile_permute(_c(B), 2, 0, FAKE, FAKE, n) == 2          # e4m3 is not a permute dtype
+    assert L.bsa_tile_permute(_c(B), 0, 7, FAKE, FAKE, n) == 1          # inverse must be 0/1
+    assert L.bsa_tile_permute(_c(B, head_dim=96), 0, 0, FAKE, FAKE, n) == 2
+    assert L.bsa_tile_permute_quant_e4m3(_c(B), FAKE, FAKE, n, n) == 1
+    big = 1 << 40
+    assert L.bsa_block_mass(_c(B), FAKE, FAKE, 0.088, FAKE, FAKE, 0, n) == 3     # no workspace
+    assert L.bsa_block_mass(_c(B), FAKE, FAKE, -1.0, FAKE, FAKE, big, n) == 1    # bad scale
+    assert L.bsa_block_mass(_c(B, q_block=96), FAKE, FAKE, 0.088, FAKE, FAKE, big, n) == 2
+    assert L.bsa_topp_select(_c(B), FAKE, 1.5, FAKE, FAKE, 10, FAKE, big, n) == 1
+    assert L.bsa_topp_select(_c(B), FAKE, 0.0, FAKE, FAKE, 10, FAKE, big, n) == 1
+    assert L.bsa_topp_select(_c(B), FAKE, float("nan"), FAKE, FAKE, 10, FAKE, big, n) == 1
+    assert L.bsa_topp_select(_c(B), FAKE, 0.99, FAKE, n, 10, FAKE, big, n) == 1  # capacity w/o buffer
+    assert L.bsa_topp_select(_c(B), FAKE, 0.99, FAKE, FAKE, 10, FAKE, 16, n) == 3
+    args = [FAKE, FAKE, FAKE, n, n, n, FAKE, FAKE, 0.088, FAKE, n, FAKE]
+    assert L.bsa_fwd(_c(B), 0, *args, 16, n) == 3                            # short workspace
+    assert L.bsa_fwd(_c(B), 2, *args, big, n) == 1                           # e4m3 without scales
+    assert L.bsa_fwd(_c(B), 1, *args, big, n) == 2                           # fp32 not an attention dtype
+    bad = list(args)
+    bad[7] = n                                                               # col_idx missing
+    assert L.bsa_fwd(_c(B), 0, *bad, big, n) == 1
+    bad = list(args)
+    bad[9] = MISALIGNED                                                      # misaligned out
+    assert L.bsa_fwd(_c(B), 0, *bad, big, n) == 1
+    bad = list(args)
+    bad[10] = ctypes.c_void_p(0x10002)                                       # lse not 4-byte aligned
+    assert L.bsa_fwd(_c(B), 0, *bad, big, n) == 1
+    assert L.bsa_fwd(_c(B, T=30), 0, *args, big, n) == 1                     # T > Tp
+
+
+def test_status_strings(B):
+    L = B.lib()
+    for code in range(7):
+        assert L.bsa_status_string(code)
+    assert b"sm_100a" in L.bsa_version()
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import block_sparse_attention_25_b200.bsattn as m
+    monkeypatch.setattr(m, "_lib_handle", None)
+    monkeypatch.setattr(m, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        m.lib()
