@@ -302,7 +302,7 @@ def run_ours(args, world, rank, local, pg):
         "roofline": {
             "bound": "tensor", "achieved": round(fwd_tflops, 2), "peak": peak, "unit": "TFLOP/s",
             "frac": round(fwd_tflops / peak, 4), "traffic": None,
-            "kernel": "bsattn_fwd_bf16_kernel<128>" if not fp8 else "bsattn_fwd_e4m3_kernel",
+            "kernel": f"bsattn_fwd_kernel<{s.head_dim},{'true' if fp8 else 'false'}>",
             "peak_source": peak_note,
         },
         "gpu_launches": launches_per_step * args.steps,
@@ -318,7 +318,12 @@ def run_e2e(args, bsa, s, draws, n_reuse, row_ptr, col_idx, flops_call, dev, str
     """Same cycle through the public API, every input copied in from pinned host memory and
     every output copied back, inside the timed region."""
     import torch
-    host = [tuple(x.to("cpu").pin_memory() for x in d) for d in draws]
+    def pinned_copy(x):
+        h = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+        h.copy_(x)
+        return h
+
+    host = [tuple(pinned_copy(x) for x in d) for d in draws]
     out_host = [torch.empty((s.batch, s.S, s.heads, s.head_dim), dtype=torch.bfloat16).pin_memory()
                 for _ in range(n_reuse)]
     dq = torch.empty_like(draws[0][0])

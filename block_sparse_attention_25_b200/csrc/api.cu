@@ -243,6 +243,9 @@ bsa_status bsa_fwd(const bsa_shape* shape, bsa_dtype dtype, const void* q, const
     return BSA_ERR_INVALID_ARG;
   if (dtype == BSA_E4M3) {
     if (q_scales == nullptr || k_scales == nullptr || v_scales == nullptr) return BSA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(q_scales) | reinterpret_cast<uintptr_t>(k_scales) |
+         reinterpret_cast<uintptr_t>(v_scales)) & 3u)
+      return BSA_ERR_INVALID_ARG;
     if (shape->head_dim != 128) return BSA_ERR_UNSUPPORTED;
   } else if (dtype != BSA_BF16) {
     return BSA_ERR_UNSUPPORTED;

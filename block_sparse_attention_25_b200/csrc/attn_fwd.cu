@@ -49,9 +49,12 @@ __global__ void __launch_bounds__(256) bsattn_schedule_kernel(AttnDims a,
                                                               const int32_t* __restrict__ col_idx,
                                                               int32_t* __restrict__ counts,
                                                               uint32_t* __restrict__ entries,
+                                                              const float* __restrict__ v_scales,
+                                                              float* __restrict__ sigma,
                                                               uint32_t* status) {
   __shared__ uint32_t bm[4][128];  // up to 4096 kv blocks per query block
   __shared__ int warp_tot[8];
+  __shared__ float warp_max[8];
   const int cta = blockIdx.x;
   const int bh = cta / a.n_cta_per_head;
   const int c = cta - bh * a.n_cta_per_head;
@@ -81,6 +84,8 @@ __global__ void __launch_bounds__(256) bsattn_schedule_kernel(AttnDims a,
   }
   __syncthreads();
   uint32_t* out = entries + static_cast<long long>(cta) * a.n_kb;
+  const float* vsc = v_scales ? v_scales + static_cast<long long>(bh) * a.n_kb : nullptr;
+  float vmax = 0.f;
   int base = 0;
   for (int j0 = 0; j0 < a.n_kb; j0 += 256) {
     const int j = j0 + tid;
@@ -103,30 +108,52 @@ __global__ void __launch_bounds__(256) bsattn_schedule_kernel(AttnDims a,
     if (any) {
       const uint32_t pad = tile_has_pad(a.g, j) ? 1u : 0u;
       out[base + before + wpos] = (static_cast<uint32_t>(j) << 5) | (pad << 4) | keep;
+      if (vsc) vmax = fmaxf(vmax, vsc[j]);
     }
     base += tot;
     __syncthreads();
   }
   if (tid == 0) counts[cta] = base;
+  if (sigma != nullptr) {
+    // Largest V tile scale over the CTA's list: P is quantised relative to it.
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    if (lane_id() == 0) warp_max[tid >> 5] = vmax;
+    __syncthreads();
+    if (tid == 0) {
+      float m = 0.f;
+      for (int w = 0; w < 8; ++w) m = fmaxf(m, warp_max[w]);
+      sigma[cta] = m > 0.f ? m : 1.f;
+    }
+  }
 }
 
 struct FwdParams {
   AttnDims a;
   const int32_t* counts;
   const uint32_t* entries;
+  const float* q_scales;  // e4m3 only: per (bh, 64-token tile)
+  const float* k_scales;
+  const float* v_scales;
+  const float* sigma;     // e4m3 only: per CTA, max V tile scale over its list
   __nv_bfloat16* out;
   float* lse;
   uint32_t* status;
   float scale_log2;  // softmax_scale * log2(e)
 };
 
-template <int D>
+// Shared-memory plan.  Every operand row is cut into 128-byte swizzle chunks (64 bf16 or
+// 128 e4m3 elements); a 128-row tile of one chunk is 16 KB.
+template <int D, bool FP8>
 struct FwdSmem {
-  static constexpr int kChunks = D / 64;             // 128-byte swizzle chunks per row
-  static constexpr int kQTile = 128 * D * 2;         // one 128-row Q tile
-  static constexpr int kKVStage = 128 * D * 2;       // two 64-row kv blocks
-  static constexpr int kKStages = (D == 128) ? 3 : 4;
-  static constexpr int kVStages = (D == 128) ? 2 : 4;
+  static constexpr int kElem = FP8 ? 1 : 2;
+  static constexpr int kRowBytes = D * kElem;
+  static constexpr int kChunks = kRowBytes / 128;
+  static constexpr int kChunkElems = 128 / kElem;
+  static constexpr int kQTile = 128 * kRowBytes;     // one 128-row Q tile
+  static constexpr int kKVStage = 128 * kRowBytes;   // two 64-row kv blocks
+  static constexpr int kKStages = (kRowBytes == 256) ? 3 : 4;
+  static constexpr int kVStages = (kRowBytes == 256) ? 2 : 4;
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + 2 * kQTile;
   static constexpr int kVOff = kKOff + kKStages * kKVStage;
@@ -135,12 +162,17 @@ struct FwdSmem {
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
-template <int D>
+// e4m3 P is stored as P * (s_v / sigma) * kPScale: with the lazy rescale P <= 256, so the
+// largest code is 256 * 1.75 = 448, the e4m3 maximum.
+constexpr float kPScale = 1.75f;
+
+template <int D, bool FP8>
 __global__ void __launch_bounds__(fwd::kThreads, 1)
-    bsattn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
-                           const __grid_constant__ CUtensorMap tm_k,
-                           const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using L = FwdSmem<D>;
+    bsattn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdSmem<D, FP8>;
+  constexpr int CE = L::kChunkElems;
   constexpr int KS = L::kKStages, VS = L::kVStages;
   extern __shared__ uint8_t smem_raw[];
   // 128-byte-swizzled operand tiles need 1024-byte alignment in the shared window.
@@ -202,7 +234,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       mbar_arrive_expect_tx(bar_q, 2 * L::kQTile);
       for (int t = 0; t < 2; ++t)
         for (int ch = 0; ch < L::kChunks; ++ch)
-          tma_load_3d(smem + L::kQOff + t * L::kQTile + ch * (128 * 128), &tm_q, bar_q, ch * 64,
+          tma_load_3d(smem + L::kQOff + t * L::kQTile + ch * (128 * 128), &tm_q, bar_q, ch * CE,
                       row0 + t * 128, bh);
       for (int s = 0; s < nsteps; ++s) {
         const int nb = (2 * s + 1 < n_ent) ? 2 : 1;
@@ -212,24 +244,24 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         if (s >= KS && !mbar_wait(bar_kempty + ks, ((s / KS) - 1) & 1, abort_flag, p.status,
                                   DETAIL_WAIT_K_EMPTY))
           break;
-        mbar_arrive_expect_tx(bar_kfull + ks, nb * 64 * D * 2);
+        mbar_arrive_expect_tx(bar_kfull + ks, nb * 64 * L::kRowBytes);
         uint8_t* kst = smem + L::kKOff + ks * L::kKVStage;
         for (int ch = 0; ch < L::kChunks; ++ch) {
-          tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * 64, j0 * 64, bh);
+          tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * CE, j0 * 64, bh);
           if (nb == 2)
-            tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * 64,
+            tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * CE,
                         j1 * 64, bh);
         }
         const int vs = s % VS;
         if (s >= VS && !mbar_wait(bar_vempty + vs, ((s / VS) - 1) & 1, abort_flag, p.status,
                                   DETAIL_WAIT_V_EMPTY))
           break;
-        mbar_arrive_expect_tx(bar_vfull + vs, nb * 64 * D * 2);
+        mbar_arrive_expect_tx(bar_vfull + vs, nb * 64 * L::kRowBytes);
         uint8_t* vst = smem + L::kVOff + vs * L::kKVStage;
         for (int ch = 0; ch < L::kChunks; ++ch) {
-          tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * 64, j0 * 64, bh);
+          tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * CE, j0 * 64, bh);
           if (nb == 2)
-            tma_load_3d(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch * 64,
+            tma_load_3d(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch * CE,
                         j1 * 64, bh);
         }
       }
@@ -240,23 +272,30 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       const uint32_t q_base = smem_u32(smem + L::kQOff);
       const uint32_t k_base = smem_u32(smem + L::kKOff);
       const uint32_t v_base = smem_u32(smem + L::kVOff);
-      const uint32_t idesc_pv = make_idesc(1u, 1u, 128u, static_cast<uint32_t>(D));
+      constexpr uint32_t kFmt = FP8 ? 0u : 1u;  // e4m3 / bf16
+      const uint32_t idesc_pv = make_idesc(kFmt, 1u, 128u, static_cast<uint32_t>(D));
       bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, DETAIL_WAIT_Q);
       auto issue_pv = [&](int t, int sp) {
-        // O_t (+)= P_t(sp) V(sp); K dimension = keys of step sp (64 or 128).
+        // O_t (+)= P_t(sp) V(sp); K dimension = keys of step sp (64 or 128).  One MMA takes
+        // 32 bytes of K: 16 keys (bf16) or 32 keys (e4m3), i.e. 8 TMEM columns of P and
+        // 16 or 32 rows (2 or 4 swizzle atoms) of V.
+        constexpr int kKeysPerMma = 32 / L::kElem;
         const int nbp = (2 * sp + 1 < n_ent) ? 2 : 1;
         const uint32_t vb = v_base + (sp % VS) * L::kKVStage;
         const uint32_t p_tmem = tmem + t * 128;
         const uint32_t o_tmem = tmem + 256 + t * D;
-        for (int kk = 0; kk < nbp * 4; ++kk) {
-          const uint64_t bdesc = make_sdesc_sw128(vb + kk * 2048, 128 * 128, 1024);
-          mma_f16_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (sp > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < nbp * 64 / kKeysPerMma; ++kk) {
+          const uint64_t bdesc = make_sdesc_sw128(vb + kk * kKeysPerMma * 128, 128 * 128, 1024);
+          if constexpr (FP8)
+            mma_f8_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (sp > 0 || kk > 0) ? 1u : 0u);
+          else
+            mma_f16_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (sp > 0 || kk > 0) ? 1u : 0u);
         }
       };
       for (int s = 0; s < nsteps && ok; ++s) {
         const int ks = s % KS;
         const int nb = (2 * s + 1 < n_ent) ? 2 : 1;
-        const uint32_t idesc_qk = make_idesc(1u, 0u, 128u, static_cast<uint32_t>(nb * 64));
+        const uint32_t idesc_qk = make_idesc(kFmt, 0u, 128u, static_cast<uint32_t>(nb * 64));
         if (!mbar_wait(bar_kfull + ks, (s / KS) & 1, abort_flag, p.status, DETAIL_WAIT_K_FULL)) {
           ok = false;
           break;
@@ -280,11 +319,15 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           }
           const uint32_t qb = q_base + t * L::kQTile;
           const uint32_t s_tmem = tmem + t * 128;
-          for (int kk = 0; kk < D / 16; ++kk) {
+          // K (= head dim) advances 32 bytes per MMA inside each 128-byte swizzle chunk.
+          for (int kk = 0; kk < L::kRowBytes / 32; ++kk) {
             const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
             const uint64_t adesc = make_sdesc_sw128(qb + off, 16, 1024);
             const uint64_t bdesc = make_sdesc_sw128(kb + off, 16, 1024);
-            mma_f16_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+            if constexpr (FP8)
+              mma_f8_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+            else
+              mma_f16_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar_sfull + t);
         }
@@ -326,6 +369,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     const uint32_t s_addr = lane_base + t * 128;
     const uint32_t o_addr = lane_base + 256 + t * D;
     const float c = p.scale_log2;
+    // e4m3: logits carry the Q tile scale of this row and the K tile scale of each block.
+    float cq = c;
+    float sig = 1.f;
+    if constexpr (FP8) {
+      const long long tbase = static_cast<long long>(bh) * a.n_kb;
+      cq = c * (in_range ? p.q_scales[tbase + (slot >> 6)] : 0.f);
+      sig = p.sigma[cta];
+    }
     float m_run = -INFINITY;  // running max, scaled log2 units
     float l_run = 0.f;
     bool ok = true;
@@ -366,14 +417,30 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 128; ++i) sv[i] = ((mw[i >> 5] >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
       }
+      // log2-domain multiplier of each half (block) of the step
+      float fb0 = c, fb1 = c, pv0 = 1.f, pv1 = 1.f;
+      if constexpr (FP8) {
+        const long long tbase = static_cast<long long>(bh) * a.n_kb;
+        const int j0 = fwd::entry_block(e0), j1 = fwd::entry_block(e1);
+        fb0 = cq * p.k_scales[tbase + j0];
+        fb1 = nb == 2 ? cq * p.k_scales[tbase + j1] : 0.f;
+        pv0 = p.v_scales[tbase + j0] / sig * kPScale;
+        pv1 = nb == 2 ? p.v_scales[tbase + j1] / sig * kPScale : 0.f;
+      }
       float mx[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+      for (int i = 0; i < 4; ++i) mx[i] = sv[i];
 #pragma unroll
-      for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
-      float mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      const float m_new = mrow * c;
+      for (int i = 4; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], sv[i]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mx[4 + i] = sv[64 + i];
+#pragma unroll
+      for (int i = 68; i < 128; ++i) mx[4 + (i & 3)] = fmaxf(mx[4 + (i & 3)], sv[i]);
+      const float mh0 = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float mh1 = fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+      // multipliers are > 0, so the scaled max is the max of the scaled half maxima
+      const float m_new = fmaxf(mh0 == -INFINITY ? -INFINITY : mh0 * fb0,
+                                mh1 == -INFINITY ? -INFINITY : mh1 * fb1);
       float factor = 1.f;
       bool resc = false;
       if (m_new > m_run + fwd::kRescaleLog2 || (m_run == -INFINITY && m_new != -INFINITY)) {
@@ -383,21 +450,45 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         }
         m_run = m_new;
       }
-      // P = exp2(S*c - m), packed to bf16 pairs and stored over S_t 16 columns at a time.
+      // P = exp2(S*f - m), stored over S_t as it is produced: bf16 pairs, 16 columns per 32
+      // keys; or e4m3 quads (P scaled by the block's V scale), 16 columns per 64 keys.
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (!FP8) {
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        if (ch >= 2 && nb == 1) break;
-        uint32_t pk[16];
+        for (int ch = 0; ch < 4; ++ch) {
+          if (ch >= 2 && nb == 1) break;
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(fmaf(sv[32 * ch + 2 * i], c, -m_use));
-          const float p1 = fast_exp2(fmaf(sv[32 * ch + 2 * i + 1], c, -m_use));
-          ls[i & 3] += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = fast_exp2(fmaf(sv[32 * ch + 2 * i], c, -m_use));
+            const float p1 = fast_exp2(fmaf(sv[32 * ch + 2 * i + 1], c, -m_use));
+            ls[i & 3] += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          BSA_TMEM_ST_X16(s_addr + 16 * ch, pk);
         }
-        BSA_TMEM_ST_X16(s_addr + 16 * ch, pk);
+      } else {
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          if (b == 1 && nb == 1) break;
+          const float fb = b ? fb1 : fb0;
+          const float pv = b ? pv1 : pv0;
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float pq[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              pq[u] = fast_exp2(fmaf(sv[64 * b + 4 * i + u], fb, -m_use));
+              ls[u] += pq[u];
+            }
+            const uint32_t lo = pack_e4m3x2(pq[0] * pv, pq[1] * pv);
+            const uint32_t hi = pack_e4m3x2(pq[2] * pv, pq[3] * pv);
+            pk[i] = lo | (hi << 16);
+          }
+          BSA_TMEM_ST_X16(s_addr + 16 * b, pk);
+        }
       }
       // factor is 1 unless this row's reference max moved; it scales only the old sum.
       l_run = fmaf(l_run, factor, (ls[0] + ls[1]) + (ls[2] + ls[3]));
@@ -421,7 +512,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     }
 
     // ------------------------------------------------------------ epilogue
-    const float inv_l = (l_run > 0.f && q_valid) ? 1.f / l_run : 0.f;
+    // e4m3: O was accumulated from P * s_v / sigma * kPScale and V / s_v.
+    const float o_mult = FP8 ? sig / kPScale : 1.f;
+    const float inv_l = (l_run > 0.f && q_valid) ? o_mult / l_run : 0.f;
     bool have_o = ok && nsteps > 0;
     if (have_o) {
       have_o = __all_sync(0xffffffffu,
@@ -465,28 +558,32 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   }
 }
 
+// Scratch after the status header: counts int32 [ctas], sigma fp32 [ctas] (e4m3 only),
+// entries uint32 [ctas][n_kb].
 size_t fwd_scratch_bytes(const AttnDims& a) {
   const long long ctas = static_cast<long long>(a.batch) * a.heads * a.n_cta_per_head;
   const size_t counts = (static_cast<size_t>(ctas) * 4 + 255) & ~static_cast<size_t>(255);
-  return counts + static_cast<size_t>(ctas) * a.n_kb * 4;
+  return 2 * counts + static_cast<size_t>(ctas) * a.n_kb * 4;
 }
 
-template <int D>
-static cudaError_t launch_fwd_bf16(const AttnDims& a, const void* q, const void* k, const void* v,
-                                   const FwdParams& prm, long long ctas, cudaStream_t stream) {
-  using L = FwdSmem<D>;
+template <int D, bool FP8>
+static cudaError_t launch_fwd(const AttnDims& a, const void* q, const void* k, const void* v,
+                              const FwdParams& prm, long long ctas, cudaStream_t stream) {
+  using L = FwdSmem<D, FP8>;
   CUtensorMap tq, tk, tv;
   const int bh = a.batch * a.heads;
-  cudaError_t e = encode_tmap_3d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.g.Np, bh, 64, 128);
+  const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int eb = L::kElem, ce = L::kChunkElems;
+  cudaError_t e = encode_tmap_3d(&tq, q, dt, eb, D, a.g.Np, bh, ce, 128);
   if (e != cudaSuccess) return e;
-  e = encode_tmap_3d(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.g.Np, bh, 64, 64);
+  e = encode_tmap_3d(&tk, k, dt, eb, D, a.g.Np, bh, ce, 64);
   if (e != cudaSuccess) return e;
-  e = encode_tmap_3d(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.g.Np, bh, 64, 64);
+  e = encode_tmap_3d(&tv, v, dt, eb, D, a.g.Np, bh, ce, 64);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(bsattn_fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(bsattn_fwd_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            L::kAlloc);
   if (e != cudaSuccess) return e;
-  bsattn_fwd_bf16_kernel<D><<<static_cast<unsigned>(ctas), fwd::kThreads, L::kAlloc, stream>>>(
+  bsattn_fwd_kernel<D, FP8><<<static_cast<unsigned>(ctas), fwd::kThreads, L::kAlloc, stream>>>(
       tq, tk, tv, prm);
   return cudaGetLastError();
 }
@@ -496,31 +593,35 @@ cudaError_t launch_bsattn_fwd(const AttnDims& a, int fp8, const void* q, const v
                               const float* v_scales, const int32_t* row_ptr,
                               const int32_t* col_idx, float softmax_scale, void* out, float* lse,
                               void* ws, cudaStream_t stream) {
-  (void)q_scales;
-  (void)k_scales;
-  (void)v_scales;
-  if (fp8) return cudaErrorNotSupported;
+  if (fp8 && a.head_dim != 128) return cudaErrorNotSupported;
   uint8_t* base = static_cast<uint8_t*>(ws);
   uint32_t* status = reinterpret_cast<uint32_t*>(base);
   const long long ctas = static_cast<long long>(a.batch) * a.heads * a.n_cta_per_head;
   if (ctas == 0) return cudaSuccess;
   const size_t counts_bytes = (static_cast<size_t>(ctas) * 4 + 255) & ~static_cast<size_t>(255);
   int32_t* counts = reinterpret_cast<int32_t*>(base + kStatusBytes);
-  uint32_t* entries = reinterpret_cast<uint32_t*>(base + kStatusBytes + counts_bytes);
-  bsattn_schedule_kernel<<<static_cast<unsigned>(ctas), 256, 0, stream>>>(a, row_ptr, col_idx,
-                                                                         counts, entries, status);
+  float* sigma = reinterpret_cast<float*>(base + kStatusBytes + counts_bytes);
+  uint32_t* entries = reinterpret_cast<uint32_t*>(base + kStatusBytes + 2 * counts_bytes);
+  bsattn_schedule_kernel<<<static_cast<unsigned>(ctas), 256, 0, stream>>>(
+      a, row_ptr, col_idx, counts, entries, fp8 ? v_scales : nullptr, fp8 ? sigma : nullptr,
+      status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   FwdParams prm;
   prm.a = a;
   prm.counts = counts;
   prm.entries = entries;
+  prm.q_scales = q_scales;
+  prm.k_scales = k_scales;
+  prm.v_scales = v_scales;
+  prm.sigma = sigma;
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.lse = lse;
   prm.status = status;
   prm.scale_log2 = softmax_scale * 1.4426950408889634f;
-  if (a.head_dim == 128) return launch_fwd_bf16<128>(a, q, k, v, prm, ctas, stream);
-  return launch_fwd_bf16<64>(a, q, k, v, prm, ctas, stream);
+  if (fp8) return launch_fwd<128, true>(a, q, k, v, prm, ctas, stream);
+  if (a.head_dim == 128) return launch_fwd<128, false>(a, q, k, v, prm, ctas, stream);
+  return launch_fwd<64, false>(a, q, k, v, prm, ctas, stream);
 }
 
 }  // namespace bsa

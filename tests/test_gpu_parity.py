@@ -289,3 +289,75 @@ def test_pipeline_calibrate_then_reuse(B, wl):
     rows = np.repeat(same.reshape(s.batch, s.heads, n_qb), wl.q_block, axis=2)
     e = Hp.attn_errors(got[rows], o_ref[rows])
     assert e["max_abs"] <= Hp.ATTN_MAX_ABS and e["mean_abs"] <= Hp.ATTN_MEAN_ABS, e
+
+
+# ------------------------------------------------------------------ FP8 attention
+FP8_WLS = [w for w in WLS if w.head_dim == 128]
+
+
+def _fp8_compare(B, wl, q, k, v, rp, ci):
+    """GPU: quantise (bit-exact against the oracle's quantiser) and attend in e4m3.
+    Oracle: its own quantisation, dequantised to fp64, masked attention."""
+    g = Hp.grid_of(wl)
+    s = _shape(B, wl)
+    gq = [B.tile_permute_quant_e4m3(x.cuda(), s) for x in (q, k, v)]
+    deq = []
+    for x, (codes, scales) in zip((q, k, v), gq):
+        rc, rs = O.quant_e4m3_tiles(O.permute_forward(x.float().numpy(), g))
+        assert np.array_equal(codes.cpu().numpy(), rc)
+        assert np.array_equal(scales.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+        deq.append(O.dequant_e4m3_tiles(rc, rs))
+    rp_d, ci_d = Hp.csr_to_device(rp, ci, "cuda")
+    ws = B.new_workspace(s, B.OP_FWD)
+    out, lse = B.bsattn_fwd(gq[0][0], gq[1][0], gq[2][0], rp_d, ci_d, s,
+                            scales=(gq[0][1], gq[1][1], gq[2][1]), want_lse=True, ws=ws)
+    assert B.device_status(ws) == 0, B.device_status_words(ws)
+    o_ref, lse_ref = O.masked_attention(deq[0], deq[1], deq[2], g, wl.q_block, 64, rp, ci,
+                                        Hp.scale_of(wl))
+    got = out.cpu().double().numpy()
+    e = Hp.attn_errors(got, o_ref)
+    assert e["max_abs"] <= Hp.FP8_MAX_ABS, e
+    zero = ~np.isfinite(lse_ref)
+    assert np.all(got[zero] == 0)
+    lg = lse.cpu().double().numpy()
+    if (~zero).any():
+        assert np.abs(lg[~zero] - lse_ref[~zero]).max() <= 1e-3
+    return e
+
+
+@pytest.mark.parametrize("wl", FP8_WLS, ids=[w.name for w in FP8_WLS])
+@pytest.mark.parametrize("sharp", [1.0, 6.0])
+def test_fwd_fp8_parity_oracle_csr(B, wl, sharp):
+    g = Hp.grid_of(wl)
+    q, k, v = Hp.draw(wl, value_scale=1.0, sharp=sharp)
+    mass = O.block_mass(Hp.oracle_tiled(q, g), Hp.oracle_tiled(k, g), g, wl.q_block, 64,
+                        Hp.scale_of(wl))
+    rp, ci = Hp.csr_from_oracle(mass, 0.99)
+    _fp8_compare(B, wl, q, k, v, rp, ci)
+
+
+@pytest.mark.parametrize("wl", FP8_WLS, ids=[w.name for w in FP8_WLS])
+def test_fwd_fp8_parity_random_csr(B, wl):
+    q, k, v = Hp.draw(wl, value_scale=1.0, sharp=4.0)
+    n_qb, n_kb = wl.Np // wl.q_block, wl.Np // 64
+    R = wl.batch * wl.heads * n_qb
+    rp, ci = synth.draw_keep_csr(R, n_kb, 0.5, seed=wl.seed + 200, empty_rows=(1,))
+    _fp8_compare(B, wl, q, k, v, rp.numpy(), ci.numpy())
+
+
+def test_fwd_fp8_rescale_path(B):
+    """Growing logits across kv blocks exercise the lazy rescale with e4m3 P."""
+    wl = FP8_WLS[0]
+    g = Hp.grid_of(wl)
+    q, k, v = Hp.draw(wl, value_scale=1.0)
+    kt = O.permute_forward(k.float().numpy(), g)
+    n_kb = wl.Np // 64
+    for j in range(n_kb):
+        kt[:, :, j * 64:(j + 1) * 64] *= (1.0 + 1.5 * j)
+    k2 = torch.from_numpy(O.permute_inverse(kt, g)).to(torch.bfloat16)
+    q2 = (q.float() * 4.0).to(torch.bfloat16)
+    n_qb = wl.Np // wl.q_block
+    R = wl.batch * wl.heads * n_qb
+    rp = np.arange(R + 1) * n_kb
+    ci = np.tile(np.arange(n_kb), R)
+    _fp8_compare(B, wl, q2, k2, v, rp, ci)
