@@ -105,6 +105,7 @@ def lib() -> ctypes.CDLL:
         "bsa_tile_permute_quant_e4m3": (I, [SP, P, P, P, P]),
         "bsa_block_mass": (I, [SP, P, P, F, P, P, S, P]),
         "bsa_topp_select": (I, [SP, P, F, P, P, L64, P, S, P]),
+        "bsa_topp_select_noalloc": (I, [SP, P, F, P, P, L64, P, P]),
         "bsa_fwd": (I, [SP, I, P, P, P, P, P, P, P, P, F, P, P, P, S, P]),
         "bsa_version": (ctypes.c_char_p, []),
     }
@@ -119,7 +120,7 @@ def lib() -> ctypes.CDLL:
 EXPORTED_SYMBOLS = ("bsa_workspace_bytes", "bsa_clear_status", "bsa_device_status",
                     "bsa_device_status_words", "bsa_status_string", "bsa_tile_permute",
                     "bsa_tile_permute_quant_e4m3", "bsa_block_mass", "bsa_topp_select", "bsa_fwd",
-                    "bsa_version")
+                    "bsa_topp_select_noalloc", "bsa_version")
 
 
 def _check(status: int, what: str):
@@ -245,6 +246,24 @@ def topp_select(mass, shape: Shape, threshold: float = 0.99, col_capacity=None, 
     _check(lib().bsa_topp_select(ctypes.byref(shape.c()), _ptr(mass), float(threshold),
                                  _ptr(row_ptr), _ptr(col_idx), cap, _ptr(ws), ws.numel(),
                                  _stream(stream)), "bsa_topp_select")
+    return row_ptr, col_idx
+
+
+def topp_select_noalloc(mass, shape: Shape, threshold: float = 0.99, row_ptr=None, col_idx=None,
+                        col_capacity=None, status=None, stream=None):
+    """bsa_topp_select_noalloc: the same selection with the library's own fixed scratch (for
+    callers that cannot provide a workspace).  status: optional int32/uint32 CUDA tensor of
+    4 words receiving the device-side flags."""
+    R = shape.rows
+    _need(mass, torch.float32, (shape.batch, shape.heads, shape.n_qb, shape.n_kb), "mass")
+    cap = R * shape.n_kb if col_capacity is None else int(col_capacity)
+    if row_ptr is None:
+        row_ptr = torch.empty(R + 1, dtype=torch.int32, device=mass.device)
+    if col_idx is None:
+        col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=mass.device)
+    _check(lib().bsa_topp_select_noalloc(ctypes.byref(shape.c()), _ptr(mass), float(threshold),
+                                         _ptr(row_ptr), _ptr(col_idx), cap, _ptr(status),
+                                         _stream(stream)), "bsa_topp_select_noalloc")
     return row_ptr, col_idx
 
 

@@ -228,6 +228,25 @@ bsa_status bsa_topp_select(const bsa_shape* shape, const float* mass, float thre
                                            col_capacity, ws, stream));
 }
 
+bsa_status bsa_topp_select_noalloc(const bsa_shape* shape, const float* mass, float threshold,
+                                   int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                   uint32_t* status, bsa_stream_t stream) {
+  bsa_status st = check_shape(shape, true);
+  if (st != BSA_OK) return st;
+  if (mass == nullptr || row_ptr == nullptr || (reinterpret_cast<uintptr_t>(mass) & 3u) ||
+      (status != nullptr && (reinterpret_cast<uintptr_t>(status) & 3u)))
+    return BSA_ERR_INVALID_ARG;
+  if (col_capacity < 0 || (col_capacity > 0 && col_idx == nullptr)) return BSA_ERR_INVALID_ARG;
+  if (!(threshold > 0.f && threshold <= 1.f)) return BSA_ERR_INVALID_ARG;
+  const AttnDims a = make_attn(shape);
+  const long long rows = 1LL * a.batch * a.heads * a.n_qb;
+  // The scratch is the library's fixed per-device array: larger problems are refused.
+  if (bsa::topp_scratch_bytes(rows, a.n_kb) > bsa::topp_noalloc_capacity_bytes())
+    return BSA_ERR_CAPACITY;
+  return from_cuda(bsa::launch_topp_select_noalloc(mass, rows, a.n_kb, threshold, row_ptr, col_idx,
+                                                   col_capacity, status, stream));
+}
+
 bsa_status bsa_fwd(const bsa_shape* shape, bsa_dtype dtype, const void* q, const void* k,
                    const void* v, const float* q_scales, const float* k_scales,
                    const float* v_scales, const int32_t* row_ptr, const int32_t* col_idx,

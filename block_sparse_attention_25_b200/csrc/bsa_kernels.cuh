@@ -96,6 +96,13 @@ cudaError_t launch_topp_select(const float* mass, long long rows, int n_kb, floa
                                int32_t* row_ptr, int32_t* col_idx, long long col_capacity,
                                void* ws, cudaStream_t stream);
 
+// Allocation-free selection: scratch in a fixed device array owned by the library
+// (kNoAllocScratchBytes per device); status is a caller buffer of 4 words or null.
+size_t topp_noalloc_capacity_bytes();
+cudaError_t launch_topp_select_noalloc(const float* mass, long long rows, int n_kb, float threshold,
+                                       int32_t* row_ptr, int32_t* col_idx, long long col_capacity,
+                                       uint32_t* status, cudaStream_t stream);
+
 // Block-sparse forward.  Scratch after the status header: per-CTA schedule.
 size_t fwd_scratch_bytes(const AttnDims& a);
 cudaError_t launch_bsattn_fwd(const AttnDims& a, int fp8, const void* q, const void* k,

@@ -17,6 +17,8 @@
 // Kernels: (1) select, one 256-thread CTA per row -> kept bitmap + count in the
 // workspace; (2) exclusive scan of the counts -> row_ptr; (3) compaction, one warp per
 // row -> col_idx ascending.
+#include <mutex>
+
 #include "bsa_kernels.cuh"
 
 namespace bsa {
@@ -289,6 +291,75 @@ cudaError_t launch_topp_select(const float* mass, long long rows, int n_kb, floa
   topp_select_rows_kernel<<<static_cast<unsigned>(rows), kToppThreads, 0, stream>>>(
       mass, n_kb, static_cast<double>(threshold), counts, bitmaps, words, status);
   cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  topp_scan_kernel<<<1, 1024, 0, stream>>>(counts, rows, row_ptr);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  topp_fill_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+      bitmaps, words, rows, row_ptr, col_idx, col_capacity, status);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------------------
+// Allocation-free variant of the selection.
+//
+// Some callers cannot hand the library a workspace: a plugin inside a serving engine whose
+// memory planner reserves all device memory up front and forbids ad-hoc cudaMalloc, code
+// on a latency-critical path where cudaMalloc's implicit synchronisation would stall the
+// stream, or a runtime that owns every device allocation through its own pool.  For them
+// the selection's scratch (per-row counts and kept bitmaps) lives in a fixed array in the
+// library's own device memory, sized for the largest shapes this library targets.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
+
+// Every GPU that loads the library holds this array until the process exits.  In host
+// code its name is only a host-side stand-in; the device address comes from
+// cudaGetSymbolAddress below.
+static __device__ __align__(256) uint8_t g_topp_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {nullptr};
+
+// Device address of the scratch array for the current device, looked up once per device
+// (with that device current) and cached.
+cudaError_t noalloc_scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_topp_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+size_t topp_noalloc_capacity_bytes() { return kNoAllocScratchBytes; }
+
+cudaError_t launch_topp_select_noalloc(const float* mass, long long rows, int n_kb, float threshold,
+                                       int32_t* row_ptr, int32_t* col_idx, long long col_capacity,
+                                       uint32_t* status, cudaStream_t stream) {
+  void* scratch = nullptr;
+  cudaError_t e = noalloc_scratch_address(&scratch);
+  if (e != cudaSuccess) return e;
+  if (rows == 0) return cudaMemsetAsync(row_ptr, 0, sizeof(int32_t), stream);
+  // Same layout as the workspace scratch: counts int32 [rows] (256-byte aligned), then
+  // bitmaps uint32 [rows][words].  Both are fully rewritten by every call.
+  const int words = (n_kb + 31) / 32;
+  const size_t counts_bytes = (static_cast<size_t>(rows) * 4 + 255) & ~static_cast<size_t>(255);
+  int32_t* counts = static_cast<int32_t*>(scratch);
+  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(scratch) + counts_bytes);
+  topp_select_rows_kernel<<<static_cast<unsigned>(rows), kToppThreads, 0, stream>>>(
+      mass, n_kb, static_cast<double>(threshold), counts, bitmaps, words, status);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   topp_scan_kernel<<<1, 1024, 0, stream>>>(counts, rows, row_ptr);
   e = cudaGetLastError();

@@ -135,6 +135,32 @@ BSA_API bsa_status bsa_topp_select(const bsa_shape* shape, const float* mass, fl
                            int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
                            void* ws, size_t ws_bytes, bsa_stream_t stream);
 
+/* Allocation-free variant of bsa_topp_select.  No counterpart in the papers: this is an
+ * interface for callers that cannot give the library a workspace -- for example a plugin
+ * inside a serving engine whose memory planner owns all device memory and forbids ad-hoc
+ * cudaMalloc, or code on a latency-critical path where cudaMalloc's implicit device
+ * synchronisation would stall the stream.  Inputs, outputs and results are exactly those
+ * of bsa_topp_select; only the scratch (per-row counts and kept bitmaps) differs: it lives
+ * in a fixed 16 MiB array in the library's own device memory, which every GPU that loads
+ * the library holds until the process exits.  This call allocates nothing (no cudaMalloc,
+ * no cudaFree, no allocating library routine).
+ *   - Size limit: R*4 rounded up to 256 bytes, plus R*ceil((Np/64)/32)*4 bytes, must fit in
+ *     16 MiB (R = B*Hh*Np/q_block); larger problems return BSA_ERR_CAPACITY and launch
+ *     nothing.  The 720p 40-head shape needs 10.6 MB.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current) and caches it; make that first call before any stream
+ *     capture.
+ *   - Every call shares the one array and leaves its contents behind; each call rewrites
+ *     all of the scratch it reads, so nothing needs clearing, but calls that overlap on the
+ *     GPU (different streams, or several host threads) race on it and must be serialised
+ *     by the caller.
+ *   - status: null, or a caller-owned device buffer of 4 uint32 words that receives the
+ *     device-side flags (same encoding as a workspace status header; zero it first). */
+BSA_API bsa_status bsa_topp_select_noalloc(const bsa_shape* shape, const float* mass,
+                                           float threshold, int32_t* row_ptr, int32_t* col_idx,
+                                           int64_t col_capacity, uint32_t* status,
+                                           bsa_stream_t stream);
+
 /* Block-sparse attention forward over frozen CSR block lists ("LoSA", Abstract: the
  * frozen block indices are reused for all remaining steps).  For each query slot of
  * row r = (b*Hh + h)*(Np/q_block) + p/q_block: softmax(softmax_scale * q.k) over the
