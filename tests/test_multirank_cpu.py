@@ -1,0 +1,65 @@
+"""The bench's multi-GPU plumbing on CPU: two gloo ranks, no GPU.
+
+The path shards with no exchange step (each GPU runs an independent problem), so the
+process group only carries the start/stop barrier and the max-over-ranks reduction of
+the timed region.  These tests run that plumbing as two processes on the host.
+"""
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    from block_sparse_attention_25_b200 import synth
+    w, r, local, pg = bench.dist_setup(None)
+    assert (w, r, local) == (world, rank, rank) and pg is not None
+    bench.barrier(pg)
+    # the timed region is the slowest rank's
+    out[rank] = bench.max_over_ranks(1.5 + rank, pg)
+    # each rank draws its own problem (different seeds), as the bench does
+    wl = synth.WORKLOADS["tiny"]
+    q, _, _ = synth.draw_qkv(wl.scaled(seed=wl.seed + 7919 * rank))
+    out[world + rank] = float(q.double().sum())
+    bench.barrier(pg)
+    pg.destroy_process_group()
+
+
+def test_two_gloo_ranks_reduce_max_and_draw_independent_problems():
+    world = 2
+    ctx = mp.get_context("spawn")
+    out = ctx.Array("d", 2 * world)
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    assert list(out[:world]) == [1.5 + world - 1] * world
+    assert out[world] != out[world + 1]
+
+
+def test_single_rank_needs_no_process_group(monkeypatch):
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    sys.path.insert(0, ROOT)
+    import bench
+    w, r, local, pg = bench.dist_setup(None)
+    assert (w, r, local, pg) == (1, 0, 0, None)
+    assert bench.max_over_ranks(3.25, pg) == 3.25
