@@ -381,14 +381,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     float l_run = 0.f;
     bool ok = true;
 
-    uint32_t e0n = nsteps > 0 ? ent[0] : 0u;
-    uint32_t e1n = n_ent > 1 ? ent[1] : 0u;
+    uint32_t e0n = nsteps > 0 ? ld_early_u32(ent) : 0u;
+    uint32_t e1n = n_ent > 1 ? ld_early_u32(ent + 1) : 0u;
     for (int s = 0; s < nsteps; ++s) {
       const int nb = (2 * s + 1 < n_ent) ? 2 : 1;
       const uint32_t e0 = e0n, e1 = e1n;
       if (s + 1 < nsteps) {
-        e0n = ent[2 * s + 2];
-        e1n = (2 * s + 3 < n_ent) ? ent[2 * s + 3] : 0u;
+        e0n = ld_early_u32(ent + 2 * s + 2);
+        e1n = (2 * s + 3 < n_ent) ? ld_early_u32(ent + 2 * s + 3) : 0u;
       }
       const bool got = __all_sync(
           0xffffffffu, mbar_wait(bar_sfull + t, s & 1, abort_flag, p.status, DETAIL_WAIT_S_FULL));

@@ -7,190 +7,163 @@
 //
 // Per row the masses become integers q = rint(m * 2^40) and the target is
 // ceil(tau * sum q) (one fp64 multiply).  The shortest prefix of the (q desc, index asc)
-// order that reaches the target is found without sorting: an exact MSB-first radix
-// select on q (8-bit digits, per-digit sums in shared memory) finds the value t* of the
-// last kept element and the sum A of everything above it; all blocks with q > t* are
-// kept, plus the ceil((target - A) / t*) lowest-index blocks with q == t*.  Integer
+// order that reaches the target is found without sorting: an exact radix select over the
+// row's value range (256 bins per level, per-bin sums in shared memory) finds the value t*
+// of the last kept element and the sum A of everything above it; all blocks with q > t*
+// are kept, plus the ceil((target - A) / t*) lowest-index blocks with q == t*.  Integer
 // arithmetic makes the result independent of reduction order, so it is bit-identical to
 // a sequential sort-and-scan.
 //
-// Kernels: (1) select, one 256-thread CTA per row -> kept bitmap + count in the
-// workspace; (2) exclusive scan of the counts -> row_ptr; (3) compaction, one warp per
-// row -> col_idx ascending.
+// Kernels: (1) select, one warp per row -> kept bitmap + count in the workspace;
+// (2) exclusive scan of the counts -> row_ptr; (3) compaction, one warp per row ->
+// col_idx ascending.
 #include <mutex>
 
 #include "bsa_kernels.cuh"
 
 namespace bsa {
 
-constexpr int kToppThreads = 256;
-constexpr int kToppMaxKb = 4096;
-constexpr int kToppMaxE = kToppMaxKb / kToppThreads;  // elements per thread
 
-__device__ __forceinline__ unsigned long long warp_incl_scan_u64(unsigned long long v) {
+// One warp per row, kSelWarps rows per CTA, warp-synchronous (no CTA barriers).
+// Shared memory per warp: the row's fixed-point masses (n_kb uint64) and a 256-bin
+// histogram of uint64 sums.
+constexpr int kSelWarps = 4;
+
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long n = __shfl_up_sync(0xffffffffu, v, o);
-    if (static_cast<int>(lane_id()) >= o) v += n;
-  }
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
-
-// Block-wide inclusive scan of one uint64 per thread (256 threads).  Returns the
-// inclusive value; *total receives the block total.
-__device__ __forceinline__ unsigned long long block_incl_scan_u64(unsigned long long v,
-                                                                  unsigned long long* sm8,
-                                                                  unsigned long long* total) {
-  const int w = threadIdx.x >> 5;
-  unsigned long long inc = warp_incl_scan_u64(v);
-  if (lane_id() == 31) sm8[w] = inc;
-  __syncthreads();
-  unsigned long long before = 0, tot = 0;
-#pragma unroll
-  for (int i = 0; i < kToppThreads / 32; ++i) {
-    const unsigned long long s = sm8[i];
-    if (i < w) before += s;
-    tot += s;
-  }
-  __syncthreads();
-  *total = tot;
-  return inc + before;
-}
-
-__device__ __forceinline__ unsigned long long block_max_u64(unsigned long long v,
-                                                            unsigned long long* sm8) {
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const unsigned long long n = __shfl_xor_sync(0xffffffffu, v, o);
     v = n > v ? n : v;
   }
-  if (lane_id() == 0) sm8[threadIdx.x >> 5] = v;
-  __syncthreads();
-  unsigned long long m = 0;
+  return v;
+}
+__device__ __forceinline__ unsigned long long warp_min_u64(unsigned long long v) {
 #pragma unroll
-  for (int i = 0; i < kToppThreads / 32; ++i) m = sm8[i] > m ? sm8[i] : m;
-  __syncthreads();
-  return m;
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long n = __shfl_xor_sync(0xffffffffu, v, o);
+    v = n < v ? n : v;
+  }
+  return v;
 }
 
-__global__ void __launch_bounds__(kToppThreads) topp_select_rows_kernel(
-    const float* __restrict__ mass, int n_kb, double tau, int32_t* __restrict__ counts,
-    uint32_t* __restrict__ bitmaps, int words, uint32_t* status) {
-  __shared__ float sm_m[kToppMaxKb];
-  __shared__ unsigned long long h_sum[256];
-  __shared__ unsigned long long sm8[kToppThreads / 32];
-  __shared__ uint32_t sm_bits[kToppMaxKb / 32];
-  __shared__ int sh_first;
-
-  const long long r = blockIdx.x;
-  const int tid = threadIdx.x;
+// Radix select over the row's own value range: each level splits the candidate range
+// [lo, hi] into 256 bins of width 2^shift (relative to lo, so similar masses still spread
+// over many bins), sums the masses per bin, and keeps the bin where the running sum from
+// the top crosses the target.  Each lane scans 8 consecutive bins; a warp scan of the
+// lane totals finds the crossing.  The final pass walks the row 32 blocks at a time, so
+// a ballot of the keep decisions is one bitmap word, in index order (ties go to the lower
+// index).
+__global__ void __launch_bounds__(32 * kSelWarps) topp_select_rows_kernel(
+    const float* __restrict__ mass, long long rows, int n_kb, double tau,
+    int32_t* __restrict__ counts, uint32_t* __restrict__ bitmaps, int words, uint32_t* status) {
+  extern __shared__ unsigned long long sel_smem[];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long r = static_cast<long long>(blockIdx.x) * kSelWarps + warp;
+  if (r >= rows) return;
+  unsigned long long* qrow = sel_smem + static_cast<size_t>(warp) * (n_kb + 256);
+  unsigned long long* hist = qrow + n_kb;
   const float* row = mass + r * n_kb;
-  for (int j = tid; j < n_kb; j += kToppThreads) sm_m[j] = row[j];
-  for (int j = tid; j < words; j += kToppThreads) sm_bits[j] = 0u;
-  __syncthreads();
 
-  // Contiguous ownership: thread tid holds blocks [tid*E, tid*E + n_mine).
-  const int E = (n_kb + kToppThreads - 1) / kToppThreads;
-  const int first = tid * E;
-  const int n_mine = max(0, min(E, n_kb - first));
-  unsigned long long q[kToppMaxE];
-  unsigned long long my_sum = 0, my_max = 0;
+  // fixed-point masses into shared memory; sum, max, min
+  unsigned long long sum = 0, mx = 0, mn = ~0ull;
   bool bad = false;
-#pragma unroll
-  for (int e = 0; e < kToppMaxE; ++e) {
-    q[e] = 0ull;
-    if (e < n_mine) {
-      const float m = sm_m[first + e];
-      // valid: finite and 0 <= m <= 4096 (NaN fails both comparisons)
-      if (m >= 0.f && m <= 4096.f) {
-        q[e] = static_cast<unsigned long long>(__double2ll_rn(static_cast<double>(m) * 1099511627776.0));
-      } else {
-        bad = true;
-      }
-      my_sum += q[e];
-      my_max = q[e] > my_max ? q[e] : my_max;
-    }
+  for (int j = lane; j < n_kb; j += 32) {
+    const float m = row[j];
+    unsigned long long q = 0;
+    // valid: finite and 0 <= m <= 4096 (NaN fails both comparisons)
+    if (m >= 0.f && m <= 4096.f)
+      q = static_cast<unsigned long long>(__double2ll_rn(static_cast<double>(m) * 1099511627776.0));
+    else
+      bad = true;
+    qrow[j] = q;
+    sum += q;
+    mx = q > mx ? q : mx;
+    mn = q < mn ? q : mn;
   }
   if (bad) record_status(status, FLAG_DEVICE_INPUT, DETAIL_MASS_VALUE, static_cast<uint32_t>(r), 0u);
-
-  unsigned long long S;
-  (void)block_incl_scan_u64(my_sum, sm8, &S);
-  const unsigned long long Mx = block_max_u64(my_max, sm8);
+  sum = warp_sum_u64(sum);
+  unsigned long long hi = warp_max_u64(mx);
+  unsigned long long lo = warp_min_u64(mn);
   const unsigned long long target =
-      static_cast<unsigned long long>(ceil(__dmul_rn(tau, static_cast<double>(S))));
+      static_cast<unsigned long long>(ceil(__dmul_rn(tau, static_cast<double>(sum))));
+  __syncwarp();
 
-  unsigned long long tstar = 0, A = 0;
-  if (target > 0) {
-    const int nbits = 64 - __clzll(static_cast<long long>(Mx));
-    int shift = ((nbits + 7) / 8 - 1) * 8;
-    if (shift < 0) shift = 0;
-    unsigned long long prefix = 0;
-    for (; shift >= 0; shift -= 8) {
-      h_sum[tid] = 0ull;
-      __syncthreads();
-      const unsigned long long hi = prefix >> (shift + 8);
+  // Invariant: elements above hi are all kept, their sum is A < target, and the value of
+  // the last kept element lies in [lo, hi].
+  unsigned long long A = 0;
+  while (target > 0 && hi > lo) {
+    const unsigned long long span = hi - lo;
+    const int nbits = 64 - __clzll(static_cast<long long>(span));
+    const int shift = nbits > 8 ? nbits - 8 : 0;
 #pragma unroll
-      for (int e = 0; e < kToppMaxE; ++e) {
-        if (e < n_mine && (q[e] >> (shift + 8)) == hi) {
-          atomicAdd(&h_sum[(q[e] >> shift) & 255ull], q[e]);
-        }
-      }
-      __syncthreads();
-      // Thread tid looks at digit 255 - tid (descending); inclusive scan from the top.
-      const unsigned long long v = h_sum[255 - tid];
-      unsigned long long tot;
-      const unsigned long long inc = block_incl_scan_u64(v, sm8, &tot);
-      if (tid == 0) sh_first = kToppThreads;
-      __syncthreads();
-      if (A + inc >= target) atomicMin(&sh_first, tid);
-      __syncthreads();
-      const int f = sh_first;
-      // Broadcast the sum strictly above the crossing digit from thread f.
-      if (tid == f) {
-        h_sum[0] = A + inc - v;  // reuse slot 0 (the histogram is read already)
-        sm8[0] = static_cast<unsigned long long>(255 - f);
-      }
-      __syncthreads();
-      A = h_sum[0];
-      prefix |= sm8[0] << shift;
-      __syncthreads();
+    for (int i = 0; i < 8; ++i) hist[lane * 8 + i] = 0ull;
+    __syncwarp();
+    for (int j = lane; j < n_kb; j += 32) {
+      const unsigned long long q = qrow[j];
+      if (q >= lo && q <= hi) atomicAdd(&hist[(q - lo) >> shift], q);
     }
-    tstar = prefix;
+    __syncwarp();
+    // lane l owns bins 255-8l .. 248-8l (descending); inclusive sums from the top
+    unsigned long long b[8];
+    unsigned long long run = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      run += hist[255 - 8 * lane - i];
+      b[i] = run;
+    }
+    unsigned long long before = run;  // exclusive warp scan of lane totals
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long n = __shfl_up_sync(0xffffffffu, before, o);
+      if (lane >= o) before += n;
+    }
+    before -= run;
+    int first = 8;
+#pragma unroll
+    for (int i = 7; i >= 0; --i)
+      if (A + before + b[i] >= target) first = i;
+    const unsigned bal = __ballot_sync(0xffffffffu, first < 8);
+    const int src = __ffs(bal) - 1;  // the crossing exists (see the invariant)
+    unsigned long long above = before;  // sum of the bins strictly above the crossing bin
+#pragma unroll
+    for (int i = 1; i < 8; ++i)
+      if (first == i) above = before + b[i - 1];
+    const int dbin = 255 - 8 * lane - first;
+    above = __shfl_sync(0xffffffffu, above, src);
+    const int d_src = __shfl_sync(0xffffffffu, dbin, src);
+    A += above;
+    const unsigned long long nlo = lo + (static_cast<unsigned long long>(d_src) << shift);
+    const unsigned long long nhi = nlo + ((1ull << shift) - 1ull);
+    lo = nlo;
+    hi = nhi < hi ? nhi : hi;
+    __syncwarp();
   }
+  const unsigned long long tstar = lo;
 
-  // Keep q > t*, and the lowest-index c elements with q == t*.
-  unsigned long long c = 0;
-  if (target > 0) c = (target - A + tstar - 1) / tstar;
-  int my_eq = 0, my_gt = 0;
-#pragma unroll
-  for (int e = 0; e < kToppMaxE; ++e) {
-    if (e < n_mine && target > 0) {
-      my_gt += q[e] > tstar;
-      my_eq += q[e] == tstar;
-    }
-  }
-  unsigned long long tot_eq;
-  const unsigned long long eq_incl = block_incl_scan_u64(static_cast<unsigned long long>(my_eq), sm8, &tot_eq);
-  unsigned long long tot_gt;
-  (void)block_incl_scan_u64(static_cast<unsigned long long>(my_gt), sm8, &tot_gt);
-  unsigned long long rank = eq_incl - my_eq;
-  if (target > 0) {
-#pragma unroll
-    for (int e = 0; e < kToppMaxE; ++e) {
-      if (e < n_mine) {
-        bool keep = q[e] > tstar;
-        if (q[e] == tstar) {
-          keep = rank < c;
-          ++rank;
-        }
-        if (keep) atomicOr(&sm_bits[(first + e) >> 5], 1u << ((first + e) & 31));
-      }
-    }
-  }
-  __syncthreads();
+  // Keep q > t*, and the c lowest-index blocks with q == t*.
+  const unsigned long long c = target > 0 ? (target - A + tstar - 1) / tstar : 0ull;
+  unsigned long long ties_before = 0;
+  unsigned long long kept = 0;
   uint32_t* out_bits = bitmaps + r * words;
-  for (int j = tid; j < words; j += kToppThreads) out_bits[j] = sm_bits[j];
-  if (tid == 0) counts[r] = static_cast<int32_t>(target > 0 ? tot_gt + c : 0ull);
+  for (int j0 = 0; j0 < n_kb; j0 += 32) {
+    const int j = j0 + lane;
+    const unsigned long long q = j < n_kb ? qrow[j] : 0ull;
+    const bool is_tie = target > 0 && j < n_kb && q == tstar;
+    const unsigned tb = __ballot_sync(0xffffffffu, is_tie);
+    const unsigned long long rank = ties_before + __popc(tb & ((1u << lane) - 1u));
+    const bool keep = target > 0 && j < n_kb && (q > tstar || (is_tie && rank < c));
+    const unsigned kb = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) out_bits[j0 >> 5] = kb;
+    ties_before += __popc(tb);
+    kept += __popc(kb);
+  }
+  if (lane == 0) counts[r] = static_cast<int32_t>(kept);
 }
 
 // Exclusive scan of counts[0..R) into row_ptr[0..R] with one 1024-thread CTA.
@@ -269,6 +242,20 @@ __global__ void __launch_bounds__(256) topp_fill_kernel(const uint32_t* __restri
   if (overflow) record_status(status, FLAG_CAPACITY, DETAIL_COL_CAPACITY, static_cast<uint32_t>(r), 0u);
 }
 
+static cudaError_t launch_select_rows(const float* mass, long long rows, int n_kb, float threshold,
+                                      int32_t* counts, uint32_t* bitmaps, int words,
+                                      uint32_t* status, cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(kSelWarps) * (n_kb + 256) * sizeof(unsigned long long);
+  cudaError_t e = cudaFuncSetAttribute(topp_select_rows_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const long long ctas = (rows + kSelWarps - 1) / kSelWarps;
+  topp_select_rows_kernel<<<static_cast<unsigned>(ctas), 32 * kSelWarps, smem, stream>>>(
+      mass, rows, n_kb, static_cast<double>(threshold), counts, bitmaps, words, status);
+  return cudaGetLastError();
+}
+
 size_t topp_scratch_bytes(long long rows, int n_kb) {
   const long long words = (n_kb + 31) / 32;
   const size_t counts = static_cast<size_t>(rows) * 4;
@@ -288,9 +275,8 @@ cudaError_t launch_topp_select(const float* mass, long long rows, int n_kb, floa
   if (rows == 0) {
     return cudaMemsetAsync(row_ptr, 0, sizeof(int32_t), stream);
   }
-  topp_select_rows_kernel<<<static_cast<unsigned>(rows), kToppThreads, 0, stream>>>(
-      mass, n_kb, static_cast<double>(threshold), counts, bitmaps, words, status);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_select_rows(mass, rows, n_kb, threshold, counts, bitmaps, words, status,
+                                     stream);
   if (e != cudaSuccess) return e;
   topp_scan_kernel<<<1, 1024, 0, stream>>>(counts, rows, row_ptr);
   e = cudaGetLastError();
@@ -357,9 +343,7 @@ cudaError_t launch_topp_select_noalloc(const float* mass, long long rows, int n_
   const size_t counts_bytes = (static_cast<size_t>(rows) * 4 + 255) & ~static_cast<size_t>(255);
   int32_t* counts = static_cast<int32_t*>(scratch);
   uint32_t* bitmaps = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(scratch) + counts_bytes);
-  topp_select_rows_kernel<<<static_cast<unsigned>(rows), kToppThreads, 0, stream>>>(
-      mass, n_kb, static_cast<double>(threshold), counts, bitmaps, words, status);
-  e = cudaGetLastError();
+  e = launch_select_rows(mass, rows, n_kb, threshold, counts, bitmaps, words, status, stream);
   if (e != cudaSuccess) return e;
   topp_scan_kernel<<<1, 1024, 0, stream>>>(counts, rows, row_ptr);
   e = cudaGetLastError();
