@@ -342,3 +342,110 @@ def dequant_e4m3_tiles(codes, scales) -> np.ndarray:
     B, Hh, Np, D = v.shape
     s = np.repeat(np.asarray(scales, dtype=np.float64), TILE_TOKENS, axis=2)
     return v * s[..., None]
+
+
+# --------------------------------------------------------------------------- static patterns
+# "Sparse-vDiT: Unleashing the Power of Sparse Attention to Accelerate Video Diffusion
+# Transformers", Abstract: recurring diagonal, multi-diagonal and vertical-stripe attention
+# structures.  "GRAT" (grouping attention for large images/videos), Abstract: queries of a
+# group share keys restricted to surrounding blocks or to criss-cross regions.
+#
+# Readings (the pages name the structures only): everything is at kv-block (= tile)
+# granularity in tile-major order; a query block covers its own tiles (one for 64-token
+# blocks, two for 128-token blocks) and keeps kv block j when the predicate holds for any
+# of them.
+#   DIAGONAL        |j - u| <= w
+#   MULTI_DIAGONAL  |j - (u + k L)| <= w for some k in [-K, K], k != 0; L defaults to the
+#                   tiles of one temporal layer (Hp/4 * Wp/4): the same place in other frames
+#   VERTICAL_STRIPE j % stride == offset (the same kv blocks for every query block)
+#   SURROUNDING     |jt - ut| <= rt and |jh - uh| <= rh and |jw - uw| <= rw (tile coords)
+#   CRISS_CROSS     tile j shares at least two of its three tile coordinates with u
+# The kept set is the union over the enabled kinds.
+PAT_DIAGONAL = 1
+PAT_MULTI_DIAGONAL = 2
+PAT_VERTICAL_STRIPE = 4
+PAT_SURROUNDING = 8
+PAT_CRISS_CROSS = 16
+
+
+def _tile_coords(g: Grid, j: int):
+    nth, ntw = g.Hp // TILE, g.Wp // TILE
+    return j // (nth * ntw), (j // ntw) % nth, j % ntw
+
+
+def pattern_keeps(g: Grid, q_block: int, i: int, j: int, kinds: int, diag_width=0,
+                  multi_count=0, multi_period=0, stripe_stride=0, stripe_offset=0,
+                  radius=(0, 0, 0)) -> bool:
+    """Whether query block i keeps kv block j under the enabled structured patterns."""
+    per = q_block // TILE_TOKENS
+    L = multi_period if multi_period > 0 else (g.Hp // TILE) * (g.Wp // TILE)
+    jt, jh, jw = _tile_coords(g, j)
+    if kinds & PAT_VERTICAL_STRIPE and stripe_stride > 0 and j % stripe_stride == stripe_offset:
+        return True
+    for u in range(i * per, (i + 1) * per):
+        if kinds & PAT_DIAGONAL and abs(j - u) <= diag_width:
+            return True
+        if kinds & PAT_MULTI_DIAGONAL:
+            for k in range(-multi_count, multi_count + 1):
+                if k != 0 and abs(j - (u + k * L)) <= diag_width:
+                    return True
+        ut, uh, uw = _tile_coords(g, u)
+        if kinds & PAT_SURROUNDING and abs(jt - ut) <= radius[0] and abs(jh - uh) <= radius[1] \
+                and abs(jw - uw) <= radius[2]:
+            return True
+        if kinds & PAT_CRISS_CROSS and (int(jt == ut) + int(jh == uh) + int(jw == uw)) >= 2:
+            return True
+    return False
+
+
+def pattern_csr(g: Grid, q_block: int, batch: int, heads: int, kinds: int, **params):
+    """CSR (row_ptr, col_idx) of the structured pattern, identical for every (b, h)."""
+    n_qb, n_kb = g.Np // q_block, g.Np // 64
+    rows = []
+    for i in range(n_qb):
+        rows.append([j for j in range(n_kb) if pattern_keeps(g, q_block, i, j, kinds, **params)])
+    kept = [r for _ in range(batch * heads) for r in rows]
+    row_ptr = np.zeros(len(kept) + 1, dtype=np.int64)
+    row_ptr[1:] = np.cumsum([len(r) for r in kept])
+    col_idx = np.array([j for r in kept for j in r], dtype=np.int64)
+    return row_ptr, col_idx
+
+
+# --------------------------------------------------------------------------- pooled estimate
+# "Sparse VideoGen2", Abstract: top-p dynamic budget control over cluster-level attention;
+# the related-work entry on head-wise adaptive sparse attention (online top-p).  Reading R8:
+# with the 4x4x4 tiles as the clusters, a kv block is represented by the mean of its valid
+# keys and weighted by its number of valid keys, a query block by the mean of its valid
+# queries, and the estimated block mass is the softmax over kv blocks of those block-level
+# logits, each weighted by its key count:
+#   M_est[i, j] = n_j exp(scale qbar_i . kbar_j) / sum_j' n_j' exp(scale qbar_i . kbar_j')
+# Blocks without valid keys get 0; query blocks without valid queries get an all-zero row.
+def pooled_block_mass(qt, kt, g: Grid, q_block: int, kv_block: int, scale: float) -> np.ndarray:
+    """Estimated block masses float64 [B, Hh, Np // q_block, Np // kv_block] (reading R8)."""
+    B, Hh = qt.shape[0], qt.shape[1]
+    valid = valid_slots(g)
+    n_qb, n_kb = g.Np // q_block, g.Np // kv_block
+    out = np.zeros((B, Hh, n_qb, n_kb), dtype=np.float64)
+    n_keys = np.array([valid[j * kv_block:(j + 1) * kv_block].sum() for j in range(n_kb)], float)
+    for b in range(B):
+        for h in range(Hh):
+            k = kt[b, h].astype(np.float64)
+            kbar = np.zeros((n_kb, k.shape[-1]))
+            for j in range(n_kb):
+                rows = np.arange(j * kv_block, (j + 1) * kv_block)
+                rows = rows[valid[rows]]
+                if rows.size:
+                    kbar[j] = k[rows].mean(axis=0)
+            q = qt[b, h].astype(np.float64)
+            for i in range(n_qb):
+                rows = np.arange(i * q_block, (i + 1) * q_block)
+                rows = rows[valid[rows]]
+                if rows.size == 0:
+                    continue
+                qbar = q[rows].mean(axis=0)
+                logits = scale * (kbar @ qbar)
+                keep = n_keys > 0
+                z = logits[keep] - logits[keep].max()
+                w = n_keys[keep] * np.exp(z)
+                out[b, h, i, keep] = w / w.sum()
+    return out

@@ -397,3 +397,106 @@ def test_quant_tiles_scale_and_error_bound():
     err = np.abs(deq - x.astype(np.float64))
     rel_bound = 2.0 ** -4 * np.abs(x) * (1 + 1e-6) + s * 2.0 ** -10 + 1e-12
     assert np.all(err <= rel_bound)
+
+
+# ------------------------------------------------------------------ structured patterns
+def _rows(rp, ci):
+    return [ci[rp[r]:rp[r + 1]].tolist() for r in range(len(rp) - 1)]
+
+
+def test_pattern_diagonal_band_closed_form():
+    g = O.Grid(8, 8, 12, 8, 8, 12)          # 2 x 2 x 3 tiles = 12 blocks
+    n = g.Np // 64
+    for w in (0, 1, 3):
+        rows = _rows(*O.pattern_csr(g, 64, 1, 1, O.PAT_DIAGONAL, diag_width=w))
+        for i, r in enumerate(rows):
+            assert r == list(range(max(0, i - w), min(n - 1, i + w) + 1))
+
+
+def test_pattern_diagonal_128_token_query_blocks_cover_both_tiles():
+    g = O.Grid(8, 8, 12, 8, 8, 12)
+    rows = _rows(*O.pattern_csr(g, 128, 1, 1, O.PAT_DIAGONAL, diag_width=0))
+    assert rows == [[2 * i, 2 * i + 1] for i in range(6)]
+
+
+def test_pattern_multi_diagonal_hits_same_place_in_other_frames():
+    g = O.Grid(12, 8, 8, 12, 8, 8)          # 3 temporal layers of 2 x 2 tiles
+    rows = _rows(*O.pattern_csr(g, 64, 1, 1, O.PAT_MULTI_DIAGONAL, multi_count=2))
+    # layer stride 4: block u also sees u - 8, u - 4, u + 4, u + 8 (within range), not itself
+    for u, r in enumerate(rows):
+        assert r == sorted(v for v in (u - 8, u - 4, u + 4, u + 8) if 0 <= v < 12)
+
+
+def test_pattern_vertical_stripes_are_the_same_for_every_row():
+    g = O.Grid(8, 8, 12, 8, 8, 12)
+    rows = _rows(*O.pattern_csr(g, 64, 2, 3, O.PAT_VERTICAL_STRIPE, stripe_stride=5,
+                                stripe_offset=2))
+    assert len(rows) == 2 * 3 * 12 and all(r == [2, 7] for r in rows)
+
+
+def test_pattern_surrounding_counts_closed_form():
+    g = O.Grid(12, 12, 12, 12, 12, 12)      # 3 x 3 x 3 tiles
+    rows = _rows(*O.pattern_csr(g, 64, 1, 1, O.PAT_SURROUNDING, radius=(1, 1, 1)))
+    for u, r in enumerate(rows):
+        t, h, w = u // 9, (u // 3) % 3, u % 3
+        expect = 1
+        for c in (t, h, w):
+            expect *= 3 - (c == 0) - (c == 2)   # neighbours along one axis, edges have 2
+        assert len(r) == expect
+    assert len(rows[13]) == 27                 # the centre tile sees the whole 3x3x3 cube
+    rows0 = _rows(*O.pattern_csr(g, 64, 1, 1, O.PAT_SURROUNDING, radius=(0, 0, 0)))
+    assert rows0 == [[u] for u in range(27)]
+
+
+def test_pattern_criss_cross_is_three_axis_lines():
+    g = O.Grid(12, 12, 16, 12, 12, 16)      # 3 x 3 x 4 tiles
+    rows = _rows(*O.pattern_csr(g, 64, 1, 1, O.PAT_CRISS_CROSS))
+    for r in rows:
+        assert len(r) == 1 + 2 + 2 + 3     # itself + other t + other h + other w
+
+
+def test_pattern_union_of_kinds():
+    g = O.Grid(8, 8, 12, 8, 8, 12)
+    a = _rows(*O.pattern_csr(g, 64, 1, 1, O.PAT_DIAGONAL, diag_width=1))
+    b = _rows(*O.pattern_csr(g, 64, 1, 1, O.PAT_VERTICAL_STRIPE, stripe_stride=4))
+    u = _rows(*O.pattern_csr(g, 64, 1, 1, O.PAT_DIAGONAL | O.PAT_VERTICAL_STRIPE,
+                             diag_width=1, stripe_stride=4))
+    assert u == [sorted(set(x) | set(y)) for x, y in zip(a, b)]
+
+
+# ------------------------------------------------------------------ pooled estimate
+def test_pooled_estimate_is_exact_when_blocks_are_constant():
+    """With every key of a block equal (and every query of a block equal), block-level
+    attention is exact: the estimate equals the exact block mass."""
+    g = O.Grid(3, 5, 6, 4, 8, 8)
+    rng = np.random.default_rng(9)
+    n_kb = g.Np // 64
+    kb = rng.standard_normal((n_kb, 8))
+    qb = rng.standard_normal((n_kb, 8)) * 2
+    k = np.repeat(kb, 64, axis=0)[None, None]
+    q = np.repeat(qb, 64, axis=0)[None, None]
+    valid = O.valid_slots(g)
+    k = np.where(valid[None, None, :, None], k, 0.0)
+    q = np.where(valid[None, None, :, None], q, 0.0)
+    est = O.pooled_block_mass(q, k, g, 64, 64, 0.7)
+    exact = O.block_mass(q, k, g, 64, 64, 0.7)
+    assert np.allclose(est, exact, atol=1e-13, rtol=0)
+
+
+def test_pooled_estimate_rows_and_zero_scale():
+    g = O.Grid(5, 4, 9, 8, 4, 12)
+    q, k = _qk(g, heads=2, D=16, scale_qk=1.5, seed=11)
+    est = O.pooled_block_mass(q, k, g, 128, 64, 0.4)
+    valid = O.valid_slots(g)
+    for i in range(g.Np // 128):
+        s = est[0, :, i].sum(axis=-1)
+        if valid[i * 128:(i + 1) * 128].any():
+            assert np.allclose(s, 1.0, atol=1e-12, rtol=0)
+        else:
+            assert np.all(est[0, :, i] == 0)
+    # scale -> 0: every valid key weighs the same, so the estimate is the key-count share
+    z = O.pooled_block_mass(q, k, g, 64, 64, 0.0)
+    nvk = np.array([valid[j * 64:(j + 1) * 64].sum() for j in range(g.Np // 64)], float)
+    for i in range(g.Np // 64):
+        if valid[i * 64:(i + 1) * 64].any():
+            assert np.allclose(z[0, 0, i], nvk / nvk.sum(), atol=1e-14, rtol=0)
