@@ -59,6 +59,29 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
 
 
+def measured_traffic(fp8: bool):
+    """DRAM bytes per bsattn_fwd launch from the committed full-size ncu capture, or None when
+    the kernel sources have changed since it was taken (or for a variant not captured)."""
+    if fp8:
+        return None
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", "bsattn_fwd_wan14b_720p_dram.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
+    if not m:
+        return None
+    csrc = os.path.join(ROOT, "block_sparse_attention_25_b200", "csrc")
+    for name in ("attn_fwd.cu", "bsa_common.cuh"):
+        h = re.search(r"source_sha256 " + re.escape(name) + r":\s*([0-9a-f]{64})", text)
+        cur = hashlib.sha256(open(os.path.join(csrc, name), "rb").read()).hexdigest()
+        if not h or h.group(1) != cur:
+            return None
+    return int(m.group(1))
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
 
@@ -301,7 +324,10 @@ def run_ours(args, world, rank, local, pg):
         },
         "roofline": {
             "bound": "tensor", "achieved": round(fwd_tflops, 2), "peak": peak, "unit": "TFLOP/s",
-            "frac": round(fwd_tflops / peak, 4), "traffic": None,
+            "frac": round(fwd_tflops / peak, 4),
+            "traffic": (measured_traffic(fp8) if wl.name == synth.WORKLOADS["wan14b_720p"].name
+                        else None),
+            "traffic_unit": "bytes per launch (dram read + write, one full-size ncu capture)",
             "kernel": f"bsattn_fwd_kernel<{s.head_dim},{'true' if fp8 else 'false'}>",
             "peak_source": peak_note,
         },

@@ -23,13 +23,20 @@ BSA_OK = 0
 STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "capacity too small",
                 4: "CUDA error", 5: "device wait timed out", 6: "device-side input check failed"}
 BSA_BF16, BSA_FP32, BSA_E4M3 = 0, 1, 2
-OP_BLOCK_MASS, OP_TOPP_SELECT, OP_FWD = 0, 1, 2
+OP_BLOCK_MASS, OP_TOPP_SELECT, OP_FWD, OP_PATTERN, OP_POOLED_MASS = 0, 1, 2, 3, 4
+PAT_DIAGONAL, PAT_MULTI_DIAGONAL, PAT_VERTICAL_STRIPE, PAT_SURROUNDING, PAT_CRISS_CROSS = 1, 2, 4, 8, 16
 
 
 class BsaError(RuntimeError):
     def __init__(self, status: int, what: str):
         super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} (status {status})")
         self.status = status
+
+
+class _Pattern(ctypes.Structure):
+    _fields_ = [("kinds", ctypes.c_uint32)] + [(n, ctypes.c_int32) for n in (
+        "diag_width", "multi_count", "multi_period", "stripe_stride", "stripe_offset",
+        "radius_t", "radius_h", "radius_w")]
 
 
 class _Shape(ctypes.Structure):
@@ -104,8 +111,11 @@ def lib() -> ctypes.CDLL:
         "bsa_tile_permute": (I, [SP, I, I, P, P, P]),
         "bsa_tile_permute_quant_e4m3": (I, [SP, P, P, P, P]),
         "bsa_block_mass": (I, [SP, P, P, F, P, P, S, P]),
+        "bsa_dense_fwd_mass": (I, [SP, P, P, P, F, P, P, P, P, S, P]),
+        "bsa_pooled_mass": (I, [SP, P, P, F, P, P, S, P]),
         "bsa_topp_select": (I, [SP, P, F, P, P, L64, P, S, P]),
         "bsa_topp_select_noalloc": (I, [SP, P, F, P, P, L64, P, P]),
+        "bsa_pattern_csr": (I, [SP, ctypes.POINTER(_Pattern), P, P, L64, P, S, P]),
         "bsa_fwd": (I, [SP, I, P, P, P, P, P, P, P, P, F, P, P, P, S, P]),
         "bsa_version": (ctypes.c_char_p, []),
     }
@@ -120,7 +130,8 @@ def lib() -> ctypes.CDLL:
 EXPORTED_SYMBOLS = ("bsa_workspace_bytes", "bsa_clear_status", "bsa_device_status",
                     "bsa_device_status_words", "bsa_status_string", "bsa_tile_permute",
                     "bsa_tile_permute_quant_e4m3", "bsa_block_mass", "bsa_topp_select", "bsa_fwd",
-                    "bsa_topp_select_noalloc", "bsa_version")
+                    "bsa_topp_select_noalloc", "bsa_pattern_csr", "bsa_dense_fwd_mass",
+                    "bsa_pooled_mass", "bsa_version")
 
 
 def _check(status: int, what: str):
@@ -227,6 +238,45 @@ def block_mass(q, k, shape: Shape, softmax_scale=None, out=None, ws=None, stream
     return out
 
 
+def dense_fwd_mass(q, k, v, shape: Shape, softmax_scale=None, want_lse=False, out=None, lse=None,
+                   mass=None, ws=None, stream=None):
+    """bsa_dense_fwd_mass: dense attention output and exact block masses in one call.
+    Returns (out, mass) or (out, mass, lse)."""
+    tiled = (shape.batch, shape.heads, shape.Np, shape.head_dim)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, tiled, n)
+    if out is None:
+        out = torch.empty(tiled, dtype=torch.bfloat16, device=q.device)
+    if mass is None:
+        mass = torch.empty((shape.batch, shape.heads, shape.n_qb, shape.n_kb), dtype=torch.float32,
+                           device=q.device)
+    if want_lse and lse is None:
+        lse = torch.empty((shape.batch, shape.heads, shape.Np), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = new_workspace(shape, OP_BLOCK_MASS, q.device)
+    scale = default_scale(shape) if softmax_scale is None else float(softmax_scale)
+    _check(lib().bsa_dense_fwd_mass(ctypes.byref(shape.c()), _ptr(q), _ptr(k), _ptr(v), scale,
+                                    _ptr(out), _ptr(lse), _ptr(mass), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "bsa_dense_fwd_mass")
+    return (out, mass, lse) if want_lse else (out, mass)
+
+
+def pooled_mass(q, k, shape: Shape, softmax_scale=None, out=None, ws=None, stream=None):
+    """bsa_pooled_mass: block-level estimate of the block masses (feed to topp_select)."""
+    tiled = (shape.batch, shape.heads, shape.Np, shape.head_dim)
+    _need(q, torch.bfloat16, tiled, "q")
+    _need(k, torch.bfloat16, tiled, "k")
+    if out is None:
+        out = torch.empty((shape.batch, shape.heads, shape.n_qb, shape.n_kb), dtype=torch.float32,
+                          device=q.device)
+    if ws is None:
+        ws = new_workspace(shape, OP_POOLED_MASS, q.device)
+    scale = default_scale(shape) if softmax_scale is None else float(softmax_scale)
+    _check(lib().bsa_pooled_mass(ctypes.byref(shape.c()), _ptr(q), _ptr(k), scale, _ptr(out),
+                                 _ptr(ws), ws.numel(), _stream(stream)), "bsa_pooled_mass")
+    return out
+
+
 def topp_select(mass, shape: Shape, threshold: float = 0.99, col_capacity=None, ws=None,
                 row_ptr=None, col_idx=None, stream=None):
     """CSR (row_ptr int32 [R+1], col_idx int32 [capacity]) of the kept kv blocks.
@@ -264,6 +314,26 @@ def topp_select_noalloc(mass, shape: Shape, threshold: float = 0.99, row_ptr=Non
     _check(lib().bsa_topp_select_noalloc(ctypes.byref(shape.c()), _ptr(mass), float(threshold),
                                          _ptr(row_ptr), _ptr(col_idx), cap, _ptr(status),
                                          _stream(stream)), "bsa_topp_select_noalloc")
+    return row_ptr, col_idx
+
+
+def pattern_csr(shape: Shape, kinds: int, diag_width=0, multi_count=0, multi_period=0,
+                stripe_stride=0, stripe_offset=0, radius=(0, 0, 0), col_capacity=None, ws=None,
+                row_ptr=None, col_idx=None, device="cuda", stream=None):
+    """bsa_pattern_csr: static structured kv-block lists (union of the enabled kinds)."""
+    R = shape.rows
+    cap = R * shape.n_kb if col_capacity is None else int(col_capacity)
+    if row_ptr is None:
+        row_ptr = torch.empty(R + 1, dtype=torch.int32, device=device)
+    if col_idx is None:
+        col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=device)
+    if ws is None:
+        ws = new_workspace(shape, OP_PATTERN, device)
+    pat = _Pattern(int(kinds), diag_width, multi_count, multi_period, stripe_stride, stripe_offset,
+                   *radius)
+    _check(lib().bsa_pattern_csr(ctypes.byref(shape.c()), ctypes.byref(pat), _ptr(row_ptr),
+                                 _ptr(col_idx), cap, _ptr(ws), ws.numel(), _stream(stream)),
+           "bsa_pattern_csr")
     return row_ptr, col_idx
 
 

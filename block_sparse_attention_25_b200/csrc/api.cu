@@ -120,6 +120,11 @@ size_t workspace_bytes(const bsa_shape* s, int op) {
              bsa::topp_scratch_bytes(1LL * a.batch * a.heads * a.n_qb, a.n_kb);
     case BSA_OP_FWD:
       return bsa::kStatusBytes + bsa::fwd_scratch_bytes(a);
+    case BSA_OP_POOLED_MASS:
+      return bsa::kStatusBytes + bsa::pooled_scratch_bytes(a);
+    case BSA_OP_PATTERN:
+      return bsa::kStatusBytes +
+             bsa::topp_scratch_bytes(1LL * a.batch * a.heads * a.n_qb, a.n_kb);
     default:
       return 0;
   }
@@ -211,6 +216,40 @@ bsa_status bsa_block_mass(const bsa_shape* shape, const void* q, const void* k, 
   return from_cuda(bsa::launch_block_mass(a, q, k, softmax_scale, mass, ws, stream));
 }
 
+bsa_status bsa_dense_fwd_mass(const bsa_shape* shape, const void* q, const void* k, const void* v,
+                              float softmax_scale, void* out, float* lse, float* mass, void* ws,
+                              size_t ws_bytes, bsa_stream_t stream) {
+  bsa_status st = check_shape(shape, true);
+  if (st != BSA_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || mass == nullptr ||
+      ws == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (!bsa::aligned16(q) || !bsa::aligned16(k) || !bsa::aligned16(v) || !bsa::aligned16(out) ||
+      !bsa::aligned16(ws) || (reinterpret_cast<uintptr_t>(mass) & 3u) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return BSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f)) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(shape, BSA_OP_BLOCK_MASS)) return BSA_ERR_CAPACITY;
+  const AttnDims a = make_attn(shape);
+  return from_cuda(
+      bsa::launch_calib_dense_mass(a, q, k, v, softmax_scale, out, lse, mass, ws, stream));
+}
+
+bsa_status bsa_pooled_mass(const bsa_shape* shape, const void* q, const void* k,
+                           float softmax_scale, float* mass_est, void* ws, size_t ws_bytes,
+                           bsa_stream_t stream) {
+  bsa_status st = check_shape(shape, true);
+  if (st != BSA_OK) return st;
+  if (q == nullptr || k == nullptr || mass_est == nullptr || ws == nullptr ||
+      !bsa::aligned16(q) || !bsa::aligned16(k) || !bsa::aligned16(ws) ||
+      (reinterpret_cast<uintptr_t>(mass_est) & 3u))
+    return BSA_ERR_INVALID_ARG;
+  if (!(softmax_scale >= 0.f) || !(softmax_scale < 1e30f)) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(shape, BSA_OP_POOLED_MASS)) return BSA_ERR_CAPACITY;
+  const AttnDims a = make_attn(shape);
+  return from_cuda(bsa::launch_pooled_mass(a, q, k, softmax_scale, mass_est, ws, stream));
+}
+
 bsa_status bsa_topp_select(const bsa_shape* shape, const float* mass, float threshold,
                            int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, void* ws,
                            size_t ws_bytes, bsa_stream_t stream) {
@@ -226,6 +265,38 @@ bsa_status bsa_topp_select(const bsa_shape* shape, const float* mass, float thre
   const long long rows = 1LL * a.batch * a.heads * a.n_qb;
   return from_cuda(bsa::launch_topp_select(mass, rows, a.n_kb, threshold, row_ptr, col_idx,
                                            col_capacity, ws, stream));
+}
+
+bsa_status bsa_pattern_csr(const bsa_shape* shape, const bsa_pattern* pattern, int32_t* row_ptr,
+                           int32_t* col_idx, int64_t col_capacity, void* ws, size_t ws_bytes,
+                           bsa_stream_t stream) {
+  bsa_status st = check_shape(shape, true);
+  if (st != BSA_OK) return st;
+  if (pattern == nullptr || row_ptr == nullptr || ws == nullptr || !bsa::aligned16(ws))
+    return BSA_ERR_INVALID_ARG;
+  if (col_capacity < 0 || (col_capacity > 0 && col_idx == nullptr)) return BSA_ERR_INVALID_ARG;
+  const uint32_t all = BSA_PAT_DIAGONAL | BSA_PAT_MULTI_DIAGONAL | BSA_PAT_VERTICAL_STRIPE |
+                       BSA_PAT_SURROUNDING | BSA_PAT_CRISS_CROSS;
+  if (pattern->kinds & ~all) return BSA_ERR_INVALID_ARG;
+  if (pattern->diag_width < 0 || pattern->multi_count < 0 || pattern->stripe_stride < 0 ||
+      pattern->radius_t < 0 || pattern->radius_h < 0 || pattern->radius_w < 0)
+    return BSA_ERR_INVALID_ARG;
+  if (pattern->stripe_stride > 0 &&
+      (pattern->stripe_offset < 0 || pattern->stripe_offset >= pattern->stripe_stride))
+    return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(shape, BSA_OP_PATTERN)) return BSA_ERR_CAPACITY;
+  bsa::PatternParams pp;
+  pp.kinds = pattern->kinds;
+  pp.diag_width = pattern->diag_width;
+  pp.multi_count = pattern->multi_count;
+  pp.multi_period = pattern->multi_period;
+  pp.stripe_stride = pattern->stripe_stride;
+  pp.stripe_offset = pattern->stripe_offset;
+  pp.radius_t = pattern->radius_t;
+  pp.radius_h = pattern->radius_h;
+  pp.radius_w = pattern->radius_w;
+  const AttnDims a = make_attn(shape);
+  return from_cuda(bsa::launch_pattern_csr(a, pp, row_ptr, col_idx, col_capacity, ws, stream));
 }
 
 bsa_status bsa_topp_select_noalloc(const bsa_shape* shape, const float* mass, float threshold,

@@ -275,17 +275,25 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       constexpr uint32_t kFmt = FP8 ? 0u : 1u;  // e4m3 / bf16
       const uint32_t idesc_pv = make_idesc(kFmt, 1u, 128u, static_cast<uint32_t>(D));
       bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, DETAIL_WAIT_Q);
+      // Shared-memory descriptors: built once; the start-address field is the low bits, so
+      // a byte offset inside the operand region is added as offset >> 4.
+      const uint64_t q_desc0 = make_sdesc_sw128(q_base, 16, 1024);
+      const uint64_t k_desc0 = make_sdesc_sw128(k_base, 16, 1024);
+      const uint64_t v_desc0 = make_sdesc_sw128(v_base, 128 * 128, 1024);
       auto issue_pv = [&](int t, int sp) {
         // O_t (+)= P_t(sp) V(sp); K dimension = keys of step sp (64 or 128).  One MMA takes
         // 32 bytes of K: 16 keys (bf16) or 32 keys (e4m3), i.e. 8 TMEM columns of P and
         // 16 or 32 rows (2 or 4 swizzle atoms) of V.
         constexpr int kKeysPerMma = 32 / L::kElem;
-        const int nbp = (2 * sp + 1 < n_ent) ? 2 : 1;
-        const uint32_t vb = v_base + (sp % VS) * L::kKVStage;
+        constexpr int kMmas = 128 / kKeysPerMma;  // for a 2-block step
+        const int nmma = (2 * sp + 1 < n_ent) ? kMmas : kMmas / 2;
+        const uint64_t vd = v_desc0 + static_cast<uint64_t>(((sp % VS) * L::kKVStage) >> 4);
         const uint32_t p_tmem = tmem + t * 128;
         const uint32_t o_tmem = tmem + 256 + t * D;
-        for (int kk = 0; kk < nbp * 64 / kKeysPerMma; ++kk) {
-          const uint64_t bdesc = make_sdesc_sw128(vb + kk * kKeysPerMma * 128, 128 * 128, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kMmas; ++kk) {
+          if (kk >= nmma) break;
+          const uint64_t bdesc = vd + static_cast<uint64_t>((kk * kKeysPerMma * 128) >> 4);
           if constexpr (FP8)
             mma_f8_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (sp > 0 || kk > 0) ? 1u : 0u);
           else
@@ -301,7 +309,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t kb = k_base + ks * L::kKVStage;
+        const uint64_t kd = k_desc0 + static_cast<uint64_t>((ks * L::kKVStage) >> 4);
         for (int t = 0; t < 2; ++t) {
           if (s > 0) {
             if (!mbar_wait(bar_pfull + t, (s - 1) & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL)) {
@@ -317,13 +325,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             issue_pv(t, s - 1);
             if (t == 1) mma_commit(bar_vempty + ((s - 1) % VS));
           }
-          const uint32_t qb = q_base + t * L::kQTile;
+          const uint64_t qd = q_desc0 + static_cast<uint64_t>((t * L::kQTile) >> 4);
           const uint32_t s_tmem = tmem + t * 128;
           // K (= head dim) advances 32 bytes per MMA inside each 128-byte swizzle chunk.
+#pragma unroll
           for (int kk = 0; kk < L::kRowBytes / 32; ++kk) {
-            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            const uint64_t adesc = make_sdesc_sw128(qb + off, 16, 1024);
-            const uint64_t bdesc = make_sdesc_sw128(kb + off, 16, 1024);
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
+            const uint64_t adesc = qd + off;
+            const uint64_t bdesc = kd + off;
             if constexpr (FP8)
               mma_f8_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
             else

@@ -89,6 +89,28 @@ cudaError_t launch_tile_permute_quant_e4m3(const GridDims& g, int batch, int hea
                                            const void* src, uint8_t* dst, float* scales,
                                            cudaStream_t stream);
 
+// Structured patterns (mirrors bsa_pattern in the C header).
+enum : uint32_t {
+  PAT_DIAGONAL = 1u,
+  PAT_MULTI_DIAGONAL = 2u,
+  PAT_VERTICAL_STRIPE = 4u,
+  PAT_SURROUNDING = 8u,
+  PAT_CRISS_CROSS = 16u,
+};
+struct PatternParams {
+  uint32_t kinds;
+  int diag_width, multi_count, multi_period, stripe_stride, stripe_offset;
+  int radius_t, radius_h, radius_w;
+};
+cudaError_t launch_pattern_csr(const AttnDims& a, const PatternParams& pp, int32_t* row_ptr,
+                               int32_t* col_idx, long long col_capacity, void* ws,
+                               cudaStream_t stream);
+
+// Per-row kept bitmaps + counts -> CSR (exclusive scan, then warp-per-row compaction).
+cudaError_t launch_bitmap_to_csr(const int32_t* counts, const uint32_t* bitmaps, long long rows,
+                                 int words, int32_t* row_ptr, int32_t* col_idx,
+                                 long long col_capacity, uint32_t* status, cudaStream_t stream);
+
 // Top-p selection.  Workspace layout after the status header: counts int32 [R],
 // bitmaps uint32 [R][words].
 size_t topp_scratch_bytes(long long rows, int n_kb);
@@ -115,6 +137,16 @@ cudaError_t launch_bsattn_fwd(const AttnDims& a, int fp8, const void* q, const v
 size_t mass_scratch_bytes(const AttnDims& a);
 cudaError_t launch_block_mass(const AttnDims& a, const void* q, const void* k, float softmax_scale,
                               float* mass, void* ws, cudaStream_t stream);
+
+// Fused calibration: dense attention output and block masses in one call.
+cudaError_t launch_calib_dense_mass(const AttnDims& a, const void* q, const void* k, const void* v,
+                                    float softmax_scale, void* out, float* lse, float* mass,
+                                    void* ws, cudaStream_t stream);
+
+// Pooled (block-level) estimate of the block masses.
+size_t pooled_scratch_bytes(const AttnDims& a);
+cudaError_t launch_pooled_mass(const AttnDims& a, const void* q, const void* k, float softmax_scale,
+                               float* mass, void* ws, cudaStream_t stream);
 
 // Encode a rank-3 bf16/e4m3 tensor map over [bh][Np][D] with a (box_d x box_rows x 1) box
 // and 128-byte swizzle.

@@ -1,0 +1,443 @@
+// Fused calibration step: the dense attention output and the exact block masses in one
+// call, sm_100a.
+//
+// "LoSA: Near-Lossless Sparse Attention for Training-Free Video Diffusion Acceleration",
+// Abstract: the calibration step runs dense attention and measures the exact block masses
+// on it.  Computing them separately costs two QK^T passes for the masses plus a QK^T and a
+// PV pass for the output; here
+//   pass 1: S = Q K^T over every kv block -> exact row log-sum-exp (online max and sum);
+//   pass 2: S again, P = exp2(S*c - lse2) -- the exact softmax probabilities, <= 1 -- used
+//           both for the per-block mass sums and, stored to TMEM as bf16, for O += P V.
+// Since P is already normalised, O needs no rescaling and no final division.
+//
+// Layout and roles follow the block-sparse forward (attn_fwd.cu): 256 query slots per CTA
+// in two M=128 tiles, 320 threads (warps 0-7 row owners, warp 8 TMA, warp 9 MMA), TMEM
+// S0 S1 O0 O1.  In pass 1 the MMA of S_t(s+1) waits until the rows of S_t(s) have been
+// read (S_free); in pass 2 the order is PV_t(s-1), S_t(s) as in the forward.
+#include "bsa_kernels.cuh"
+
+namespace bsa {
+
+namespace calib {
+constexpr int kThreads = 320;
+constexpr int kRowsPerCta = 256;
+}  // namespace calib
+
+struct CalibParams {
+  AttnDims a;
+  __nv_bfloat16* out;
+  float* lse;
+  float* mass;
+  uint32_t* status;
+  float scale_log2;
+};
+
+template <int D>
+struct CalibSmem {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kQTile = 128 * D * 2;
+  static constexpr int kKVStage = 128 * D * 2;
+  static constexpr int kKStages = (D == 128) ? 3 : 4;
+  static constexpr int kVStages = (D == 128) ? 2 : 4;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = 2 * kQTile;
+  static constexpr int kVOff = kKOff + kKStages * kKVStage;
+  static constexpr int kRedOff = kVOff + kVStages * kKVStage;  // float [2 parity][2 tile][4 warp][2 blk]
+  static constexpr int kBarOff = kRedOff + 2 * 2 * 4 * 2 * 4;
+  static constexpr int kBytes = kBarOff + 256;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(calib::kThreads, 1)
+    calib_dense_mass_kernel(const __grid_constant__ CUtensorMap tm_q,
+                            const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, const CalibParams p) {
+  using L = CalibSmem<D>;
+  constexpr int KS = L::kKStages, VS = L::kVStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_kfull = bars + 1;
+  uint64_t* bar_kempty = bar_kfull + KS;
+  uint64_t* bar_vfull = bar_kempty + KS;
+  uint64_t* bar_vempty = bar_vfull + VS;
+  uint64_t* bar_sfull = bar_vempty + VS;  // [2]
+  uint64_t* bar_sfree = bar_sfull + 2;    // [2] pass 1: rows of S_t read
+  uint64_t* bar_pfull = bar_sfree + 2;    // [2] pass 2: P_t stored
+  uint64_t* bar_ofull = bar_pfull + 2;
+  uint64_t* bar_drain = bar_ofull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* nvalid_sm = reinterpret_cast<int*>(tmem_slot + 2);  // [2 tile][4 warp]
+  float* red = reinterpret_cast<float*>(smem + L::kRedOff);
+
+  const AttnDims& a = p.a;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int cta = blockIdx.x;
+  const int bh = cta / a.n_cta_per_head;
+  const int row0 = (cta - bh * a.n_cta_per_head) * calib::kRowsPerCta;
+  const int npass = (a.n_kb + 1) >> 1;  // steps per pass
+  const int nsteps = 2 * npass;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < KS; ++i) {
+      mbar_init(bar_kfull + i, 1);
+      mbar_init(bar_kempty + i, 1);
+    }
+    for (int i = 0; i < VS; ++i) {
+      mbar_init(bar_vfull + i, 1);
+      mbar_init(bar_vempty + i, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_sfull + t, 1);
+      mbar_init(bar_sfree + t, 128);
+      mbar_init(bar_pfull + t, 128);
+    }
+    mbar_init(bar_ofull, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      mbar_arrive_expect_tx(bar_q, 2 * L::kQTile);
+      for (int t = 0; t < 2; ++t)
+        for (int ch = 0; ch < L::kChunks; ++ch)
+          tma_load_3d(smem + L::kQOff + t * L::kQTile + ch * (128 * 128), &tm_q, bar_q, ch * 64,
+                      row0 + t * 128, bh);
+      for (int s = 0; s < nsteps; ++s) {
+        const int st = s % npass;
+        const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+        const int ks = s % KS;
+        if (s >= KS && !mbar_wait(bar_kempty + ks, ((s / KS) - 1) & 1, abort_flag, p.status,
+                                  DETAIL_WAIT_K_EMPTY))
+          break;
+        mbar_arrive_expect_tx(bar_kfull + ks, nb * 64 * D * 2);
+        uint8_t* kst = smem + L::kKOff + ks * L::kKVStage;
+        for (int ch = 0; ch < L::kChunks; ++ch) {
+          tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * 64, 2 * st * 64, bh);
+          if (nb == 2)
+            tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * 64,
+                        (2 * st + 1) * 64, bh);
+        }
+        if (s < npass) continue;  // V is needed in pass 2 only
+        const int u = s - npass;
+        const int vs = u % VS;
+        if (u >= VS && !mbar_wait(bar_vempty + vs, ((u / VS) - 1) & 1, abort_flag, p.status,
+                                  DETAIL_WAIT_V_EMPTY))
+          break;
+        mbar_arrive_expect_tx(bar_vfull + vs, nb * 64 * D * 2);
+        uint8_t* vst = smem + L::kVOff + vs * L::kKVStage;
+        for (int ch = 0; ch < L::kChunks; ++ch) {
+          tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * 64, 2 * st * 64, bh);
+          if (nb == 2)
+            tma_load_3d(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch * 64,
+                        (2 * st + 1) * 64, bh);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint64_t q_desc0 = make_sdesc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
+      const uint64_t k_desc0 = make_sdesc_sw128(smem_u32(smem + L::kKOff), 16, 1024);
+      const uint64_t v_desc0 = make_sdesc_sw128(smem_u32(smem + L::kVOff), 128 * 128, 1024);
+      const uint32_t idesc_pv = make_idesc(1u, 1u, 128u, static_cast<uint32_t>(D));
+      bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, DETAIL_WAIT_Q);
+      auto issue_pv = [&](int t, int u) {
+        // O_t (+)= P_t V over the keys of pass-2 step u (64 or 128 keys, 16 per MMA).
+        const int nbp = (2 * u + 1 < a.n_kb) ? 2 : 1;
+        const uint64_t vd = v_desc0 + static_cast<uint64_t>(((u % VS) * L::kKVStage) >> 4);
+        const uint32_t p_tmem = tmem + t * 128;
+        const uint32_t o_tmem = tmem + 256 + t * D;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          if (kk >= nbp * 4) break;
+          mma_f16_ts(o_tmem, p_tmem + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4),
+                     idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      for (int s = 0; s < nsteps && ok; ++s) {
+        const int st = s % npass;
+        const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+        const int ks = s % KS;
+        const uint32_t idesc_qk = make_idesc(1u, 0u, 128u, static_cast<uint32_t>(nb * 64));
+        if (!mbar_wait(bar_kfull + ks, (s / KS) & 1, abort_flag, p.status, DETAIL_WAIT_K_FULL)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t kd = k_desc0 + static_cast<uint64_t>((ks * L::kKVStage) >> 4);
+        for (int t = 0; t < 2; ++t) {
+          if (s >= 1 && s <= npass) {
+            // S_t is free once its rows of the previous step were read (pass 1 and the
+            // first step of pass 2)
+            if (!mbar_wait(bar_sfree + t, (s - 1) & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL)) {
+              ok = false;
+              break;
+            }
+          } else if (s > npass) {
+            const int u = s - 1 - npass;  // pass-2 step whose P is consumed now
+            if (!mbar_wait(bar_pfull + t, u & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL)) {
+              ok = false;
+              break;
+            }
+            if (t == 0 && !mbar_wait(bar_vfull + (u % VS), (u / VS) & 1, abort_flag, p.status,
+                                     DETAIL_WAIT_V_FULL)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(t, u);
+            if (t == 1) mma_commit(bar_vempty + (u % VS));
+          }
+          tc_fence_after();
+          const uint64_t qd = q_desc0 + static_cast<uint64_t>((t * L::kQTile) >> 4);
+          const uint32_t s_tmem = tmem + t * 128;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
+            mma_f16_ss(s_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_sfull + t);
+        }
+        if (!ok) break;
+        mma_commit(bar_kempty + ks);
+      }
+      if (ok) {
+        const int u = npass - 1;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!mbar_wait(bar_pfull + t, u & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL)) {
+            ok = false;
+            break;
+          }
+          if (t == 0 && !mbar_wait(bar_vfull + (u % VS), (u / VS) & 1, abort_flag, p.status,
+                                   DETAIL_WAIT_V_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(t, u);
+        }
+        if (ok) mma_commit(bar_ofull);
+      }
+      mma_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0, p.status, DETAIL_WAIT_O_FULL);
+    }
+  } else {
+    // ------------------------------------------------------------ row owners
+    const int t = warp >> 2;
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const int slot = row0 + t * 128 + row;
+    const bool in_range = slot < a.g.Np;
+    const bool q_valid = in_range && slot_valid(a.g, slot);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t s_addr = lane_base + t * 128;
+    const uint32_t o_addr = lane_base + 256 + t * D;
+    const float c = p.scale_log2;
+    const int wcount = __popc(__ballot_sync(0xffffffffu, q_valid));
+    if (lane == 0) nvalid_sm[t * 4 + wq] = wcount;
+    named_bar_sync(1 + t, 128);
+    const int warps_per_qb = a.q_block / 32;  // 2 or 4
+    const int qb_first_warp = (wq / warps_per_qb) * warps_per_qb;
+    int nvq = 0;
+    for (int i = 0; i < warps_per_qb; ++i) nvq += nvalid_sm[t * 4 + qb_first_warp + i];
+    const int qb_global = (row0 + t * 128 + qb_first_warp * 32) / a.q_block;
+    const bool writer = (wq == qb_first_warp) && lane < 2 && qb_global < a.n_qb;
+    float* mass_row = p.mass + (static_cast<long long>(bh) * a.n_qb + qb_global) * a.n_kb;
+    const float inv_nvq = nvq > 0 ? 1.f / static_cast<float>(nvq) : 0.f;
+
+    float m_run = -INFINITY, l_run = 0.f, lse2 = 0.f;
+    bool ok = true;
+    for (int s = 0; s < nsteps; ++s) {
+      const int st = s % npass;
+      const bool pass2 = s >= npass;
+      const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+      if (s == npass) lse2 = (l_run > 0.f) ? m_run + log2f(l_run) : INFINITY;
+      // A warp that gives up keeps stepping (without touching TMEM) so that every warp of
+      // the group passes the same named barriers.
+      bool got = ok ? mbar_wait(bar_sfull + t, s & 1, abort_flag, p.status, DETAIL_WAIT_S_FULL)
+                    : false;
+      got = __all_sync(0xffffffffu, got);
+      ok = got;
+      float rs[2] = {0.f, 0.f};
+      if (got) {
+        tc_fence_after();
+        float sv[128];
+        tmem_ld32(s_addr + 0, sv + 0);
+        tmem_ld32(s_addr + 32, sv + 32);
+        if (nb == 2) {
+          tmem_ld32(s_addr + 64, sv + 64);
+          tmem_ld32(s_addr + 96, sv + 96);
+        }
+        tmem_ld_wait();
+        if (!pass2) {
+          tc_fence_before();
+          mbar_arrive(bar_sfree + t);
+        }
+        // pad keys and the absent half of a 1-block step -> -inf
+        const int j0 = 2 * st;
+        const uint64_t mk0 = tile_has_pad(a.g, j0) ? tile_valid_mask(a.g, j0) : ~0ull;
+        const uint64_t mk1 =
+            nb == 2 ? (tile_has_pad(a.g, j0 + 1) ? tile_valid_mask(a.g, j0 + 1) : ~0ull) : 0ull;
+        if ((mk0 & mk1) != ~0ull) {
+          const uint32_t mw[4] = {static_cast<uint32_t>(mk0), static_cast<uint32_t>(mk0 >> 32),
+                                  static_cast<uint32_t>(mk1), static_cast<uint32_t>(mk1 >> 32)};
+#pragma unroll
+          for (int i = 0; i < 128; ++i) sv[i] = ((mw[i >> 5] >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
+        }
+        if (!pass2) {
+          float mx[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+#pragma unroll
+          for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
+          const float mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+          const float m_new = fmaxf(m_run, mrow * c);
+          if (m_new != -INFINITY) {
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 128; ++i) ls[i & 3] += fast_exp2(fmaf(sv[i], c, -m_new));
+            l_run = l_run * fast_exp2(m_run - m_new) + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+            m_run = m_new;
+          }
+        } else {
+          // exact probabilities; pad query rows contribute nothing to the masses
+          float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            if (ch >= 2 && nb == 1) break;
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float p0 = fast_exp2(fmaf(sv[32 * ch + 2 * i], c, -lse2));
+              const float p1 = fast_exp2(fmaf(sv[32 * ch + 2 * i + 1], c, -lse2));
+              acc[ch >> 1][i & 1] += p0 + p1;
+              pk[i] = pack_bf16x2(p0, p1);
+            }
+            BSA_TMEM_ST_X16(s_addr + 16 * ch, pk);
+          }
+          if (q_valid) {
+            rs[0] = acc[0][0] + acc[0][1];
+            rs[1] = acc[1][0] + acc[1][1];
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(bar_pfull + t);
+        }
+      }
+      if (pass2) {
+        // per-(query block, kv block) sums: warp shuffles, then the 2 or 4 warps of the
+        // query block through shared memory in a fixed order (deterministic)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          rs[0] += __shfl_xor_sync(0xffffffffu, rs[0], o);
+          rs[1] += __shfl_xor_sync(0xffffffffu, rs[1], o);
+        }
+        float* rbuf = red + ((s & 1) * 2 + t) * 8;
+        if (lane < 2) rbuf[wq * 2 + lane] = lane == 0 ? rs[0] : rs[1];
+        named_bar_sync(1 + t, 128);
+        if (writer && (lane < nb)) {
+          float tot = 0.f;
+          for (int i = 0; i < warps_per_qb; ++i) tot += rbuf[(qb_first_warp + i) * 2 + lane];
+          mass_row[2 * st + lane] = tot * inv_nvq;
+        }
+      }
+    }
+
+    // ------------------------------------------------------------ epilogue
+    bool have_o = ok && npass > 0;
+    if (have_o) {
+      have_o = __all_sync(0xffffffffu,
+                          mbar_wait(bar_ofull, 0, abort_flag, p.status, DETAIL_WAIT_O_FULL));
+      tc_fence_after();
+    }
+    const float omul = (q_valid && l_run > 0.f) ? 1.f : 0.f;
+    __nv_bfloat16* orow = p.out + (static_cast<long long>(bh) * a.g.Np + slot) * D;
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      float ov[32];
+      if (have_o) {
+        tmem_ld32(o_addr + c0, ov);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] = 0.f;
+      }
+      if (in_range) {
+        uint4 w[4];
+        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) wp[i] = pack_bf16x2(ov[2 * i] * omul, ov[2 * i + 1] * omul);
+        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = w[i];
+      }
+    }
+    if (p.lse != nullptr && in_range)
+      p.lse[static_cast<long long>(bh) * a.g.Np + slot] =
+          (q_valid && l_run > 0.f) ? lse2 * 0.6931471805599453f : -INFINITY;
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+static cudaError_t launch_calib(const AttnDims& a, const void* q, const void* k, const void* v,
+                                const CalibParams& prm, long long ctas, cudaStream_t stream) {
+  using L = CalibSmem<D>;
+  CUtensorMap tq, tk, tv;
+  const int bh = a.batch * a.heads;
+  cudaError_t e = encode_tmap_3d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.g.Np, bh, 64, 128);
+  if (e != cudaSuccess) return e;
+  e = encode_tmap_3d(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.g.Np, bh, 64, 64);
+  if (e != cudaSuccess) return e;
+  e = encode_tmap_3d(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.g.Np, bh, 64, 64);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(calib_dense_mass_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           L::kAlloc);
+  if (e != cudaSuccess) return e;
+  calib_dense_mass_kernel<D><<<static_cast<unsigned>(ctas), calib::kThreads, L::kAlloc, stream>>>(
+      tq, tk, tv, prm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_calib_dense_mass(const AttnDims& a, const void* q, const void* k, const void* v,
+                                    float softmax_scale, void* out, float* lse, float* mass,
+                                    void* ws, cudaStream_t stream) {
+  const long long ctas = static_cast<long long>(a.batch) * a.heads * a.n_cta_per_head;
+  if (ctas == 0) return cudaSuccess;
+  CalibParams prm;
+  prm.a = a;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.mass = mass;
+  prm.status = static_cast<uint32_t*>(ws);
+  prm.scale_log2 = softmax_scale * 1.4426950408889634f;
+  if (a.head_dim == 128) return launch_calib<128>(a, q, k, v, prm, ctas, stream);
+  return launch_calib<64>(a, q, k, v, prm, ctas, stream);
+}
+
+}  // namespace bsa

@@ -26,7 +26,7 @@ namespace bsa {
 
 // One warp per row, kSelWarps rows per CTA, warp-synchronous (no CTA barriers).
 // Shared memory per warp: the row's fixed-point masses (n_kb uint64) and a 256-bin
-// histogram of uint64 sums.
+// histogram (counts and remainder sums, 32-bit).
 constexpr int kSelWarps = 4;
 
 __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
@@ -66,8 +66,8 @@ __global__ void __launch_bounds__(32 * kSelWarps) topp_select_rows_kernel(
   const int lane = threadIdx.x & 31;
   const long long r = static_cast<long long>(blockIdx.x) * kSelWarps + warp;
   if (r >= rows) return;
-  unsigned long long* qrow = sel_smem + static_cast<size_t>(warp) * (n_kb + 256);
-  unsigned long long* hist = qrow + n_kb;
+  unsigned long long* qrow = sel_smem + static_cast<size_t>(warp) * (n_kb + 512);
+  unsigned long long* hist = qrow + n_kb;  // 4 KB: 256 counts + 3 x 256 remainder sums
   const float* row = mass + r * n_kb;
 
   // fixed-point masses into shared memory; sum, max, min
@@ -96,17 +96,36 @@ __global__ void __launch_bounds__(32 * kSelWarps) topp_select_rows_kernel(
 
   // Invariant: elements above hi are all kept, their sum is A < target, and the value of
   // the last kept element lies in [lo, hi].
+  // Bin sums use only native 32-bit shared atomics: inside a level every candidate is
+  // q = lo + (d << shift) + rem with rem < 2^shift, so a bin's exact sum is
+  // count * (lo + (d << shift)) + sum(rem), and sum(rem) is kept as up to three 32-bit
+  // sums of 16-bit pieces of rem (each at most 4096 * 2^16).
   unsigned long long A = 0;
+  uint32_t* hcnt = reinterpret_cast<uint32_t*>(hist);   // [256]
+  uint32_t* hrem = hcnt + 256;                          // [3][256]
   while (target > 0 && hi > lo) {
     const unsigned long long span = hi - lo;
     const int nbits = 64 - __clzll(static_cast<long long>(span));
     const int shift = nbits > 8 ? nbits - 8 : 0;
+    const int pieces = (shift + 15) >> 4;  // 16-bit pieces of rem (<= 3: shift <= 45)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) hist[lane * 8 + i] = 0ull;
+    for (int i = 0; i < 8; ++i) {
+      hcnt[lane * 8 + i] = 0u;
+      hrem[lane * 8 + i] = 0u;
+      hrem[256 + lane * 8 + i] = 0u;
+      hrem[512 + lane * 8 + i] = 0u;
+    }
     __syncwarp();
     for (int j = lane; j < n_kb; j += 32) {
       const unsigned long long q = qrow[j];
-      if (q >= lo && q <= hi) atomicAdd(&hist[(q - lo) >> shift], q);
+      if (q >= lo && q <= hi) {
+        const unsigned long long x = q - lo;
+        const int d = static_cast<int>(x >> shift);
+        const unsigned long long rem = x & ((1ull << shift) - 1ull);
+        atomicAdd(&hcnt[d], 1u);
+        for (int k = 0; k < pieces; ++k)
+          atomicAdd(&hrem[256 * k + d], static_cast<uint32_t>((rem >> (16 * k)) & 0xFFFFull));
+      }
     }
     __syncwarp();
     // lane l owns bins 255-8l .. 248-8l (descending); inclusive sums from the top
@@ -114,7 +133,13 @@ __global__ void __launch_bounds__(32 * kSelWarps) topp_select_rows_kernel(
     unsigned long long run = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      run += hist[255 - 8 * lane - i];
+      const int d = 255 - 8 * lane - i;
+      const unsigned long long cnt = hcnt[d];
+      unsigned long long bs = cnt * (lo + (static_cast<unsigned long long>(d) << shift));
+      bs += static_cast<unsigned long long>(hrem[d]);
+      bs += static_cast<unsigned long long>(hrem[256 + d]) << 16;
+      bs += static_cast<unsigned long long>(hrem[512 + d]) << 32;
+      run += bs;
       b[i] = run;
     }
     unsigned long long before = run;  // exclusive warp scan of lane totals
@@ -245,7 +270,7 @@ __global__ void __launch_bounds__(256) topp_fill_kernel(const uint32_t* __restri
 static cudaError_t launch_select_rows(const float* mass, long long rows, int n_kb, float threshold,
                                       int32_t* counts, uint32_t* bitmaps, int words,
                                       uint32_t* status, cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(kSelWarps) * (n_kb + 256) * sizeof(unsigned long long);
+  const size_t smem = static_cast<size_t>(kSelWarps) * (n_kb + 512) * sizeof(unsigned long long);
   cudaError_t e = cudaFuncSetAttribute(topp_select_rows_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -253,6 +278,17 @@ static cudaError_t launch_select_rows(const float* mass, long long rows, int n_k
   const long long ctas = (rows + kSelWarps - 1) / kSelWarps;
   topp_select_rows_kernel<<<static_cast<unsigned>(ctas), 32 * kSelWarps, smem, stream>>>(
       mass, rows, n_kb, static_cast<double>(threshold), counts, bitmaps, words, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bitmap_to_csr(const int32_t* counts, const uint32_t* bitmaps, long long rows,
+                                 int words, int32_t* row_ptr, int32_t* col_idx,
+                                 long long col_capacity, uint32_t* status, cudaStream_t stream) {
+  topp_scan_kernel<<<1, 1024, 0, stream>>>(counts, rows, row_ptr);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  topp_fill_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+      bitmaps, words, rows, row_ptr, col_idx, col_capacity, status);
   return cudaGetLastError();
 }
 

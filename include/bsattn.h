@@ -67,7 +67,32 @@ typedef enum {
 
 typedef enum { BSA_BF16 = 0, BSA_FP32 = 1, BSA_E4M3 = 2 } bsa_dtype;
 
-typedef enum { BSA_OP_BLOCK_MASS = 0, BSA_OP_TOPP_SELECT = 1, BSA_OP_FWD = 2 } bsa_op;
+typedef enum {
+  BSA_OP_BLOCK_MASS = 0,
+  BSA_OP_TOPP_SELECT = 1,
+  BSA_OP_FWD = 2,
+  BSA_OP_PATTERN = 3,
+  BSA_OP_POOLED_MASS = 4
+} bsa_op;
+
+/* Structured kv-block patterns for bsa_pattern_csr (bit flags, combined by union). */
+typedef enum {
+  BSA_PAT_DIAGONAL = 1,         /* |j - u| <= diag_width                                   */
+  BSA_PAT_MULTI_DIAGONAL = 2,   /* |j - (u + k*L)| <= diag_width, 0 < |k| <= multi_count   */
+  BSA_PAT_VERTICAL_STRIPE = 4,  /* j % stripe_stride == stripe_offset, for every row        */
+  BSA_PAT_SURROUNDING = 8,      /* tile of j within (radius_t, radius_h, radius_w) of u     */
+  BSA_PAT_CRISS_CROSS = 16      /* tile of j shares at least two tile coordinates with u    */
+} bsa_pattern_kind;
+
+typedef struct {
+  uint32_t kinds;               /* OR of bsa_pattern_kind */
+  int32_t diag_width;           /* half width of every diagonal band, in blocks (>= 0) */
+  int32_t multi_count;          /* extra diagonals on each side (>= 0) */
+  int32_t multi_period;         /* L in blocks; <= 0 means the tiles of one temporal layer */
+  int32_t stripe_stride;        /* > 0 enables stripes */
+  int32_t stripe_offset;        /* 0 <= offset < stride */
+  int32_t radius_t, radius_h, radius_w;  /* >= 0, in tiles */
+} bsa_pattern;
 
 typedef struct {
   int32_t batch, heads, head_dim; /* B, Hh, D */
@@ -121,10 +146,37 @@ BSA_API bsa_status bsa_block_mass(const bsa_shape* shape, const void* q, const v
                           float softmax_scale, float* mass, void* ws, size_t ws_bytes,
                           bsa_stream_t stream);
 
+/* Fused calibration step: the dense attention output and the exact block masses in one
+ * call ("LoSA", Abstract: the calibration step is a dense attention step on which the
+ * block masses are measured).  Pass 1 computes each query row's exact log-sum-exp; pass 2
+ * forms the exact probabilities once and uses them for both the masses (as
+ * bsa_block_mass) and out = P V.  q, k, v: tile-major bf16 [B,Hh,Np,D].  out: bf16
+ * tile-major (pad query slots zero); lse (nullable): fp32 [B,Hh,Np] natural log; mass:
+ * fp32 [B,Hh,Np/q_block,Np/64].  Workspace as for BSA_OP_BLOCK_MASS. */
+BSA_API bsa_status bsa_dense_fwd_mass(const bsa_shape* shape, const void* q, const void* k,
+                                      const void* v, float softmax_scale, void* out, float* lse,
+                                      float* mass, void* ws, size_t ws_bytes,
+                                      bsa_stream_t stream);
+
+/* Pooled estimate of the block masses, for per-step ("online") selection without a dense
+ * pass ("Sparse VideoGen2", Abstract: top-p dynamic budget control on attention between
+ * token clusters).  With the 4x4x4 tiles as clusters: qbar_i = mean of the valid queries
+ * of query block i, kbar_j = mean of the valid keys of kv block j, n_j = its valid keys;
+ * mass_est[b,h,i,j] = n_j exp(s qbar_i.kbar_j) / sum_j' n_j' exp(s qbar_i.kbar_j'), with
+ * s = softmax_scale; 0 for blocks without valid keys; zero rows for query blocks without
+ * valid queries.  Feed the result to bsa_topp_select.  q, k: tile-major bf16; mass_est:
+ * fp32 [B,Hh,Np/q_block,Np/64].  Workspace: bsa_workspace_bytes(shape,
+ * BSA_OP_POOLED_MASS). */
+BSA_API bsa_status bsa_pooled_mass(const bsa_shape* shape, const void* q, const void* k,
+                                   float softmax_scale, float* mass_est, void* ws,
+                                   size_t ws_bytes, bsa_stream_t stream);
+
 /* Retained-mass (top-p) block selection ("LoSA", Abstract: per head and query block,
  * the fewest kv blocks whose mass reaches the threshold are kept; "Sparse VideoGen2",
  * Abstract: top-p dynamic budget control).  mass: fp32 [R, Np/64] with
- * R = B*Hh*(Np/q_block), values finite in [0, 4096].  Per row, masses become integers
+ * R = B*Hh*(Np/q_block), values finite in [0, 4096] (others are flagged DEVICE_INPUT and
+ * count as 0) with each row summing to less than 2^22 (block masses are probabilities; a
+ * row sums to 1).  Per row, masses become integers
  * q = rint(m * 2^40); target = ceil(threshold * sum q) (one fp64 multiply); blocks are
  * ranked by (q desc, index asc) and the shortest prefix reaching the target is kept.
  * Output CSR: row_ptr int32 [R+1] (row_ptr[0] = 0), col_idx int32 ascending within a
@@ -160,6 +212,17 @@ BSA_API bsa_status bsa_topp_select_noalloc(const bsa_shape* shape, const float* 
                                            float threshold, int32_t* row_ptr, int32_t* col_idx,
                                            int64_t col_capacity, uint32_t* status,
                                            bsa_stream_t stream);
+
+/* Static structured kv-block lists ("Sparse-vDiT", Abstract: diagonal, multi-diagonal and
+ * vertical-stripe attention structures; "GRAT", Abstract: key regions restricted to
+ * surrounding blocks or criss-cross lines).  Blocks are 4x4x4 tiles in tile-major order;
+ * u ranges over the tile(s) of query block i (one for q_block 64, two for 128); kv block j
+ * is kept when any enabled kind holds for some u.  Output CSR as bsa_topp_select (same
+ * lists for every batch and head; ascending within a row).  Workspace:
+ * bsa_workspace_bytes(shape, BSA_OP_PATTERN). */
+BSA_API bsa_status bsa_pattern_csr(const bsa_shape* shape, const bsa_pattern* pattern,
+                                   int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                   void* ws, size_t ws_bytes, bsa_stream_t stream);
 
 /* Block-sparse attention forward over frozen CSR block lists ("LoSA", Abstract: the
  * frozen block indices are reused for all remaining steps).  For each query slot of

@@ -125,6 +125,13 @@ def test_rejections_before_launch(B):
     bad[10] = ctypes.c_void_p(0x10002)                                       # lse not 4-byte aligned
     assert L.bsa_fwd(_c(B), 0, *bad, big, n) == 1
     assert L.bsa_fwd(_c(B, T=30), 0, *args, big, n) == 1                     # T > Tp
+    P = B.bsattn._Pattern
+    assert L.bsa_pattern_csr(_c(B), None, FAKE, FAKE, 10, FAKE, big, n) == 1
+    assert L.bsa_pattern_csr(_c(B), ctypes.byref(P(64)), FAKE, FAKE, 10, FAKE, big, n) == 1
+    assert L.bsa_pattern_csr(_c(B), ctypes.byref(P(1, -1)), FAKE, FAKE, 10, FAKE, big, n) == 1
+    assert L.bsa_pattern_csr(_c(B), ctypes.byref(P(4, 0, 0, 0, 5, 5)), FAKE, FAKE, 10, FAKE, big,
+                             n) == 1                                          # offset >= stride
+    assert L.bsa_pattern_csr(_c(B), ctypes.byref(P(1)), FAKE, FAKE, 10, FAKE, 16, n) == 3
 
 
 def test_status_strings(B):

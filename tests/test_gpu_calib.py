@@ -1,0 +1,65 @@
+"""GPU parity of the fused calibration call: dense attention output and block masses in one
+pass pair, against the oracle's dense attention (every block kept) and its block masses."""
+import numpy as np
+import pytest
+
+import helpers as Hp
+from oracle import bsa_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+WLS = Hp.small_workloads()
+
+
+@pytest.fixture(scope="module")
+def B(cuda_device):
+    from block_sparse_attention_25_b200 import build
+    build.build()
+    import block_sparse_attention_25_b200 as b
+    return b
+
+
+@pytest.mark.parametrize("wl", WLS, ids=[w.name for w in WLS])
+@pytest.mark.parametrize("sharp", [1.0, 6.0])
+def test_dense_fwd_mass_parity(B, wl, sharp):
+    g = Hp.grid_of(wl)
+    s = B.Shape.of(wl)
+    q, k, v = Hp.draw(wl, value_scale=1.0, sharp=sharp)
+    qt, kt, vt = (B.tile_permute(x.cuda(), s) for x in (q, k, v))
+    ws = B.new_workspace(s, B.OP_BLOCK_MASS)
+    out, mass, lse = B.dense_fwd_mass(qt, kt, vt, s, want_lse=True, ws=ws)
+    assert B.device_status(ws) == 0, B.device_status_words(ws)
+    qo, ko, vo = (Hp.oracle_tiled(x, g) for x in (q, k, v))
+    m_ref = O.block_mass(qo, ko, g, wl.q_block, 64, Hp.scale_of(wl))
+    got_m = mass.cpu().double().numpy()
+    assert np.abs(got_m - m_ref).max() <= Hp.MASS_ABS
+    assert np.all(got_m[m_ref == 0] == 0)
+    n_qb, n_kb = wl.Np // wl.q_block, wl.Np // 64
+    R = wl.batch * wl.heads * n_qb
+    rp = np.arange(R + 1) * n_kb
+    ci = np.tile(np.arange(n_kb), R)
+    o_ref, lse_ref = O.masked_attention(qo, ko, vo, g, wl.q_block, 64, rp, ci, Hp.scale_of(wl))
+    e = Hp.attn_errors(out.cpu().double().numpy(), o_ref)
+    assert e["max_abs"] <= Hp.ATTN_MAX_ABS and e["mean_abs"] <= Hp.ATTN_MEAN_ABS, e
+    zero = ~np.isfinite(lse_ref)
+    lg = lse.cpu().double().numpy()
+    assert np.all(np.isneginf(lg[zero]))
+    assert np.abs(lg[~zero] - lse_ref[~zero]).max() <= 1e-3
+
+
+def test_dense_fwd_mass_matches_separate_calls(B):
+    """The fused masses equal bsa_block_mass's within fp32 rounding, and its output equals
+    bsa_fwd over the full list."""
+    wl = WLS[0]
+    s = B.Shape.of(wl)
+    q, k, v = Hp.draw(wl, value_scale=1.0, sharp=4.0)
+    qt, kt, vt = (B.tile_permute(x.cuda(), s) for x in (q, k, v))
+    out, mass = B.dense_fwd_mass(qt, kt, vt, s)
+    m2 = B.block_mass(qt, kt, s)
+    assert float((mass - m2).abs().max()) <= 1e-6
+    import torch
+    R, n_kb = s.rows, s.n_kb
+    rp = (torch.arange(R + 1, dtype=torch.int32) * n_kb).cuda()
+    ci = torch.arange(n_kb, dtype=torch.int32).repeat(R).cuda()
+    o2 = B.bsattn_fwd(qt, kt, vt, rp, ci, s)
+    assert float((out.float() - o2.float()).abs().max()) <= 1e-2
