@@ -1,0 +1,155 @@
+"""Per-call timing of every entry point on one workload, one JSON line per call.
+
+    python -m block_sparse_attention_25_b200.microbench [--config wan14b_720p] [--iters 5]
+
+Each call is timed alone with CUDA events on the launch stream (median of --iters timed
+launches after two warm-up launches); inputs are seeded synthetic draws resident in HBM.
+Every line carries the call's algorithmic work (bytes for the memory-bound calls, FLOPs for
+the contractions), the achieved rate and its fraction of the peak: the measured copy
+bandwidth or the measured burst bf16 rate from MEASURED_PEAKS.json at the repository root
+(the e4m3 peak is taken as twice the bf16 one, the nominal ratio).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+
+import torch
+
+from . import bsattn as B
+from . import build, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, source="fallback")
+
+
+def _time(fn, iters: int) -> float:
+    stream = torch.cuda.current_stream()
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(iters):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms.append(a.elapsed_time(b))
+    return sorted(ms)[len(ms) // 2]
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--config", default="wan14b_720p")
+    ap.add_argument("--iters", type=int, default=5)
+    ap.add_argument("--tau", type=float, default=0.99)
+    args = ap.parse_args(argv)
+    build.build()
+    dev = torch.device("cuda")
+    wl = synth.WORKLOADS[args.config]
+    s = B.Shape.of(wl)
+    pk = _peaks()
+    q, k, v = synth.draw_qkv(wl, device=dev)
+    e = 2  # bf16 bytes
+    S, Np, Hh, D, R, nkb = s.S * s.batch, s.Np * s.batch, s.heads, s.head_dim, s.rows, s.n_kb
+
+    def line(name, ms, work, unit, bound, peak, extra=None):
+        rate = work / (ms * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
+        d = {"call": name, "workload": wl.name, "ms": round(ms, 4), "work": work,
+             "work_unit": "bytes" if unit == "GB/s" else "FLOP", "achieved": round(rate, 2),
+             "unit": unit, "bound": bound, "peak": peak, "frac": round(rate / peak, 4),
+             "peak_source": pk["source"]}
+        if extra:
+            d.update(extra)
+        print(json.dumps(d), flush=True)
+
+    qt, kt, vt = (B.tile_permute(x, s) for x in (q, k, v))
+    out_r = torch.empty_like(q)
+    line("tile_permute", _time(lambda: B.tile_permute(q, s, out=qt), args.iters),
+         S * Hh * D * e + Np * Hh * D * e, "GB/s", "hbm", pk["hbm"])
+    line("tile_permute_inverse", _time(lambda: B.tile_permute(qt, s, inverse=True, out=out_r), args.iters),
+         2 * S * Hh * D * e, "GB/s", "hbm", pk["hbm"])
+    if D == 128:
+        q8 = torch.empty(qt.shape, dtype=torch.uint8, device=dev)
+        sc = torch.empty((s.batch, Hh, s.Np // 64), dtype=torch.float32, device=dev)
+        line("tile_permute_quant_e4m3",
+             _time(lambda: B.tile_permute_quant_e4m3(q, s, out=q8, scales=sc), args.iters),
+             S * Hh * D * e + Np * Hh * D + 4 * Hh * Np // 64, "GB/s", "hbm", pk["hbm"])
+
+    mass = torch.empty((s.batch, Hh, s.n_qb, nkb), dtype=torch.float32, device=dev)
+    ws_m = B.new_workspace(s, B.OP_BLOCK_MASS, dev)
+    dense_qk = 2.0 * 2 * Np * s.Np * D * Hh  # two QK^T passes over all slot pairs
+    line("block_mass", _time(lambda: B.block_mass(qt, kt, s, out=mass, ws=ws_m), args.iters),
+         dense_qk, "TFLOP/s", "tensor", pk["bf16"])
+    out_t = torch.empty_like(qt)
+    mass2 = torch.empty_like(mass)
+    line("dense_fwd_mass",
+         _time(lambda: B.dense_fwd_mass(qt, kt, vt, s, out=out_t, mass=mass2, ws=ws_m), args.iters),
+         1.5 * dense_qk, "TFLOP/s", "tensor", pk["bf16"])
+
+    ws_t = B.new_workspace(s, B.OP_TOPP_SELECT, dev)
+    row_ptr = torch.empty(R + 1, dtype=torch.int32, device=dev)
+    col_idx = torch.empty(R * nkb, dtype=torch.int32, device=dev)
+    ms = _time(lambda: B.topp_select(mass, s, args.tau, ws=ws_t, row_ptr=row_ptr, col_idx=col_idx),
+               args.iters)
+    nnz = int(row_ptr[-1])
+    line("topp_select", ms, 4 * R * nkb + 4 * (R + 1 + nnz), "GB/s", "hbm", pk["hbm"],
+         {"kept_fraction": round(nnz / (R * nkb), 5)})
+
+    ws_p = B.new_workspace(s, B.OP_POOLED_MASS, dev)
+    pmass = torch.empty_like(mass)
+    line("pooled_mass", _time(lambda: B.pooled_mass(qt, kt, s, out=pmass, ws=ws_p), args.iters),
+         2 * Np * Hh * D * e + 4 * R * nkb, "GB/s", "hbm", pk["hbm"])
+
+    ws_pt = B.new_workspace(s, B.OP_PATTERN, dev)
+    prp = torch.empty(R + 1, dtype=torch.int32, device=dev)
+    pci = torch.empty(R * nkb, dtype=torch.int32, device=dev)
+    kinds = B.PAT_DIAGONAL | B.PAT_MULTI_DIAGONAL | B.PAT_VERTICAL_STRIPE | B.PAT_SURROUNDING
+
+    def pat():
+        B.pattern_csr(s, kinds, diag_width=2, multi_count=2, stripe_stride=16, radius=(1, 2, 2),
+                      ws=ws_pt, row_ptr=prp, col_idx=pci, device=dev)
+    ms = _time(pat, args.iters)
+    pnnz = int(prp[-1])
+    line("pattern_csr", ms, 4 * (R + 1 + pnnz), "GB/s", "hbm", pk["hbm"],
+         {"kept_fraction": round(pnnz / (R * nkb), 5)})
+
+    ws_f = B.new_workspace(s, B.OP_FWD, dev)
+    out_t = torch.empty_like(qt)
+    fl = 4.0 * nnz * s.q_block * 64 * D
+    line("bsattn_fwd", _time(lambda: B.bsattn_fwd(qt, kt, vt, row_ptr, col_idx, s, out=out_t, ws=ws_f),
+                             args.iters), fl, "TFLOP/s", "tensor", pk["bf16"],
+         {"kept_fraction": round(nnz / (R * nkb), 5)})
+    if D == 128:
+        k8, v8 = torch.empty_like(q8), torch.empty_like(q8)
+        scs = [sc, torch.empty_like(sc), torch.empty_like(sc)]
+        B.tile_permute_quant_e4m3(q, s, out=q8, scales=scs[0])
+        B.tile_permute_quant_e4m3(k, s, out=k8, scales=scs[1])
+        B.tile_permute_quant_e4m3(v, s, out=v8, scales=scs[2])
+        line("bsattn_fwd_e4m3",
+             _time(lambda: B.bsattn_fwd(q8, k8, v8, row_ptr, col_idx, s, scales=scs, out=out_t, ws=ws_f),
+                   args.iters), fl, "TFLOP/s", "tensor", 2 * pk["bf16"],
+             {"kept_fraction": round(nnz / (R * nkb), 5)})
+    # structured lists through the same attention kernel
+    pfl = 4.0 * pnnz * s.q_block * 64 * D
+    line("bsattn_fwd_pattern", _time(lambda: B.bsattn_fwd(qt, kt, vt, prp, pci, s, out=out_t, ws=ws_f),
+                                     args.iters), pfl, "TFLOP/s", "tensor", pk["bf16"],
+         {"kept_fraction": round(pnnz / (R * nkb), 5)})
+    for w in (ws_m, ws_t, ws_p, ws_pt, ws_f):
+        st = B.device_status(w)
+        if st != 0:
+            raise RuntimeError(f"device status {st}: {B.device_status_words(w)}")
+
+
+if __name__ == "__main__":
+    main()
