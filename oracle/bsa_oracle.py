@@ -449,3 +449,97 @@ def pooled_block_mass(qt, kt, g: Grid, q_block: int, kv_block: int, scale: float
                 w = n_keys[keep] * np.exp(z)
                 out[b, h, i, keep] = w / w.sum()
     return out
+
+
+# --------------------------------------------------------------------------- semantic clusters
+# "Sparse VideoGen2", Abstract: semantic-aware permutation -- tokens are clustered by
+# k-means on their vectors and reordered so that each cluster is contiguous, with no
+# padding; cluster representatives identify the critical clusters (top-p dynamic budget
+# control) and the attention runs over the densified layout.  Reading R10:
+#   * per (batch, head), queries and keys are clustered separately by Lloyd's k-means from
+#     given initial centroids for a fixed number of rounds; a round assigns every token to
+#     the nearest centroid (squared Euclidean distance, ties to the lowest index) and then
+#     replaces each centroid by the mean of its tokens (an empty cluster keeps its centroid);
+#   * the assignment is an integer decided by floating point, so it is taken in float32 as
+#     argmin_c (|c|^2 - 2 x.c), the kernel's precision; the means are float64 here;
+#   * cluster order: clusters by index, tokens of one cluster in their raster order;
+#   * cluster-level estimate as in R8 with clusters for tiles: weights n_j exp(s qc_i . kc_j)
+#     over the key clusters, normalised per query cluster (qc, kc the final centroids);
+#   * the selection is R3 applied to those rows; a query token attends to every key of the
+#     key clusters selected for its cluster, softmax renormalised over them (R4).
+def kmeans_assign(x, centroids) -> np.ndarray:
+    """Nearest centroid of every row of x, decided in float32 (reading R10)."""
+    x32 = np.asarray(x, dtype=np.float32)
+    c32 = np.asarray(centroids, dtype=np.float32)
+    d = (c32 * c32).sum(axis=1, dtype=np.float32)[None, :] - np.float32(2.0) * (x32 @ c32.T)
+    return np.argmin(d, axis=1).astype(np.int64)  # first minimum: the lowest index
+
+
+def kmeans_lloyd(x, init, rounds: int):
+    """(labels, centroids float64 [C, D], counts) after `rounds` assign-then-update rounds."""
+    x = np.asarray(x, dtype=np.float64)
+    c = np.array(init, dtype=np.float64)
+    labels = np.zeros(x.shape[0], dtype=np.int64)
+    for _ in range(rounds):
+        labels = kmeans_assign(x, c)
+        for j in range(c.shape[0]):
+            member = labels == j
+            if member.any():
+                c[j] = x[member].mean(axis=0)
+    counts = np.bincount(labels, minlength=c.shape[0])
+    return labels, c, counts
+
+
+def cluster_layout(labels, n_clusters: int):
+    """(starts, token_of_slot, slot_of_token): clusters in index order, tokens of a cluster
+    in raster order (a stable sort by cluster id)."""
+    labels = np.asarray(labels, dtype=np.int64)
+    counts = np.bincount(labels, minlength=n_clusters)
+    starts = np.concatenate([[0], np.cumsum(counts)[:-1]]).astype(np.int64)
+    token_of_slot = np.argsort(labels, kind="stable").astype(np.int64)
+    slot_of_token = np.empty_like(token_of_slot)
+    slot_of_token[token_of_slot] = np.arange(labels.size)
+    return starts, token_of_slot, slot_of_token
+
+
+def cluster_mass(qc, q_counts, kc, k_counts, scale: float) -> np.ndarray:
+    """Estimated mass [Cq, Ck] of key cluster j for query cluster i (reading R10)."""
+    qc = np.asarray(qc, dtype=np.float64)
+    kc = np.asarray(kc, dtype=np.float64)
+    nk = np.asarray(k_counts, dtype=np.float64)
+    out = np.zeros((qc.shape[0], kc.shape[0]))
+    keep = nk > 0
+    if not keep.any():
+        return out
+    for i in range(qc.shape[0]):
+        if q_counts[i] == 0:
+            continue
+        logits = scale * (kc[keep] @ qc[i])
+        w = nk[keep] * np.exp(logits - logits.max())
+        out[i, keep] = w / w.sum()
+    return out
+
+
+def cluster_attention(q, k, v, q_starts, q_counts, k_starts, k_counts, row_ptr, col_idx,
+                      scale: float, rows=None) -> np.ndarray:
+    """Attention in cluster order [S, D]: the queries of cluster i attend to the keys of the
+    key clusters col_idx[row_ptr[i]:row_ptr[i+1]] (reading R10).  `rows` restricts the
+    computation to those query slots (others stay zero)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    out = np.zeros((q.shape[0], v.shape[1]))
+    want = None if rows is None else set(int(r) for r in rows)
+    for i in range(len(q_starts)):
+        keys = np.concatenate([np.arange(k_starts[j], k_starts[j] + k_counts[j])
+                               for j in col_idx[row_ptr[i]:row_ptr[i + 1]]] or [np.zeros(0, int)])
+        keys = keys.astype(np.int64)
+        for p in range(int(q_starts[i]), int(q_starts[i] + q_counts[i])):
+            if want is not None and p not in want:
+                continue
+            if keys.size == 0:
+                continue
+            logits = scale * (k[keys] @ q[p])
+            w = np.exp(logits - logits.max())
+            out[p] = (w / w.sum()) @ v[keys]
+    return out

@@ -500,3 +500,135 @@ def test_pooled_estimate_rows_and_zero_scale():
     for i in range(g.Np // 64):
         if valid[i * 64:(i + 1) * 64].any():
             assert np.allclose(z[0, 0, i], nvk / nvk.sum(), atol=1e-14, rtol=0)
+
+
+# ------------------------------------------------------------------ semantic clusters
+def _blobs(seed, n_per, centers, spread):
+    """Well-separated Gaussian blobs; returns points, ground-truth ids, one seed point per blob."""
+    rng = np.random.default_rng(seed)
+    pts, ids = [], []
+    for j, c in enumerate(centers):
+        pts.append(c + spread * rng.standard_normal((n_per[j], len(c))))
+        ids += [j] * n_per[j]
+    x = np.concatenate(pts)
+    ids = np.array(ids)
+    perm = rng.permutation(x.shape[0])
+    x, ids = x[perm], ids[perm]
+    init = np.stack([x[np.flatnonzero(ids == j)[0]] for j in range(len(centers))])
+    return x, ids, init
+
+
+def test_kmeans_recovers_separated_blobs():
+    rng = np.random.default_rng(1)
+    centers = 10.0 * rng.standard_normal((5, 16))
+    x, ids, init = _blobs(2, [30, 1, 12, 40, 7], centers, 0.05)
+    labels, c, counts = O.kmeans_lloyd(x, init, rounds=4)
+    assert np.array_equal(labels, ids)
+    assert counts.tolist() == [30, 1, 12, 40, 7]
+    for j in range(5):   # the centroids are the blob means of the generating partition
+        np.testing.assert_allclose(c[j], x[ids == j].mean(axis=0), rtol=0, atol=1e-12)
+
+
+def test_kmeans_matches_sklearn_lloyd():
+    from sklearn.cluster import KMeans
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((400, 8))
+    init = x[rng.choice(400, 6, replace=False)]
+    def fit(rounds):
+        return KMeans(n_clusters=6, init=init, n_init=1, max_iter=rounds, tol=0.0,
+                      algorithm="lloyd").fit(x)
+    for rounds in (2, 4, 10):
+        labels, c, _ = O.kmeans_lloyd(x, init, rounds)
+        np.testing.assert_allclose(c, fit(rounds).cluster_centers_, rtol=0, atol=1e-9)
+        # sklearn's labels_ come from one more assignment against its final centres, so the
+        # oracle's last assignment (against the centres of round - 1) is sklearn's labels_
+        # after rounds - 1 rounds
+        assert np.array_equal(labels, fit(rounds - 1).labels_)
+    # one round: the assignment against the initial centres, by brute-force distances
+    labels, _, _ = O.kmeans_lloyd(x, init, 1)
+    d = np.array([[((xi - cj) ** 2).sum() for cj in init] for xi in x])
+    assert np.array_equal(labels, d.argmin(axis=1))
+
+
+def test_kmeans_inertia_never_increases_and_empty_cluster_keeps_centroid():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((200, 4))
+    far = np.full(4, 1e3)                      # a centroid no point is nearest to
+    init = np.concatenate([x[:3], far[None]])
+    prev = np.inf
+    for rounds in range(1, 6):
+        labels, c, counts = O.kmeans_lloyd(x, init, rounds)
+        inertia = ((x - c[labels]) ** 2).sum()
+        assert inertia <= prev + 1e-9
+        prev = inertia
+        assert counts[3] == 0 and np.array_equal(c[3], far)
+
+
+def test_kmeans_ties_go_to_lowest_index():
+    x = np.array([[0.0, 0.0], [2.0, 0.0]])
+    c = np.array([[1.0, 1.0], [1.0, -1.0], [1.0, 1.0]])   # every point equidistant
+    assert O.kmeans_assign(x, c).tolist() == [0, 0]
+
+
+def test_cluster_layout_is_stable_counting_sort():
+    rng = np.random.default_rng(5)
+    labels = rng.integers(0, 7, size=300)
+    labels[labels == 4] = 5                                 # an empty cluster
+    starts, tos, sot = O.cluster_layout(labels, 7)
+    # brute force: walk the clusters in order, tokens in raster order
+    expect = [t for j in range(7) for t in range(300) if labels[t] == j]
+    assert tos.tolist() == expect
+    assert np.array_equal(sot[tos], np.arange(300))
+    counts = np.bincount(labels, minlength=7)
+    for j in range(7):
+        assert np.all(labels[tos[starts[j]:starts[j] + counts[j]]] == j)
+    assert starts[4] == starts[5]
+
+
+def test_cluster_mass_is_exact_for_constant_clusters():
+    # every token equals its cluster's centroid: the estimate is the exact softmax mass
+    rng = np.random.default_rng(6)
+    D, Cq, Ck = 8, 3, 4
+    qc, kc = rng.standard_normal((Cq, D)), rng.standard_normal((Ck, D))
+    nq, nk = np.array([2, 5, 1]), np.array([3, 1, 4, 2])
+    q = np.repeat(qc, nq, axis=0)
+    k = np.repeat(kc, nk, axis=0)
+    scale = 0.7
+    est = O.cluster_mass(qc, nq, kc, nk, scale)
+    kid = np.repeat(np.arange(Ck), nk)
+    qid = np.repeat(np.arange(Cq), nq)
+    p = torch.softmax(torch.tensor(scale * q @ k.T), dim=-1).numpy()
+    for i in range(Cq):
+        exact = [p[qid == i][:, kid == j].sum(axis=1).mean() for j in range(Ck)]
+        np.testing.assert_allclose(est[i], exact, rtol=1e-12, atol=1e-15)
+
+
+def test_cluster_mass_empty_clusters():
+    est = O.cluster_mass(np.ones((2, 3)), np.array([0, 4]), np.ones((3, 3)), np.array([2, 0, 2]), 1.0)
+    assert np.all(est[0] == 0) and est[1, 1] == 0
+    np.testing.assert_allclose(est[1].sum(), 1.0)
+
+
+def test_cluster_attention_matches_masked_sdpa():
+    rng = np.random.default_rng(7)
+    S, D = 60, 8
+    labels_q = rng.integers(0, 4, size=S)
+    labels_k = rng.integers(0, 5, size=S)
+    q, k, v = (rng.standard_normal((S, D)) for _ in range(3))
+    qs, qtos, _ = O.cluster_layout(labels_q, 4)
+    ks, ktos, _ = O.cluster_layout(labels_k, 5)
+    qn, kn = np.bincount(labels_q, minlength=4), np.bincount(labels_k, minlength=5)
+    sel = [[0, 2], [1], [0, 1, 2, 3, 4], []]               # cluster 3 keeps nothing
+    row_ptr = np.concatenate([[0], np.cumsum([len(r) for r in sel])])
+    col_idx = np.array([j for r in sel for j in r])
+    scale = 0.4
+    out = O.cluster_attention(q[qtos], k[ktos], v[ktos], qs, qn, ks, kn, row_ptr, col_idx, scale)
+    # reference: SDPA in raster order with the boolean mask of selected cluster pairs
+    allowed = np.zeros((S, S), dtype=bool)
+    for t in range(S):
+        allowed[t] = np.isin(labels_k, sel[labels_q[t]])
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q)[None], torch.tensor(k)[None], torch.tensor(v)[None],
+        attn_mask=torch.tensor(allowed)[None], scale=scale)[0].numpy()
+    ref[~allowed.any(axis=1)] = 0.0
+    np.testing.assert_allclose(out, ref[qtos], rtol=1e-10, atol=1e-12)
