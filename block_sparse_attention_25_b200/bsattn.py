@@ -5,7 +5,10 @@ PyTorch provides device memory and the current CUDA stream.  There is no fallbac
 the library cannot be loaded every call raises.
 
 Names follow the C ABI in include/bsattn.h:
-    tile_permute, tile_permute_quant_e4m3, block_mass, topp_select, bsattn_fwd
+    tile_permute, tile_permute_quant_e4m3, block_mass, dense_fwd_mass, pooled_mass,
+    topp_select, topp_select_noalloc, pattern_csr, bsattn_fwd;
+    cluster order: kmeans, cluster_layout, cluster_permute, cluster_mass,
+    topp_select_rows, cluster_fwd
 """
 from __future__ import annotations
 
@@ -25,6 +28,26 @@ STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "capa
 BSA_BF16, BSA_FP32, BSA_E4M3 = 0, 1, 2
 OP_BLOCK_MASS, OP_TOPP_SELECT, OP_FWD, OP_PATTERN, OP_POOLED_MASS = 0, 1, 2, 3, 4
 PAT_DIAGONAL, PAT_MULTI_DIAGONAL, PAT_VERTICAL_STRIPE, PAT_SURROUNDING, PAT_CRISS_CROSS = 1, 2, 4, 8, 16
+
+
+class _ClusterShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("batch", "heads", "head_dim", "n_tokens",
+                                              "n_q_clusters", "n_k_clusters")]
+
+
+@dataclass(frozen=True)
+class ClusterShape:
+    """bsa_cluster_shape: S tokens per (batch, head), clustered separately for queries and keys."""
+    batch: int
+    heads: int
+    head_dim: int
+    n_tokens: int
+    n_q_clusters: int
+    n_k_clusters: int
+
+    def c(self) -> _ClusterShape:
+        return _ClusterShape(self.batch, self.heads, self.head_dim, self.n_tokens,
+                             self.n_q_clusters, self.n_k_clusters)
 
 
 class BsaError(RuntimeError):
@@ -102,6 +125,7 @@ def lib() -> ctypes.CDLL:
     L = ctypes.CDLL(LIB_PATH)
     P, I, S, F, L64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float, ctypes.c_int64
     SP = ctypes.POINTER(_Shape)
+    CSP = ctypes.POINTER(_ClusterShape)
     sig = {
         "bsa_workspace_bytes": (S, [SP, I]),
         "bsa_clear_status": (I, [P, P]),
@@ -118,6 +142,15 @@ def lib() -> ctypes.CDLL:
         "bsa_pattern_csr": (I, [SP, ctypes.POINTER(_Pattern), P, P, L64, P, S, P]),
         "bsa_fwd": (I, [SP, I, P, P, P, P, P, P, P, P, F, P, P, P, S, P]),
         "bsa_version": (ctypes.c_char_p, []),
+        "bsa_kmeans_workspace_bytes": (S, [CSP, I]),
+        "bsa_cluster_fwd_workspace_bytes": (S, [CSP]),
+        "bsa_topp_rows_workspace_bytes": (S, [L64, I]),
+        "bsa_kmeans": (I, [CSP, I, P, I, P, P, P, P, S, P]),
+        "bsa_cluster_layout": (I, [CSP, I, P, P, P, P, P, P, S, P]),
+        "bsa_cluster_permute": (I, [CSP, I, P, P, P, P]),
+        "bsa_cluster_mass": (I, [CSP, P, P, P, P, F, P, P]),
+        "bsa_topp_select_rows": (I, [P, L64, I, F, P, P, L64, P, S, P]),
+        "bsa_cluster_fwd": (I, [CSP, P, P, P, P, P, P, P, P, P, F, P, P, P, S, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -131,7 +164,10 @@ EXPORTED_SYMBOLS = ("bsa_workspace_bytes", "bsa_clear_status", "bsa_device_statu
                     "bsa_device_status_words", "bsa_status_string", "bsa_tile_permute",
                     "bsa_tile_permute_quant_e4m3", "bsa_block_mass", "bsa_topp_select", "bsa_fwd",
                     "bsa_topp_select_noalloc", "bsa_pattern_csr", "bsa_dense_fwd_mass",
-                    "bsa_pooled_mass", "bsa_version")
+                    "bsa_pooled_mass", "bsa_version", "bsa_kmeans_workspace_bytes",
+                    "bsa_cluster_fwd_workspace_bytes", "bsa_topp_rows_workspace_bytes",
+                    "bsa_kmeans", "bsa_cluster_layout", "bsa_cluster_permute", "bsa_cluster_mass",
+                    "bsa_topp_select_rows", "bsa_cluster_fwd")
 
 
 def _check(status: int, what: str):
@@ -365,4 +401,145 @@ def bsattn_fwd(q, k, v, row_ptr, col_idx, shape: Shape, softmax_scale=None, scal
     _check(lib().bsa_fwd(ctypes.byref(shape.c()), BSA_E4M3 if fp8 else BSA_BF16, _ptr(q), _ptr(k),
                          _ptr(v), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(row_ptr), _ptr(col_idx), scale,
                          _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)), "bsa_fwd")
+    return (out, lse) if want_lse else out
+
+
+# ------------------------------------------------------------------ cluster order
+def _i32(t, shape, name):
+    _need(t, torch.int32, shape, name)
+
+
+def kmeans(x, cs: ClusterShape, n_clusters: int, init, rounds: int, labels=None, counts=None,
+           ws=None, stream=None):
+    """bsa_kmeans on raster bf16 x [B, S, Hh, D].  init (fp32 [B, Hh, C, D]) is updated in
+    place to the final centroids.  Returns (centroids, labels int32 [B,Hh,S], counts)."""
+    B, Hh, S, D = cs.batch, cs.heads, cs.n_tokens, cs.head_dim
+    _need(x, torch.bfloat16, (B, S, Hh, D), "x")
+    _need(init, torch.float32, (B, Hh, n_clusters, D), "centroids")
+    if labels is None:
+        labels = torch.empty((B, Hh, S), dtype=torch.int32, device=x.device)
+    if counts is None:
+        counts = torch.empty((B, Hh, n_clusters), dtype=torch.int32, device=x.device)
+    if ws is None:
+        ws = new_cluster_workspace(cs, n_clusters, x.device)
+    _check(lib().bsa_kmeans(ctypes.byref(cs.c()), int(n_clusters), _ptr(x), int(rounds), _ptr(init),
+                            _ptr(labels), _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)),
+           "bsa_kmeans")
+    return init, labels, counts
+
+
+def new_cluster_workspace(cs: ClusterShape, n_clusters: int, device="cuda") -> torch.Tensor:
+    n = int(lib().bsa_kmeans_workspace_bytes(ctypes.byref(cs.c()), int(n_clusters)))
+    if n == 0:
+        raise BsaError(1, "cluster workspace size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _check(lib().bsa_clear_status(_ptr(ws), _stream()), "bsa_clear_status")
+    return ws
+
+
+def cluster_layout(labels, cs: ClusterShape, n_clusters: int, ws=None, stream=None):
+    """bsa_cluster_layout: (counts, starts, token_of_slot, slot_of_token), int32."""
+    B, Hh, S = cs.batch, cs.heads, cs.n_tokens
+    _i32(labels, (B, Hh, S), "labels")
+    dev = labels.device
+    counts = torch.empty((B, Hh, n_clusters), dtype=torch.int32, device=dev)
+    starts = torch.empty_like(counts)
+    tos = torch.empty((B, Hh, S), dtype=torch.int32, device=dev)
+    sot = torch.empty_like(tos)
+    if ws is None:
+        ws = new_cluster_workspace(cs, n_clusters, dev)
+    _check(lib().bsa_cluster_layout(ctypes.byref(cs.c()), int(n_clusters), _ptr(labels), _ptr(counts),
+                                    _ptr(starts), _ptr(tos), _ptr(sot), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "bsa_cluster_layout")
+    return counts, starts, tos, sot
+
+
+def cluster_permute(x, cs: ClusterShape, token_of_slot, inverse: bool = False, out=None, stream=None):
+    """bsa_cluster_permute: raster [B,S,Hh,D] -> cluster order [B,Hh,S,D], or back."""
+    B, Hh, S, D = cs.batch, cs.heads, cs.n_tokens, cs.head_dim
+    raster, perm = (B, S, Hh, D), (B, Hh, S, D)
+    _need(x, torch.bfloat16, perm if inverse else raster, "src")
+    _i32(token_of_slot, (B, Hh, S), "token_of_slot")
+    if out is None:
+        out = torch.zeros(raster if inverse else perm, dtype=torch.bfloat16, device=x.device)
+    _check(lib().bsa_cluster_permute(ctypes.byref(cs.c()), int(bool(inverse)), _ptr(token_of_slot),
+                                     _ptr(x), _ptr(out), _stream(stream)), "bsa_cluster_permute")
+    return out
+
+
+def cluster_mass(cs: ClusterShape, q_centroids, q_counts, k_centroids, k_counts, softmax_scale=None,
+                 out=None, stream=None):
+    """bsa_cluster_mass: fp32 [B, Hh, Cq, Ck]."""
+    B, Hh, D, Cq, Ck = cs.batch, cs.heads, cs.head_dim, cs.n_q_clusters, cs.n_k_clusters
+    _need(q_centroids, torch.float32, (B, Hh, Cq, D), "q_centroids")
+    _need(k_centroids, torch.float32, (B, Hh, Ck, D), "k_centroids")
+    _i32(q_counts, (B, Hh, Cq), "q_counts")
+    _i32(k_counts, (B, Hh, Ck), "k_counts")
+    if out is None:
+        out = torch.empty((B, Hh, Cq, Ck), dtype=torch.float32, device=q_centroids.device)
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
+    _check(lib().bsa_cluster_mass(ctypes.byref(cs.c()), _ptr(q_centroids), _ptr(q_counts),
+                                  _ptr(k_centroids), _ptr(k_counts), scale, _ptr(out),
+                                  _stream(stream)), "bsa_cluster_mass")
+    return out
+
+
+def topp_select_rows(mass, threshold: float = 0.99, col_capacity=None, ws=None, row_ptr=None,
+                     col_idx=None, stream=None):
+    """bsa_topp_select_rows on a [..., cols] fp32 tensor viewed as rows x cols."""
+    if mass.dtype != torch.float32 or not mass.is_cuda or not mass.is_contiguous():
+        raise TypeError("mass: contiguous float32 CUDA tensor")
+    cols = int(mass.shape[-1])
+    rows = mass.numel() // cols
+    cap = rows * cols if col_capacity is None else int(col_capacity)
+    if row_ptr is None:
+        row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=mass.device)
+    if col_idx is None:
+        col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=mass.device)
+    if ws is None:
+        n = int(lib().bsa_topp_rows_workspace_bytes(rows, cols))
+        if n == 0:
+            raise BsaError(2, "topp rows workspace size")
+        ws = torch.empty(n, dtype=torch.uint8, device=mass.device)
+        _check(lib().bsa_clear_status(_ptr(ws), _stream()), "bsa_clear_status")
+    _check(lib().bsa_topp_select_rows(_ptr(mass), rows, cols, float(threshold), _ptr(row_ptr),
+                                      _ptr(col_idx), cap, _ptr(ws), ws.numel(), _stream(stream)),
+           "bsa_topp_select_rows")
+    return row_ptr, col_idx
+
+
+def new_cluster_fwd_workspace(cs: ClusterShape, device="cuda") -> torch.Tensor:
+    n = int(lib().bsa_cluster_fwd_workspace_bytes(ctypes.byref(cs.c())))
+    if n == 0:
+        raise BsaError(1, "cluster fwd workspace size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _check(lib().bsa_clear_status(_ptr(ws), _stream()), "bsa_clear_status")
+    return ws
+
+
+def cluster_fwd(q, k, v, cs: ClusterShape, q_starts, q_counts, k_starts, k_counts, row_ptr,
+                col_idx, softmax_scale=None, want_lse=False, out=None, lse=None, ws=None,
+                stream=None):
+    """bsa_cluster_fwd: attention in cluster order; returns out (or (out, lse))."""
+    B, Hh, S, D, Cq, Ck = cs.batch, cs.heads, cs.n_tokens, cs.head_dim, cs.n_q_clusters, cs.n_k_clusters
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, (B, Hh, S, D), n)
+    _i32(q_starts, (B, Hh, Cq), "q_starts")
+    _i32(q_counts, (B, Hh, Cq), "q_counts")
+    _i32(k_starts, (B, Hh, Ck), "k_starts")
+    _i32(k_counts, (B, Hh, Ck), "k_counts")
+    _i32(row_ptr, (B * Hh * Cq + 1,), "row_ptr")
+    if col_idx.dtype != torch.int32 or not col_idx.is_cuda:
+        raise TypeError("col_idx: int32 CUDA tensor")
+    if out is None:
+        out = torch.empty((B, Hh, S, D), dtype=torch.bfloat16, device=q.device)
+    if want_lse and lse is None:
+        lse = torch.empty((B, Hh, S), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = new_cluster_fwd_workspace(cs, q.device)
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
+    _check(lib().bsa_cluster_fwd(ctypes.byref(cs.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(q_starts),
+                                 _ptr(q_counts), _ptr(k_starts), _ptr(k_counts), _ptr(row_ptr),
+                                 _ptr(col_idx), scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                 _stream(stream)), "bsa_cluster_fwd")
     return (out, lse) if want_lse else out

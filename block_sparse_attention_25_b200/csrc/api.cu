@@ -53,6 +53,7 @@ cudaError_t encode_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataTy
 
 using bsa::AttnDims;
 using bsa::GridDims;
+using bsa::ClusterDims;
 
 namespace {
 
@@ -348,6 +349,164 @@ bsa_status bsa_fwd(const bsa_shape* shape, bsa_dtype dtype, const void* q, const
                              row_ptr, col_idx, softmax_scale, out, lse, ws, stream);
   if (e == cudaErrorNotSupported) return BSA_ERR_UNSUPPORTED;
   return from_cuda(e);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- semantic clusters
+namespace {
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+bsa_status check_cluster_shape(const bsa_cluster_shape* s) {
+  if (s == nullptr) return BSA_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->heads < 1 || s->n_tokens < 1 || s->n_q_clusters < 1 ||
+      s->n_k_clusters < 1)
+    return BSA_ERR_INVALID_ARG;
+  if (s->head_dim != 64 && s->head_dim != 128) return BSA_ERR_UNSUPPORTED;
+  if (s->n_tokens > (1 << 24) || s->n_q_clusters > 1024 || s->n_k_clusters > 1024)
+    return BSA_ERR_UNSUPPORTED;
+  const long long bh = 1LL * s->batch * s->heads;
+  // every per-head array and every flat row index fits in 31 bits
+  if (bh * s->n_tokens * (s->head_dim / 8) >= (1LL << 31)) return BSA_ERR_UNSUPPORTED;
+  if (bh * s->n_q_clusters * s->n_k_clusters >= (1LL << 31)) return BSA_ERR_UNSUPPORTED;
+  return BSA_OK;
+}
+
+ClusterDims cluster_dims(const bsa_cluster_shape* s, int C) {
+  ClusterDims cd;
+  cd.batch = s->batch;
+  cd.heads = s->heads;
+  cd.head_dim = s->head_dim;
+  cd.S = s->n_tokens;
+  cd.C = C;
+  return cd;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t bsa_kmeans_workspace_bytes(const bsa_cluster_shape* shape, int32_t n_clusters) {
+  if (check_cluster_shape(shape) != BSA_OK || n_clusters < 1 || n_clusters > 1024) return 0;
+  return bsa::kStatusBytes + bsa::cluster_scratch_bytes(cluster_dims(shape, n_clusters));
+}
+
+size_t bsa_cluster_fwd_workspace_bytes(const bsa_cluster_shape* shape) {
+  if (check_cluster_shape(shape) != BSA_OK) return 0;
+  return bsa::kStatusBytes + bsa::cluster_fwd_scratch_bytes(shape->batch * shape->heads,
+                                                            shape->n_tokens, shape->n_q_clusters,
+                                                            shape->n_k_clusters);
+}
+
+size_t bsa_topp_rows_workspace_bytes(int64_t rows, int32_t cols) {
+  if (rows < 0 || cols < 1 || cols > 4096 || rows * cols >= (1LL << 31)) return 0;
+  return bsa::kStatusBytes + bsa::topp_scratch_bytes(rows, cols);
+}
+
+bsa_status bsa_kmeans(const bsa_cluster_shape* shape, int32_t n_clusters, const void* x,
+                      int32_t rounds, float* centroids, int32_t* labels, int32_t* counts, void* ws,
+                      size_t ws_bytes, bsa_stream_t stream) {
+  bsa_status st = check_cluster_shape(shape);
+  if (st != BSA_OK) return st;
+  if (n_clusters < 1 || n_clusters > 1024) return BSA_ERR_UNSUPPORTED;
+  if (rounds < 1 || rounds > 10000) return BSA_ERR_INVALID_ARG;
+  if (x == nullptr || centroids == nullptr || labels == nullptr || counts == nullptr ||
+      ws == nullptr || !bsa::aligned16(x) || !aligned4(centroids) || !aligned4(labels) ||
+      !aligned4(counts) || !bsa::aligned16(ws))
+    return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < bsa_kmeans_workspace_bytes(shape, n_clusters)) return BSA_ERR_CAPACITY;
+  return from_cuda(bsa::launch_kmeans(cluster_dims(shape, n_clusters), x, rounds, centroids,
+                                      labels, counts, ws, stream));
+}
+
+bsa_status bsa_cluster_layout(const bsa_cluster_shape* shape, int32_t n_clusters,
+                              const int32_t* labels, int32_t* counts, int32_t* starts,
+                              int32_t* token_of_slot, int32_t* slot_of_token, void* ws,
+                              size_t ws_bytes, bsa_stream_t stream) {
+  bsa_status st = check_cluster_shape(shape);
+  if (st != BSA_OK) return st;
+  if (n_clusters < 1 || n_clusters > 1024) return BSA_ERR_UNSUPPORTED;
+  if (labels == nullptr || counts == nullptr || starts == nullptr || token_of_slot == nullptr ||
+      slot_of_token == nullptr || ws == nullptr || !aligned4(labels) || !aligned4(counts) ||
+      !aligned4(starts) || !aligned4(token_of_slot) || !aligned4(slot_of_token) ||
+      !bsa::aligned16(ws))
+    return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < bsa_kmeans_workspace_bytes(shape, n_clusters)) return BSA_ERR_CAPACITY;
+  return from_cuda(bsa::launch_cluster_layout(cluster_dims(shape, n_clusters), labels, counts,
+                                              starts, token_of_slot, slot_of_token, ws, stream));
+}
+
+bsa_status bsa_cluster_permute(const bsa_cluster_shape* shape, int inverse,
+                               const int32_t* token_of_slot, const void* src, void* dst,
+                               bsa_stream_t stream) {
+  bsa_status st = check_cluster_shape(shape);
+  if (st != BSA_OK) return st;
+  if (inverse != 0 && inverse != 1) return BSA_ERR_INVALID_ARG;
+  if (token_of_slot == nullptr || src == nullptr || dst == nullptr || !aligned4(token_of_slot) ||
+      !bsa::aligned16(src) || !bsa::aligned16(dst) || src == dst)
+    return BSA_ERR_INVALID_ARG;
+  return from_cuda(bsa::launch_cluster_permute(cluster_dims(shape, 1), inverse, token_of_slot, src,
+                                               dst, stream));
+}
+
+bsa_status bsa_cluster_mass(const bsa_cluster_shape* shape, const float* q_centroids,
+                            const int32_t* q_counts, const float* k_centroids,
+                            const int32_t* k_counts, float softmax_scale, float* mass,
+                            bsa_stream_t stream) {
+  bsa_status st = check_cluster_shape(shape);
+  if (st != BSA_OK) return st;
+  if (q_centroids == nullptr || q_counts == nullptr || k_centroids == nullptr ||
+      k_counts == nullptr || mass == nullptr || !aligned4(q_centroids) || !aligned4(q_counts) ||
+      !aligned4(k_centroids) || !aligned4(k_counts) || !aligned4(mass))
+    return BSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f)) return BSA_ERR_INVALID_ARG;
+  return from_cuda(bsa::launch_cluster_mass(shape->batch, shape->heads, shape->head_dim,
+                                            shape->n_q_clusters, shape->n_k_clusters, q_centroids,
+                                            q_counts, k_centroids, k_counts, softmax_scale, mass,
+                                            stream));
+}
+
+bsa_status bsa_topp_select_rows(const float* mass, int64_t rows, int32_t cols, float threshold,
+                                int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, void* ws,
+                                size_t ws_bytes, bsa_stream_t stream) {
+  if (rows < 0 || cols < 1) return BSA_ERR_INVALID_ARG;
+  if (cols > 4096 || rows * cols >= (1LL << 31)) return BSA_ERR_UNSUPPORTED;
+  if (mass == nullptr || row_ptr == nullptr || ws == nullptr || !bsa::aligned16(ws) ||
+      !aligned4(mass) || !aligned4(row_ptr))
+    return BSA_ERR_INVALID_ARG;
+  if (col_capacity < 0 || (col_capacity > 0 && (col_idx == nullptr || !aligned4(col_idx))))
+    return BSA_ERR_INVALID_ARG;
+  if (!(threshold > 0.f && threshold <= 1.f)) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < bsa_topp_rows_workspace_bytes(rows, cols)) return BSA_ERR_CAPACITY;
+  return from_cuda(bsa::launch_topp_select(mass, rows, cols, threshold, row_ptr, col_idx,
+                                           col_capacity, ws, stream));
+}
+
+bsa_status bsa_cluster_fwd(const bsa_cluster_shape* shape, const void* q, const void* k,
+                           const void* v, const int32_t* q_starts, const int32_t* q_counts,
+                           const int32_t* k_starts, const int32_t* k_counts,
+                           const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale,
+                           void* out, float* lse, void* ws, size_t ws_bytes,
+                           bsa_stream_t stream) {
+  bsa_status st = check_cluster_shape(shape);
+  if (st != BSA_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || q_starts == nullptr ||
+      q_counts == nullptr || k_starts == nullptr || k_counts == nullptr || row_ptr == nullptr ||
+      col_idx == nullptr || ws == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (!bsa::aligned16(q) || !bsa::aligned16(k) || !bsa::aligned16(v) || !bsa::aligned16(out) ||
+      !bsa::aligned16(ws) || !aligned4(q_starts) || !aligned4(q_counts) || !aligned4(k_starts) ||
+      !aligned4(k_counts) || !aligned4(row_ptr) || !aligned4(col_idx) ||
+      (lse != nullptr && !aligned4(lse)))
+    return BSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f)) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < bsa_cluster_fwd_workspace_bytes(shape)) return BSA_ERR_CAPACITY;
+  return from_cuda(bsa::launch_cluster_fwd(shape->batch, shape->heads, shape->head_dim,
+                                           shape->n_tokens, shape->n_q_clusters,
+                                           shape->n_k_clusters, q, k, v, q_starts, q_counts,
+                                           k_starts, k_counts, row_ptr, col_idx, softmax_scale,
+                                           out, lse, ws, stream));
 }
 
 }  // extern "C"

@@ -40,6 +40,13 @@ constexpr float kRescaleLog2 = 8.0f;
 // Schedule entry: (j << 5) | (has_pad_keys << 4) | keep bits for the CTA's <= 4 query blocks.
 __device__ __forceinline__ int entry_block(uint32_t e) { return static_cast<int>(e >> 5); }
 
+// Cluster order: an entry is a run of 1..64 consecutive keys, (first slot << 7) | length.
+__device__ __forceinline__ int entry_start(uint32_t e) { return static_cast<int>(e >> 7); }
+__device__ __forceinline__ uint64_t entry_len_mask(uint32_t e) {
+  const uint32_t len = e & 127u;
+  return len >= 64u ? ~0ull : ((1ull << len) - 1ull);
+}
+
 }  // namespace fwd
 
 // Build, per CTA, the ascending union of its query blocks' kv lists with keep bits.
@@ -140,6 +147,16 @@ struct FwdParams {
   float* lse;
   uint32_t* status;
   float scale_log2;  // softmax_scale * log2(e)
+  // cluster order only (tokens of a query cluster are consecutive slots; the CTAs of one
+  // head cover its clusters 256 rows at a time, cta_base[bh][c] = first CTA of cluster c)
+  int S;            // slots per (batch, head)
+  int n_qc;         // query clusters per (batch, head)
+  int cap;          // CTAs launched per (batch, head); those past cta_base[bh][n_qc] exit
+  int max_ent;      // entry capacity per query cluster
+  const int32_t* q_starts;
+  const int32_t* q_counts;
+  const int32_t* cta_base;   // [bh][n_qc + 1]
+  const int32_t* ent_counts; // [bh][n_qc]
 };
 
 // Shared-memory plan.  Every operand row is cut into 128-byte swizzle chunks (64 bf16 or
@@ -166,7 +183,7 @@ struct FwdSmem {
 // largest code is 256 * 1.75 = 448, the e4m3 maximum.
 constexpr float kPScale = 1.75f;
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool VARLEN>
 __global__ void __launch_bounds__(fwd::kThreads, 1)
     bsattn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -194,11 +211,40 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
-  const int bh = cta / a.n_cta_per_head;
-  const int row0 = (cta - bh * a.n_cta_per_head) * fwd::kRowsPerCta;
-  const int n_ent = p.counts[cta];
+  int bh, row0, n_ent, rows_here;
+  const uint32_t* ent;
+  if constexpr (VARLEN) {
+    // Which query cluster, and which 256 rows of it, this CTA owns.
+    bh = cta / p.cap;
+    const int local_cta = cta - bh * p.cap;
+    const int32_t* base = p.cta_base + static_cast<long long>(bh) * (p.n_qc + 1);
+    if (local_cta >= base[p.n_qc]) return;  // uniform: before any barrier or allocation
+    int lo = 0, hi = p.n_qc - 1;              // last cluster with base <= local_cta
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (base[mid] <= local_cta) lo = mid; else hi = mid - 1;
+    }
+    const int tile = local_cta - base[lo];
+    const long long qrow = static_cast<long long>(bh) * p.n_qc + lo;
+    const int qs = p.q_starts[qrow], qn = p.q_counts[qrow];
+    row0 = qs + tile * fwd::kRowsPerCta;
+    rows_here = min(fwd::kRowsPerCta, qn - tile * fwd::kRowsPerCta);
+    n_ent = p.ent_counts[qrow];
+    ent = p.entries + qrow * p.max_ent;
+    if (qs < 0 || qn < 0 || qs > p.S - qn) {  // the cluster's slots must lie inside the head
+      if (threadIdx.x == 0)
+        record_status(p.status, FLAG_DEVICE_INPUT, DETAIL_CLUSTER_RANGE, static_cast<uint32_t>(qrow), 0u);
+      rows_here = 0;
+      n_ent = 0;
+    }
+  } else {
+    bh = cta / a.n_cta_per_head;
+    row0 = (cta - bh * a.n_cta_per_head) * fwd::kRowsPerCta;
+    rows_here = fwd::kRowsPerCta;
+    n_ent = p.counts[cta];
+    ent = p.entries + static_cast<long long>(cta) * a.n_kb;
+  }
   const int nsteps = (n_ent + 1) >> 1;
-  const uint32_t* ent = p.entries + static_cast<long long>(cta) * a.n_kb;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -238,8 +284,11 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
                       row0 + t * 128, bh);
       for (int s = 0; s < nsteps; ++s) {
         const int nb = (2 * s + 1 < n_ent) ? 2 : 1;
-        const int j0 = fwd::entry_block(ent[2 * s]);
-        const int j1 = nb == 2 ? fwd::entry_block(ent[2 * s + 1]) : 0;
+        // first key row of each of the step's (one or two) 64-row boxes
+        const int j0 = VARLEN ? fwd::entry_start(ent[2 * s]) : fwd::entry_block(ent[2 * s]) * 64;
+        const int j1 = nb == 2 ? (VARLEN ? fwd::entry_start(ent[2 * s + 1])
+                                         : fwd::entry_block(ent[2 * s + 1]) * 64)
+                               : 0;
         const int ks = s % KS;
         if (s >= KS && !mbar_wait(bar_kempty + ks, ((s / KS) - 1) & 1, abort_flag, p.status,
                                   DETAIL_WAIT_K_EMPTY))
@@ -247,10 +296,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         mbar_arrive_expect_tx(bar_kfull + ks, nb * 64 * L::kRowBytes);
         uint8_t* kst = smem + L::kKOff + ks * L::kKVStage;
         for (int ch = 0; ch < L::kChunks; ++ch) {
-          tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * CE, j0 * 64, bh);
+          tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * CE, j0, bh);
           if (nb == 2)
             tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * CE,
-                        j1 * 64, bh);
+                        j1, bh);
         }
         const int vs = s % VS;
         if (s >= VS && !mbar_wait(bar_vempty + vs, ((s / VS) - 1) & 1, abort_flag, p.status,
@@ -259,10 +308,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         mbar_arrive_expect_tx(bar_vfull + vs, nb * 64 * L::kRowBytes);
         uint8_t* vst = smem + L::kVOff + vs * L::kKVStage;
         for (int ch = 0; ch < L::kChunks; ++ch) {
-          tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * CE, j0 * 64, bh);
+          tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * CE, j0, bh);
           if (nb == 2)
             tma_load_3d(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch * CE,
-                        j1 * 64, bh);
+                        j1, bh);
         }
       }
     }
@@ -371,9 +420,11 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     const int row = wq * 32 + lane;    // row inside the tile
     const int local = t * 128 + row;   // row inside the CTA
     const int slot = row0 + local;     // query slot inside the head
-    const int qsel = local / a.q_block;
-    const bool in_range = slot < a.g.Np;
-    const bool q_valid = in_range && slot_valid(a.g, slot);
+    const int qsel = VARLEN ? 0 : local / a.q_block;
+    // in_range: the row is this CTA's to write; q_valid: it holds a token
+    const bool in_range = VARLEN ? local < rows_here : slot < a.g.Np;
+    const bool q_valid = VARLEN ? in_range : (in_range && slot_valid(a.g, slot));
+    const long long head_slots = VARLEN ? p.S : a.g.Np;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t s_addr = lane_base + t * 128;
     const uint32_t o_addr = lane_base + 256 + t * D;
@@ -417,9 +468,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       // Column masks (warp-uniform: a warp's rows share one query block).  A block this
       // query block did not keep, or a pad key, or the absent half of a 1-block step -> -inf.
       uint64_t mk0 = 0ull, mk1 = 0ull;
-      if ((e0 >> qsel) & 1u) mk0 = ((e0 >> 4) & 1u) ? tile_valid_mask(a.g, fwd::entry_block(e0)) : ~0ull;
-      if (nb == 2 && ((e1 >> qsel) & 1u))
-        mk1 = ((e1 >> 4) & 1u) ? tile_valid_mask(a.g, fwd::entry_block(e1)) : ~0ull;
+      if constexpr (VARLEN) {  // every row keeps every run; a short run masks its tail
+        mk0 = fwd::entry_len_mask(e0);
+        if (nb == 2) mk1 = fwd::entry_len_mask(e1);
+      } else {
+        if ((e0 >> qsel) & 1u) mk0 = ((e0 >> 4) & 1u) ? tile_valid_mask(a.g, fwd::entry_block(e0)) : ~0ull;
+        if (nb == 2 && ((e1 >> qsel) & 1u))
+          mk1 = ((e1 >> 4) & 1u) ? tile_valid_mask(a.g, fwd::entry_block(e1)) : ~0ull;
+      }
       if ((mk0 & mk1) != ~0ull) {
         const uint32_t mw[4] = {static_cast<uint32_t>(mk0), static_cast<uint32_t>(mk0 >> 32),
                                 static_cast<uint32_t>(mk1), static_cast<uint32_t>(mk1 >> 32)};
@@ -530,7 +586,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
                           mbar_wait(bar_ofull, 0, abort_flag, p.status, DETAIL_WAIT_O_FULL));
       tc_fence_after();
     }
-    __nv_bfloat16* orow = p.out + (static_cast<long long>(bh) * a.g.Np + slot) * D;
+    __nv_bfloat16* orow = p.out + (static_cast<long long>(bh) * head_slots + slot) * D;
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       float ov[32];
@@ -554,7 +610,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     if (p.lse != nullptr && in_range) {
       const float lse = (l_run > 0.f && q_valid) ? (m_run + __log2f(l_run)) * 0.6931471805599453f
                                                  : -INFINITY;
-      p.lse[static_cast<long long>(bh) * a.g.Np + slot] = lse;
+      p.lse[static_cast<long long>(bh) * head_slots + slot] = lse;
     }
   }
 
@@ -575,25 +631,26 @@ size_t fwd_scratch_bytes(const AttnDims& a) {
   return 2 * counts + static_cast<size_t>(ctas) * a.n_kb * 4;
 }
 
-template <int D, bool FP8>
-static cudaError_t launch_fwd(const AttnDims& a, const void* q, const void* k, const void* v,
-                              const FwdParams& prm, long long ctas, cudaStream_t stream) {
+template <int D, bool FP8, bool VARLEN>
+static cudaError_t launch_fwd(const AttnDims& a, int rows_per_head, const void* q, const void* k,
+                              const void* v, const FwdParams& prm, long long ctas,
+                              cudaStream_t stream) {
   using L = FwdSmem<D, FP8>;
   CUtensorMap tq, tk, tv;
   const int bh = a.batch * a.heads;
   const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const int eb = L::kElem, ce = L::kChunkElems;
-  cudaError_t e = encode_tmap_3d(&tq, q, dt, eb, D, a.g.Np, bh, ce, 128);
+  cudaError_t e = encode_tmap_3d(&tq, q, dt, eb, D, rows_per_head, bh, ce, 128);
   if (e != cudaSuccess) return e;
-  e = encode_tmap_3d(&tk, k, dt, eb, D, a.g.Np, bh, ce, 64);
+  e = encode_tmap_3d(&tk, k, dt, eb, D, rows_per_head, bh, ce, 64);
   if (e != cudaSuccess) return e;
-  e = encode_tmap_3d(&tv, v, dt, eb, D, a.g.Np, bh, ce, 64);
+  e = encode_tmap_3d(&tv, v, dt, eb, D, rows_per_head, bh, ce, 64);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(bsattn_fwd_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           L::kAlloc);
+  e = cudaFuncSetAttribute(bsattn_fwd_kernel<D, FP8, VARLEN>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
-  bsattn_fwd_kernel<D, FP8><<<static_cast<unsigned>(ctas), fwd::kThreads, L::kAlloc, stream>>>(
-      tq, tk, tv, prm);
+  bsattn_fwd_kernel<D, FP8, VARLEN>
+      <<<static_cast<unsigned>(ctas), fwd::kThreads, L::kAlloc, stream>>>(tq, tk, tv, prm);
   return cudaGetLastError();
 }
 
@@ -628,9 +685,189 @@ cudaError_t launch_bsattn_fwd(const AttnDims& a, int fp8, const void* q, const v
   prm.lse = lse;
   prm.status = status;
   prm.scale_log2 = softmax_scale * 1.4426950408889634f;
-  if (fp8) return launch_fwd<128, true>(a, q, k, v, prm, ctas, stream);
-  if (a.head_dim == 128) return launch_fwd<128, false>(a, q, k, v, prm, ctas, stream);
-  return launch_fwd<64, false>(a, q, k, v, prm, ctas, stream);
+  prm.S = 0;
+  prm.n_qc = 0;
+  prm.cap = 0;
+  prm.max_ent = 0;
+  prm.q_starts = prm.q_counts = prm.cta_base = prm.ent_counts = nullptr;
+  if (fp8) return launch_fwd<128, true, false>(a, a.g.Np, q, k, v, prm, ctas, stream);
+  if (a.head_dim == 128) return launch_fwd<128, false, false>(a, a.g.Np, q, k, v, prm, ctas, stream);
+  return launch_fwd<64, false, false>(a, a.g.Np, q, k, v, prm, ctas, stream);
+}
+
+// ---------------------------------------------------------------------------------------
+// Cluster order ("Sparse VideoGen2", Abstract: semantic-aware permutation, densified layout
+// without padding).  Q, K and V are [B, Hh, S, D] with the tokens of every cluster in
+// consecutive slots; query cluster c of head bh owns slots [q_starts, q_starts + q_counts)
+// and attends to the key clusters listed in CSR row bh * n_qc + c.
+
+// Per (bh, query cluster): the runs of <= 64 keys covering its selected key clusters, in
+// list order.  One CTA per CSR row; validates the row like bsattn_schedule_kernel.
+__global__ void __launch_bounds__(256) cluster_schedule_kernel(
+    int n_rows, int n_kc, int max_ent, int S, const int32_t* __restrict__ row_ptr,
+    const int32_t* __restrict__ col_idx, const int32_t* __restrict__ k_starts,
+    const int32_t* __restrict__ k_counts, int32_t* __restrict__ ent_counts,
+    uint32_t* __restrict__ entries, uint32_t* status) {
+  __shared__ int warp_tot[8];
+  const int r = blockIdx.x;
+  const int bh = r / n_rows;  // n_rows = query clusters per head
+  const int tid = threadIdx.x;
+  const int beg = row_ptr[r], end = row_ptr[r + 1];
+  if (beg < 0 || end < beg || end - beg > n_kc) {
+    if (tid == 0) {
+      record_status(status, FLAG_DEVICE_INPUT, DETAIL_CSR_ROWPTR, static_cast<uint32_t>(r), 0u);
+      ent_counts[r] = 0;
+    }
+    return;
+  }
+  uint32_t* out = entries + static_cast<long long>(r) * max_ent;
+  int base = 0;
+  for (int e0 = beg; e0 < end; e0 += 256) {
+    const int e = e0 + tid;
+    int kc = -1, nrun = 0, start = 0, cnt = 0;
+    if (e < end) {
+      kc = col_idx[e];
+      if (kc < 0 || kc >= n_kc) {
+        record_status(status, FLAG_DEVICE_INPUT, DETAIL_CSR_RANGE, static_cast<uint32_t>(r),
+                      static_cast<uint32_t>(e));
+        kc = -1;
+      } else {
+        if (e > beg && col_idx[e - 1] >= kc)
+          record_status(status, FLAG_DEVICE_INPUT, DETAIL_CSR_ORDER, static_cast<uint32_t>(r),
+                        static_cast<uint32_t>(e));
+        start = k_starts[static_cast<long long>(bh) * n_kc + kc];
+        cnt = k_counts[static_cast<long long>(bh) * n_kc + kc];
+        if (start < 0 || cnt < 0 || start > S - cnt) {  // runs must lie inside the head
+          record_status(status, FLAG_DEVICE_INPUT, DETAIL_CLUSTER_RANGE, static_cast<uint32_t>(r),
+                        static_cast<uint32_t>(e));
+          cnt = 0;
+        }
+        nrun = cnt > 0 ? (cnt + 63) >> 6 : 0;
+      }
+    }
+    // exclusive scan of the run counts over the 256 entries of this chunk
+    int incl = nrun;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane_id() >= static_cast<uint32_t>(o)) incl += y;
+    }
+    if (lane_id() == 31) warp_tot[tid >> 5] = incl;
+    __syncthreads();
+    int before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      if (w < (tid >> 5)) before += warp_tot[w];
+      tot += warp_tot[w];
+    }
+    const int pos = base + before + incl - nrun;
+    for (int u = 0; u < nrun; ++u) {
+      const int len = min(64, cnt - 64 * u);
+      if (pos + u < max_ent)
+        out[pos + u] = (static_cast<uint32_t>(start + 64 * u) << 7) | static_cast<uint32_t>(len);
+    }
+    base += tot;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    if (base > max_ent) {
+      record_status(status, FLAG_CAPACITY, DETAIL_COL_CAPACITY, static_cast<uint32_t>(r), 0u);
+      base = max_ent;
+    }
+    ent_counts[r] = base;
+  }
+}
+
+// cta_base[bh][c] = first CTA of query cluster c (256 rows per CTA); [bh][n_qc] = total.
+__global__ void __launch_bounds__(1024) cluster_cta_base_kernel(int n_qc,
+                                                                const int32_t* __restrict__ q_counts,
+                                                                int32_t* __restrict__ cta_base) {
+  __shared__ int warp_tot[32];
+  const int bh = blockIdx.x;
+  const int tid = threadIdx.x;
+  int base = 0;
+  for (int c0 = 0; c0 < n_qc; c0 += 1024) {
+    const int c = c0 + tid;
+    const int n = c < n_qc ? max(q_counts[static_cast<long long>(bh) * n_qc + c], 0) : 0;
+    const int tiles = (n + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+    int incl = tiles;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane_id() >= static_cast<uint32_t>(o)) incl += y;
+    }
+    if (lane_id() == 31) warp_tot[tid >> 5] = incl;
+    __syncthreads();
+    int before = 0, tot = 0;
+    for (int w = 0; w < 32; ++w) {
+      if (w < (tid >> 5)) before += warp_tot[w];
+      tot += warp_tot[w];
+    }
+    if (c < n_qc) cta_base[static_cast<long long>(bh) * (n_qc + 1) + c] = base + before + incl - tiles;
+    base += tot;
+    __syncthreads();
+  }
+  if (tid == 0) cta_base[static_cast<long long>(bh) * (n_qc + 1) + n_qc] = base;
+}
+
+int cluster_max_entries(int S, int n_kc) { return (S + 63) / 64 + n_kc; }
+int cluster_ctas_per_head(int S, int n_qc) { return n_qc + (S + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta; }
+
+// Scratch after the status header: ent_counts int32 [BH * n_qc], cta_base int32
+// [BH * (n_qc + 1)], entries uint32 [BH * n_qc][max_ent].
+size_t cluster_fwd_scratch_bytes(int bhn, int S, int n_qc, int n_kc) {
+  const size_t a = (static_cast<size_t>(bhn) * n_qc * 4 + 255) & ~static_cast<size_t>(255);
+  const size_t b = (static_cast<size_t>(bhn) * (n_qc + 1) * 4 + 255) & ~static_cast<size_t>(255);
+  return a + b + static_cast<size_t>(bhn) * n_qc * cluster_max_entries(S, n_kc) * 4;
+}
+
+cudaError_t launch_cluster_fwd(int batch, int heads, int head_dim, int S, int n_qc, int n_kc,
+                               const void* q, const void* k, const void* v,
+                               const int32_t* q_starts, const int32_t* q_counts,
+                               const int32_t* k_starts, const int32_t* k_counts,
+                               const int32_t* row_ptr, const int32_t* col_idx,
+                               float softmax_scale, void* out, float* lse, void* ws,
+                               cudaStream_t stream) {
+  const int bhn = batch * heads;
+  if (bhn == 0 || S == 0) return cudaSuccess;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base);
+  const size_t a_bytes = (static_cast<size_t>(bhn) * n_qc * 4 + 255) & ~static_cast<size_t>(255);
+  const size_t b_bytes = (static_cast<size_t>(bhn) * (n_qc + 1) * 4 + 255) & ~static_cast<size_t>(255);
+  int32_t* ent_counts = reinterpret_cast<int32_t*>(base + kStatusBytes);
+  int32_t* cta_base = reinterpret_cast<int32_t*>(base + kStatusBytes + a_bytes);
+  uint32_t* entries = reinterpret_cast<uint32_t*>(base + kStatusBytes + a_bytes + b_bytes);
+  const int max_ent = cluster_max_entries(S, n_kc);
+  cluster_schedule_kernel<<<static_cast<unsigned>(bhn * n_qc), 256, 0, stream>>>(
+      n_qc, n_kc, max_ent, S, row_ptr, col_idx, k_starts, k_counts, ent_counts, entries, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  cluster_cta_base_kernel<<<static_cast<unsigned>(bhn), 1024, 0, stream>>>(n_qc, q_counts, cta_base);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  AttnDims a{};
+  a.batch = batch;
+  a.heads = heads;
+  a.head_dim = head_dim;
+  a.q_block = 64;
+  FwdParams prm{};
+  prm.a = a;
+  prm.entries = entries;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.status = status;
+  prm.scale_log2 = softmax_scale * 1.4426950408889634f;
+  prm.S = S;
+  prm.n_qc = n_qc;
+  prm.cap = cluster_ctas_per_head(S, n_qc);
+  prm.max_ent = max_ent;
+  prm.q_starts = q_starts;
+  prm.q_counts = q_counts;
+  prm.cta_base = cta_base;
+  prm.ent_counts = ent_counts;
+  const long long ctas = static_cast<long long>(bhn) * prm.cap;
+  if (head_dim == 128) return launch_fwd<128, false, true>(a, S, q, k, v, prm, ctas, stream);
+  return launch_fwd<64, false, true>(a, S, q, k, v, prm, ctas, stream);
 }
 
 }  // namespace bsa

@@ -34,6 +34,7 @@ enum : uint32_t {
   DETAIL_CSR_RANGE = 0x201,
   DETAIL_CSR_ORDER = 0x202,
   DETAIL_CSR_ROWPTR = 0x203,
+  DETAIL_CLUSTER_RANGE = 0x204,
   DETAIL_COL_CAPACITY = 0x300,
 };
 

@@ -148,6 +148,38 @@ size_t pooled_scratch_bytes(const AttnDims& a);
 cudaError_t launch_pooled_mass(const AttnDims& a, const void* q, const void* k, float softmax_scale,
                                float* mass, void* ws, cudaStream_t stream);
 
+// Semantic-aware clustering (one clustering of S tokens into C clusters per (batch, head)).
+struct ClusterDims {
+  int batch, heads, head_dim;
+  int S;  // tokens per (batch, head)
+  int C;  // clusters
+};
+size_t cluster_scratch_bytes(const ClusterDims& cd);
+cudaError_t launch_kmeans(const ClusterDims& cd, const void* x, int rounds, float* centroids,
+                          int32_t* labels, int32_t* counts, void* ws, cudaStream_t stream);
+cudaError_t launch_cluster_layout(const ClusterDims& cd, const int32_t* labels, int32_t* counts,
+                                  int32_t* starts, int32_t* token_of_slot, int32_t* slot_of_token,
+                                  void* ws, cudaStream_t stream);
+cudaError_t launch_cluster_permute(const ClusterDims& cd, int inverse, const int32_t* token_of_slot,
+                                   const void* src, void* dst, cudaStream_t stream);
+cudaError_t launch_cluster_mass(int batch, int heads, int head_dim, int n_qc, int n_kc,
+                                const float* qc, const int32_t* q_counts, const float* kc,
+                                const int32_t* k_counts, float softmax_scale, float* mass,
+                                cudaStream_t stream);
+
+// Attention in cluster order.  Scratch after the status header: per query cluster, its
+// runs of <= 64 keys, and the CTA offsets of the clusters.
+int cluster_max_entries(int S, int n_kc);
+int cluster_ctas_per_head(int S, int n_qc);
+size_t cluster_fwd_scratch_bytes(int bhn, int S, int n_qc, int n_kc);
+cudaError_t launch_cluster_fwd(int batch, int heads, int head_dim, int S, int n_qc, int n_kc,
+                               const void* q, const void* k, const void* v,
+                               const int32_t* q_starts, const int32_t* q_counts,
+                               const int32_t* k_starts, const int32_t* k_counts,
+                               const int32_t* row_ptr, const int32_t* col_idx,
+                               float softmax_scale, void* out, float* lse, void* ws,
+                               cudaStream_t stream);
+
 // Encode a rank-3 bf16/e4m3 tensor map over [bh][Np][D] with a (box_d x box_rows x 1) box
 // and 128-byte swizzle.
 cudaError_t encode_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,

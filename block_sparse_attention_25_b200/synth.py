@@ -227,3 +227,34 @@ def draw_keep_csr(n_rows: int, n_kb: int, keep_prob: float, seed: int, empty_row
     row_ptr[1:] = torch.cumsum(counts, 0)
     col_idx = keep.nonzero()[:, 1]
     return row_ptr.to(torch.int32), col_idx.to(torch.int32)
+
+
+def draw_cluster_labels(batch: int, heads: int, n_tokens: int, n_clusters: int, seed: int,
+                        empty=(), device="cpu") -> torch.Tensor:
+    """Seeded cluster labels int32 [B, Hh, S] with uneven cluster sizes (sizes drawn from a
+    power-law mixture, so some clusters span several 256-row tiles and others hold a few
+    tokens); the clusters in `empty` receive no token."""
+    g = _gen(seed, "cpu")
+    weights = torch.rand((batch, heads, n_clusters), generator=g, dtype=torch.float64) ** 3 + 1e-3
+    for c in empty:
+        weights[..., c] = 0.0
+    probs = weights / weights.sum(dim=-1, keepdim=True)
+    labels = torch.multinomial(probs.view(-1, n_clusters), n_tokens, replacement=True, generator=g)
+    return labels.view(batch, heads, n_tokens).to(torch.int32).to(device)
+
+
+def draw_blobs(batch: int, heads: int, n_tokens: int, n_clusters: int, head_dim: int, seed: int,
+               spread: float = 0.02):
+    """Tokens in well-separated Gaussian blobs, raster bf16 [B, S, Hh, D], with the blob of
+    every token ([B, Hh, S] int64) and initial centroids (one member token of each blob,
+    fp32 [B, Hh, C, D]).  Every blob holds at least one token."""
+    g = _gen(seed, "cpu")
+    centers = 4.0 * torch.randn((batch, heads, n_clusters, head_dim), generator=g)
+    ids = torch.randint(0, n_clusters, (batch, heads, n_tokens), generator=g)
+    ids[..., :n_clusters] = torch.arange(n_clusters)  # every blob non-empty
+    pts = torch.gather(centers, 2, ids[..., None].expand(-1, -1, -1, head_dim))
+    pts = pts + spread * torch.randn(pts.shape, generator=g)
+    x = pts.permute(0, 2, 1, 3).contiguous().to(torch.bfloat16)   # [B, S, Hh, D]
+    xf = x.float().permute(0, 2, 1, 3)                             # the stored values
+    init = xf[:, :, :n_clusters, :].contiguous()                   # token c is in blob c
+    return x, ids, init

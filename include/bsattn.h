@@ -241,6 +241,94 @@ BSA_API bsa_status bsa_fwd(const bsa_shape* shape, bsa_dtype dtype,
                    const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale,
                    void* out, float* lse, void* ws, size_t ws_bytes, bsa_stream_t stream);
 
+/* ------------------------------------------------------------------------------------
+ * Semantic-aware permutation ("Sparse VideoGen2: Accelerate Video Generation with Sparse
+ * Attention via Semantic-Aware Permutation", Abstract: tokens are clustered by k-means on
+ * their vectors and reordered so that every cluster is contiguous, without padding; the
+ * cluster representatives identify the critical clusters under top-p budget control, and
+ * the attention runs on the densified layout).  Per (batch, head), queries and keys are
+ * clustered separately: n_q_clusters query clusters, n_k_clusters key clusters.
+ *
+ * Layouts: raster tokens [B, S, Hh, D] bf16; cluster order [B, Hh, S, D] bf16, where the
+ * tokens of cluster c of head (b, h) occupy slots [starts[b,h,c], starts + counts) in
+ * raster order; per-head int32 arrays [B, Hh, S] or [B, Hh, C]; centroids fp32
+ * [B, Hh, C, D].  All pointers are device pointers owned by the caller; tensors of bf16
+ * rows must be 16-byte aligned, int32 and fp32 arrays 4-byte aligned. */
+typedef struct {
+  int32_t batch, heads;
+  int32_t head_dim;                    /* 64 or 128 */
+  int32_t n_tokens;                    /* S, 1 .. 2^24 */
+  int32_t n_q_clusters, n_k_clusters;  /* 1 .. 1024 each */
+} bsa_cluster_shape;
+
+/* Bytes of workspace for bsa_kmeans / bsa_cluster_layout with n_clusters clusters. */
+BSA_API size_t bsa_kmeans_workspace_bytes(const bsa_cluster_shape* shape, int32_t n_clusters);
+/* Bytes of workspace for bsa_cluster_fwd. */
+BSA_API size_t bsa_cluster_fwd_workspace_bytes(const bsa_cluster_shape* shape);
+/* Bytes of workspace for bsa_topp_select_rows. */
+BSA_API size_t bsa_topp_rows_workspace_bytes(int64_t rows, int32_t cols);
+
+/* Lloyd's k-means over the S tokens of every (batch, head), `rounds` rounds of: assign
+ * every token to the nearest centroid (argmin_c |c|^2 - 2 x.c in fp32, ties to the lowest
+ * c), then replace every centroid by the mean of its tokens, summed in cluster order in
+ * fp32 (deterministic); a cluster with no token keeps its centroid.  x: raster bf16.
+ * centroids: in = initial, out = final (the means of the last assignment).  labels:
+ * int32 [B, Hh, S], the last assignment; counts: int32 [B, Hh, n_clusters]. */
+BSA_API bsa_status bsa_kmeans(const bsa_cluster_shape* shape, int32_t n_clusters, const void* x,
+                              int32_t rounds, float* centroids, int32_t* labels, int32_t* counts,
+                              void* ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* Cluster order of every (batch, head) from labels in [0, n_clusters): counts, starts
+ * (exclusive scan of counts), token_of_slot [B,Hh,S] (raster token held by each slot; -1
+ * for slots left over by out-of-range labels, which raise DEVICE_INPUT) and slot_of_token
+ * [B,Hh,S] (-1 for such tokens).  A stable counting sort: tokens of a cluster keep their
+ * raster order. */
+BSA_API bsa_status bsa_cluster_layout(const bsa_cluster_shape* shape, int32_t n_clusters,
+                                      const int32_t* labels, int32_t* counts, int32_t* starts,
+                                      int32_t* token_of_slot, int32_t* slot_of_token, void* ws,
+                                      size_t ws_bytes, bsa_stream_t stream);
+
+/* Row gather into cluster order (inverse = 0): dst[b,h,p,:] = src[b, token_of_slot[b,h,p],
+ * h, :] (zeros for a -1 slot); or scatter back (inverse = 1): dst[b, token_of_slot[b,h,p],
+ * h, :] = src[b,h,p,:] (raster rows no slot points at are left untouched). */
+BSA_API bsa_status bsa_cluster_permute(const bsa_cluster_shape* shape, int inverse,
+                                       const int32_t* token_of_slot, const void* src, void* dst,
+                                       bsa_stream_t stream);
+
+/* Cluster-level estimate of the attention mass, to feed bsa_topp_select_rows:
+ * mass[b,h,i,j] = n_j exp(s qc_i.kc_j) / sum_j' n_j' exp(s qc_i.kc_j') with s =
+ * softmax_scale, qc/kc the query/key centroids (fp32 [B,Hh,C,D]) and n_j = k_counts; 0
+ * for key clusters without tokens; zero rows for query clusters without tokens.
+ * mass: fp32 [B, Hh, n_q_clusters, n_k_clusters]. */
+BSA_API bsa_status bsa_cluster_mass(const bsa_cluster_shape* shape, const float* q_centroids,
+                                    const int32_t* q_counts, const float* k_centroids,
+                                    const int32_t* k_counts, float softmax_scale, float* mass,
+                                    bsa_stream_t stream);
+
+/* bsa_topp_select on any rows x cols fp32 matrix (same rule, same precondition on the
+ * values): CSR of the smallest column set of each row reaching threshold of its mass.
+ * cols <= 4096, rows * cols < 2^31. */
+BSA_API bsa_status bsa_topp_select_rows(const float* mass, int64_t rows, int32_t cols,
+                                        float threshold, int32_t* row_ptr, int32_t* col_idx,
+                                        int64_t col_capacity, void* ws, size_t ws_bytes,
+                                        bsa_stream_t stream);
+
+/* Attention in cluster order: every query of cluster i of head (b, h) attends to all keys
+ * of the key clusters col_idx[row_ptr[r] .. row_ptr[r+1]), r = (b*Hh + h)*n_q_clusters + i
+ * (strictly ascending, < n_k_clusters; checked on the device), softmax(softmax_scale q.k)
+ * renormalised over those keys.  q, k, v: cluster order bf16 [B,Hh,S,D] (q by the query
+ * clustering, k and v by the key clustering); q_starts/q_counts and k_starts/k_counts:
+ * int32 [B,Hh,C] cluster extents (checked to lie inside [0, S) on the device).  out: bf16
+ * cluster order [B,Hh,S,D]; lse (nullable) fp32 [B,Hh,S]; rows of a cluster with no kept
+ * key are zero (lse -inf).  The tensor-core kernel of bsa_fwd, walking each selected key
+ * cluster in runs of <= 64 keys that start at the cluster's first slot. */
+BSA_API bsa_status bsa_cluster_fwd(const bsa_cluster_shape* shape, const void* q, const void* k,
+                                   const void* v, const int32_t* q_starts, const int32_t* q_counts,
+                                   const int32_t* k_starts, const int32_t* k_counts,
+                                   const int32_t* row_ptr, const int32_t* col_idx,
+                                   float softmax_scale, void* out, float* lse, void* ws,
+                                   size_t ws_bytes, bsa_stream_t stream);
+
 /* Library build identification (static string). */
 BSA_API const char* bsa_version(void);
 

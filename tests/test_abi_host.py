@@ -134,6 +134,61 @@ def test_rejections_before_launch(B):
     assert L.bsa_pattern_csr(_c(B), ctypes.byref(P(1)), FAKE, FAKE, 10, FAKE, 16, n) == 3
 
 
+def test_cluster_rejections_before_launch(B):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("fake-pointer validation checks run on hosts without a GPU only")
+    L = B.lib()
+    n = None
+    big = 1 << 40
+
+    def cs(**kw):
+        d = dict(batch=1, heads=40, head_dim=128, n_tokens=75600, n_q_clusters=256, n_k_clusters=256)
+        d.update(kw)
+        return ctypes.byref(B.ClusterShape(**d).c())
+
+    # workspace sizes: positive for good shapes, 0 for bad ones
+    assert L.bsa_kmeans_workspace_bytes(cs(), 256) > 0
+    assert L.bsa_kmeans_workspace_bytes(cs(), 2000) == 0
+    assert L.bsa_kmeans_workspace_bytes(cs(head_dim=96), 16) == 0
+    assert L.bsa_cluster_fwd_workspace_bytes(cs()) > 0
+    assert L.bsa_cluster_fwd_workspace_bytes(cs(n_tokens=0)) == 0
+    assert L.bsa_topp_rows_workspace_bytes(100, 5000) == 0
+    # k-means
+    assert L.bsa_kmeans(cs(), 256, FAKE, 5, FAKE, FAKE, FAKE, FAKE, 16, n) == 3       # short ws
+    assert L.bsa_kmeans(cs(), 256, FAKE, 0, FAKE, FAKE, FAKE, FAKE, big, n) == 1      # no round
+    assert L.bsa_kmeans(cs(), 1025, FAKE, 5, FAKE, FAKE, FAKE, FAKE, big, n) == 2
+    assert L.bsa_kmeans(cs(head_dim=96), 8, FAKE, 5, FAKE, FAKE, FAKE, FAKE, big, n) == 2
+    assert L.bsa_kmeans(cs(), 256, MISALIGNED, 5, FAKE, FAKE, FAKE, FAKE, big, n) == 1
+    assert L.bsa_kmeans(cs(n_tokens=1 << 25), 8, FAKE, 5, FAKE, FAKE, FAKE, FAKE, big, n) == 2
+    # layout, permute, mass
+    assert L.bsa_cluster_layout(cs(), 256, FAKE, FAKE, FAKE, n, FAKE, FAKE, big, n) == 1
+    assert L.bsa_cluster_layout(cs(), 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, n) == 3
+    assert L.bsa_cluster_permute(cs(), 2, FAKE, FAKE, ctypes.c_void_p(0x20000), n) == 1
+    assert L.bsa_cluster_permute(cs(), 0, FAKE, FAKE, FAKE, n) == 1                   # in place
+    assert L.bsa_cluster_permute(cs(), 0, FAKE, MISALIGNED, ctypes.c_void_p(0x20000), n) == 1
+    assert L.bsa_cluster_mass(cs(), FAKE, FAKE, FAKE, FAKE, 0.0, FAKE, n) == 1         # bad scale
+    assert L.bsa_cluster_mass(cs(n_k_clusters=0), FAKE, FAKE, FAKE, FAKE, 0.1, FAKE, n) == 1
+    # row selection
+    assert L.bsa_topp_select_rows(FAKE, 10, 5000, 0.9, FAKE, FAKE, 10, FAKE, big, n) == 2
+    assert L.bsa_topp_select_rows(FAKE, 10, 8, 1.5, FAKE, FAKE, 10, FAKE, big, n) == 1
+    assert L.bsa_topp_select_rows(FAKE, 10, 8, 0.9, FAKE, n, 10, FAKE, big, n) == 1
+    assert L.bsa_topp_select_rows(FAKE, 10, 8, 0.9, FAKE, FAKE, 10, FAKE, 16, n) == 3
+    # attention in cluster order
+    args = [FAKE] * 9 + [0.088, FAKE, n, FAKE]      # q..col_idx, scale, out, lse, ws
+    assert L.bsa_cluster_fwd(cs(), *args, 16, n) == 3
+    bad = list(args)
+    bad[2] = MISALIGNED
+    assert L.bsa_cluster_fwd(cs(), *bad, big, n) == 1
+    bad = list(args)
+    bad[8] = n                                                                 # col_idx missing
+    assert L.bsa_cluster_fwd(cs(), *bad, big, n) == 1
+    bad = list(args)
+    bad[9] = -1.0
+    assert L.bsa_cluster_fwd(cs(), *bad, big, n) == 1
+    assert L.bsa_cluster_fwd(cs(head_dim=32), *args, big, n) == 2
+
+
 def test_status_strings(B):
     L = B.lib()
     for code in range(7):

@@ -1,0 +1,258 @@
+"""GPU parity of the semantic-aware permutation path (k-means, cluster layout, gather and
+scatter, cluster-level estimate, row top-p, attention in cluster order) against the oracle.
+
+Integer work (layouts, permutations, selections) is compared bit for bit.  k-means labels
+are integers decided by float32 distances; on separated blobs they are unique and compared
+exactly, on general data the GPU's choice is checked to be a nearest centroid within the
+float32 rounding of the distance.  No oracle input comes from the GPU: both sides start
+from the same seeded draws.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import helpers as Hp
+from block_sparse_attention_25_b200 import synth
+from oracle import bsa_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def B(cuda_device):
+    from block_sparse_attention_25_b200 import build
+    build.build()
+    import block_sparse_attention_25_b200 as b
+    return b
+
+
+def _np(t):
+    return t.detach().cpu().double().numpy()
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("rounds", [1, 4])
+def test_kmeans_separated_blobs_exact(B, D, rounds):
+    Bt, Hh, S, C = 2, 3, 700, 37
+    cs = B.ClusterShape(Bt, Hh, D, S, C, C)
+    x, ids, init = synth.draw_blobs(Bt, Hh, S, C, D, seed=11 + D)
+    cent = init.clone().cuda()
+    cent, labels, counts = B.kmeans(x.cuda(), cs, C, cent, rounds)
+    xf = x.float().permute(0, 2, 1, 3).double().numpy()   # [B, Hh, S, D]
+    for b in range(Bt):
+        for h in range(Hh):
+            lab, c, n = O.kmeans_lloyd(xf[b, h], init[b, h].double().numpy(), rounds)
+            assert np.array_equal(labels[b, h].cpu().numpy(), lab)
+            assert np.array_equal(counts[b, h].cpu().numpy(), n)
+            np.testing.assert_allclose(_np(cent[b, h]), c, rtol=0, atol=2e-5)
+            assert np.array_equal(lab, ids[b, h].numpy())   # the generating partition
+
+
+def test_kmeans_general_data_is_nearest_within_rounding(B):
+    """One round on video-like tokens: every GPU label is a nearest initial centroid up to
+    float32 rounding of the distance, and the centroids are the means of the labels."""
+    wl = synth.WORKLOADS["wan13b_480p"].scaled(heads=2)
+    x, _, _ = synth.draw_qkv(wl, seed=5)
+    S, Hh, D, C = x.shape[1], 2, 128, 64
+    cs = B.ClusterShape(1, Hh, D, S, C, C)
+    g = torch.Generator().manual_seed(3)
+    pick = torch.randint(0, S, (Hh, C), generator=g)
+    xf = x.float().permute(0, 2, 1, 3)[0]                  # [Hh, S, D]
+    init = torch.stack([xf[h, pick[h]] for h in range(Hh)])[None].contiguous()
+    cent, labels, counts = B.kmeans(x.cuda(), cs, C, init.clone().cuda(), 1)
+    for h in range(Hh):
+        X = xf[h].double().numpy()
+        C0 = init[0, h].double().numpy()
+        d = (C0 * C0).sum(1)[None, :] - 2.0 * X @ C0.T      # float64 distances
+        lab = labels[0, h].cpu().numpy().astype(np.int64)
+        chosen = d[np.arange(S), lab]
+        scale = np.abs(X).max() * np.abs(C0).max() * D
+        assert np.all(chosen <= d.min(axis=1) + 2e-5 * scale)
+        ref = O.kmeans_assign(X, C0)
+        assert (lab == ref).mean() > 0.999
+        n = np.bincount(lab, minlength=C)
+        assert np.array_equal(counts[0, h].cpu().numpy(), n)
+        means = np.stack([X[lab == j].mean(0) if n[j] else C0[j] for j in range(C)])
+        np.testing.assert_allclose(_np(cent[0, h]), means, rtol=0, atol=2e-5)
+
+
+@pytest.mark.parametrize("S,C", [(1, 1), (100, 7), (5000, 300), (3001, 1024)])
+def test_cluster_layout_bit_exact(B, S, C):
+    Bt, Hh = 2, 2
+    cs = B.ClusterShape(Bt, Hh, 64, S, C, C)
+    labels = synth.draw_cluster_labels(Bt, Hh, S, C, seed=S + C, empty=(0,) if C > 1 else ())
+    counts, starts, tos, sot = B.cluster_layout(labels.cuda(), cs, C)
+    for b in range(Bt):
+        for h in range(Hh):
+            st, t, s_ = O.cluster_layout(labels[b, h].numpy(), C)
+            assert np.array_equal(starts[b, h].cpu().numpy(), st)
+            assert np.array_equal(counts[b, h].cpu().numpy(), np.bincount(labels[b, h].numpy(), minlength=C))
+            assert np.array_equal(tos[b, h].cpu().numpy(), t)
+            assert np.array_equal(sot[b, h].cpu().numpy(), s_)
+
+
+def test_cluster_layout_flags_bad_labels(B):
+    cs = B.ClusterShape(1, 1, 64, 50, 4, 4)
+    labels = torch.zeros((1, 1, 50), dtype=torch.int32)
+    labels[0, 0, 7] = 9
+    ws = B.new_cluster_workspace(cs, 4)
+    counts, starts, tos, sot = B.cluster_layout(labels.cuda(), cs, 4, ws=ws)
+    assert B.device_status(ws) & 2
+    assert int(counts.sum()) == 49 and int(sot[0, 0, 7]) == -1
+    t = tos[0, 0].cpu().numpy()
+    assert t[-1] == -1 and sorted(t[:49].tolist()) == [i for i in range(50) if i != 7]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_cluster_permute_round_trip(B, D):
+    Bt, Hh, S, C = 2, 3, 777, 20
+    cs = B.ClusterShape(Bt, Hh, D, S, C, C)
+    x = torch.randn((Bt, S, Hh, D), generator=torch.Generator().manual_seed(D)).to(torch.bfloat16)
+    labels = synth.draw_cluster_labels(Bt, Hh, S, C, seed=4)
+    _, _, tos, _ = B.cluster_layout(labels.cuda(), cs, C)
+    y = B.cluster_permute(x.cuda(), cs, tos)
+    xr = x.permute(0, 2, 1, 3)                              # [B, Hh, S, D]
+    for b in range(Bt):
+        for h in range(Hh):
+            _, t, _ = O.cluster_layout(labels[b, h].numpy(), C)
+            assert torch.equal(y[b, h].cpu(), xr[b, h][torch.from_numpy(t)])
+    z = B.cluster_permute(y, cs, tos, inverse=True)
+    assert torch.equal(z.cpu(), x)
+
+
+def test_cluster_mass_parity(B):
+    Bt, Hh, D, Cq, Ck = 1, 3, 128, 40, 70
+    cs = B.ClusterShape(Bt, Hh, D, 1000, Cq, Ck)
+    g = torch.Generator().manual_seed(8)
+    qc = torch.randn((Bt, Hh, Cq, D), generator=g)
+    kc = torch.randn((Bt, Hh, Ck, D), generator=g)
+    qn = torch.randint(0, 50, (Bt, Hh, Cq), generator=g, dtype=torch.int32)
+    kn = torch.randint(0, 50, (Bt, Hh, Ck), generator=g, dtype=torch.int32)
+    qn[0, 0, 3] = 0
+    kn[0, 1, :5] = 0
+    scale = 1.5 / math.sqrt(D)
+    m = B.cluster_mass(cs, qc.cuda(), qn.cuda(), kc.cuda(), kn.cuda(), scale)
+    for h in range(Hh):
+        ref = O.cluster_mass(qc[0, h].double().numpy(), qn[0, h].numpy(), kc[0, h].double().numpy(),
+                             kn[0, h].numpy(), scale)
+        got = _np(m[0, h])
+        assert np.abs(got - ref).max() <= 1e-5
+        assert np.all(got[ref == 0] == 0)
+
+
+@pytest.mark.parametrize("cols", [1, 37, 256, 1440])
+def test_topp_select_rows_bit_exact(B, cols):
+    rows = 300
+    m = synth.draw_mass_rows(rows, cols, seed=cols, kind="dirichlet", zero_frac=0.1)
+    rp, ci = B.topp_select_rows(m.cuda(), 0.95)
+    ref_rp, ref_ci = O.topp_select(m.double().numpy(), np.float32(0.95))
+    assert np.array_equal(rp.cpu().numpy(), ref_rp)
+    n = int(ref_rp[-1])
+    assert np.array_equal(ci[:n].cpu().numpy(), ref_ci)
+
+
+def _cluster_case(B, Bt, Hh, S, D, Cq, Ck, seed, keep_prob, sharp):
+    cs = B.ClusterShape(Bt, Hh, D, S, Cq, Ck)
+    g = torch.Generator().manual_seed(seed)
+    q, k, v = (torch.randn((Bt, Hh, S, D), generator=g) for _ in range(3))
+    # |v| ~ 0.25 keeps outputs at the scale the bf16 bar (max abs 2e-2) is set for
+    q, k, v = q * sharp, k * sharp, v * 0.25
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))     # already in cluster order
+    lq = synth.draw_cluster_labels(Bt, Hh, S, Cq, seed=seed + 1, empty=(1,))
+    lk = synth.draw_cluster_labels(Bt, Hh, S, Ck, seed=seed + 2, empty=(2,))
+    qn = torch.stack([torch.bincount(lq[b, h].long(), minlength=Cq) for b in range(Bt) for h in range(Hh)])
+    kn = torch.stack([torch.bincount(lk[b, h].long(), minlength=Ck) for b in range(Bt) for h in range(Hh)])
+    qn, kn = qn.view(Bt, Hh, Cq).to(torch.int32), kn.view(Bt, Hh, Ck).to(torch.int32)
+    qs = (torch.cumsum(qn, -1) - qn).to(torch.int32)
+    ks = (torch.cumsum(kn, -1) - kn).to(torch.int32)
+    rp, ci = synth.draw_keep_csr(Bt * Hh * Cq, Ck, keep_prob, seed=seed + 3, empty_rows=(0,))
+    return cs, q, k, v, qs, qn, ks, kn, rp, ci
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("keep_prob,sharp", [(1.0, 1.0), (0.3, 3.0), (0.05, 3.0)])
+def test_cluster_fwd_parity(B, D, keep_prob, sharp):
+    Bt, Hh, S, Cq, Ck = 1, 2, 1500, 9, 23
+    cs, q, k, v, qs, qn, ks, kn, rp, ci = _cluster_case(B, Bt, Hh, S, D, Cq, Ck, 40 + D, keep_prob, sharp)
+    dev = lambda t: t.cuda()
+    ws = B.new_cluster_fwd_workspace(cs)
+    out, lse = B.cluster_fwd(dev(q), dev(k), dev(v), cs, dev(qs), dev(qn), dev(ks), dev(kn),
+                             dev(rp), dev(ci), want_lse=True, ws=ws)
+    assert B.device_status(ws) == 0
+    scale = 1.0 / math.sqrt(D)
+    for b in range(Bt):
+        for h in range(Hh):
+            r0 = (b * Hh + h) * Cq
+            rows = rp[r0:r0 + Cq + 1].numpy() - rp[r0].numpy()
+            cols = ci[rp[r0]:rp[r0 + Cq]].numpy()
+            ref = O.cluster_attention(q[b, h].double().numpy(), k[b, h].double().numpy(),
+                                      v[b, h].double().numpy(), qs[b, h].numpy(), qn[b, h].numpy(),
+                                      ks[b, h].numpy(), kn[b, h].numpy(), rows, cols, scale)
+            e = Hp.attn_errors(_np(out[b, h]), ref)
+            assert e["max_abs"] <= Hp.ATTN_MAX_ABS and e["mean_abs"] <= Hp.ATTN_MEAN_ABS, e
+            # rows of cluster 0 (no kept key cluster) are zero with lse -inf
+            z = slice(int(qs[b, h, 0]), int(qs[b, h, 0] + qn[b, h, 0]))
+            if b == 0 and h == 0:
+                assert torch.all(out[b, h, z] == 0) and torch.all(torch.isinf(lse[b, h, z]))
+
+
+def test_cluster_fwd_flags_bad_extents(B):
+    Bt, Hh, S, D, Cq, Ck = 1, 1, 300, 64, 4, 4
+    cs, q, k, v, qs, qn, ks, kn, rp, ci = _cluster_case(B, Bt, Hh, S, D, Cq, Ck, 77, 1.0, 1.0)
+    qs = qs.clone()
+    qs[0, 0, 2] = S - 1                     # runs past the end of the head
+    ks = ks.clone()
+    ks[0, 0, 1] = -5
+    ws = B.new_cluster_fwd_workspace(cs)
+    out = torch.full((Bt, Hh, S, D), 7.0, dtype=torch.bfloat16, device="cuda")
+    B.cluster_fwd(q.cuda(), k.cuda(), v.cuda(), cs, qs.cuda(), qn.cuda(), ks.cuda(), kn.cuda(),
+                  rp.cuda(), ci.cuda(), out=out, ws=ws)
+    assert B.device_status(ws) & 2
+    assert torch.isfinite(out.float()).all()
+
+
+def test_semantic_pipeline_on_blobs_matches_oracle(B):
+    """k-means (queries and keys) -> layout -> gather -> cluster estimate -> top-p ->
+    attention -> scatter, on the GPU and in the oracle, from the same seeded blobs."""
+    Bt, Hh, S, D, C = 1, 2, 900, 64, 12
+    cs = B.ClusterShape(Bt, Hh, D, S, C, C)
+    xq, _, iq = synth.draw_blobs(Bt, Hh, S, C, D, seed=21, spread=0.3)
+    xk, _, ik = synth.draw_blobs(Bt, Hh, S, C, D, seed=22, spread=0.3)
+    xv = torch.randn((Bt, S, Hh, D), generator=torch.Generator().manual_seed(23)).to(torch.bfloat16)
+    scale, tau, rounds = 0.05, 0.9, 3
+    cq, lq, nq = B.kmeans(xq.cuda(), cs, C, iq.clone().cuda(), rounds)
+    ck, lk, nk = B.kmeans(xk.cuda(), cs, C, ik.clone().cuda(), rounds)
+    _, sq, tq, _ = B.cluster_layout(lq, cs, C)
+    _, sk, tk, _ = B.cluster_layout(lk, cs, C)
+    qp, kp, vp = B.cluster_permute(xq.cuda(), cs, tq), B.cluster_permute(xk.cuda(), cs, tk), \
+        B.cluster_permute(xv.cuda(), cs, tk)
+    m = B.cluster_mass(cs, cq, nq, ck, nk, scale)
+    rp, ci = B.topp_select_rows(m, tau)
+    o = B.cluster_fwd(qp, kp, vp, cs, sq, nq, sk, nk, rp, ci, softmax_scale=scale)
+    out = B.cluster_permute(o, cs, tq, inverse=True)        # back to raster
+    for h in range(Hh):
+        Xq = xq[0, :, h].double().numpy()
+        Xk = xk[0, :, h].double().numpy()
+        Xv = xv[0, :, h].double().numpy()
+        Lq, Cq_, Nq = O.kmeans_lloyd(Xq, iq[0, h].double().numpy(), rounds)
+        Lk, Ck_, Nk = O.kmeans_lloyd(Xk, ik[0, h].double().numpy(), rounds)
+        assert np.array_equal(lq[0, h].cpu().numpy(), Lq) and np.array_equal(lk[0, h].cpu().numpy(), Lk)
+        Sq, Tq, _ = O.cluster_layout(Lq, C)
+        Sk, Tk, _ = O.cluster_layout(Lk, C)
+        M = O.cluster_mass(Cq_, Nq, Ck_, Nk, scale)
+        np.testing.assert_allclose(_np(m[0, h]), M, rtol=0, atol=1e-5)
+        r, c_ = O.topp_select(M.astype(np.float32).astype(np.float64), np.float32(tau))
+        # the selections are integers from float masses that differ by rounding: compare
+        # them cluster by cluster and the outputs of the clusters where they agree
+        g_rp = rp.cpu().numpy()[h * C:(h + 1) * C + 1]
+        g_ci = ci.cpu().numpy()
+        same = [np.array_equal(g_ci[g_rp[i]:g_rp[i + 1]], c_[r[i]:r[i + 1]]) for i in range(C)]
+        assert np.mean(same) >= 0.9
+        ref_p = O.cluster_attention(Xq[Tq], Xk[Tk], Xv[Tk], Sq, Nq, Sk, Nk, r, c_, scale)
+        ref = np.empty_like(ref_p)
+        ref[Tq] = ref_p
+        rows = np.isin(Lq, np.flatnonzero(same))
+        e = Hp.attn_errors(out[0, :, h].cpu().double().numpy()[rows], ref[rows])
+        assert e["max_abs"] <= Hp.ATTN_MAX_ABS and e["mean_abs"] <= Hp.ATTN_MEAN_ABS, e
