@@ -53,6 +53,9 @@ def main(argv=None):
     ap.add_argument("--config", default="wan14b_720p")
     ap.add_argument("--iters", type=int, default=5)
     ap.add_argument("--tau", type=float, default=0.99)
+    ap.add_argument("--q-clusters", type=int, default=64, help="k-means clusters of the queries")
+    ap.add_argument("--k-clusters", type=int, default=256, help="k-means clusters of the keys")
+    ap.add_argument("--rounds", type=int, default=10, help="k-means rounds")
     args = ap.parse_args(argv)
     build.build()
     dev = torch.device("cuda")
@@ -146,6 +149,93 @@ def main(argv=None):
                                      args.iters), pfl, "TFLOP/s", "tensor", pk["bf16"],
          {"kept_fraction": round(pnnz / (R * nkb), 5)})
     for w in (ws_m, ws_t, ws_p, ws_pt, ws_f):
+        st = B.device_status(w)
+        if st != 0:
+            raise RuntimeError(f"device status {st}: {B.device_status_words(w)}")
+    del qt, kt, vt, out_t, mass, mass2, pmass, col_idx, pci, ws_m, ws_t, ws_p, ws_pt, ws_f
+    torch.cuda.empty_cache()
+    semantic(args, wl, q, k, v, line, pk)
+
+
+def semantic(args, wl, q, k, v, line, pk):
+    """The semantic-aware permutation path on the same tokens: k-means of queries and of
+    keys, cluster order, cluster-level estimate, top-p over key clusters, attention in
+    cluster order, scatter back."""
+    s = B.Shape.of(wl)
+    Bt, Hh, D, S = s.batch, s.heads, s.head_dim, s.S
+    Cq, Ck, rounds = args.q_clusters, args.k_clusters, args.rounds
+    cs = B.ClusterShape(Bt, Hh, D, S, Cq, Ck)
+    dev = q.device
+    g = torch.Generator(device="cpu").manual_seed(17)
+
+    def init_of(x, C):  # C seeded tokens of every head as initial centroids
+        pick = torch.randint(0, S, (Bt, Hh, C), generator=g).to(dev)
+        xh = x.float().permute(0, 2, 1, 3)                       # [B, Hh, S, D]
+        return torch.gather(xh, 2, pick[..., None].expand(-1, -1, -1, D)).contiguous()
+
+    iq, ik = init_of(q, Cq), init_of(k, Ck)
+    ws_q = B.new_cluster_workspace(cs, Cq, dev)
+    ws_k = B.new_cluster_workspace(cs, Ck, dev)
+    cq, ck = iq.clone(), ik.clone()
+    lq = torch.empty((Bt, Hh, S), dtype=torch.int32, device=dev)
+    nq = torch.empty((Bt, Hh, Cq), dtype=torch.int32, device=dev)
+    lk = torch.empty_like(lq)
+    nk = torch.empty((Bt, Hh, Ck), dtype=torch.int32, device=dev)
+    # fp32 CUDA-core peak: 148 SMs x 128 FMA lanes x 2 FLOP at the boost clock
+    alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+
+    def km(x, init, cent, C, labels, counts, ws):
+        cent.copy_(init)
+        B.kmeans(x, cs, C, cent, rounds, labels=labels, counts=counts, ws=ws)
+    for name, x, init, cent, C, lab, cnt, ws in (("kmeans_q", q, iq, cq, Cq, lq, nq, ws_q),
+                                                 ("kmeans_k", k, ik, ck, Ck, lk, nk, ws_k)):
+        ms = _time(lambda: km(x, init, cent, C, lab, cnt, ws), args.iters)
+        line(name, ms, 2.0 * Bt * Hh * S * C * D * rounds, "TFLOP/s", "alu", alu_peak,
+             {"rounds": rounds, "clusters": C, "ms_per_round": round(ms / rounds, 4),
+              "peak_note": "fp32 FMA lanes x boost clock (nominal)"})
+    lay = {}
+
+    def layout():
+        lay["q"] = B.cluster_layout(lq, cs, Cq, ws=ws_q)
+    ms = _time(layout, args.iters)
+    line("cluster_layout", ms, 3 * 4 * Bt * Hh * S, "GB/s", "hbm", pk["hbm"])
+    lay["k"] = B.cluster_layout(lk, cs, Ck, ws=ws_k)
+    _, sq, tq, _ = lay["q"]
+    _, sk, tk, _ = lay["k"]
+    qp = torch.empty((Bt, Hh, S, D), dtype=torch.bfloat16, device=dev)
+    kp, vp, op = torch.empty_like(qp), torch.empty_like(qp), torch.empty_like(qp)
+    ms = _time(lambda: B.cluster_permute(q, cs, tq, out=qp), args.iters)
+    line("cluster_permute", ms, 2 * Bt * Hh * S * D * 2 + 4 * Bt * Hh * S, "GB/s", "hbm", pk["hbm"])
+    B.cluster_permute(k, cs, tk, out=kp)
+    B.cluster_permute(v, cs, tk, out=vp)
+    mass = torch.empty((Bt, Hh, Cq, Ck), dtype=torch.float32, device=dev)
+    ms = _time(lambda: B.cluster_mass(cs, cq, nq, ck, nk, out=mass), args.iters)
+    line("cluster_mass", ms, 2.0 * Bt * Hh * Cq * Ck * D, "TFLOP/s", "alu", alu_peak)
+    rows = Bt * Hh * Cq
+    rp = torch.empty(rows + 1, dtype=torch.int32, device=dev)
+    ci = torch.empty(rows * Ck, dtype=torch.int32, device=dev)
+    ms = _time(lambda: B.topp_select_rows(mass, args.tau, row_ptr=rp, col_idx=ci), args.iters)
+    nnz = int(rp[-1])
+    line("topp_select_rows", ms, 4 * rows * Ck + 4 * (rows + 1 + nnz), "GB/s", "hbm", pk["hbm"],
+         {"kept_fraction": round(nnz / (rows * Ck), 5)})
+    # algorithmic FLOPs: every (query, key) pair of the selected cluster pairs, 4 D each
+    rpc, cic = rp.cpu().long(), ci[:nnz].cpu().long()
+    nqc, nkc = nq.cpu().long().view(-1), nk.cpu().long().view(Bt * Hh, Ck)
+    head = torch.arange(rows) // Cq
+    sel_keys = torch.zeros(rows, dtype=torch.long)
+    for r in range(rows):
+        sel_keys[r] = nkc[head[r], cic[rpc[r]:rpc[r + 1]]].sum()
+    pairs = float((nqc * sel_keys).sum())
+    ws_f = B.new_cluster_fwd_workspace(cs, dev)
+    ms = _time(lambda: B.cluster_fwd(qp, kp, vp, cs, sq, nq, sk, nk, rp, ci, out=op, ws=ws_f),
+               args.iters)
+    line("cluster_fwd", ms, 4.0 * D * pairs, "TFLOP/s", "tensor", pk["bf16"],
+         {"kept_pair_fraction": round(pairs / (Bt * Hh * float(S) * S), 5)})
+    out = torch.empty_like(q)
+    ms = _time(lambda: B.cluster_permute(op, cs, tq, inverse=True, out=out), args.iters)
+    line("cluster_permute_inverse", ms, 2 * Bt * Hh * S * D * 2 + 4 * Bt * Hh * S, "GB/s", "hbm",
+         pk["hbm"])
+    for w in (ws_q, ws_k, ws_f):
         st = B.device_status(w)
         if st != 0:
             raise RuntimeError(f"device status {st}: {B.device_status_words(w)}")
