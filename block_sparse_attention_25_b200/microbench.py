@@ -56,6 +56,8 @@ def main(argv=None):
     ap.add_argument("--q-clusters", type=int, default=64, help="k-means clusters of the queries")
     ap.add_argument("--k-clusters", type=int, default=256, help="k-means clusters of the keys")
     ap.add_argument("--rounds", type=int, default=10, help="k-means rounds")
+    ap.add_argument("--only", choices=["all", "tiles", "semantic"], default="all",
+                    help="the 3D-tile path, the semantic-aware permutation path, or both")
     args = ap.parse_args(argv)
     build.build()
     dev = torch.device("cuda")
@@ -76,6 +78,9 @@ def main(argv=None):
             d.update(extra)
         print(json.dumps(d), flush=True)
 
+    if args.only == "semantic":
+        semantic(args, wl, q, k, v, line, pk)
+        return
     qt, kt, vt = (B.tile_permute(x, s) for x in (q, k, v))
     out_r = torch.empty_like(q)
     line("tile_permute", _time(lambda: B.tile_permute(q, s, out=qt), args.iters),
@@ -154,7 +159,8 @@ def main(argv=None):
             raise RuntimeError(f"device status {st}: {B.device_status_words(w)}")
     del qt, kt, vt, out_t, mass, mass2, pmass, col_idx, pci, ws_m, ws_t, ws_p, ws_pt, ws_f
     torch.cuda.empty_cache()
-    semantic(args, wl, q, k, v, line, pk)
+    if args.only == "all":
+        semantic(args, wl, q, k, v, line, pk)
 
 
 def semantic(args, wl, q, k, v, line, pk):
