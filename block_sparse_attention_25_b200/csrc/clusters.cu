@@ -8,8 +8,8 @@
 //
 // Per (batch, head) one clustering of S tokens into C clusters:
 //   kmeans_assign_kernel   label = argmin_c (|c|^2 - 2 x.c) in float32, ties to the lowest c;
-//                          one thread per token, centroids staged 32 at a time in shared
-//                          memory and read as broadcasts.
+//                          four tokens per thread, centroids staged 16 at a time in shared
+//                          memory and read as broadcasts (each feeds 32 FMAs).
 //   layout_hist_kernel     per chunk of 1024 tokens, the tokens of each cluster.
 //   layout_scan_kernel     per head: cluster sizes, cluster starts (exclusive scan) and each
 //                          chunk's first slot inside every cluster.
@@ -27,7 +27,8 @@ namespace bsa {
 namespace {
 
 constexpr int kAsgThreads = 128;
-constexpr int kAsgChunk = 32;
+constexpr int kAsgChunk = 16;   // centroids per shared-memory stage
+constexpr int kAsgTokens = 4;   // tokens per thread
 constexpr int kLayoutChunk = 1024;  // tokens per histogram chunk
 constexpr int kScatterWarps = 8;
 
@@ -48,18 +49,27 @@ template <int D>
 __global__ void __launch_bounds__(kAsgThreads) kmeans_assign_kernel(
     const __nv_bfloat16* __restrict__ x, ClusterDims cd, const float* __restrict__ cent,
     int32_t* __restrict__ labels) {
+  constexpr int TPT = kAsgTokens;  // tokens per thread: each centroid broadcast feeds 4 x 8 FMAs
   __shared__ __align__(16) float cs[kAsgChunk][D];
   __shared__ float cn[kAsgChunk];
-  const int per_bh = (cd.S + kAsgThreads - 1) / kAsgThreads;
+  const int per_bh = (cd.S + kAsgThreads * TPT - 1) / (kAsgThreads * TPT);
   const int bh = blockIdx.x / per_bh;
-  const int s = (blockIdx.x - bh * per_bh) * kAsgThreads + threadIdx.x;
+  const int s0 = (blockIdx.x - bh * per_bh) * kAsgThreads * TPT + threadIdx.x;
   const int b = bh / cd.heads, h = bh - b * cd.heads;
-  const bool live = s < cd.S;
-  const __nv_bfloat16* xr =
-      x + ((static_cast<long long>(b) * cd.S + (live ? s : 0)) * cd.heads + h) * D;
+  const __nv_bfloat16* xr[TPT];
+#pragma unroll
+  for (int u = 0; u < TPT; ++u) {
+    const int s = s0 + u * kAsgThreads;
+    xr[u] = x + ((static_cast<long long>(b) * cd.S + (s < cd.S ? s : 0)) * cd.heads + h) * D;
+  }
   const float* cb = cent + static_cast<long long>(bh) * cd.C * D;
-  float best = INFINITY;
-  int best_c = 0;
+  float best[TPT];
+  int best_c[TPT];
+#pragma unroll
+  for (int u = 0; u < TPT; ++u) {
+    best[u] = INFINITY;
+    best_c[u] = 0;
+  }
   for (int c0 = 0; c0 < cd.C; c0 += kAsgChunk) {
     const int nc = min(kAsgChunk, cd.C - c0);
     __syncthreads();
@@ -68,45 +78,68 @@ __global__ void __launch_bounds__(kAsgThreads) kmeans_assign_kernel(
       cs[j][d] = j < nc ? cb[static_cast<long long>(c0 + j) * D + d] : 0.f;
     }
     __syncthreads();
-    if (threadIdx.x < kAsgChunk) {
+    {  // |c|^2: 8 lanes per centroid; lane p sums dims 8m + p, m = 0 .. D/8 - 1, starting at
+       // m = j mod 4 so the warp's four centroids fall in distinct banks; fixed order.
+      constexpr int kPart = D / 8;
+      const int j = threadIdx.x >> 3, part = threadIdx.x & 7;
       float n = 0.f;
-      for (int d = 0; d < D; ++d) n = fmaf(cs[threadIdx.x][d], cs[threadIdx.x][d], n);
-      cn[threadIdx.x] = n;
+#pragma unroll 4
+      for (int m = 0; m < kPart; ++m) {
+        const float c = cs[j][8 * ((m + (j & 3)) % kPart) + part];
+        n = fmaf(c, c, n);
+      }
+      n += __shfl_xor_sync(0xffffffffu, n, 1);
+      n += __shfl_xor_sync(0xffffffffu, n, 2);
+      n += __shfl_xor_sync(0xffffffffu, n, 4);
+      if (part == 0) cn[j] = n;
     }
     __syncthreads();
-    float acc[kAsgChunk];
+    float acc[TPT][kAsgChunk];
 #pragma unroll
-    for (int j = 0; j < kAsgChunk; ++j) acc[j] = 0.f;
+    for (int u = 0; u < TPT; ++u)
+#pragma unroll
+      for (int j = 0; j < kAsgChunk; ++j) acc[u][j] = 0.f;
 #pragma unroll 1
     for (int d = 0; d < D; d += 8) {
-      float xv[8];
-      bf16x8_to_float(*reinterpret_cast<const uint4*>(xr + d), xv);
+      float xv[TPT][8];
+#pragma unroll
+      for (int u = 0; u < TPT; ++u) bf16x8_to_float(*reinterpret_cast<const uint4*>(xr[u] + d), xv[u]);
 #pragma unroll
       for (int j = 0; j < kAsgChunk; ++j) {
-        const float4 u = *reinterpret_cast<const float4*>(&cs[j][d]);
-        const float4 w = *reinterpret_cast<const float4*>(&cs[j][d + 4]);
-        float a = acc[j];
-        a = fmaf(xv[0], u.x, a);
-        a = fmaf(xv[1], u.y, a);
-        a = fmaf(xv[2], u.z, a);
-        a = fmaf(xv[3], u.w, a);
-        a = fmaf(xv[4], w.x, a);
-        a = fmaf(xv[5], w.y, a);
-        a = fmaf(xv[6], w.z, a);
-        a = fmaf(xv[7], w.w, a);
-        acc[j] = a;
+        const float4 c0v = *reinterpret_cast<const float4*>(&cs[j][d]);
+        const float4 c1v = *reinterpret_cast<const float4*>(&cs[j][d + 4]);
+#pragma unroll
+        for (int u = 0; u < TPT; ++u) {
+          float a = acc[u][j];
+          a = fmaf(xv[u][0], c0v.x, a);
+          a = fmaf(xv[u][1], c0v.y, a);
+          a = fmaf(xv[u][2], c0v.z, a);
+          a = fmaf(xv[u][3], c0v.w, a);
+          a = fmaf(xv[u][4], c1v.x, a);
+          a = fmaf(xv[u][5], c1v.y, a);
+          a = fmaf(xv[u][6], c1v.z, a);
+          a = fmaf(xv[u][7], c1v.w, a);
+          acc[u][j] = a;
+        }
       }
     }
 #pragma unroll
     for (int j = 0; j < kAsgChunk; ++j) {
-      const float dist = fmaf(-2.f, acc[j], cn[j]);
-      if (j < nc && dist < best) {  // strict: the lowest index wins a tie
-        best = dist;
-        best_c = c0 + j;
+#pragma unroll
+      for (int u = 0; u < TPT; ++u) {
+        const float dist = fmaf(-2.f, acc[u][j], cn[j]);
+        if (j < nc && dist < best[u]) {  // strict: the lowest index wins a tie
+          best[u] = dist;
+          best_c[u] = c0 + j;
+        }
       }
     }
   }
-  if (live) labels[static_cast<long long>(bh) * cd.S + s] = best_c;
+#pragma unroll
+  for (int u = 0; u < TPT; ++u) {
+    const int s = s0 + u * kAsgThreads;
+    if (s < cd.S) labels[static_cast<long long>(bh) * cd.S + s] = best_c[u];
+  }
 }
 
 // Tokens of each cluster in every chunk of kLayoutChunk tokens: hist[bh][chunk][C].
@@ -388,7 +421,8 @@ cudaError_t launch_kmeans(const ClusterDims& cd, const void* x, int rounds, floa
   p += al256(static_cast<size_t>(bhn) * cd.S * 4);
   int32_t* sot = reinterpret_cast<int32_t*>(p);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  const unsigned asg_ctas = static_cast<unsigned>(bhn * ((cd.S + kAsgThreads - 1) / kAsgThreads));
+  const unsigned asg_ctas =
+      static_cast<unsigned>(bhn * ((cd.S + kAsgThreads * kAsgTokens - 1) / (kAsgThreads * kAsgTokens)));
   const unsigned upd_ctas = static_cast<unsigned>(bhn * cd.C);
   for (int r = 0; r < rounds; ++r) {
     if (cd.head_dim == 128)
