@@ -9,10 +9,9 @@
 //
 // Kernels (fp32 CUDA-core math: the estimate is ~Np^2/4096 * D multiply-adds per head):
 //   pool_tiles_kernel   one warp per (bh, tile): sums of the valid rows of Q and K.
-//   pooled_logits_kernel one CTA per (bh, 8 query blocks): qbar from the tile sums, kbar
-//                        in chunks of 32 tiles staged in shared memory (rows padded to
-//                        D+1 floats, so 32 threads reading 32 rows hit 32 banks); writes
-//                        the log2-domain logits into the output tensor.
+//   pooled_logits_kernel a register-tiled qbar . kbar product per (bh): 64 x 64 logits per
+//                        CTA, 4 x 4 per thread; writes the log2-domain logits into the
+//                        output tensor.
 //   pooled_softmax_kernel one warp per row: weighted softmax in place.
 #include "bsa_kernels.cuh"
 
@@ -57,65 +56,107 @@ __global__ void __launch_bounds__(256) pool_tiles_kernel(const __nv_bfloat16* __
 }
 
 // Logits in log2 units: scale * log2(e) * qbar_i . kbar_j, -inf for tiles without valid keys
-// (the softmax kernel adds log2(n_j)).  One thread per (query block, kv tile) of a chunk.
+// (the softmax kernel adds log2(n_j)).  A register-tiled product per (bh): a CTA of 256
+// threads computes a 64 x 64 tile of (query block, kv block) logits, 4 x 4 per thread; the
+// head dimension is staged 16 at a time in shared memory as [d][block] so each thread
+// reads its four qbar and four kbar values with two 16-byte loads.  qbar and kbar are formed
+// while staging: sums of the block's tiles times 1 / valid count (0 for an empty block).
+// Every logit sums over d in order 0..D-1 (deterministic).
+constexpr int kLgTile = 64;
+constexpr int kLgK = 16;
+
 template <int D>
 __global__ void __launch_bounds__(256) pooled_logits_kernel(const float* __restrict__ qsum,
                                                             const float* __restrict__ ksum,
                                                             AttnDims a, float scale_log2,
                                                             float* __restrict__ out) {
-  __shared__ float sq[8][D];
-  __shared__ float sk[32][D + 1];
-  __shared__ float s_inv[8];     // 1 / valid queries of each query block (0 if none)
-  __shared__ float s_kinv[32];   // 1 / valid keys of each tile of the chunk (0 if none)
-  const int groups = (a.n_qb + 7) / 8;
-  const int bh = blockIdx.x / groups;
-  const int i0 = (blockIdx.x % groups) * 8;
+  __shared__ __align__(16) float sa[kLgK][kLgTile];
+  __shared__ __align__(16) float sb[kLgK][kLgTile];
+  __shared__ float s_qinv[kLgTile];
+  __shared__ float s_kinv[kLgTile];
+  const int ti = (a.n_qb + kLgTile - 1) / kLgTile;
+  const int tj = (a.n_kb + kLgTile - 1) / kLgTile;
+  const int per_bh = ti * tj;
+  const int bh = blockIdx.x / per_bh;
+  const int rem = blockIdx.x - bh * per_bh;
+  const int i0 = (rem / tj) * kLgTile;
+  const int j0 = (rem % tj) * kLgTile;
   const int tid = threadIdx.x;
   const int per = a.q_block / 64;  // tiles per query block
   const long long tbase = static_cast<long long>(bh) * a.n_kb;
-  if (tid < 8) {
+  if (tid < kLgTile) {
     const int i = i0 + tid;
     int cnt = 0;
     if (i < a.n_qb)
       for (int u = i * per; u < (i + 1) * per; ++u) cnt += tile_valid_count(a.g, u);
-    s_inv[tid] = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
+    s_qinv[tid] = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
+  } else if (tid < 2 * kLgTile) {
+    const int j = j0 + tid - kLgTile;
+    const int cnt = j < a.n_kb ? tile_valid_count(a.g, j) : 0;
+    s_kinv[tid - kLgTile] = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
   }
-  __syncthreads();
-  // qbar of the CTA's 8 query blocks (0 for a block without valid queries)
-  for (int x = tid; x < 8 * D; x += 256) {
-    const int qi = x / D, d = x % D;
-    const int i = i0 + qi;
-    float sum = 0.f;
-    if (i < a.n_qb)
-      for (int u = i * per; u < (i + 1) * per; ++u) sum += qsum[(tbase + u) * D + d];
-    sq[qi][d] = sum * s_inv[qi];
-  }
-  const int qi = tid >> 5, jl = tid & 31;
-  const int i = i0 + qi;
-  for (int j0 = 0; j0 < a.n_kb; j0 += 32) {
+  const int ty = tid >> 4, tx = tid & 15;  // rows 4ty.., cols 4tx..
+  float acc[4][4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+  for (int d0 = 0; d0 < D; d0 += kLgK) {
     __syncthreads();
-    if (tid < 32) {
-      const int j = j0 + tid;
-      const int cnt = j < a.n_kb ? tile_valid_count(a.g, j) : 0;
-      s_kinv[tid] = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
-    }
-    __syncthreads();
-    for (int x = tid; x < 32 * D; x += 256) {
-      const int r = x / D, d = x % D;
-      const int j = j0 + r;
-      sk[r][d] = j < a.n_kb ? ksum[(tbase + j) * D + d] * s_kinv[r] : 0.f;
-    }
-    __syncthreads();
-    const int j = j0 + jl;
-    if (i < a.n_qb && j < a.n_kb) {
-      float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 8
-      for (int d = 0; d < D; d += 2) {
-        acc0 = fmaf(sq[qi][d], sk[jl][d], acc0);
-        acc1 = fmaf(sq[qi][d + 1], sk[jl][d + 1], acc1);
+    // stage 64 blocks x 16 dims of qbar and kbar, transposed to [d][block]: one 16-byte
+    // load of four consecutive dims per thread and matrix (64 x 16 = 256 x 4)
+    {
+      const int blk = tid >> 2, dq = (tid & 3) * 4;
+      const int i = i0 + blk, j = j0 + blk;
+      float4 qv = make_float4(0.f, 0.f, 0.f, 0.f), kv = qv;
+      if (i < a.n_qb) {
+        for (int u = i * per; u < (i + 1) * per; ++u) {
+          const float4 t = *reinterpret_cast<const float4*>(qsum + (tbase + u) * D + d0 + dq);
+          qv.x += t.x;
+          qv.y += t.y;
+          qv.z += t.z;
+          qv.w += t.w;
+        }
+        const float f = s_qinv[blk];
+        qv = make_float4(qv.x * f, qv.y * f, qv.z * f, qv.w * f);
       }
-      out[(static_cast<long long>(bh) * a.n_qb + i) * a.n_kb + j] =
-          s_kinv[jl] > 0.f ? (acc0 + acc1) * scale_log2 : -INFINITY;
+      if (j < a.n_kb) {
+        const float4 t = *reinterpret_cast<const float4*>(ksum + (tbase + j) * D + d0 + dq);
+        const float f = s_kinv[blk];
+        kv = make_float4(t.x * f, t.y * f, t.z * f, t.w * f);
+      }
+      sa[dq + 0][blk] = qv.x;
+      sa[dq + 1][blk] = qv.y;
+      sa[dq + 2][blk] = qv.z;
+      sa[dq + 3][blk] = qv.w;
+      sb[dq + 0][blk] = kv.x;
+      sb[dq + 1][blk] = kv.y;
+      sb[dq + 2][blk] = kv.z;
+      sb[dq + 3][blk] = kv.w;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int d = 0; d < kLgK; ++d) {
+      const float4 av = *reinterpret_cast<const float4*>(&sa[d][4 * ty]);
+      const float4 bv = *reinterpret_cast<const float4*>(&sb[d][4 * tx]);
+      const float ar[4] = {av.x, av.y, av.z, av.w};
+      const float br[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(ar[r], br[c], acc[r][c]);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int i = i0 + 4 * ty + r;
+    if (i >= a.n_qb) continue;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int j = j0 + 4 * tx + c;
+      if (j < a.n_kb)
+        out[(static_cast<long long>(bh) * a.n_qb + i) * a.n_kb + j] =
+            s_kinv[4 * tx + c] > 0.f ? acc[r][c] * scale_log2 : -INFINITY;
     }
   }
 }
@@ -165,7 +206,9 @@ cudaError_t launch_pooled_mass(const AttnDims& a, const void* q, const void* k, 
   float* ksum = qsum + tiles * a.head_dim;
   const float sl2 = softmax_scale * 1.4426950408889634f;
   const unsigned pool_ctas = static_cast<unsigned>((tiles + 7) / 8);
-  const unsigned logit_ctas = static_cast<unsigned>(1LL * a.batch * a.heads * ((a.n_qb + 7) / 8));
+  const unsigned logit_ctas = static_cast<unsigned>(1LL * a.batch * a.heads *
+                                                    ((a.n_qb + kLgTile - 1) / kLgTile) *
+                                                    ((a.n_kb + kLgTile - 1) / kLgTile));
   const unsigned sm_ctas = static_cast<unsigned>((rows + 7) / 8);
   const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
   const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
