@@ -530,7 +530,12 @@ def run_reference(args, world, rank, pg):
         "value": val, "unit": "TFLOP/s (executed, kept blocks)", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": wl.name},
+        "data": "synthetic",
+        "config": {"workload": wl.name,
+                   "grid": f"{wl.T}x{wl.H}x{wl.W} padded {wl.Tp}x{wl.Hp}x{wl.Wp}",
+                   "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
+                   "q_block": wl.q_block, "kv_block": 64, "tokens": wl.S, "slots": wl.Np,
+                   "threshold": args.tau},
         "cpu_baseline": {"value": val, "unit": "TFLOP/s (executed, kept blocks)", "cores": 1,
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": val, "unit": "TFLOP/s (executed, kept blocks)", "h2d_bytes_per_step": 0,

@@ -256,3 +256,81 @@ def test_semantic_pipeline_on_blobs_matches_oracle(B):
         rows = np.isin(Lq, np.flatnonzero(same))
         e = Hp.attn_errors(out[0, :, h].cpu().double().numpy()[rows], ref[rows])
         assert e["max_abs"] <= Hp.ATTN_MAX_ABS and e["mean_abs"] <= Hp.ATTN_MEAN_ABS, e
+
+
+# ------------------------------------------------------------------ full size (720p tokens)
+FULL_WL = synth.WORKLOADS["wan14b_720p"]
+
+
+def test_cluster_path_full_size_sampled_rows(B):
+    """The 720p token count and head count: cluster order from seeded labels on both sides
+    (bit-exact), then attention in cluster order on sampled query rows against the oracle."""
+    S, Hh, D = FULL_WL.T * FULL_WL.H * FULL_WL.W, FULL_WL.heads, 128
+    Cq, Ck = 64, 256
+    cs = B.ClusterShape(1, Hh, D, S, Cq, Ck)
+    q, k, v = synth.draw_qkv(FULL_WL, device="cuda")            # raster bf16
+    lq = synth.draw_cluster_labels(1, Hh, S, Cq, seed=101, empty=(5,))
+    lk = synth.draw_cluster_labels(1, Hh, S, Ck, seed=102, empty=(7,))
+    nq, sq, tq, _ = B.cluster_layout(lq.cuda(), cs, Cq)
+    nk, sk, tk, _ = B.cluster_layout(lk.cuda(), cs, Ck)
+    rp, ci = synth.draw_keep_csr(Hh * Cq, Ck, 0.6, seed=103, empty_rows=(3,))
+    qp, kp, vp = (B.cluster_permute(x, cs, t) for x, t in ((q, tq), (k, tk), (v, tk)))
+    ws = B.new_cluster_fwd_workspace(cs)
+    out = B.cluster_fwd(qp, kp, vp, cs, sq, nq, sk, nk, rp.cuda(), ci.cuda(), ws=ws)
+    back = B.cluster_permute(out, cs, tq, inverse=True)          # raster order again
+    assert B.device_status(ws) == 0
+    scale = 1.0 / math.sqrt(D)
+    g = torch.Generator().manual_seed(104)
+    errs = []
+    for h in (0, Hh // 2, Hh - 1):
+        st_q, tos_q, _ = O.cluster_layout(lq[0, h].numpy(), Cq)
+        st_k, tos_k, _ = O.cluster_layout(lk[0, h].numpy(), Ck)
+        assert np.array_equal(tq[0, h].cpu().numpy(), tos_q)
+        assert np.array_equal(tk[0, h].cpu().numpy(), tos_k)
+        cq_ = np.bincount(lq[0, h].numpy(), minlength=Cq)
+        ck_ = np.bincount(lk[0, h].numpy(), minlength=Ck)
+        r0 = h * Cq
+        rows = rp[r0:r0 + Cq + 1].numpy() - rp[r0].numpy()
+        cols = ci[rp[r0]:rp[r0 + Cq]].numpy()
+        toks = torch.randint(0, S, (24,), generator=g).numpy()   # sampled raster tokens
+        slots = np.empty(S, dtype=np.int64)
+        slots[tos_q] = np.arange(S)
+        Xq = q[0, :, h].float().cpu().double().numpy()[tos_q]
+        Xk = k[0, :, h].float().cpu().double().numpy()[tos_k]
+        Xv = v[0, :, h].float().cpu().double().numpy()[tos_k]
+        ref = O.cluster_attention(Xq, Xk, Xv, st_q, cq_, st_k, ck_, rows, cols, scale,
+                                  rows=slots[toks])
+        got = back[0, torch.from_numpy(toks), h].float().cpu().double().numpy()
+        errs.append(Hp.attn_errors(got, ref[slots[toks]]))
+    for e in errs:
+        assert e["max_abs"] <= Hp.ATTN_MAX_ABS and e["mean_abs"] <= Hp.ATTN_MEAN_ABS, e
+
+
+def test_kmeans_full_size_properties(B):
+    """k-means at the 720p size: labels in range, counts and layout consistent with them,
+    centroids the means of their tokens (sampled clusters, float64 check)."""
+    S, Hh, D, C = FULL_WL.T * FULL_WL.H * FULL_WL.W, FULL_WL.heads, 128, 256
+    cs = B.ClusterShape(1, Hh, D, S, C, C)
+    k = synth.draw_qkv(FULL_WL, device="cuda")[1]
+    g = torch.Generator().manual_seed(105)
+    pick = torch.randint(0, S, (1, Hh, C), generator=g).cuda()
+    kh = k.float().permute(0, 2, 1, 3)
+    init = torch.gather(kh, 2, pick[..., None].expand(-1, -1, -1, D)).contiguous()
+    ws = B.new_cluster_workspace(cs, C)
+    cent, labels, counts = B.kmeans(k, cs, C, init.clone(), 3, ws=ws)
+    assert B.device_status(ws) == 0
+    lab = labels.cpu().long()
+    assert int(lab.min()) >= 0 and int(lab.max()) < C
+    for h in (0, Hh - 1):
+        assert torch.equal(torch.bincount(lab[0, h], minlength=C), counts[0, h].cpu().long())
+        X = kh[0, h].cpu().double()
+        for c in torch.randint(0, C, (6,), generator=g).tolist():
+            m = lab[0, h] == c
+            if m.any():
+                np.testing.assert_allclose(cent[0, h, c].cpu().double().numpy(),
+                                           X[m].mean(0).numpy(), rtol=0, atol=5e-5)
+    n2, st2, tos2, sot2 = B.cluster_layout(labels, cs, C, ws=ws)
+    assert torch.equal(n2, counts)
+    t = tos2[0, 0].cpu().long()
+    assert torch.equal(torch.sort(t).values, torch.arange(S))
+    assert torch.equal(sot2[0, 0].cpu().long()[t], torch.arange(S))
