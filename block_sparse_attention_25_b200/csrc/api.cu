@@ -49,6 +49,22 @@ cudaError_t encode_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataTy
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t encode_tmap_3d_strided(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                                   const unsigned long long dims[3],
+                                   const unsigned long long strides_bytes[2],
+                                   const unsigned box[3]) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorInitializationError;
+  const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  const cuuint64_t st[2] = {strides_bytes[0], strides_bytes[1]};
+  const cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = fn(map, dtype, 3, const_cast<void*>(base), d, st, bx, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace bsa
 
 using bsa::AttnDims;

@@ -184,5 +184,10 @@ cudaError_t launch_cluster_fwd(int batch, int heads, int head_dim, int S, int n_
 // and 128-byte swizzle.
 cudaError_t encode_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                            int elem_bytes, int D, int Np, int bh, int box_d, int box_rows);
+// Same with explicit extents (innermost first), byte strides of dims 1 and 2, and box.
+cudaError_t encode_tmap_3d_strided(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                                   const unsigned long long dims[3],
+                                   const unsigned long long strides_bytes[2],
+                                   const unsigned box[3]);
 
 }  // namespace bsa

@@ -7,16 +7,18 @@
 // representatives identify the critical clusters for the top-p budget control.
 //
 // Per (batch, head) one clustering of S tokens into C clusters:
-//   kmeans_assign_kernel   label = argmin_c (|c|^2 - 2 x.c) in float32, ties to the lowest c;
-//                          four tokens per thread, centroids staged 16 at a time in shared
-//                          memory and read as broadcasts (each feeds 32 FMAs).
+//   kmeans_split_kernel    centroids -> three bf16 parts (hi, mid, lo) and |c|^2.
+//   kmeans_assign_tc_kernel label = argmin_c (|c|^2 - 2 x.c), ties to the lowest c: x.c on
+//                          the tensor cores as x.hi + x.mid + x.lo (tcgen05, fp32 accumulate
+//                          in TMEM), 128 tokens per CTA, argmin by one thread per TMEM lane.
 //   layout_hist_kernel     per chunk of 1024 tokens, the tokens of each cluster.
 //   layout_scan_kernel     per head: cluster sizes, cluster starts (exclusive scan) and each
 //                          chunk's first slot inside every cluster.
 //   layout_scatter_kernel  one warp per chunk walks its tokens in order: rank among equal
 //                          labels by __match_any_sync, so the order is stable.
-//   kmeans_update_kernel   centroid = sum of the cluster's tokens in cluster order / size,
-//                          a fixed summation order (deterministic); empty clusters keep theirs.
+//   kmeans_update_kernel   centroid = sum of the cluster's tokens / size: 8 warps over fixed
+//                          segments of the cluster order, partial sums added in a fixed order
+//                          (deterministic); empty clusters keep theirs.
 //   cluster_gather/scatter row copies between raster [B, S, Hh, D] and cluster order
 //                          [B, Hh, S, D].
 //   cluster_mass_kernel    one CTA per (bh, query cluster): weighted softmax over key clusters.
@@ -26,119 +28,216 @@ namespace bsa {
 
 namespace {
 
-constexpr int kAsgThreads = 128;
-constexpr int kAsgChunk = 16;   // centroids per shared-memory stage
-constexpr int kAsgTokens = 4;   // tokens per thread
 constexpr int kLayoutChunk = 1024;  // tokens per histogram chunk
 constexpr int kScatterWarps = 8;
 
-// Eight bf16 values (little-endian pairs in four words) to float: a bf16 is the upper half
-// of the float with the same bits.
-__device__ __forceinline__ void bf16x8_to_float(const uint4& raw, float* f) {
-  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-
 }  // namespace
 
+// ---- assignment on the tensor cores
+// Every centroid is split into three bf16 parts, hi = bf16(c), mid = bf16(c - hi),
+// lo = bf16(c - hi - mid), whose sum is c to within ~2^-24 relative; x is bf16, so the
+// tensor cores form x.hi + x.mid + x.lo from exact products with fp32 accumulation: the
+// dot products of the fp32 centroids to float32 accuracy.  dist = |c|^2 - 2 x.c is then
+// reduced per token (one thread per TMEM lane), ties to the lowest centroid index.
+
+// One warp per (bh, padded centroid row): the three parts [bh][part][c_pad][D] and |c|^2
+// (lanes over d, then a fixed xor-shuffle tree).  Rows c >= C are zero.
 template <int D>
-__global__ void __launch_bounds__(kAsgThreads) kmeans_assign_kernel(
-    const __nv_bfloat16* __restrict__ x, ClusterDims cd, const float* __restrict__ cent,
-    int32_t* __restrict__ labels) {
-  constexpr int TPT = kAsgTokens;  // tokens per thread: each centroid broadcast feeds 4 x 8 FMAs
-  __shared__ __align__(16) float cs[kAsgChunk][D];
-  __shared__ float cn[kAsgChunk];
-  const int per_bh = (cd.S + kAsgThreads * TPT - 1) / (kAsgThreads * TPT);
+__global__ void __launch_bounds__(256) kmeans_split_kernel(ClusterDims cd, int c_pad,
+                                                           const float* __restrict__ cent,
+                                                           __nv_bfloat16* __restrict__ parts,
+                                                           float* __restrict__ norms) {
+  const long long w = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<long long>(cd.batch) * cd.heads * c_pad) return;  // warp-uniform
+  const int bh = static_cast<int>(w / c_pad);
+  const int c = static_cast<int>(w - static_cast<long long>(bh) * c_pad);
+  const long long plane = static_cast<long long>(c_pad) * D;
+  __nv_bfloat16* out = parts + static_cast<long long>(bh) * 3 * plane + static_cast<long long>(c) * D;
+  float n = 0.f;
+#pragma unroll
+  for (int d = lane; d < D; d += 32) {
+    const float v = c < cd.C ? cent[(static_cast<long long>(bh) * cd.C + c) * D + d] : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+    out[d] = hi;
+    out[plane + d] = mid;
+    out[2 * plane + d] = lo;
+    n = fmaf(v, v, n);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+  if (lane == 0) norms[static_cast<long long>(bh) * c_pad + c] = n;
+}
+
+constexpr int kTcRows = 128;     // tokens per CTA = TMEM lanes
+constexpr int kTcStages = 3;     // centroid-part ring
+constexpr int kTcThreads = 160;  // warps 0-3: distances and argmin; warp 4: TMA + MMA
+
+template <int D>
+struct AssignSmem {
+  static constexpr int kChunks = D / 64;         // 128-byte chunks of a bf16 row
+  static constexpr int kXChunk = kTcRows * 128;  // one chunk of the token tile
+  static size_t bytes(int n_tile, int c_pad) {
+    return 1024 + kChunks * kXChunk + static_cast<size_t>(kTcStages) * n_tile * 128 +
+           static_cast<size_t>(c_pad) * 4 + 256;
+  }
+};
+
+// One CTA per (bh, 128 tokens).  The token tile is loaded once; the parts of each tile of
+// n_tile centroids stream through a 3-stage ring as (part, 64-dim chunk) steps, each step
+// 4 MMAs of K = 16 into TMEM buffer (tile & 1); the epilogue warps reduce a finished buffer
+// while the next tile accumulates in the other.
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1) kmeans_assign_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_c,
+    ClusterDims cd, int n_tile, int c_pad, const float* __restrict__ norms,
+    int32_t* __restrict__ labels, uint32_t* status) {
+  using L = AssignSmem<D>;
+  constexpr int CH = L::kChunks;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const int bstage = n_tile * 128;
+  uint8_t* xs = smem;
+  uint8_t* bs = smem + CH * L::kXChunk;
+  float* sn = reinterpret_cast<float*>(bs + kTcStages * bstage);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sn + c_pad);  // c_pad is a multiple of 16
+  uint64_t* bar_x = bars;
+  uint64_t* bar_full = bars + 1;
+  uint64_t* bar_empty = bar_full + kTcStages;
+  uint64_t* bar_acc = bar_empty + kTcStages;  // [2] accumulator complete
+  uint64_t* bar_drained = bar_acc + 2;        // [2] epilogue done with the buffer
+  uint64_t* bar_drain = bar_drained + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per_bh = (cd.S + kTcRows - 1) / kTcRows;
   const int bh = blockIdx.x / per_bh;
-  const int s0 = (blockIdx.x - bh * per_bh) * kAsgThreads * TPT + threadIdx.x;
+  const int s0 = (blockIdx.x - bh * per_bh) * kTcRows;
   const int b = bh / cd.heads, h = bh - b * cd.heads;
-  const __nv_bfloat16* xr[TPT];
-#pragma unroll
-  for (int u = 0; u < TPT; ++u) {
-    const int s = s0 + u * kAsgThreads;
-    xr[u] = x + ((static_cast<long long>(b) * cd.S + (s < cd.S ? s : 0)) * cd.heads + h) * D;
-  }
-  const float* cb = cent + static_cast<long long>(bh) * cd.C * D;
-  float best[TPT];
-  int best_c[TPT];
-#pragma unroll
-  for (int u = 0; u < TPT; ++u) {
-    best[u] = INFINITY;
-    best_c[u] = 0;
-  }
-  for (int c0 = 0; c0 < cd.C; c0 += kAsgChunk) {
-    const int nc = min(kAsgChunk, cd.C - c0);
-    __syncthreads();
-    for (int i = threadIdx.x; i < kAsgChunk * D; i += kAsgThreads) {
-      const int j = i / D, d = i - j * D;
-      cs[j][d] = j < nc ? cb[static_cast<long long>(c0 + j) * D + d] : 0.f;
+  const int n_tiles = c_pad / n_tile;
+  const int per_tile = 3 * CH;  // ring steps per centroid tile
+  const int T = n_tiles * per_tile;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_x, 1);
+    for (int i = 0; i < kTcStages; ++i) {
+      mbar_init(bar_full + i, 1);
+      mbar_init(bar_empty + i, 1);
     }
-    __syncthreads();
-    {  // |c|^2: 8 lanes per centroid; lane p sums dims 8m + p, m = 0 .. D/8 - 1, starting at
-       // m = j mod 4 so the warp's four centroids fall in distinct banks; fixed order.
-      constexpr int kPart = D / 8;
-      const int j = threadIdx.x >> 3, part = threadIdx.x & 7;
-      float n = 0.f;
-#pragma unroll 4
-      for (int m = 0; m < kPart; ++m) {
-        const float c = cs[j][8 * ((m + (j & 3)) % kPart) + part];
-        n = fmaf(c, c, n);
-      }
-      n += __shfl_xor_sync(0xffffffffu, n, 1);
-      n += __shfl_xor_sync(0xffffffffu, n, 2);
-      n += __shfl_xor_sync(0xffffffffu, n, 4);
-      if (part == 0) cn[j] = n;
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_acc + i, 1);
+      mbar_init(bar_drained + i, 4);
     }
-    __syncthreads();
-    float acc[TPT][kAsgChunk];
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < c_pad; i += kTcThreads) sn[i] = norms[static_cast<long long>(bh) * c_pad + i];
+  if (warp == 4) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tensormap(&tm_x);
+      prefetch_tensormap(&tm_c);
+      auto load_step = [&](int k) {  // centroid tile k / per_tile, part, 64-dim chunk
+        const int st = k % kTcStages;
+        const int n = k / per_tile, part = (k / CH) % 3, ch = k % CH;
+        mbar_arrive_expect_tx(bar_full + st, bstage);
+        tma_load_3d(bs + st * bstage, &tm_c, bar_full + st, ch * 64, n * n_tile, bh * 3 + part);
+      };
+      mbar_arrive_expect_tx(bar_x, CH * L::kXChunk);
+      for (int ch = 0; ch < CH; ++ch)
+        tma_load_3d(xs + ch * L::kXChunk, &tm_x, bar_x, ch * 64, h, b * cd.S + s0);
+      for (int k = 0; k < T && k < kTcStages; ++k) load_step(k);
+      const uint32_t idesc = make_idesc(1u, 0u, 128u, static_cast<uint32_t>(n_tile));
+      const uint64_t x_desc0 = make_sdesc_sw128(smem_u32(xs), 16, 1024);
+      const uint64_t b_desc0 = make_sdesc_sw128(smem_u32(bs), 16, 1024);
+      bool ok = mbar_wait(bar_x, 0, abort_flag, status, DETAIL_WAIT_Q);
+      for (int k = 0; k < T && ok; ++k) {
+        const int st = k % kTcStages;
+        const int n = k / per_tile, kin = k - n * per_tile, ch = k % CH;
+        const int buf = n & 1;
+        if (kin == 0 && n >= 2 &&
+            !mbar_wait(bar_drained + buf, ((n - 2) >> 1) & 1, abort_flag, status, DETAIL_WAIT_O_FULL)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(bar_full + st, (k / kTcStages) & 1, abort_flag, status, DETAIL_WAIT_K_FULL)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t xd = x_desc0 + static_cast<uint64_t>((ch * L::kXChunk) >> 4);
+        const uint64_t bd = b_desc0 + static_cast<uint64_t>((st * bstage) >> 4);
 #pragma unroll
-    for (int u = 0; u < TPT; ++u)
-#pragma unroll
-      for (int j = 0; j < kAsgChunk; ++j) acc[u][j] = 0.f;
-#pragma unroll 1
-    for (int d = 0; d < D; d += 8) {
-      float xv[TPT][8];
-#pragma unroll
-      for (int u = 0; u < TPT; ++u) bf16x8_to_float(*reinterpret_cast<const uint4*>(xr[u] + d), xv[u]);
-#pragma unroll
-      for (int j = 0; j < kAsgChunk; ++j) {
-        const float4 c0v = *reinterpret_cast<const float4*>(&cs[j][d]);
-        const float4 c1v = *reinterpret_cast<const float4*>(&cs[j][d + 4]);
-#pragma unroll
-        for (int u = 0; u < TPT; ++u) {
-          float a = acc[u][j];
-          a = fmaf(xv[u][0], c0v.x, a);
-          a = fmaf(xv[u][1], c0v.y, a);
-          a = fmaf(xv[u][2], c0v.z, a);
-          a = fmaf(xv[u][3], c0v.w, a);
-          a = fmaf(xv[u][4], c1v.x, a);
-          a = fmaf(xv[u][5], c1v.y, a);
-          a = fmaf(xv[u][6], c1v.z, a);
-          a = fmaf(xv[u][7], c1v.w, a);
-          acc[u][j] = a;
+        for (int kk = 0; kk < 4; ++kk)  // 16 dims (32 bytes) per MMA inside the chunk
+          mma_f16_ss(tmem + buf * n_tile, xd + 2 * kk, bd + 2 * kk, idesc, (kin > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar_empty + st);
+        if (kin == per_tile - 1) mma_commit(bar_acc + buf);
+        // refill the stage of step k - 1 (its MMAs were issued before this step's)
+        if (k >= 1 && k - 1 + kTcStages < T) {
+          const int st2 = (k - 1) % kTcStages;
+          if (!mbar_wait(bar_empty + st2, ((k - 1) / kTcStages) & 1, abort_flag, status,
+                         DETAIL_WAIT_K_EMPTY)) {
+            ok = false;
+            break;
+          }
+          load_step(k - 1 + kTcStages);
         }
       }
+      // Whatever happened, let every issued MMA finish before TMEM is released.
+      mma_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0, status, DETAIL_WAIT_O_FULL);
     }
+  } else {
+    // ------------------------------------------------ distances and argmin, one token per thread
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float best = INFINITY;
+    int best_c = 0;
+    bool ok = true;
+    for (int n = 0; n < n_tiles; ++n) {
+      const int buf = n & 1;
+      const bool got = ok && __all_sync(0xffffffffu, mbar_wait(bar_acc + buf, (n >> 1) & 1, abort_flag,
+                                                                status, DETAIL_WAIT_S_FULL));
+      ok = got;
+      tc_fence_after();
+      if (got) {
+        for (int c0 = 0; c0 < n_tile; c0 += 32) {
+          float v[32];
+          tmem_ld32(lane_base + buf * n_tile + c0, v);
+          tmem_ld_wait();
 #pragma unroll
-    for (int j = 0; j < kAsgChunk; ++j) {
-#pragma unroll
-      for (int u = 0; u < TPT; ++u) {
-        const float dist = fmaf(-2.f, acc[u][j], cn[j]);
-        if (j < nc && dist < best[u]) {  // strict: the lowest index wins a tie
-          best[u] = dist;
-          best_c[u] = c0 + j;
+          for (int j = 0; j < 32; ++j) {
+            const int idx = n * n_tile + c0 + j;
+            const float dist = fmaf(-2.f, v[j], sn[idx]);
+            if (idx < cd.C && dist < best) {  // strict: the lowest index wins a tie
+              best = dist;
+              best_c = idx;
+            }
+          }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_drained + buf);
     }
+    const int s = s0 + warp * 32 + lane;
+    if (s < cd.S && ok) labels[static_cast<long long>(bh) * cd.S + s] = best_c;
   }
-#pragma unroll
-  for (int u = 0; u < TPT; ++u) {
-    const int s = s0 + u * kAsgThreads;
-    if (s < cd.S) labels[static_cast<long long>(bh) * cd.S + s] = best_c[u];
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -247,34 +346,57 @@ __global__ void __launch_bounds__(32 * kScatterWarps) layout_scatter_kernel(
   }
 }
 
-// centroid[bh][c] = mean of the cluster's tokens, summed in cluster order: 4 partial sums by
-// slot index mod 4, combined in a fixed order.  One CTA of D threads per (bh, cluster).
+// centroid[bh][c] = mean of the cluster's tokens.  One CTA of 8 warps per (bh, cluster):
+// warp w sums the w-th of 8 contiguous segments of the cluster's slots (lane l holds dims
+// D/32 * l ..), the 8 partial sums are added in warp order: a fixed summation order
+// (deterministic).  An empty cluster keeps its centroid.
 template <int D>
-__global__ void __launch_bounds__(D) kmeans_update_kernel(ClusterDims cd,
-                                                          const __nv_bfloat16* __restrict__ x,
-                                                          const int32_t* __restrict__ token_of_slot,
-                                                          const int32_t* __restrict__ starts,
-                                                          const int32_t* __restrict__ counts,
-                                                          float* __restrict__ cent) {
+__global__ void __launch_bounds__(256) kmeans_update_kernel(ClusterDims cd,
+                                                            const __nv_bfloat16* __restrict__ x,
+                                                            const int32_t* __restrict__ token_of_slot,
+                                                            const int32_t* __restrict__ starts,
+                                                            const int32_t* __restrict__ counts,
+                                                            float* __restrict__ cent) {
+  constexpr int PER = D / 32;  // dims per lane: 4 (D = 128) or 2 (D = 64)
+  __shared__ float part[8][D];
   const int bh = blockIdx.x / cd.C;
   const int c = blockIdx.x - bh * cd.C;
   const int b = bh / cd.heads, h = bh - b * cd.heads;
-  const int d = threadIdx.x;
   const int n = counts[static_cast<long long>(bh) * cd.C + c];
-  if (n <= 0) return;  // empty cluster: keeps its centroid
+  if (n <= 0) return;  // uniform over the CTA
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int st = starts[static_cast<long long>(bh) * cd.C + c];
+  const int seg = (n + 7) / 8;
+  const int lo = min(n, warp * seg), hi = min(n, lo + seg);
   const int32_t* tos = token_of_slot + static_cast<long long>(bh) * cd.S + st;
-  const __nv_bfloat16* xb = x + static_cast<long long>(b) * cd.S * cd.heads * D + h * D + d;
+  const __nv_bfloat16* xb = x + static_cast<long long>(b) * cd.S * cd.heads * D + h * D + lane * PER;
   const long long row = static_cast<long long>(cd.heads) * D;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  int i = 0;
-  for (; i + 4 <= n; i += 4) {
+  float acc[PER];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) acc[u] += __bfloat162float(xb[tos[i + u] * row]);
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  for (int i = lo; i < hi; ++i) {
+    const __nv_bfloat16* r = xb + tos[i] * row;
+    if constexpr (PER == 4) {
+      const uint2 w = *reinterpret_cast<const uint2*>(r);
+      acc[0] += __uint_as_float(w.x << 16);
+      acc[1] += __uint_as_float(w.x & 0xFFFF0000u);
+      acc[2] += __uint_as_float(w.y << 16);
+      acc[3] += __uint_as_float(w.y & 0xFFFF0000u);
+    } else {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(r);
+      acc[0] += __uint_as_float(w << 16);
+      acc[1] += __uint_as_float(w & 0xFFFF0000u);
+    }
   }
-  for (; i < n; ++i) acc[i & 3] += __bfloat162float(xb[tos[i] * row]);
-  const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-  cent[(static_cast<long long>(bh) * cd.C + c) * D + d] = __fdiv_rn(sum, static_cast<float>(n));
+#pragma unroll
+  for (int e = 0; e < PER; ++e) part[warp][lane * PER + e] = acc[e];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) sum += part[w][threadIdx.x];
+    cent[(static_cast<long long>(bh) * cd.C + c) * D + threadIdx.x] = __fdiv_rn(sum, static_cast<float>(n));
+  }
 }
 
 // Row copies: forward dst[bh][p] = src[b][token_of_slot[bh][p]][h] (zeros for an empty
@@ -368,10 +490,55 @@ __global__ void __launch_bounds__(256) cluster_mass_kernel(int heads, int D, int
 // three internally; the layout call writes them to the caller's arrays instead).
 static size_t al256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 
+// Centroid tile of the tensor-core assignment: all clusters in one MMA when C <= 256; a
+// multiple of 32 so the epilogue reads whole 32-column groups of it.
+static int assign_n_tile(int C) { return C >= 256 ? 256 : ((C + 31) / 32) * 32; }
+static int assign_c_pad(int C) {
+  const int n = assign_n_tile(C);
+  return ((C + n - 1) / n) * n;
+}
+
+// Workspace after the status header: hist, starts, token_of_slot, slot_of_token (the
+// cluster order), then the centroid parts bf16 [BH][3][c_pad][D] and norms fp32 [BH][c_pad].
 size_t cluster_scratch_bytes(const ClusterDims& cd) {
   const size_t bhn = static_cast<size_t>(cd.batch) * cd.heads;
   const size_t nchunks = (cd.S + kLayoutChunk - 1) / kLayoutChunk;
-  return al256(bhn * nchunks * cd.C * 4) + al256(bhn * cd.C * 4) + 2 * al256(bhn * cd.S * 4);
+  const size_t c_pad = static_cast<size_t>(assign_c_pad(cd.C));
+  return al256(bhn * nchunks * cd.C * 4) + al256(bhn * cd.C * 4) + 2 * al256(bhn * cd.S * 4) +
+         al256(bhn * 3 * c_pad * cd.head_dim * 2) + al256(bhn * c_pad * 4);
+}
+
+template <int D>
+static cudaError_t launch_assign(const ClusterDims& cd, const void* x, const float* centroids,
+                                 __nv_bfloat16* parts, float* norms, int32_t* labels,
+                                 uint32_t* status, cudaStream_t stream) {
+  const long long bhn = static_cast<long long>(cd.batch) * cd.heads;
+  const int n_tile = assign_n_tile(cd.C), c_pad = assign_c_pad(cd.C);
+  kmeans_split_kernel<D><<<static_cast<unsigned>((bhn * c_pad + 7) / 8), 256, 0, stream>>>(
+      cd, c_pad, centroids, parts, norms);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // tokens: raster [B, S, Hh, D] as (D, Hh, B*S) with a 64 x 1 x 128 box
+  CUtensorMap tx, tc;
+  const unsigned long long xdims[3] = {static_cast<unsigned long long>(D),
+                                       static_cast<unsigned long long>(cd.heads),
+                                       static_cast<unsigned long long>(cd.batch) * cd.S};
+  const unsigned long long xstr[2] = {static_cast<unsigned long long>(D) * 2,
+                                      static_cast<unsigned long long>(cd.heads) * D * 2};
+  const unsigned xbox[3] = {64u, 1u, static_cast<unsigned>(kTcRows)};
+  e = encode_tmap_3d_strided(&tx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xdims, xstr, xbox);
+  if (e != cudaSuccess) return e;
+  e = encode_tmap_3d(&tc, parts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, c_pad,
+                     static_cast<int>(bhn * 3), 64, n_tile);
+  if (e != cudaSuccess) return e;
+  const size_t smem = AssignSmem<D>::bytes(n_tile, c_pad);
+  e = cudaFuncSetAttribute(kmeans_assign_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const unsigned ctas = static_cast<unsigned>(bhn * ((cd.S + kTcRows - 1) / kTcRows));
+  kmeans_assign_tc_kernel<D><<<ctas, kTcThreads, smem, stream>>>(tx, tc, cd, n_tile, c_pad, norms,
+                                                                 labels, status);
+  return cudaGetLastError();
 }
 
 static cudaError_t layout_into(const ClusterDims& cd, const int32_t* labels, int32_t* counts,
@@ -420,23 +587,23 @@ cudaError_t launch_kmeans(const ClusterDims& cd, const void* x, int rounds, floa
   int32_t* tos = reinterpret_cast<int32_t*>(p);
   p += al256(static_cast<size_t>(bhn) * cd.S * 4);
   int32_t* sot = reinterpret_cast<int32_t*>(p);
+  p += al256(static_cast<size_t>(bhn) * cd.S * 4);
+  __nv_bfloat16* parts = reinterpret_cast<__nv_bfloat16*>(p);
+  p += al256(static_cast<size_t>(bhn) * 3 * assign_c_pad(cd.C) * cd.head_dim * 2);
+  float* norms = reinterpret_cast<float*>(p);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  const unsigned asg_ctas =
-      static_cast<unsigned>(bhn * ((cd.S + kAsgThreads * kAsgTokens - 1) / (kAsgThreads * kAsgTokens)));
   const unsigned upd_ctas = static_cast<unsigned>(bhn * cd.C);
   for (int r = 0; r < rounds; ++r) {
-    if (cd.head_dim == 128)
-      kmeans_assign_kernel<128><<<asg_ctas, kAsgThreads, 0, stream>>>(xb, cd, centroids, labels);
-    else
-      kmeans_assign_kernel<64><<<asg_ctas, kAsgThreads, 0, stream>>>(xb, cd, centroids, labels);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = cd.head_dim == 128
+                        ? launch_assign<128>(cd, x, centroids, parts, norms, labels, status, stream)
+                        : launch_assign<64>(cd, x, centroids, parts, norms, labels, status, stream);
     if (e != cudaSuccess) return e;
     e = layout_into(cd, labels, counts, starts, tos, sot, hist, status, stream);
     if (e != cudaSuccess) return e;
     if (cd.head_dim == 128)
-      kmeans_update_kernel<128><<<upd_ctas, 128, 0, stream>>>(cd, xb, tos, starts, counts, centroids);
+      kmeans_update_kernel<128><<<upd_ctas, 256, 0, stream>>>(cd, xb, tos, starts, counts, centroids);
     else
-      kmeans_update_kernel<64><<<upd_ctas, 64, 0, stream>>>(cd, xb, tos, starts, counts, centroids);
+      kmeans_update_kernel<64><<<upd_ctas, 256, 0, stream>>>(cd, xb, tos, starts, counts, centroids);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
