@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(256) kmeans_split_kernel(ClusterDims cd, int c
 }
 
 constexpr int kTcRows = 128;     // tokens per CTA = TMEM lanes
-constexpr int kTcStages = 3;     // centroid-part ring
+constexpr int kTcStages = 2;     // centroid-part ring (two stages: two CTAs fit an SM at n_tile 256)
 constexpr int kTcThreads = 160;  // warps 0-3: distances and argmin; warp 4: TMA + MMA
 
 template <int D>
@@ -87,13 +87,14 @@ struct AssignSmem {
 };
 
 // One CTA per (bh, 128 tokens).  The token tile is loaded once; the parts of each tile of
-// n_tile centroids stream through a 3-stage ring as (part, 64-dim chunk) steps, each step
+// n_tile centroids stream through a 2-stage ring as (part, 64-dim chunk) steps, each step
 // 4 MMAs of K = 16 into TMEM buffer (tile & 1); the epilogue warps reduce a finished buffer
-// while the next tile accumulates in the other.
+// while the next tile accumulates in the other.  The CTA allocates only the TMEM columns
+// it uses (tmem_cols), so CTAs overlap on an SM.
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1) kmeans_assign_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_c,
-    ClusterDims cd, int n_tile, int c_pad, const float* __restrict__ norms,
+    ClusterDims cd, int n_tile, int c_pad, uint32_t tmem_cols, const float* __restrict__ norms,
     int32_t* __restrict__ labels, uint32_t* status) {
   using L = AssignSmem<D>;
   constexpr int CH = L::kChunks;
@@ -137,7 +138,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) kmeans_assign_tc_kernel(
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < c_pad; i += kTcThreads) sn[i] = norms[static_cast<long long>(bh) * c_pad + i];
-  if (warp == 4) tmem_alloc(tmem_slot, 512);
+  if (warp == 4) tmem_alloc(tmem_slot, tmem_cols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -237,7 +238,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) kmeans_assign_tc_kernel(
   __syncthreads();
   if (warp == 4) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, tmem_cols);
   }
 }
 
@@ -374,18 +375,36 @@ __global__ void __launch_bounds__(256) kmeans_update_kernel(ClusterDims cd,
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  for (int i = lo; i < hi; ++i) {
-    const __nv_bfloat16* r = xb + tos[i] * row;
-    if constexpr (PER == 4) {
-      const uint2 w = *reinterpret_cast<const uint2*>(r);
-      acc[0] += __uint_as_float(w.x << 16);
-      acc[1] += __uint_as_float(w.x & 0xFFFF0000u);
-      acc[2] += __uint_as_float(w.y << 16);
-      acc[3] += __uint_as_float(w.y & 0xFFFF0000u);
-    } else {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(r);
-      acc[0] += __uint_as_float(w << 16);
-      acc[1] += __uint_as_float(w & 0xFFFF0000u);
+  // 8 tokens' loads in flight, then their adds in slot order (the same sums as one token
+  // at a time)
+  constexpr int kBatch = 8;
+  for (int i0 = lo; i0 < hi; i0 += kBatch) {
+    uint32_t w[kBatch][PER / 2];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u;
+      if (i < hi) {
+        const __nv_bfloat16* r = xb + tos[i] * row;
+        if constexpr (PER == 4) {
+          const uint2 v = *reinterpret_cast<const uint2*>(r);
+          w[u][0] = v.x;
+          w[u][1] = v.y;
+        } else {
+          w[u][0] = *reinterpret_cast<const uint32_t*>(r);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < PER / 2; ++e) w[u][e] = 0u;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (i0 + u >= hi) break;
+#pragma unroll
+      for (int e = 0; e < PER / 2; ++e) {
+        acc[2 * e] += __uint_as_float(w[u][e] << 16);
+        acc[2 * e + 1] += __uint_as_float(w[u][e] & 0xFFFF0000u);
+      }
     }
   }
 #pragma unroll
@@ -536,8 +555,13 @@ static cudaError_t launch_assign(const ClusterDims& cd, const void* x, const flo
                            static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const unsigned ctas = static_cast<unsigned>(bhn * ((cd.S + kTcRows - 1) / kTcRows));
-  kmeans_assign_tc_kernel<D><<<ctas, kTcThreads, smem, stream>>>(tx, tc, cd, n_tile, c_pad, norms,
-                                                                 labels, status);
+  // TMEM: one accumulator of n_tile columns, two when there are several centroid tiles,
+  // rounded up to a power of two, so several CTAs can share an SM's 512 columns.
+  const int need = (c_pad / n_tile > 1) ? 2 * n_tile : n_tile;
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(need)) cols <<= 1;
+  kmeans_assign_tc_kernel<D><<<ctas, kTcThreads, smem, stream>>>(tx, tc, cd, n_tile, c_pad, cols,
+                                                                 norms, labels, status);
   return cudaGetLastError();
 }
 
