@@ -47,6 +47,8 @@ def parse_args():
     ap.add_argument("--tau", type=float, default=0.99)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-sample-rows", type=int, default=256)
+    ap.add_argument("--clock-log", default=None,
+                    help="CSV of the nvidia-smi clock samples ({rank} is replaced); default /tmp")
     return ap.parse_args()
 
 
@@ -254,8 +256,9 @@ def run_ours(args, world, rank, local, pg):
     dense_flops_call = 4.0 * s.rows * s.n_kb * s.q_block * 64 * s.head_dim
 
     # timed region
-    clk = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")) \
-        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ClockSampler(local, f"/tmp/bsa_clocks_{rank}.csv")
+    clk_path = (args.clock_log.replace("{rank}", str(rank)) if args.clock_log
+                else f"/tmp/bsa_clocks_{rank}.csv")
+    clk = ClockSampler(local, clk_path)
     barrier(pg)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
