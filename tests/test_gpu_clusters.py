@@ -334,3 +334,54 @@ def test_kmeans_full_size_properties(B):
     t = tos2[0, 0].cpu().long()
     assert torch.equal(torch.sort(t).values, torch.arange(S))
     assert torch.equal(sot2[0, 0].cpu().long()[t], torch.arange(S))
+
+
+# ------------------------------------------------------------------ edge cases
+@pytest.mark.parametrize("S,C", [(1, 1), (5, 1), (7, 12), (63, 4), (130, 130)])
+def test_kmeans_edge_shapes(B, S, C):
+    """One token, one cluster, more clusters than tokens (empty ones keep their centroid)."""
+    D = 64
+    cs = B.ClusterShape(1, 2, D, S, C, C)
+    g = torch.Generator().manual_seed(S * 31 + C)
+    x = torch.randn((1, S, 2, D), generator=g).to(torch.bfloat16)
+    init = torch.randn((1, 2, C, D), generator=g)
+    cent, labels, counts = B.kmeans(x.cuda(), cs, C, init.clone().cuda(), 3)
+    xf = x.float().permute(0, 2, 1, 3).double().numpy()
+    for h in range(2):
+        lab, c, n = O.kmeans_lloyd(xf[0, h], init[0, h].double().numpy(), 3)
+        got = labels[0, h].cpu().numpy()
+        assert np.array_equal(counts[0, h].cpu().numpy(), np.bincount(got, minlength=C))
+        # labels: nearest within rounding (random data has no exact ties at these sizes)
+        assert (got == lab).mean() >= 0.99
+        if np.array_equal(got, lab):
+            np.testing.assert_allclose(_np(cent[0, h]), c, rtol=0, atol=2e-5)
+
+
+@pytest.mark.parametrize("S", [1, 40, 64, 65, 300])
+def test_cluster_fwd_edge_shapes(B, S):
+    """Runs shorter than a 64-key chunk, single-token clusters, a 300-row query cluster."""
+    D, Cq, Ck = 64, 3, 5
+    cs = B.ClusterShape(1, 1, D, S, Cq, Ck)
+    g = torch.Generator().manual_seed(S)
+    q, k, v = (torch.randn((1, 1, S, D), generator=g) for _ in range(3))
+    q, k, v = q * 2, k * 2, v * 0.25
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    one = 1 if S > 1 else 0
+    qn = torch.tensor([[[S - S // 10 - one, one, S // 10]]], dtype=torch.int32)   # 269 rows at S = 300
+    kn = torch.tensor([[[S // 2, 0, 1 if S > 1 else 0, S - S // 2 - (1 if S > 1 else 0) - min(S // 4, 1), min(S // 4, 1)]]],
+                      dtype=torch.int32)
+    assert int(qn.sum()) == S and int(kn.sum()) == S and bool((qn >= 0).all()) and bool((kn >= 0).all())
+    qs = (torch.cumsum(qn, -1) - qn).to(torch.int32)
+    ks = (torch.cumsum(kn, -1) - kn).to(torch.int32)
+    sel = [[0, 3], [1, 2, 4], [0, 1, 2, 3, 4]]
+    rp = torch.tensor([0] + list(np.cumsum([len(r) for r in sel])), dtype=torch.int32)
+    ci = torch.tensor([j for r in sel for j in r], dtype=torch.int32)
+    ws = B.new_cluster_fwd_workspace(cs)
+    out = B.cluster_fwd(q.cuda(), k.cuda(), v.cuda(), cs, qs.cuda(), qn.cuda(), ks.cuda(), kn.cuda(),
+                        rp.cuda(), ci.cuda(), ws=ws)
+    assert B.device_status(ws) == 0
+    ref = O.cluster_attention(q[0, 0].double().numpy(), k[0, 0].double().numpy(), v[0, 0].double().numpy(),
+                              qs[0, 0].numpy(), qn[0, 0].numpy(), ks[0, 0].numpy(), kn[0, 0].numpy(),
+                              rp.numpy(), ci.numpy(), 1.0 / math.sqrt(D))
+    e = Hp.attn_errors(_np(out[0, 0]), ref)
+    assert e["max_abs"] <= Hp.ATTN_MAX_ABS and e["mean_abs"] <= Hp.ATTN_MEAN_ABS, e
