@@ -513,6 +513,48 @@ def oracle_sample(wl, n_rows: int, seed: int = 0):
     return flops, dt, desc
 
 
+def oracle_units(wl, seed: int = 0):
+    """Per-unit times of the oracle's other steps on the workload (one head drawn on the
+    host, one thread), each with its unit count per call and a labelled extrapolation to
+    one call: a query-block row of masses, a top-p row, one tensor-head of the permute."""
+    import numpy as np
+    import torch
+    from threadpoolctl import threadpool_limits
+
+    from block_sparse_attention_25_b200 import synth
+    from oracle import bsa_oracle as O
+
+    g = O.Grid(wl.T, wl.H, wl.W, wl.Tp, wl.Hp, wl.Wp)
+    q, k, _ = synth.draw_qkv(wl.scaled(heads=1), device="cpu")
+    n_qb, n_kb = wl.Np // wl.q_block, wl.Np // 64
+    rows_per_call = wl.batch * wl.heads * n_qb
+    out = {}
+
+    def unit(seconds, per_call, what):
+        return {"unit": what, "ms_per_unit": round(1e3 * seconds, 3), "units_per_call": per_call,
+                "extrapolated_call_s": round(seconds * per_call, 1)}
+
+    with threadpool_limits(limits=1):
+        t = time.perf_counter()
+        qt = O.permute_forward(q.to(torch.float64).numpy(), g)
+        out["tile_permute"] = unit(time.perf_counter() - t, 3 * wl.batch * wl.heads,
+                                   "one tensor of one head")
+        kt = O.permute_forward(k.to(torch.float64).numpy(), g)
+        rng = np.random.default_rng(seed)
+        pick = rng.choice(n_qb, 2, replace=False)
+        t = time.perf_counter()
+        for i in pick:
+            O.block_mass_row(qt, kt, g, 0, 0, int(i), wl.q_block, 64, 1.0 / math.sqrt(wl.head_dim))
+        out["block_mass"] = unit((time.perf_counter() - t) / len(pick), rows_per_call,
+                                 "one query-block row of masses")
+        m = synth.draw_mass_rows(100, n_kb, seed=seed).double().numpy()
+        t = time.perf_counter()
+        for r in m:
+            O.topp_select_row(r, np.float32(0.99))
+        out["topp_select"] = unit((time.perf_counter() - t) / len(m), rows_per_call, "one row")
+    return out
+
+
 def run_reference(args, world, rank, pg):
     from block_sparse_attention_25_b200 import synth
     wl = synth.WORKLOADS[args.config]
@@ -558,10 +600,20 @@ def main():
     if rank == 0:
         from block_sparse_attention_25_b200 import synth
         wl = synth.WORKLOADS[args.config]
-        f, t, desc = oracle_sample(wl, args.cpu_sample_rows)
-        res["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s (executed, kept blocks)",
-                               "cores": 1, "kind": "oracle", "sample": desc,
-                               "seconds": round(t, 2)}
+        res["cpu_baseline"] = None
+        if world == 1:  # the oracle baseline is taken at N = 1 only
+            f, t, desc = oracle_sample(wl, args.cpu_sample_rows)
+            n_q = wl.batch * wl.heads * wl.S
+            units = oracle_units(wl)
+            units["attention"] = {"unit": "one query row", "ms_per_unit": round(1e3 * t / args.cpu_sample_rows, 3),
+                                  "units_per_call": n_q,
+                                  "extrapolated_call_s": round(t / args.cpu_sample_rows * n_q, 1)}
+            res["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s (executed, kept blocks)",
+                                   "cores": 1, "kind": "oracle", "sample": desc,
+                                   "seconds": round(t, 2),
+                                   "units": units,
+                                   "units_note": "per-unit oracle times; extrapolated_call_s is an "
+                                                 "extrapolation to one full call, not a measurement"}
         print(json.dumps(res), flush=True)
     if pg is not None:
         pg.destroy_process_group()

@@ -148,6 +148,17 @@ def main(argv=None):
              _time(lambda: B.bsattn_fwd(q8, k8, v8, row_ptr, col_idx, s, scales=scs, out=out_t, ws=ws_f),
                    args.iters), fl, "TFLOP/s", "tensor", 2 * pk["bf16"],
              {"kept_fraction": round(nnz / (R * nkb), 5)})
+    # the same kernel over full lists (every kv block): the dense-path time of the same call
+    frp = torch.empty(R + 1, dtype=torch.int32, device=dev)
+    fci = torch.empty(R * nkb, dtype=torch.int32, device=dev)
+    B.pattern_csr(s, B.PAT_VERTICAL_STRIPE, stripe_stride=1, ws=ws_pt, row_ptr=frp, col_idx=fci,
+                  device=dev)
+    sparse_ms = _time(lambda: B.bsattn_fwd(qt, kt, vt, row_ptr, col_idx, s, out=out_t, ws=ws_f), args.iters)
+    dense_ms = _time(lambda: B.bsattn_fwd(qt, kt, vt, frp, fci, s, out=out_t, ws=ws_f), args.iters)
+    line("bsattn_fwd_full_lists", dense_ms, 4.0 * R * nkb * s.q_block * 64 * D, "TFLOP/s", "tensor",
+         pk["bf16"], {"kept_fraction": 1.0,
+                      "speedup_of_selected_lists": round(dense_ms / sparse_ms, 4)})
+    del frp, fci
     # structured lists through the same attention kernel
     pfl = 4.0 * pnnz * s.q_block * 64 * D
     line("bsattn_fwd_pattern", _time(lambda: B.bsattn_fwd(qt, kt, vt, prp, pci, s, out=out_t, ws=ws_f),
