@@ -174,7 +174,7 @@ def _cluster_case(B, Bt, Hh, S, D, Cq, Ck, seed, keep_prob, sharp):
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("keep_prob,sharp", [(1.0, 1.0), (0.3, 3.0), (0.05, 3.0)])
 def test_cluster_fwd_parity(B, D, keep_prob, sharp):
-    Bt, Hh, S, Cq, Ck = 1, 2, 1500, 9, 23
+    Bt, Hh, S, Cq, Ck = 2, 2, 1500, 9, 23
     cs, q, k, v, qs, qn, ks, kn, rp, ci = _cluster_case(B, Bt, Hh, S, D, Cq, Ck, 40 + D, keep_prob, sharp)
     dev = lambda t: t.cuda()
     ws = B.new_cluster_fwd_workspace(cs)
