@@ -151,6 +151,7 @@ def lib() -> ctypes.CDLL:
         "bsa_cluster_mass": (I, [CSP, P, P, P, P, F, P, P]),
         "bsa_topp_select_rows": (I, [P, L64, I, F, P, P, L64, P, S, P]),
         "bsa_cluster_fwd": (I, [CSP, P, P, P, P, P, P, P, P, P, F, P, P, P, S, P]),
+        "bsa_selftest_wait": (I, [P, S, L64, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -167,7 +168,7 @@ EXPORTED_SYMBOLS = ("bsa_workspace_bytes", "bsa_clear_status", "bsa_device_statu
                     "bsa_pooled_mass", "bsa_version", "bsa_kmeans_workspace_bytes",
                     "bsa_cluster_fwd_workspace_bytes", "bsa_topp_rows_workspace_bytes",
                     "bsa_kmeans", "bsa_cluster_layout", "bsa_cluster_permute", "bsa_cluster_mass",
-                    "bsa_topp_select_rows", "bsa_cluster_fwd")
+                    "bsa_topp_select_rows", "bsa_cluster_fwd", "bsa_selftest_wait")
 
 
 def _check(status: int, what: str):
@@ -543,3 +544,14 @@ def cluster_fwd(q, k, v, cs: ClusterShape, q_starts, q_counts, k_starts, k_count
                                  _ptr(col_idx), scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                  _stream(stream)), "bsa_cluster_fwd")
     return (out, lse) if want_lse else out
+
+
+def selftest_wait(ws, limit_ns: int = 20_000_000, stream=None):
+    """bsa_selftest_wait: a bounded wait that must give up (see include/bsattn.h).
+    Returns the status header words after the kernel: (flags, detail, ...) and the three
+    result words (first wait completed, second wait completed, abort flag seen)."""
+    _check(lib().bsa_selftest_wait(_ptr(ws), ws.numel(), int(limit_ns), _stream(stream)),
+           "bsa_selftest_wait")
+    torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+    words = ws[:64].view(torch.int32).cpu().tolist()
+    return words[:4], words[8:11]

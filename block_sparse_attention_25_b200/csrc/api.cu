@@ -525,4 +525,11 @@ bsa_status bsa_cluster_fwd(const bsa_cluster_shape* shape, const void* q, const 
                                            out, lse, ws, stream));
 }
 
+
+bsa_status bsa_selftest_wait(void* ws, size_t ws_bytes, int64_t limit_ns, bsa_stream_t stream) {
+  if (ws == nullptr || !bsa::aligned16(ws) || ws_bytes < bsa::kStatusBytes) return BSA_ERR_INVALID_ARG;
+  if (limit_ns < 1000 || limit_ns > 10000000000LL) return BSA_ERR_INVALID_ARG;
+  return from_cuda(bsa::launch_selftest_wait(ws, static_cast<uint64_t>(limit_ns), stream));
+}
+
 }  // extern "C"

@@ -30,6 +30,7 @@ enum : uint32_t {
   DETAIL_WAIT_S_FULL = 0x105,
   DETAIL_WAIT_P_FULL = 0x106,
   DETAIL_WAIT_O_FULL = 0x107,
+  DETAIL_SELFTEST = 0x1FF,
   DETAIL_MASS_VALUE = 0x200,
   DETAIL_CSR_RANGE = 0x201,
   DETAIL_CSR_ORDER = 0x202,
@@ -110,11 +111,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 // wait inside one CTA lasts more than microseconds.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// Wait for the phase with the given parity to complete.  Gives up after kWaitLimitNs or
-// as soon as another warp of the CTA has raised *abort; returns false then (and records
-// a TIMEOUT in the status header on the first give-up).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* status, uint32_t detail) {
+// Wait for the phase with the given parity to complete.  Gives up after limit_ns or as
+// soon as another warp of the CTA has raised *abort; returns false then (and records a
+// TIMEOUT in the status header on the first give-up, raising *abort for the others).
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              uint32_t* status, uint32_t detail, uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -123,13 +124,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(a, parity)) return true;
     if ((++spins & 63u) == 0u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         record_status(status, FLAG_TIMEOUT, detail, blockIdx.x, threadIdx.x);
         return false;
       }
     }
   }
+}
+
+// The pipeline wait of every kernel: limit kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint32_t* status, uint32_t detail) {
+  return mbar_wait_for(bar, parity, abort, status, detail, kWaitLimitNs);
 }
 
 // Same, but ignores the abort flag: used to drain in-flight tensor-core work before the

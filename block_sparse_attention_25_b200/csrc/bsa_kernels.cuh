@@ -180,6 +180,9 @@ cudaError_t launch_cluster_fwd(int batch, int heads, int head_dim, int S, int n_
                                float softmax_scale, void* out, float* lse, void* ws,
                                cudaStream_t stream);
 
+// Failure-detection self-test (bounded wait on a barrier nothing completes).
+cudaError_t launch_selftest_wait(void* ws, uint64_t limit_ns, cudaStream_t stream);
+
 // Encode a rank-3 bf16/e4m3 tensor map over [bh][Np][D] with a (box_d x box_rows x 1) box
 // and 128-byte swizzle.
 cudaError_t encode_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,

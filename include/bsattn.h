@@ -329,6 +329,19 @@ BSA_API bsa_status bsa_cluster_fwd(const bsa_cluster_shape* shape, const void* q
                                    float softmax_scale, void* out, float* lse, void* ws,
                                    size_t ws_bytes, bsa_stream_t stream);
 
+/* Self-test of the failure detection every pipelined kernel relies on.  Launches one
+ * small CTA in which one thread waits on a shared-memory barrier that nothing ever
+ * completes, with the same bounded wait the kernels use but a limit of limit_ns
+ * (1e3 .. 1e10 ns): the wait gives up, records TIMEOUT (detail 0x1FF) in the status
+ * header of ws and raises the CTA's abort flag; a second warp waiting on the same barrier
+ * with a longer limit then gives up through the abort flag.  Nothing faults or hangs: the
+ * kernel ends by itself after ~limit_ns and the context stays usable.  Words 8..10 of the
+ * header receive (first wait completed?, second wait completed?, abort flag seen), so a
+ * healthy run reads TIMEOUT from bsa_device_status and (0, 0, 1) there.  ws: >= 256
+ * bytes, 16-byte aligned. */
+BSA_API bsa_status bsa_selftest_wait(void* ws, size_t ws_bytes, int64_t limit_ns,
+                                     bsa_stream_t stream);
+
 /* Library build identification (static string). */
 BSA_API const char* bsa_version(void);
 

@@ -189,6 +189,18 @@ def test_cluster_rejections_before_launch(B):
     assert L.bsa_cluster_fwd(cs(head_dim=32), *args, big, n) == 2
 
 
+def test_selftest_rejections_before_launch(B):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("fake-pointer validation checks run on hosts without a GPU only")
+    L = B.lib()
+    assert L.bsa_selftest_wait(None, 256, 1000000, None) == 1
+    assert L.bsa_selftest_wait(FAKE, 100, 1000000, None) == 1           # header does not fit
+    assert L.bsa_selftest_wait(MISALIGNED, 256, 1000000, None) == 1
+    assert L.bsa_selftest_wait(FAKE, 256, 10, None) == 1                # limit below 1 us
+    assert L.bsa_selftest_wait(FAKE, 256, 10**11, None) == 1            # above 10 s
+
+
 def test_status_strings(B):
     L = B.lib()
     for code in range(7):
