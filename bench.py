@@ -5,13 +5,16 @@
 A step is one calibrate-then-reuse cycle of the 720p workload (the default config,
 Wan-14B-like: B=1, 40 heads, D=128, 21x45x80 tokens padded to 24x48x80, 64-token blocks):
     calibration  tile_permute(Q, K) -> block_mass -> topp_select(0.99)
-    10 x reuse   tile_permute(Q_r, K_r, V_r) -> bsattn_fwd(frozen lists) -> inverse permute
+    10 x reuse   bsattn_fwd_raster(Q_r, K_r, V_r, frozen lists): raster in, raster out, the
+                 tile permutation fused into the forward's loads and stores
+                 (--layout tiles: tile_permute x3 -> bsattn_fwd -> inverse permute; the
+                 e4m3 workload always takes tile_permute_quant_e4m3 x3 -> bsattn_fwd -> inverse)
 on seeded synthetic inputs already resident in HBM (Q/K/V of 774 MB each, far above L2).
 
 value  = executed attention TFLOP/s of the whole step: FLOPs of the kept blocks of the 10
          reuse calls (4 * 64 * 64 * D per kept (query block, kv block) pair) divided by
          the device time of the whole cycle, max over ranks.
-fwd    = the same FLOPs over the bsattn_fwd launches alone (CUDA events on the launch
+fwd    = the same FLOPs over the forward launches alone (CUDA events on the launch
          stream) -> roofline of the dominant kernel.
 e2e    = the same metric through the public API with inputs copied from pinned host
          memory and outputs copied back inside the timed region.
@@ -46,6 +49,8 @@ def parse_args():
     ap.add_argument("--reuse", type=int, default=None, help="reuse calls per step (default: the workload's)")
     ap.add_argument("--tau", type=float, default=0.99)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layout", default="raster", choices=["raster", "tiles"],
+                    help="bf16 reuse calls: fused raster forward, or permute + tile-major forward")
     ap.add_argument("--cpu-sample-rows", type=int, default=256)
     ap.add_argument("--clock-log", default=None,
                     help="CSV of the nvidia-smi clock samples ({rank} is replaced); default /tmp")
@@ -61,14 +66,16 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
 
 
-def measured_traffic(fp8: bool):
-    """DRAM bytes per bsattn_fwd launch from the committed full-size ncu capture, or None when
-    the kernel sources have changed since it was taken (or for a variant not captured)."""
+def measured_traffic(fp8: bool, raster: bool):
+    """DRAM bytes per forward launch from the committed full-size ncu capture of the variant
+    the bench times, or None when the kernel sources have changed since it was taken (or for
+    a variant not captured)."""
     if fp8:
         return None
     import hashlib
     import re
-    path = os.path.join(ROOT, "profiles", "bsattn_fwd_wan14b_720p_dram.md")
+    name = "bsattn_fwd_raster_wan14b_720p_dram.md" if raster else "bsattn_fwd_wan14b_720p_dram.md"
+    path = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -174,6 +181,7 @@ def run_ours(args, world, rank, local, pg):
     n_reuse = args.reuse if args.reuse is not None else max(wl.redraws, 1)
     s = bsa.Shape.of(wl)
     fp8 = wl.fp8
+    raster = not fp8 and args.layout == "raster"
     seed_wl = wl.scaled(seed=wl.seed + 7919 * rank)  # independent problem per rank
 
     # ---- inputs resident in HBM: the calibration draw and n_reuse correlated re-draws
@@ -227,6 +235,14 @@ def run_ours(args, world, rank, local, pg):
                 if time_fwd:
                     fwd_ev[cur["step"]][r][0].record(stream)
                 bsa.bsattn_fwd(q8, k8, v8, row_ptr, col_idx, s, scales=sc, out=out_t, ws=ws_f)
+            elif raster:
+                if time_fwd:
+                    fwd_ev[cur["step"]][r][0].record(stream)
+                bsa.bsattn_fwd_raster(q, k, v, row_ptr, col_idx, s, out=out_r[r], ws=ws_f)
+                if time_fwd:
+                    fwd_ev[cur["step"]][r][1].record(stream)
+                n += 1 + s.batch  # schedule + one forward launch per batch
+                continue
             else:
                 bsa.tile_permute(q, s, out=qt)
                 bsa.tile_permute(k, s, out=kt)
@@ -294,7 +310,7 @@ def run_ours(args, world, rank, local, pg):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, bsa, s, draws, n_reuse, row_ptr, col_idx, flops_call, dev, stream,
-                      fp8, pg, world)
+                      fp8, raster, pg, world)
 
     result = {
         "metric": "bsattn_fwd ms/call & executed TFLOPS at 99% retained mass, % of bf16 peak",
@@ -315,6 +331,8 @@ def run_ours(args, world, rank, local, pg):
             "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
             "q_block": wl.q_block, "kv_block": 64, "tokens": wl.S, "slots": wl.Np,
             "threshold": args.tau, "reuse_calls_per_step": n_reuse,
+            "layout": "raster (permutation fused into the forward)" if raster
+                      else "tile-major (separate permutation launches)",
             "kept_fraction": round(kept_frac, 5),
             "bsattn_fwd_ms_per_call": round(fwd_avg_ms, 3),
             "bsattn_fwd_tflops": round(fwd_tflops, 2),
@@ -328,10 +346,11 @@ def run_ours(args, world, rank, local, pg):
         "roofline": {
             "bound": "tensor", "achieved": round(fwd_tflops, 2), "peak": peak, "unit": "TFLOP/s",
             "frac": round(fwd_tflops / peak, 4),
-            "traffic": (measured_traffic(fp8) if wl.name == synth.WORKLOADS["wan14b_720p"].name
-                        else None),
+            "traffic": (measured_traffic(fp8, raster)
+                        if wl.name == synth.WORKLOADS["wan14b_720p"].name else None),
             "traffic_unit": "bytes per launch (dram read + write, one full-size ncu capture)",
-            "kernel": f"bsattn_fwd_kernel<{s.head_dim},{'true' if fp8 else 'false'}>",
+            "kernel": (f"bsattn_fwd_kernel<{s.head_dim},false,false,true> (raster layout)" if raster
+                       else f"bsattn_fwd_kernel<{s.head_dim},{'true' if fp8 else 'false'},false,false>"),
             "peak_source": peak_note,
         },
         "gpu_launches": launches_per_step * args.steps,
@@ -342,8 +361,8 @@ def run_ours(args, world, rank, local, pg):
     return result
 
 
-def run_e2e(args, bsa, s, draws, n_reuse, row_ptr, col_idx, flops_call, dev, stream, fp8, pg,
-            world):
+def run_e2e(args, bsa, s, draws, n_reuse, row_ptr, col_idx, flops_call, dev, stream, fp8, fused,
+            pg, world):
     """Same cycle through the public API, every input copied in from pinned host memory and
     every output copied back, inside the timed region.  The copies run on two copy streams
     and overlap the compute: the inputs of the next call land in the second of two device
@@ -409,6 +428,21 @@ def run_e2e(args, bsa, s, draws, n_reuse, row_ptr, col_idx, flops_call, dev, str
             state["set_free"][st] = e
             bsa.block_mass(qt, kt, s, out=mass, ws=ws_m)
             bsa.topp_select(mass, s, args.tau, ws=ws_t, row_ptr=rp, col_idx=ci)
+            return
+        if fused:  # the forward reads the raster set and writes the output buffer directly
+            if state["out_free"][st] is not None:
+                stream.wait_event(state["out_free"][st])
+            bsa.bsattn_fwd_raster(dq, dk, dv, rp, ci, s, out=outs[st], ws=ws_f)
+            e = ev()
+            e.record(stream)
+            state["set_free"][st] = e
+            down.wait_event(e)
+            with torch.cuda.stream(down):
+                out_host[job - 1].copy_(outs[st], non_blocking=True)
+                e = ev()
+                e.record(down)
+            state["out_free"][st] = e
+            counts["d2h"] += raster.numel() * 2
             return
         if fp8:
             bsa.tile_permute_quant_e4m3(dq, s, out=q8, scales=sc[0])

@@ -152,6 +152,7 @@ def lib() -> ctypes.CDLL:
         "bsa_topp_select_rows": (I, [P, L64, I, F, P, P, L64, P, S, P]),
         "bsa_cluster_fwd": (I, [CSP, P, P, P, P, P, P, P, P, P, F, P, P, P, S, P]),
         "bsa_selftest_wait": (I, [P, S, L64, P]),
+        "bsa_fwd_raster": (I, [SP, P, P, P, P, P, F, P, P, P, S, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -168,7 +169,8 @@ EXPORTED_SYMBOLS = ("bsa_workspace_bytes", "bsa_clear_status", "bsa_device_statu
                     "bsa_pooled_mass", "bsa_version", "bsa_kmeans_workspace_bytes",
                     "bsa_cluster_fwd_workspace_bytes", "bsa_topp_rows_workspace_bytes",
                     "bsa_kmeans", "bsa_cluster_layout", "bsa_cluster_permute", "bsa_cluster_mass",
-                    "bsa_topp_select_rows", "bsa_cluster_fwd", "bsa_selftest_wait")
+                    "bsa_topp_select_rows", "bsa_cluster_fwd", "bsa_selftest_wait",
+                    "bsa_fwd_raster")
 
 
 def _check(status: int, what: str):
@@ -372,6 +374,29 @@ def pattern_csr(shape: Shape, kinds: int, diag_width=0, multi_count=0, multi_per
                                  _ptr(col_idx), cap, _ptr(ws), ws.numel(), _stream(stream)),
            "bsa_pattern_csr")
     return row_ptr, col_idx
+
+
+def bsattn_fwd_raster(q, k, v, row_ptr, col_idx, shape: Shape, softmax_scale=None,
+                      want_lse=False, out=None, lse=None, ws=None, stream=None):
+    """bsa_fwd_raster: block-sparse attention on raster bf16 [B, S, Hh, D] (the tile
+    permutation fused into the kernel).  Returns out (raster) or (out, lse [B, Hh, S])."""
+    raster = (shape.batch, shape.S, shape.heads, shape.head_dim)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, raster, n)
+    _need(row_ptr, torch.int32, (shape.rows + 1,), "row_ptr")
+    if col_idx.dtype != torch.int32 or not col_idx.is_cuda:
+        raise TypeError("col_idx: int32 CUDA tensor")
+    if out is None:
+        out = torch.empty(raster, dtype=torch.bfloat16, device=q.device)
+    if want_lse and lse is None:
+        lse = torch.empty((shape.batch, shape.heads, shape.S), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = new_workspace(shape, OP_FWD, q.device)
+    scale = default_scale(shape) if softmax_scale is None else float(softmax_scale)
+    _check(lib().bsa_fwd_raster(ctypes.byref(shape.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
+                                _ptr(col_idx), scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                _stream(stream)), "bsa_fwd_raster")
+    return (out, lse) if want_lse else out
 
 
 def bsattn_fwd(q, k, v, row_ptr, col_idx, shape: Shape, softmax_scale=None, scales=None,

@@ -65,6 +65,26 @@ cudaError_t encode_tmap_3d_strided(CUtensorMap* map, const void* base, CUtensorM
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Raster tokens [S = T*H*W][Hh][D] of one batch as a 5D map (D, Hh, W, H, T) with a
+// (64, 1, 4, 4, 4) box: one box is one 4x4x4 tile of one head, 64 rows of 64 elements in
+// (t, h, w) row-major order, coordinates past (W, H, T) read as zeros.
+cudaError_t encode_tmap_raster_tiles(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                                     int elem_bytes, int D, int heads, int W, int H, int T) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return cudaErrorInitializationError;
+  const cuuint64_t row = static_cast<cuuint64_t>(D) * elem_bytes;
+  const cuuint64_t dims[5] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[4] = {row, row * heads, row * heads * W, row * heads * W * H};
+  const cuuint32_t box[5] = {static_cast<cuuint32_t>(128 / elem_bytes), 1u, 4u, 4u, 4u};
+  const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+  const CUresult r = fn(map, dtype, 5, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace bsa
 
 using bsa::AttnDims;
@@ -530,6 +550,27 @@ bsa_status bsa_selftest_wait(void* ws, size_t ws_bytes, int64_t limit_ns, bsa_st
   if (ws == nullptr || !bsa::aligned16(ws) || ws_bytes < bsa::kStatusBytes) return BSA_ERR_INVALID_ARG;
   if (limit_ns < 1000 || limit_ns > 10000000000LL) return BSA_ERR_INVALID_ARG;
   return from_cuda(bsa::launch_selftest_wait(ws, static_cast<uint64_t>(limit_ns), stream));
+}
+
+
+bsa_status bsa_fwd_raster(const bsa_shape* shape, const void* q, const void* k, const void* v,
+                          const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale,
+                          void* out, float* lse, void* ws, size_t ws_bytes, bsa_stream_t stream) {
+  bsa_status st = check_shape(shape, true);
+  if (st != BSA_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || row_ptr == nullptr ||
+      col_idx == nullptr || ws == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (!bsa::aligned16(q) || !bsa::aligned16(k) || !bsa::aligned16(v) || !bsa::aligned16(out) ||
+      !bsa::aligned16(ws) || (reinterpret_cast<uintptr_t>(row_ptr) & 3u) ||
+      (reinterpret_cast<uintptr_t>(col_idx) & 3u) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return BSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f)) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_bytes(shape, BSA_OP_FWD)) return BSA_ERR_CAPACITY;
+  const AttnDims a = make_attn(shape);
+  return from_cuda(bsa::launch_bsattn_fwd_raster(a, q, k, v, row_ptr, col_idx, softmax_scale, out,
+                                                 lse, ws, stream));
 }
 
 }  // extern "C"

@@ -157,6 +157,9 @@ struct FwdParams {
   const int32_t* q_counts;
   const int32_t* cta_base;   // [bh][n_qc + 1]
   const int32_t* ent_counts; // [bh][n_qc]
+  // raster layout only: the batch of this launch and its first CTA (one launch per batch)
+  int raster_b;
+  int cta_offset;
 };
 
 // Shared-memory plan.  Every operand row is cut into 128-byte swizzle chunks (64 bf16 or
@@ -183,7 +186,7 @@ struct FwdSmem {
 // largest code is 256 * 1.75 = 448, the e4m3 maximum.
 constexpr float kPScale = 1.75f;
 
-template <int D, bool FP8, bool VARLEN>
+template <int D, bool FP8, bool VARLEN, bool RASTER = false>
 __global__ void __launch_bounds__(fwd::kThreads, 1)
     bsattn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -210,7 +213,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   const AttnDims& a = p.a;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int cta = blockIdx.x;
+  const int cta = blockIdx.x + (RASTER ? p.cta_offset : 0);
   int bh, row0, n_ent, rows_here;
   const uint32_t* ent;
   if constexpr (VARLEN) {
@@ -271,6 +274,16 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Raster layout: tile u of head h as one 5D box (dims, head, w, h, t) of this batch's
+  // tensor map; tiles past the padded grid and slots past the valid grid read as zeros.
+  const int head = bh - (bh / a.heads) * a.heads;
+  auto raster_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int ch, int u) {
+    const int tw = u % a.g.ntw;
+    const int rest = u / a.g.ntw;
+    const int th = rest % a.g.nth;
+    const int tt = rest / a.g.nth;
+    tma_load_5d(dst, map, bar, ch * CE, head, tw * 4, th * 4, tt * 4);
+  };
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && nsteps > 0) {
@@ -279,9 +292,15 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       prefetch_tensormap(&tm_v);
       mbar_arrive_expect_tx(bar_q, 2 * L::kQTile);
       for (int t = 0; t < 2; ++t)
-        for (int ch = 0; ch < L::kChunks; ++ch)
-          tma_load_3d(smem + L::kQOff + t * L::kQTile + ch * (128 * 128), &tm_q, bar_q, ch * CE,
-                      row0 + t * 128, bh);
+        for (int ch = 0; ch < L::kChunks; ++ch) {
+          uint8_t* dq = smem + L::kQOff + t * L::kQTile + ch * (128 * 128);
+          if constexpr (RASTER) {  // a 128-row Q tile is two 4x4x4 tiles
+            raster_tile(dq, &tm_q, bar_q, ch, (row0 + t * 128) >> 6);
+            raster_tile(dq + 64 * 128, &tm_q, bar_q, ch, ((row0 + t * 128) >> 6) + 1);
+          } else {
+            tma_load_3d(dq, &tm_q, bar_q, ch * CE, row0 + t * 128, bh);
+          }
+        }
       for (int s = 0; s < nsteps; ++s) {
         const int nb = (2 * s + 1 < n_ent) ? 2 : 1;
         // first key row of each of the step's (one or two) 64-row boxes
@@ -296,10 +315,15 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         mbar_arrive_expect_tx(bar_kfull + ks, nb * 64 * L::kRowBytes);
         uint8_t* kst = smem + L::kKOff + ks * L::kKVStage;
         for (int ch = 0; ch < L::kChunks; ++ch) {
-          tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * CE, j0, bh);
-          if (nb == 2)
-            tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * CE,
-                        j1, bh);
+          if constexpr (RASTER) {
+            raster_tile(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch, j0 >> 6);
+            if (nb == 2) raster_tile(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch, j1 >> 6);
+          } else {
+            tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * CE, j0, bh);
+            if (nb == 2)
+              tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * CE,
+                          j1, bh);
+          }
         }
         const int vs = s % VS;
         if (s >= VS && !mbar_wait(bar_vempty + vs, ((s / VS) - 1) & 1, abort_flag, p.status,
@@ -308,10 +332,15 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         mbar_arrive_expect_tx(bar_vfull + vs, nb * 64 * L::kRowBytes);
         uint8_t* vst = smem + L::kVOff + vs * L::kKVStage;
         for (int ch = 0; ch < L::kChunks; ++ch) {
-          tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * CE, j0, bh);
-          if (nb == 2)
-            tma_load_3d(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch * CE,
-                        j1, bh);
+          if constexpr (RASTER) {
+            raster_tile(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch, j0 >> 6);
+            if (nb == 2) raster_tile(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch, j1 >> 6);
+          } else {
+            tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * CE, j0, bh);
+            if (nb == 2)
+              tma_load_3d(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch * CE,
+                          j1, bh);
+          }
         }
       }
     }
@@ -422,7 +451,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     const int slot = row0 + local;     // query slot inside the head
     const int qsel = VARLEN ? 0 : local / a.q_block;
     // in_range: the row is this CTA's to write; q_valid: it holds a token
-    const bool in_range = VARLEN ? local < rows_here : slot < a.g.Np;
+    // raster layout: the token a slot holds (-1 for a pad slot); only tokens are written
+    const int token = (RASTER && slot < a.g.Np) ? slot_to_token(a.g, slot) : -1;
+    const bool in_range = VARLEN ? local < rows_here : (RASTER ? token >= 0 : slot < a.g.Np);
     const bool q_valid = VARLEN ? in_range : (in_range && slot_valid(a.g, slot));
     const long long head_slots = VARLEN ? p.S : a.g.Np;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
@@ -586,7 +617,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
                           mbar_wait(bar_ofull, 0, abort_flag, p.status, DETAIL_WAIT_O_FULL));
       tc_fence_after();
     }
-    __nv_bfloat16* orow = p.out + (static_cast<long long>(bh) * head_slots + slot) * D;
+    __nv_bfloat16* orow =
+        RASTER ? p.out + ((static_cast<long long>(p.raster_b) * a.g.S + (token < 0 ? 0 : token)) *
+                              a.heads + head) * D
+               : p.out + (static_cast<long long>(bh) * head_slots + slot) * D;
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       float ov[32];
@@ -610,7 +644,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     if (p.lse != nullptr && in_range) {
       const float lse = (l_run > 0.f && q_valid) ? (m_run + __log2f(l_run)) * 0.6931471805599453f
                                                  : -INFINITY;
-      p.lse[static_cast<long long>(bh) * head_slots + slot] = lse;
+      if constexpr (RASTER)
+        p.lse[static_cast<long long>(bh) * a.g.S + token] = lse;
+      else
+        p.lse[static_cast<long long>(bh) * head_slots + slot] = lse;
     }
   }
 
@@ -690,9 +727,75 @@ cudaError_t launch_bsattn_fwd(const AttnDims& a, int fp8, const void* q, const v
   prm.cap = 0;
   prm.max_ent = 0;
   prm.q_starts = prm.q_counts = prm.cta_base = prm.ent_counts = nullptr;
+  prm.raster_b = 0;
+  prm.cta_offset = 0;
   if (fp8) return launch_fwd<128, true, false>(a, a.g.Np, q, k, v, prm, ctas, stream);
   if (a.head_dim == 128) return launch_fwd<128, false, false>(a, a.g.Np, q, k, v, prm, ctas, stream);
   return launch_fwd<64, false, false>(a, a.g.Np, q, k, v, prm, ctas, stream);
+}
+
+// ---------------------------------------------------------------------------------------
+// Raster layout: Q, K, V and O are [B, S, Hh, D] bf16 in token order.  The kernel loads each
+// 4x4x4 tile with one 5D TMA box (whose shared-memory image is the tile-major block) and
+// writes each query row to its token; the lists, schedule and arithmetic are those of
+// bsa_fwd, so the result equals bsa_fwd on tile-permuted inputs, permuted back.
+template <int D>
+static cudaError_t launch_fwd_raster(const AttnDims& a, const void* q, const void* k,
+                                     const void* v, FwdParams prm, cudaStream_t stream) {
+  using L = FwdSmem<D, false>;
+  cudaError_t e = cudaFuncSetAttribute(bsattn_fwd_kernel<D, false, false, true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  const long long per_batch = static_cast<long long>(a.g.S) * a.heads * D;  // elements
+  for (int b = 0; b < a.batch; ++b) {  // 5D maps cover one batch
+    CUtensorMap tq, tk, tv;
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q) + b * per_batch;
+    const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k) + b * per_batch;
+    const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(v) + b * per_batch;
+    e = encode_tmap_raster_tiles(&tq, qb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.heads, a.g.W,
+                                 a.g.H, a.g.T);
+    if (e != cudaSuccess) return e;
+    e = encode_tmap_raster_tiles(&tk, kb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.heads, a.g.W,
+                                 a.g.H, a.g.T);
+    if (e != cudaSuccess) return e;
+    e = encode_tmap_raster_tiles(&tv, vb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.heads, a.g.W,
+                                 a.g.H, a.g.T);
+    if (e != cudaSuccess) return e;
+    prm.raster_b = b;
+    prm.cta_offset = b * a.heads * a.n_cta_per_head;
+    const unsigned ctas = static_cast<unsigned>(a.heads * a.n_cta_per_head);
+    bsattn_fwd_kernel<D, false, false, true><<<ctas, fwd::kThreads, L::kAlloc, stream>>>(tq, tk, tv, prm);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_bsattn_fwd_raster(const AttnDims& a, const void* q, const void* k,
+                                     const void* v, const int32_t* row_ptr, const int32_t* col_idx,
+                                     float softmax_scale, void* out, float* lse, void* ws,
+                                     cudaStream_t stream) {
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base);
+  const long long ctas = static_cast<long long>(a.batch) * a.heads * a.n_cta_per_head;
+  if (ctas == 0) return cudaSuccess;
+  const size_t counts_bytes = (static_cast<size_t>(ctas) * 4 + 255) & ~static_cast<size_t>(255);
+  int32_t* counts = reinterpret_cast<int32_t*>(base + kStatusBytes);
+  uint32_t* entries = reinterpret_cast<uint32_t*>(base + kStatusBytes + 2 * counts_bytes);
+  bsattn_schedule_kernel<<<static_cast<unsigned>(ctas), 256, 0, stream>>>(
+      a, row_ptr, col_idx, counts, entries, nullptr, nullptr, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  FwdParams prm{};
+  prm.a = a;
+  prm.counts = counts;
+  prm.entries = entries;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.status = status;
+  prm.scale_log2 = softmax_scale * 1.4426950408889634f;
+  if (a.head_dim == 128) return launch_fwd_raster<128>(a, q, k, v, prm, stream);
+  return launch_fwd_raster<64>(a, q, k, v, prm, stream);
 }
 
 // ---------------------------------------------------------------------------------------

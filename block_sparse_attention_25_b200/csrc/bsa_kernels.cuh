@@ -180,6 +180,15 @@ cudaError_t launch_cluster_fwd(int batch, int heads, int head_dim, int S, int n_
                                float softmax_scale, void* out, float* lse, void* ws,
                                cudaStream_t stream);
 
+// Raster tokens of one batch as 4x4x4-tile boxes (see api.cu).
+cudaError_t encode_tmap_raster_tiles(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                                     int elem_bytes, int D, int heads, int W, int H, int T);
+// Block-sparse forward reading Q/K/V from and writing O to the raster layout.
+cudaError_t launch_bsattn_fwd_raster(const AttnDims& a, const void* q, const void* k,
+                                     const void* v, const int32_t* row_ptr, const int32_t* col_idx,
+                                     float softmax_scale, void* out, float* lse, void* ws,
+                                     cudaStream_t stream);
+
 // Failure-detection self-test (bounded wait on a barrier nothing completes).
 cudaError_t launch_selftest_wait(void* ws, uint64_t limit_ns, cudaStream_t stream);
 

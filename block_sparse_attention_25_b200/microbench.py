@@ -138,6 +138,13 @@ def main(argv=None):
     line("bsattn_fwd", _time(lambda: B.bsattn_fwd(qt, kt, vt, row_ptr, col_idx, s, out=out_t, ws=ws_f),
                              args.iters), fl, "TFLOP/s", "tensor", pk["bf16"],
          {"kept_fraction": round(nnz / (R * nkb), 5)})
+    # the permutation fused into the forward: raster in, raster out
+    out_r = torch.empty_like(q)
+    line("bsattn_fwd_raster",
+         _time(lambda: B.bsattn_fwd_raster(q, k, v, row_ptr, col_idx, s, out=out_r, ws=ws_f),
+               args.iters), fl, "TFLOP/s", "tensor", pk["bf16"],
+         {"kept_fraction": round(nnz / (R * nkb), 5)})
+    del out_r
     if D == 128:
         k8, v8 = torch.empty_like(q8), torch.empty_like(q8)
         scs = [sc, torch.empty_like(sc), torch.empty_like(sc)]

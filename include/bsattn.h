@@ -342,6 +342,19 @@ BSA_API bsa_status bsa_cluster_fwd(const bsa_cluster_shape* shape, const void* q
 BSA_API bsa_status bsa_selftest_wait(void* ws, size_t ws_bytes, int64_t limit_ns,
                                      bsa_stream_t stream);
 
+/* bsa_fwd on the raster layout, the tile permutation fused into the kernel: q, k, v and
+ * out are bf16 [B, S, Hh, D] in token order (S = T*H*W).  The kernel loads every 4x4x4
+ * tile of a head with one 5D TMA box over the raster tensor (the box's shared-memory
+ * image is the tile-major block; positions outside the valid grid read as zeros, which are
+ * the pad slots) and writes each query row straight to its token.  Lists, schedule and
+ * arithmetic are those of bsa_fwd: the result equals bsa_tile_permute(inverse) of bsa_fwd
+ * on tile-permuted inputs.  lse (nullable): fp32 [B, Hh, S] in token order.  Workspace as
+ * for BSA_OP_FWD.  bf16 only. */
+BSA_API bsa_status bsa_fwd_raster(const bsa_shape* shape, const void* q, const void* k,
+                                  const void* v, const int32_t* row_ptr, const int32_t* col_idx,
+                                  float softmax_scale, void* out, float* lse, void* ws,
+                                  size_t ws_bytes, bsa_stream_t stream);
+
 /* Library build identification (static string). */
 BSA_API const char* bsa_version(void);
 

@@ -161,6 +161,23 @@ def test_fwd_full_size_sampled_rows(B, full):
     assert errs.max() <= 2e-2 * refmax
 
 
+def test_fwd_raster_full_size_matches_permuted_path(B, full):
+    """The fused raster forward at full size, in the bench's launch configuration:
+    bit-identical to the tile-major forward permuted back (whose rows the oracle checks)."""
+    wl, s, (q, k, v), (qt, kt, vt) = full
+    rp, ci = synth.draw_keep_csr(s.rows, s.n_kb, 0.957, seed=wl.seed + 5,
+                                 empty_rows=(0, s.rows // 2))
+    rp, ci = rp.cuda(), ci.cuda()
+    ws = B.new_workspace(s, B.OP_FWD)
+    out = B.bsattn_fwd_raster(q, k, v, rp, ci, s, ws=ws)
+    assert B.device_status(ws) == 0, B.device_status_words(ws)
+    back = B.tile_permute(B.bsattn_fwd(qt, kt, vt, rp, ci, s, ws=ws), s, inverse=True)
+    assert B.device_status(ws) == 0, B.device_status_words(ws)
+    assert torch.equal(out.view(torch.int16), back.view(torch.int16))
+    del out, back
+    torch.cuda.empty_cache()
+
+
 def _oracle_row(qh, kh, vh, g, wl, h, s, p, rp, ci, scale):
     """Oracle row for head h: the CSR row index includes the head offset."""
     r = h * s.n_qb + p // wl.q_block
