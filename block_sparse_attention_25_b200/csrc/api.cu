@@ -128,6 +128,10 @@ GridDims make_grid(const bsa_shape* s) {
   g.ntw = s->Wp / 4;
   g.S = s->T * s->H * s->W;
   g.Np = s->Tp * s->Hp * s->Wp;
+  g.div_ntw = bsa::make_fastdiv(g.ntw);
+  g.div_nth = bsa::make_fastdiv(g.nth);
+  g.div_W = bsa::make_fastdiv(g.W);
+  g.div_H = bsa::make_fastdiv(g.H);
   return g;
 }
 

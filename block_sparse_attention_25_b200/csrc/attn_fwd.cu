@@ -278,10 +278,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   // tensor map; tiles past the padded grid and slots past the valid grid read as zeros.
   const int head = bh - (bh / a.heads) * a.heads;
   auto raster_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int ch, int u) {
-    const int tw = u % a.g.ntw;
-    const int rest = u / a.g.ntw;
-    const int th = rest % a.g.nth;
-    const int tt = rest / a.g.nth;
+    int tw, th, tt;
+    tile_coords(a.g, u, tw, th, tt);
     tma_load_5d(dst, map, bar, ch * CE, head, tw * 4, th * 4, tt * 4);
   };
   if (warp == 8) {

@@ -13,16 +13,24 @@
 //   pass 2: S again, p = exp2(S*c - lse2), per-block row sums, then a sum over the rows
 //           of each query block (warp shuffles + shared memory, fixed order, so the result
 //           is deterministic).
-// Warp roles (320 threads): warps 0-3 / 4-7 row owners of tile 0 / 1, warp 8 TMA
-// producer (K only), warp 9 MMA issuer and TMEM owner.  TMEM holds two S buffers per
-// tile (4 x 128 columns), so the tensor core computes step s+1 while step s is reduced.
+// Warp roles (576 threads): warps 0-7 and 10-17 own the rows, two threads per row: warps
+// 0-3 / 4-7 take the first kv block of each step of tile 0 / 1, warps 10-13 / 14-17 the
+// second (a warp reads the TMEM lane quarter of its sub-partition, warp % 4); warp 8 is
+// the TMA producer (K only), warp 9 the MMA issuer and TMEM owner.  Each thread keeps its
+// own running (max, sum) over its kv blocks; the two halves of a row are combined once,
+// at the end of pass 1.  Four row warps per sub-partition (instead of two) keep the
+// exponential unit fed.  TMEM holds two S buffers per tile (4 x 128 columns), so the
+// tensor core computes step s+1 while step s is reduced.
 #include "bsa_kernels.cuh"
 
 namespace bsa {
 
 namespace mass {
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
 constexpr int kRowsPerCta = 256;
+// 18 warps: 5 share sub-partitions 0 and 1, whose 16K-register files then allow 96
+// registers per thread.
+constexpr int kMaxRegs = 96;
 }  // namespace mass
 
 struct MassParams {
@@ -40,14 +48,15 @@ struct MassSmem {
   static constexpr int kKStages = (D == 128) ? 4 : 6;
   static constexpr int kQOff = 0;
   static constexpr int kKOff = 2 * kQTile;
-  static constexpr int kRedOff = kKOff + kKStages * kKStage;   // float [2 parity][2 tile][4 warp][2 blk]
-  static constexpr int kBarOff = kRedOff + 2 * 2 * 4 * 2 * 4;
-  static constexpr int kBytes = kBarOff + 256;
+  static constexpr int kRedOff = kKOff + kKStages * kKStage;   // float [2 parity][2 tile][4 warp][2 half]
+  static constexpr int kXchOff = kRedOff + 2 * 2 * 4 * 2 * 4;   // float [2 tile][2 half][128 row][2]
+  static constexpr int kBarOff = kXchOff + 2 * 2 * 128 * 2 * 4;
+  static constexpr int kBytes = kBarOff + 512;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
 template <int D>
-__global__ void __launch_bounds__(mass::kThreads, 1)
+__global__ void __maxnreg__(mass::kMaxRegs)
     block_mass_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k, const MassParams p) {
   using L = MassSmem<D>;
@@ -64,8 +73,9 @@ __global__ void __launch_bounds__(mass::kThreads, 1)
   uint64_t* bar_drain = bar_sempty + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* nvalid_sm = reinterpret_cast<int*>(tmem_slot + 2);  // [2 tile][4 warp]
+  int* nvalid_sm = reinterpret_cast<int*>(tmem_slot + 2);  // [2 half][2 tile][4 warp]
   float* red = reinterpret_cast<float*>(smem + L::kRedOff);
+  float* xch = reinterpret_cast<float*>(smem + L::kXchOff);
 
   const AttnDims& a = p.a;
   const int warp = threadIdx.x >> 5;
@@ -84,7 +94,7 @@ __global__ void __launch_bounds__(mass::kThreads, 1)
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(bar_sfull + i, 1);
-      mbar_init(bar_sempty + i, 128);
+      mbar_init(bar_sempty + i, 256);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -106,7 +116,7 @@ __global__ void __launch_bounds__(mass::kThreads, 1)
           tma_load_3d(smem + L::kQOff + t * L::kQTile + ch * (128 * 128), &tm_q, bar_q, ch * 64,
                       row0 + t * 128, bh);
       for (int s = 0; s < nsteps; ++s) {
-        const int st = s % npass;
+        const int st = s >= npass ? s - npass : s;
         const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
         const int ks = s % KS;
         if (s >= KS && !mbar_wait(bar_kempty + ks, ((s / KS) - 1) & 1, abort_flag, p.status,
@@ -128,7 +138,7 @@ __global__ void __launch_bounds__(mass::kThreads, 1)
       const uint32_t k_base = smem_u32(smem + L::kKOff);
       bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, DETAIL_WAIT_Q);
       for (int s = 0; s < nsteps && ok; ++s) {
-        const int st = s % npass;
+        const int st = s >= npass ? s - npass : s;
         const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
         const int ks = s % KS;
         const int buf = s & 1;
@@ -161,35 +171,58 @@ __global__ void __launch_bounds__(mass::kThreads, 1)
       mbar_wait_drain(bar_drain, 0, p.status, DETAIL_WAIT_O_FULL);
     }
   } else {
-    const int t = warp >> 2;
-    const int wq = warp & 3;
+    const int h = warp >= 10 ? 1 : 0;           // which kv block of each step (column half)
+    const int t = (h ? warp - 10 : warp) >> 2;  // query tile
+    const int wq = warp & 3;                    // TMEM lane quarter = the warp's sub-partition
     const int row = wq * 32 + lane;
     const int local = t * 128 + row;
     const int slot = row0 + local;
     const bool q_valid = slot < a.g.Np && slot_valid(a.g, slot);
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float c = p.scale_log2;
+    const int gbar = 1 + 2 * t + h;  // named barrier of the 4 warps of (tile, half)
     // valid queries per warp, then per query block
     const int wcount = __popc(__ballot_sync(0xffffffffu, q_valid));
-    if (lane == 0) nvalid_sm[t * 4 + wq] = wcount;
-    named_bar_sync(1 + t, 128);
+    if (lane == 0) nvalid_sm[(h * 2 + t) * 4 + wq] = wcount;
+    named_bar_sync(gbar, 128);
     const int warps_per_qb = a.q_block / 32;  // 2 or 4
     const int qb_first_warp = (wq / warps_per_qb) * warps_per_qb;
     int nvq = 0;
-    for (int i = 0; i < warps_per_qb; ++i) nvq += nvalid_sm[t * 4 + qb_first_warp + i];
+    for (int i = 0; i < warps_per_qb; ++i) nvq += nvalid_sm[(h * 2 + t) * 4 + qb_first_warp + i];
     const int qb_global = (row0 + t * 128 + qb_first_warp * 32) / a.q_block;
-    const bool writer = (wq == qb_first_warp) && lane < 2 && qb_global < a.n_qb;
+    const bool writer = (wq == qb_first_warp) && lane == 0 && qb_global < a.n_qb;
     float* mass_row = p.mass + (static_cast<long long>(bh) * a.n_qb + qb_global) * a.n_kb;
     const float inv_nvq = nvq > 0 ? 1.f / static_cast<float>(nvq) : 0.f;
 
     float m_run = -INFINITY, l_run = 0.f, lse2 = 0.f;
     bool ok = true;
+    // tile coordinates of this half's kv block 2*st + h, advanced incrementally (no
+    // division inside the loop: integer division shares the pipe of the exponentials)
+    int tw = 0, th = 0, tt = 0;
+    tile_advance(a.g, h, tw, th, tt);
     for (int s = 0; s < nsteps; ++s) {
-      const int st = s % npass;
       const bool pass2 = s >= npass;
+      const int st = pass2 ? s - npass : s;
       const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+      const bool mine = h < nb;  // this half has a kv block in this step
       const int buf = s & 1;
-      if (s == npass) lse2 = (l_run > 0.f) ? m_run + log2f(l_run) : INFINITY;
+      if (s == npass) {
+        tw = th = tt = 0;
+        tile_advance(a.g, h, tw, th, tt);
+        // Both halves' (max, sum) of the row -> the row's exact log-sum-exp (log2 units),
+        // combined in the same order by both threads.
+        float* x = xch + ((t * 2 + h) * 128 + row) * 2;
+        x[0] = m_run;
+        x[1] = l_run;
+        named_bar_sync(5 + t, 256);
+        const float* y0 = xch + ((t * 2 + 0) * 128 + row) * 2;
+        const float* y1 = xch + ((t * 2 + 1) * 128 + row) * 2;
+        const float m = fmaxf(y0[0], y1[0]);
+        const float l = (m == -INFINITY)
+                            ? 0.f
+                            : y0[1] * fast_exp2(y0[0] - m) + y1[1] * fast_exp2(y1[0] - m);
+        lse2 = (l > 0.f) ? m + log2f(l) : INFINITY;
+      }
       // A warp that gives up keeps stepping (without touching TMEM) so that every warp of
       // the group passes the same named barriers.
       bool got = ok ? mbar_wait(bar_sfull + 2 * t + buf, (s >> 1) & 1, abort_flag, p.status,
@@ -197,72 +230,63 @@ __global__ void __launch_bounds__(mass::kThreads, 1)
                     : false;
       got = __all_sync(0xffffffffu, got);
       ok = got;
-      float rs[2] = {0.f, 0.f};
+      float rs = 0.f;
       if (got) {
-        float sv[128];
+        float sv[64];
         tc_fence_after();
-        const uint32_t s_addr = lane_base + (2 * t + buf) * 128;
-        tmem_ld32(s_addr + 0, sv + 0);
-        tmem_ld32(s_addr + 32, sv + 32);
-        if (nb == 2) {
-          tmem_ld32(s_addr + 64, sv + 64);
-          tmem_ld32(s_addr + 96, sv + 96);
+        if (mine) {
+          const uint32_t s_addr = lane_base + (2 * t + buf) * 128 + 64 * h;
+          tmem_ld32(s_addr + 0, sv + 0);
+          tmem_ld32(s_addr + 32, sv + 32);
+          tmem_ld_wait();
         }
-        tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(bar_sempty + 2 * t + buf);
-        // Pad keys and the absent half of a 1-block step -> -inf (same for every row).
-        const int j0 = 2 * st;
-        const uint64_t mk0 = tile_has_pad(a.g, j0) ? tile_valid_mask(a.g, j0) : ~0ull;
-        const uint64_t mk1 =
-            nb == 2 ? (tile_has_pad(a.g, j0 + 1) ? tile_valid_mask(a.g, j0 + 1) : ~0ull) : 0ull;
-        if ((mk0 & mk1) != ~0ull) {
-          const uint32_t mw[4] = {static_cast<uint32_t>(mk0), static_cast<uint32_t>(mk0 >> 32),
-                                  static_cast<uint32_t>(mk1), static_cast<uint32_t>(mk1 >> 32)};
+        if (mine) {
+          // Pad keys -> -inf (same for every row).
+          if (4 * tt + 4 > a.g.T || 4 * th + 4 > a.g.H || 4 * tw + 4 > a.g.W) {
+            const uint64_t mk = tile_valid_mask_at(a.g, tw, th, tt);
+            const uint32_t mw[2] = {static_cast<uint32_t>(mk), static_cast<uint32_t>(mk >> 32)};
 #pragma unroll
-          for (int i = 0; i < 128; ++i) sv[i] = ((mw[i >> 5] >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
-        }
-        if (!pass2) {
-          float mx[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) mx[i] = sv[i];
-#pragma unroll
-          for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
-          const float mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-          const float m_new = fmaxf(m_run, mrow * c);
-          if (m_new != -INFINITY) {
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int i = 0; i < 128; ++i) ls[i & 3] += fast_exp2(fmaf(sv[i], c, -m_new));
-            l_run = l_run * fast_exp2(m_run - m_new) + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-            m_run = m_new;
+            for (int i = 0; i < 64; ++i) sv[i] = ((mw[i >> 5] >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
           }
-        } else if (q_valid) {
+          if (!pass2) {
+            float mx[8];
 #pragma unroll
-          for (int b = 0; b < 2; ++b) {
+            for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+#pragma unroll
+            for (int i = 8; i < 64; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
+            const float mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            const float m_new = fmaxf(m_run, mrow * c);
+            if (m_new != -INFINITY) {
+              float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int i = 0; i < 64; ++i) ls[i & 3] += fast_exp2(fmaf(sv[i], c, -m_new));
+              l_run = l_run * fast_exp2(m_run - m_new) + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+              m_run = m_new;
+            }
+          } else if (q_valid) {
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < 64; ++i) acc[i & 3] += fast_exp2(fmaf(sv[64 * b + i], c, -lse2));
-            rs[b] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            for (int i = 0; i < 64; ++i) acc[i & 3] += fast_exp2(fmaf(sv[i], c, -lse2));
+            rs = (acc[0] + acc[1]) + (acc[2] + acc[3]);
           }
         }
       }
+      tile_advance(a.g, 2, tw, th, tt);
       if (pass2) {
         // Sum the per-row block masses over the rows of each query block: warp shuffles,
         // then the 2 or 4 warps of the block through shared memory in a fixed order.
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          rs[0] += __shfl_xor_sync(0xffffffffu, rs[0], o);
-          rs[1] += __shfl_xor_sync(0xffffffffu, rs[1], o);
-        }
+        for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
         float* rbuf = red + ((s & 1) * 2 + t) * 8;
-        if (lane < 2) rbuf[wq * 2 + lane] = lane == 0 ? rs[0] : rs[1];
-        named_bar_sync(1 + t, 128);
-        if (writer && (lane < nb)) {
+        if (lane == 0) rbuf[wq * 2 + h] = rs;
+        named_bar_sync(gbar, 128);
+        if (writer && mine) {
           float tot = 0.f;
-          for (int i = 0; i < warps_per_qb; ++i) tot += rbuf[(qb_first_warp + i) * 2 + lane];
-          mass_row[2 * st + lane] = tot * inv_nvq;
+          for (int i = 0; i < warps_per_qb; ++i) tot += rbuf[(qb_first_warp + i) * 2 + h];
+          mass_row[2 * st + h] = tot * inv_nvq;
         }
       }
     }

@@ -5,12 +5,39 @@
 
 namespace bsa {
 
+// Division by a per-launch constant as a multiply and a shift ("Division by Invariant
+// Integers using Multiplication", Granlund and Montgomery, 1994): for 0 <= n < 2^31 and
+// 1 <= d < 2^31, with l = ceil(log2 d) and m = ceil(2^(32+l) / d) (below 2^34),
+// floor(n / d) = floor(n * m / 2^(32+l)) exactly, and n * m fits 64 bits.  A division by
+// a runtime value would otherwise run on the conversion/reciprocal pipe, which the
+// softmax loops need for their exponentials.
+struct FastDiv {
+  unsigned long long m;
+  int shift;  // 32 + l
+};
+
+inline FastDiv make_fastdiv(int d) {
+  int l = 0;
+  while ((1ull << l) < static_cast<unsigned long long>(d)) ++l;
+  FastDiv f;
+  f.m = ((1ull << (32 + l)) + static_cast<unsigned long long>(d) - 1ull) /
+        static_cast<unsigned long long>(d);
+  f.shift = 32 + l;
+  return f;
+}
+
+__device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
+  return static_cast<int>((static_cast<unsigned long long>(static_cast<unsigned>(n)) * f.m) >>
+                          f.shift);
+}
+
 // Token grid of one (batch, head) slice.
 struct GridDims {
   int T, H, W;     // valid grid
   int Tp, Hp, Wp;  // padded grid (multiples of 4)
   int nth, ntw;    // tiles along h and w (Hp/4, Wp/4)
   int S, Np;       // valid tokens, padded slots
+  FastDiv div_ntw, div_nth, div_W, div_H;  // division by ntw, nth, W, H
 };
 
 // Attention problem in tile-major layout.
@@ -26,13 +53,19 @@ struct AttnDims {
 // Slot p of the tile-major order: tile = p / 64, inner = p % 64; tiles run row-major over
 // (t/4, h/4, w/4), inner slots row-major over (t%4, h%4, w%4).
 
+// Coordinates of tile j (w fastest, then h, then t).
+__device__ __forceinline__ void tile_coords(const GridDims& g, int j, int& tw, int& th, int& tt) {
+  const int rest = fdiv(j, g.div_ntw);
+  tw = j - rest * g.ntw;
+  tt = fdiv(rest, g.div_nth);
+  th = rest - tt * g.nth;
+}
+
 // Raster token index held by slot p, or -1 for a pad slot.
 __device__ __forceinline__ int slot_to_token(const GridDims& g, int p) {
   const int tile = p >> 6, inner = p & 63;
-  const int tw = tile % g.ntw;
-  const int rest = tile / g.ntw;
-  const int th = rest % g.nth;
-  const int tt = rest / g.nth;
+  int tw, th, tt;
+  tile_coords(g, tile, tw, th, tt);
   const int t = tt * 4 + (inner >> 4);
   const int h = th * 4 + ((inner >> 2) & 3);
   const int w = tw * 4 + (inner & 3);
@@ -41,10 +74,10 @@ __device__ __forceinline__ int slot_to_token(const GridDims& g, int p) {
 }
 
 __device__ __forceinline__ int token_to_slot(const GridDims& g, int s) {
-  const int w = s % g.W;
-  const int rest = s / g.W;
-  const int h = rest % g.H;
-  const int t = rest / g.H;
+  const int rest = fdiv(s, g.div_W);
+  const int w = s - rest * g.W;
+  const int t = fdiv(rest, g.div_H);
+  const int h = rest - t * g.H;
   const int tile = ((t >> 2) * g.nth + (h >> 2)) * g.ntw + (w >> 2);
   return tile * 64 + (((t & 3) * 4 + (h & 3)) * 4 + (w & 3));
 }
@@ -55,10 +88,8 @@ __device__ __forceinline__ bool slot_valid(const GridDims& g, int p) {
 
 // Valid-slot mask of tile j: bit i set when slot i of the tile lies inside the grid.
 __device__ __forceinline__ uint64_t tile_valid_mask(const GridDims& g, int j) {
-  const int tw = j % g.ntw;
-  const int rest = j / g.ntw;
-  const int th = rest % g.nth;
-  const int tt = rest / g.nth;
+  int tw, th, tt;
+  tile_coords(g, j, tw, th, tt);
   const int vt = min(4, max(0, g.T - 4 * tt));
   const int vh = min(4, max(0, g.H - 4 * th));
   const int vw = min(4, max(0, g.W - 4 * tw));
@@ -70,11 +101,34 @@ __device__ __forceinline__ uint64_t tile_valid_mask(const GridDims& g, int j) {
   return m64;
 }
 
+// The same mask from the tile's coordinates (no division).
+__device__ __forceinline__ uint64_t tile_valid_mask_at(const GridDims& g, int tw, int th, int tt) {
+  const int vt = min(4, max(0, g.T - 4 * tt));
+  const int vh = min(4, max(0, g.H - 4 * th));
+  const int vw = min(4, max(0, g.W - 4 * tw));
+  const uint64_t row4 = (1ull << vw) - 1ull;
+  uint64_t m16 = 0;
+  for (int i = 0; i < vh; ++i) m16 |= row4 << (4 * i);
+  uint64_t m64 = 0;
+  for (int i = 0; i < vt; ++i) m64 |= m16 << (16 * i);
+  return m64;
+}
+
+// Moves tile coordinates (w fastest, then h, then t) forward by `by` tiles.
+__device__ __forceinline__ void tile_advance(const GridDims& g, int by, int& tw, int& th, int& tt) {
+  tw += by;
+  while (tw >= g.ntw) {
+    tw -= g.ntw;
+    if (++th == g.nth) {
+      th = 0;
+      ++tt;
+    }
+  }
+}
+
 __device__ __forceinline__ bool tile_has_pad(const GridDims& g, int j) {
-  const int tw = j % g.ntw;
-  const int rest = j / g.ntw;
-  const int th = rest % g.nth;
-  const int tt = rest / g.nth;
+  int tw, th, tt;
+  tile_coords(g, j, tw, th, tt);
   return 4 * tt + 4 > g.T || 4 * th + 4 > g.H || 4 * tw + 4 > g.W;
 }
 

@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
           tma_load_3d(smem + L::kQOff + t * L::kQTile + ch * (128 * 128), &tm_q, bar_q, ch * 64,
                       row0 + t * 128, bh);
       for (int s = 0; s < nsteps; ++s) {
-        const int st = s % npass;
+        const int st = s >= npass ? s - npass : s;
         const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
         const int ks = s % KS;
         if (s >= KS && !mbar_wait(bar_kempty + ks, ((s / KS) - 1) & 1, abort_flag, p.status,
@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
         }
       };
       for (int s = 0; s < nsteps && ok; ++s) {
-        const int st = s % npass;
+        const int st = s >= npass ? s - npass : s;
         const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
         const int ks = s % KS;
         const uint32_t idesc_qk = make_idesc(1u, 0u, 128u, static_cast<uint32_t>(nb * 64));
@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
     float m_run = -INFINITY, l_run = 0.f, lse2 = 0.f;
     bool ok = true;
     for (int s = 0; s < nsteps; ++s) {
-      const int st = s % npass;
+      const int st = s >= npass ? s - npass : s;
       const bool pass2 = s >= npass;
       const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
       if (s == npass) lse2 = (l_run > 0.f) ? m_run + log2f(l_run) : INFINITY;
