@@ -5,10 +5,10 @@
 A step is one calibrate-then-reuse cycle of the 720p workload (the default config,
 Wan-14B-like: B=1, 40 heads, D=128, 21x45x80 tokens padded to 24x48x80, 64-token blocks):
     calibration  tile_permute(Q, K) -> block_mass -> topp_select(0.99)
-    10 x reuse   bsattn_fwd_raster(Q_r, K_r, V_r, frozen lists): raster in, raster out, the
-                 tile permutation fused into the forward's loads and stores
-                 (--layout tiles: tile_permute x3 -> bsattn_fwd -> inverse permute; the
-                 e4m3 workload always takes tile_permute_quant_e4m3 x3 -> bsattn_fwd -> inverse)
+    10 x reuse   tile_permute(Q_r, K_r, V_r) -> bsattn_fwd(frozen lists) -> inverse permute
+                 (--layout raster: bsattn_fwd_raster, the permutation fused into the
+                 forward's loads and stores; the e4m3 workload always takes
+                 tile_permute_quant_e4m3 x3 -> bsattn_fwd -> inverse)
 on seeded synthetic inputs already resident in HBM (Q/K/V of 774 MB each, far above L2).
 
 value  = executed attention TFLOP/s of the whole step: FLOPs of the kept blocks of the 10
@@ -49,8 +49,9 @@ def parse_args():
     ap.add_argument("--reuse", type=int, default=None, help="reuse calls per step (default: the workload's)")
     ap.add_argument("--tau", type=float, default=0.99)
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--layout", default="raster", choices=["raster", "tiles"],
-                    help="bf16 reuse calls: fused raster forward, or permute + tile-major forward")
+    ap.add_argument("--layout", default="tiles", choices=["raster", "tiles"],
+                    help="bf16 reuse calls: permute + tile-major forward (the faster, measured), "
+                         "or the fused raster forward")
     ap.add_argument("--cpu-sample-rows", type=int, default=256)
     ap.add_argument("--clock-log", default=None,
                     help="CSV of the nvidia-smi clock samples ({rank} is replaced); default /tmp")

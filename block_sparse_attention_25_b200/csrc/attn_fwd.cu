@@ -24,9 +24,11 @@
 //
 // Per step s, the MMA thread issues for t = 0, 1:  O_t += P_t(s-1) V(s-1);  S_t(s) = Q_t K(s)^T
 // and commits S_full[t] after both, so when softmax t sees S_t(s) the previous PV into O_t
-// has completed and O_t may be rescaled in place.  Rescaling is lazy: the running max used
-// for exponentiation moves only when a row's max grows by more than 8 (log2 units), so
-// P <= 256 and, for smooth attention, O is almost never touched.
+// has completed and O_t may be rescaled in place.  The PV is issued in two halves: the
+// first kv block's keys as soon as their P is stored (P_part), the rest at P_full.
+// Rescaling is lazy: the running max used for exponentiation moves only when a row's max
+// grows by more than 8 (log2 units), so P <= 256 and, for smooth attention, O is almost
+// never touched (a threshold of 16 for bf16 measured the same: rescales are already rare).
 #include "bsa_kernels.cuh"
 
 namespace bsa {
@@ -178,8 +180,14 @@ struct FwdSmem {
   static constexpr int kKOff = kQOff + 2 * kQTile;
   static constexpr int kVOff = kKOff + kKStages * kKVStage;
   static constexpr int kBarOff = kVOff + kVStages * kKVStage;
-  static constexpr int kBytes = kBarOff + 256;
+  static constexpr int kBytes = kBarOff + 512;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+  // P of a step is released to the PV MMAs in kParts key ranges of 128 / kParts keys (bf16
+  // P is stored 32 keys at a time, e4m3 P 64 keys at a time).  Two ranges (one kv block
+  // each): four 32-key ranges measured 3% slower, each release costing the softmax a wait
+  // for its tensor-memory stores.
+  static constexpr int kParts = 2;
+  static constexpr int kChunksPerPart = 4 / kParts;  // bf16 32-key chunks per part
 };
 
 // e4m3 P is stored as P * (s_v / sigma) * kPScale: with the lazy rescale P <= 256, so the
@@ -205,7 +213,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   uint64_t* bar_vempty = bar_vfull + VS;
   uint64_t* bar_sfull = bar_vempty + VS;  // [2]
   uint64_t* bar_pfull = bar_sfull + 2;    // [2]
-  uint64_t* bar_ofull = bar_pfull + 2;
+  uint64_t* bar_ppart = bar_pfull + 2;    // [2][3] P of the step's first key ranges stored
+  uint64_t* bar_ofull = bar_ppart + 6;
   uint64_t* bar_drain = bar_ofull + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -262,6 +271,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_sfull + t, 1);
       mbar_init(bar_pfull + t, 128);
+      for (int q = 0; q < 3; ++q) mbar_init(bar_ppart + 3 * t + q, 128);
     }
     mbar_init(bar_ofull, 1);
     mbar_init(bar_drain, 1);
@@ -356,18 +366,21 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       const uint64_t q_desc0 = make_sdesc_sw128(q_base, 16, 1024);
       const uint64_t k_desc0 = make_sdesc_sw128(k_base, 16, 1024);
       const uint64_t v_desc0 = make_sdesc_sw128(v_base, 128 * 128, 1024);
-      auto issue_pv = [&](int t, int sp) {
-        // O_t (+)= P_t(sp) V(sp); K dimension = keys of step sp (64 or 128).  One MMA takes
-        // 32 bytes of K: 16 keys (bf16) or 32 keys (e4m3), i.e. 8 TMEM columns of P and
-        // 16 or 32 rows (2 or 4 swizzle atoms) of V.
+      auto issue_pv = [&](int t, int sp, int part) {
+        // O_t (+)= P_t(sp) V(sp) over key range `part` of the step (kParts ranges of 128 /
+        // kParts keys).  One MMA takes 32 bytes of K: 16 keys (bf16) or 32 keys (e4m3), i.e. 8
+        // TMEM columns of P and 16 or 32 rows (2 or 4 swizzle atoms) of V.
         constexpr int kKeysPerMma = 32 / L::kElem;
         constexpr int kMmas = 128 / kKeysPerMma;  // for a 2-block step
-        const int nmma = (2 * sp + 1 < n_ent) ? kMmas : kMmas / 2;
+        constexpr int kPerPart = kMmas / L::kParts;
+        const int kk0 = part * kPerPart;
+        const int nmma = min(kk0 + kPerPart, (2 * sp + 1 < n_ent) ? kMmas : kMmas / 2);
         const uint64_t vd = v_desc0 + static_cast<uint64_t>(((sp % VS) * L::kKVStage) >> 4);
         const uint32_t p_tmem = tmem + t * 128;
         const uint32_t o_tmem = tmem + 256 + t * D;
 #pragma unroll
         for (int kk = 0; kk < kMmas; ++kk) {
+          if (kk < kk0) continue;
           if (kk >= nmma) break;
           const uint64_t bdesc = vd + static_cast<uint64_t>((kk * kKeysPerMma * 128) >> 4);
           if constexpr (FP8)
@@ -388,17 +401,22 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         const uint64_t kd = k_desc0 + static_cast<uint64_t>((ks * L::kKVStage) >> 4);
         for (int t = 0; t < 2; ++t) {
           if (s > 0) {
-            if (!mbar_wait(bar_pfull + t, (s - 1) & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL)) {
-              ok = false;
-              break;
-            }
+            // PV of the previous step range by range, each as soon as its P is stored, while
+            // the softmax still works on the later keys.
             if (t == 0 && !mbar_wait(bar_vfull + ((s - 1) % VS), ((s - 1) / VS) & 1, abort_flag,
                                      p.status, DETAIL_WAIT_V_FULL)) {
               ok = false;
               break;
             }
-            tc_fence_after();
-            issue_pv(t, s - 1);
+            for (int q = 0; q < L::kParts && ok; ++q) {
+              const bool last = q + 1 == L::kParts;
+              ok = mbar_wait(last ? bar_pfull + t : bar_ppart + 3 * t + q, (s - 1) & 1,
+                             abort_flag, p.status, last ? DETAIL_WAIT_P_FULL : DETAIL_WAIT_P_PART);
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv(t, s - 1, q);
+            }
+            if (!ok) break;
             if (t == 1) mma_commit(bar_vempty + ((s - 1) % VS));
           }
           const uint64_t qd = q_desc0 + static_cast<uint64_t>((t * L::kQTile) >> 4);
@@ -422,17 +440,19 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       if (ok) {
         const int sl = nsteps - 1;
         for (int t = 0; t < 2 && ok; ++t) {
-          if (!mbar_wait(bar_pfull + t, sl & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL)) {
-            ok = false;
-            break;
-          }
           if (t == 0 && !mbar_wait(bar_vfull + (sl % VS), (sl / VS) & 1, abort_flag, p.status,
                                    DETAIL_WAIT_V_FULL)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          issue_pv(t, sl);
+          for (int q = 0; q < L::kParts && ok; ++q) {
+            const bool last = q + 1 == L::kParts;
+            ok = mbar_wait(last ? bar_pfull + t : bar_ppart + 3 * t + q, sl & 1, abort_flag,
+                           p.status, last ? DETAIL_WAIT_P_FULL : DETAIL_WAIT_P_PART);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(t, sl, q);
+          }
         }
         if (ok) mma_commit(bar_ofull);
       }
@@ -545,8 +565,19 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         m_run = m_new;
       }
       // P = exp2(S*f - m), stored over S_t as it is produced: bf16 pairs, 16 columns per 32
-      // keys; or e4m3 quads (P scaled by the block's V scale), 16 columns per 64 keys.
+      // keys; or e4m3 quads (P scaled by the block's V scale), 16 columns per 64 keys.  As
+      // each key range's P is stored, its barrier lets the MMA start that part of PV --
+      // unless this warp must first rescale its rows of O: then every part is released at
+      // the end.  Every part barrier is arrived at once per step (absent keys included).
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      const bool warp_resc = __any_sync(0xffffffffu, resc);
+      auto release_part = [&](int q) {
+        if (!warp_resc) {
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(bar_ppart + 3 * t + q);
+        }
+      };
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
       if constexpr (!FP8) {
 #pragma unroll
@@ -561,6 +592,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             pk[i] = pack_bf16x2(p0, p1);
           }
           BSA_TMEM_ST_X16(s_addr + 16 * ch, pk);
+          if ((ch + 1) % L::kChunksPerPart == 0 && (ch + 1) / L::kChunksPerPart < L::kParts)
+            release_part((ch + 1) / L::kChunksPerPart - 1);
         }
       } else {
 #pragma unroll
@@ -582,11 +615,12 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             pk[i] = lo | (hi << 16);
           }
           BSA_TMEM_ST_X16(s_addr + 16 * b, pk);
+          if (b == 0) release_part(0);
         }
       }
       // factor is 1 unless this row's reference max moved; it scales only the old sum.
       l_run = fmaf(l_run, factor, (ls[0] + ls[1]) + (ls[2] + ls[3]));
-      if (__any_sync(0xffffffffu, resc)) {
+      if (warp_resc) {
         // O_t is quiescent: the PV of the previous step completed before S_full fired.
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
@@ -602,6 +636,11 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       }
       tmem_st_wait();
       tc_fence_before();
+      if (warp_resc) {
+        for (int q = 0; q + 1 < L::kParts; ++q) mbar_arrive(bar_ppart + 3 * t + q);
+      } else if (!FP8 && L::kParts == 4 && nb == 1) {
+        mbar_arrive(bar_ppart + 3 * t + 2);  // keys 64-95: absent in a one-block step
+      }
       mbar_arrive(bar_pfull + t);
     }
 

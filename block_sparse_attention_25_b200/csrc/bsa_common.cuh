@@ -30,6 +30,7 @@ enum : uint32_t {
   DETAIL_WAIT_S_FULL = 0x105,
   DETAIL_WAIT_P_FULL = 0x106,
   DETAIL_WAIT_O_FULL = 0x107,
+  DETAIL_WAIT_P_PART = 0x108,
   DETAIL_SELFTEST = 0x1FF,
   DETAIL_MASS_VALUE = 0x200,
   DETAIL_CSR_RANGE = 0x201,
