@@ -35,7 +35,17 @@ namespace bsa {
 
 namespace fwd {
 
-constexpr int kThreads = 320;
+// 12 warps = 3 warpgroups: two softmax warpgroups (one per Q tile) and one producer
+// warpgroup (TMA warp, MMA warp, two idle warps).  Launched at 168 registers a thread (three
+// warps share each sub-partition's 16K registers), the producer warpgroup gives registers
+// back and the softmax warpgroups take them: 2*128*184 + 128*136 = 384*168 (the split with
+// the fewest spills over the variants).
+constexpr int kThreads = 384;
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsSoftmax = 184;
+constexpr int kRegsProducer = 136;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsProducer <= kThreads * kRegsLaunch,
+              "register shares must fit the launch total");
 constexpr int kRowsPerCta = 256;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -292,175 +302,179 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     tile_coords(a.g, u, tw, th, tt);
     tma_load_5d(dst, map, bar, ch * CE, head, tw * 4, th * 4, tt * 4);
   };
-  if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && nsteps > 0) {
-      prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
-      mbar_arrive_expect_tx(bar_q, 2 * L::kQTile);
-      for (int t = 0; t < 2; ++t)
-        for (int ch = 0; ch < L::kChunks; ++ch) {
-          uint8_t* dq = smem + L::kQOff + t * L::kQTile + ch * (128 * 128);
-          if constexpr (RASTER) {  // a 128-row Q tile is two 4x4x4 tiles
-            raster_tile(dq, &tm_q, bar_q, ch, (row0 + t * 128) >> 6);
-            raster_tile(dq + 64 * 128, &tm_q, bar_q, ch, ((row0 + t * 128) >> 6) + 1);
-          } else {
-            tma_load_3d(dq, &tm_q, bar_q, ch * CE, row0 + t * 128, bh);
+  if (warp >= 8) {
+    warpgroup_reg_dec<fwd::kRegsProducer>();
+    if (warp == 8) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0 && nsteps > 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        mbar_arrive_expect_tx(bar_q, 2 * L::kQTile);
+        for (int t = 0; t < 2; ++t)
+          for (int ch = 0; ch < L::kChunks; ++ch) {
+            uint8_t* dq = smem + L::kQOff + t * L::kQTile + ch * (128 * 128);
+            if constexpr (RASTER) {  // a 128-row Q tile is two 4x4x4 tiles
+              raster_tile(dq, &tm_q, bar_q, ch, (row0 + t * 128) >> 6);
+              raster_tile(dq + 64 * 128, &tm_q, bar_q, ch, ((row0 + t * 128) >> 6) + 1);
+            } else {
+              tma_load_3d(dq, &tm_q, bar_q, ch * CE, row0 + t * 128, bh);
+            }
           }
-        }
-      for (int s = 0; s < nsteps; ++s) {
-        const int nb = (2 * s + 1 < n_ent) ? 2 : 1;
-        // first key row of each of the step's (one or two) 64-row boxes
-        const int j0 = VARLEN ? fwd::entry_start(ent[2 * s]) : fwd::entry_block(ent[2 * s]) * 64;
-        const int j1 = nb == 2 ? (VARLEN ? fwd::entry_start(ent[2 * s + 1])
-                                         : fwd::entry_block(ent[2 * s + 1]) * 64)
-                               : 0;
-        const int ks = s % KS;
-        if (s >= KS && !mbar_wait(bar_kempty + ks, ((s / KS) - 1) & 1, abort_flag, p.status,
-                                  DETAIL_WAIT_K_EMPTY))
-          break;
-        mbar_arrive_expect_tx(bar_kfull + ks, nb * 64 * L::kRowBytes);
-        uint8_t* kst = smem + L::kKOff + ks * L::kKVStage;
-        for (int ch = 0; ch < L::kChunks; ++ch) {
-          if constexpr (RASTER) {
-            raster_tile(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch, j0 >> 6);
-            if (nb == 2) raster_tile(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch, j1 >> 6);
-          } else {
-            tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * CE, j0, bh);
-            if (nb == 2)
-              tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * CE,
-                          j1, bh);
+        for (int s = 0; s < nsteps; ++s) {
+          const int nb = (2 * s + 1 < n_ent) ? 2 : 1;
+          // first key row of each of the step's (one or two) 64-row boxes
+          const int j0 = VARLEN ? fwd::entry_start(ent[2 * s]) : fwd::entry_block(ent[2 * s]) * 64;
+          const int j1 = nb == 2 ? (VARLEN ? fwd::entry_start(ent[2 * s + 1])
+                                           : fwd::entry_block(ent[2 * s + 1]) * 64)
+                                 : 0;
+          const int ks = s % KS;
+          if (s >= KS && !mbar_wait(bar_kempty + ks, ((s / KS) - 1) & 1, abort_flag, p.status,
+                                    DETAIL_WAIT_K_EMPTY))
+            break;
+          mbar_arrive_expect_tx(bar_kfull + ks, nb * 64 * L::kRowBytes);
+          uint8_t* kst = smem + L::kKOff + ks * L::kKVStage;
+          for (int ch = 0; ch < L::kChunks; ++ch) {
+            if constexpr (RASTER) {
+              raster_tile(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch, j0 >> 6);
+              if (nb == 2) raster_tile(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch, j1 >> 6);
+            } else {
+              tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * CE, j0, bh);
+              if (nb == 2)
+                tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * CE,
+                            j1, bh);
+            }
           }
-        }
-        const int vs = s % VS;
-        if (s >= VS && !mbar_wait(bar_vempty + vs, ((s / VS) - 1) & 1, abort_flag, p.status,
-                                  DETAIL_WAIT_V_EMPTY))
-          break;
-        mbar_arrive_expect_tx(bar_vfull + vs, nb * 64 * L::kRowBytes);
-        uint8_t* vst = smem + L::kVOff + vs * L::kKVStage;
-        for (int ch = 0; ch < L::kChunks; ++ch) {
-          if constexpr (RASTER) {
-            raster_tile(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch, j0 >> 6);
-            if (nb == 2) raster_tile(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch, j1 >> 6);
-          } else {
-            tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * CE, j0, bh);
-            if (nb == 2)
-              tma_load_3d(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch * CE,
-                          j1, bh);
+          const int vs = s % VS;
+          if (s >= VS && !mbar_wait(bar_vempty + vs, ((s / VS) - 1) & 1, abort_flag, p.status,
+                                    DETAIL_WAIT_V_EMPTY))
+            break;
+          mbar_arrive_expect_tx(bar_vfull + vs, nb * 64 * L::kRowBytes);
+          uint8_t* vst = smem + L::kVOff + vs * L::kKVStage;
+          for (int ch = 0; ch < L::kChunks; ++ch) {
+            if constexpr (RASTER) {
+              raster_tile(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch, j0 >> 6);
+              if (nb == 2) raster_tile(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch, j1 >> 6);
+            } else {
+              tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * CE, j0, bh);
+              if (nb == 2)
+                tma_load_3d(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch * CE,
+                            j1, bh);
+            }
           }
         }
       }
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nsteps > 0) {
-      const uint32_t q_base = smem_u32(smem + L::kQOff);
-      const uint32_t k_base = smem_u32(smem + L::kKOff);
-      const uint32_t v_base = smem_u32(smem + L::kVOff);
-      constexpr uint32_t kFmt = FP8 ? 0u : 1u;  // e4m3 / bf16
-      const uint32_t idesc_pv = make_idesc(kFmt, 1u, 128u, static_cast<uint32_t>(D));
-      bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, DETAIL_WAIT_Q);
-      // Shared-memory descriptors: built once; the start-address field is the low bits, so
-      // a byte offset inside the operand region is added as offset >> 4.
-      const uint64_t q_desc0 = make_sdesc_sw128(q_base, 16, 1024);
-      const uint64_t k_desc0 = make_sdesc_sw128(k_base, 16, 1024);
-      const uint64_t v_desc0 = make_sdesc_sw128(v_base, 128 * 128, 1024);
-      auto issue_pv = [&](int t, int sp, int part) {
-        // O_t (+)= P_t(sp) V(sp) over key range `part` of the step (kParts ranges of 128 /
-        // kParts keys).  One MMA takes 32 bytes of K: 16 keys (bf16) or 32 keys (e4m3), i.e. 8
-        // TMEM columns of P and 16 or 32 rows (2 or 4 swizzle atoms) of V.
-        constexpr int kKeysPerMma = 32 / L::kElem;
-        constexpr int kMmas = 128 / kKeysPerMma;  // for a 2-block step
-        constexpr int kPerPart = kMmas / L::kParts;
-        const int kk0 = part * kPerPart;
-        const int nmma = min(kk0 + kPerPart, (2 * sp + 1 < n_ent) ? kMmas : kMmas / 2);
-        const uint64_t vd = v_desc0 + static_cast<uint64_t>(((sp % VS) * L::kKVStage) >> 4);
-        const uint32_t p_tmem = tmem + t * 128;
-        const uint32_t o_tmem = tmem + 256 + t * D;
-#pragma unroll
-        for (int kk = 0; kk < kMmas; ++kk) {
-          if (kk < kk0) continue;
-          if (kk >= nmma) break;
-          const uint64_t bdesc = vd + static_cast<uint64_t>((kk * kKeysPerMma * 128) >> 4);
-          if constexpr (FP8)
-            mma_f8_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (sp > 0 || kk > 0) ? 1u : 0u);
-          else
-            mma_f16_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (sp > 0 || kk > 0) ? 1u : 0u);
+    } else if (warp == 9) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0 && nsteps > 0) {
+        const uint32_t q_base = smem_u32(smem + L::kQOff);
+        const uint32_t k_base = smem_u32(smem + L::kKOff);
+        const uint32_t v_base = smem_u32(smem + L::kVOff);
+        constexpr uint32_t kFmt = FP8 ? 0u : 1u;  // e4m3 / bf16
+        const uint32_t idesc_pv = make_idesc(kFmt, 1u, 128u, static_cast<uint32_t>(D));
+        bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, DETAIL_WAIT_Q);
+        // Shared-memory descriptors: built once; the start-address field is the low bits, so
+        // a byte offset inside the operand region is added as offset >> 4.
+        const uint64_t q_desc0 = make_sdesc_sw128(q_base, 16, 1024);
+        const uint64_t k_desc0 = make_sdesc_sw128(k_base, 16, 1024);
+        const uint64_t v_desc0 = make_sdesc_sw128(v_base, 128 * 128, 1024);
+        auto issue_pv = [&](int t, int sp, int part) {
+          // O_t (+)= P_t(sp) V(sp) over key range `part` of the step (kParts ranges of 128 /
+          // kParts keys).  One MMA takes 32 bytes of K: 16 keys (bf16) or 32 keys (e4m3), i.e. 8
+          // TMEM columns of P and 16 or 32 rows (2 or 4 swizzle atoms) of V.
+          constexpr int kKeysPerMma = 32 / L::kElem;
+          constexpr int kMmas = 128 / kKeysPerMma;  // for a 2-block step
+          constexpr int kPerPart = kMmas / L::kParts;
+          const int kk0 = part * kPerPart;
+          const int nmma = min(kk0 + kPerPart, (2 * sp + 1 < n_ent) ? kMmas : kMmas / 2);
+          const uint64_t vd = v_desc0 + static_cast<uint64_t>(((sp % VS) * L::kKVStage) >> 4);
+          const uint32_t p_tmem = tmem + t * 128;
+          const uint32_t o_tmem = tmem + 256 + t * D;
+  #pragma unroll
+          for (int kk = 0; kk < kMmas; ++kk) {
+            if (kk < kk0) continue;
+            if (kk >= nmma) break;
+            const uint64_t bdesc = vd + static_cast<uint64_t>((kk * kKeysPerMma * 128) >> 4);
+            if constexpr (FP8)
+              mma_f8_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (sp > 0 || kk > 0) ? 1u : 0u);
+            else
+              mma_f16_ts(o_tmem, p_tmem + kk * 8, bdesc, idesc_pv, (sp > 0 || kk > 0) ? 1u : 0u);
+          }
+        };
+        for (int s = 0; s < nsteps && ok; ++s) {
+          const int ks = s % KS;
+          const int nb = (2 * s + 1 < n_ent) ? 2 : 1;
+          const uint32_t idesc_qk = make_idesc(kFmt, 0u, 128u, static_cast<uint32_t>(nb * 64));
+          if (!mbar_wait(bar_kfull + ks, (s / KS) & 1, abort_flag, p.status, DETAIL_WAIT_K_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t kd = k_desc0 + static_cast<uint64_t>((ks * L::kKVStage) >> 4);
+          for (int t = 0; t < 2; ++t) {
+            if (s > 0) {
+              // PV of the previous step range by range, each as soon as its P is stored, while
+              // the softmax still works on the later keys.
+              if (t == 0 && !mbar_wait(bar_vfull + ((s - 1) % VS), ((s - 1) / VS) & 1, abort_flag,
+                                       p.status, DETAIL_WAIT_V_FULL)) {
+                ok = false;
+                break;
+              }
+              for (int q = 0; q < L::kParts && ok; ++q) {
+                const bool last = q + 1 == L::kParts;
+                ok = mbar_wait(last ? bar_pfull + t : bar_ppart + 3 * t + q, (s - 1) & 1,
+                               abort_flag, p.status, last ? DETAIL_WAIT_P_FULL : DETAIL_WAIT_P_PART);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(t, s - 1, q);
+              }
+              if (!ok) break;
+              if (t == 1) mma_commit(bar_vempty + ((s - 1) % VS));
+            }
+            const uint64_t qd = q_desc0 + static_cast<uint64_t>((t * L::kQTile) >> 4);
+            const uint32_t s_tmem = tmem + t * 128;
+            // K (= head dim) advances 32 bytes per MMA inside each 128-byte swizzle chunk.
+  #pragma unroll
+            for (int kk = 0; kk < L::kRowBytes / 32; ++kk) {
+              const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
+              const uint64_t adesc = qd + off;
+              const uint64_t bdesc = kd + off;
+              if constexpr (FP8)
+                mma_f8_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+              else
+                mma_f16_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar_sfull + t);
+          }
+          if (!ok) break;
+          mma_commit(bar_kempty + ks);
         }
-      };
-      for (int s = 0; s < nsteps && ok; ++s) {
-        const int ks = s % KS;
-        const int nb = (2 * s + 1 < n_ent) ? 2 : 1;
-        const uint32_t idesc_qk = make_idesc(kFmt, 0u, 128u, static_cast<uint32_t>(nb * 64));
-        if (!mbar_wait(bar_kfull + ks, (s / KS) & 1, abort_flag, p.status, DETAIL_WAIT_K_FULL)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint64_t kd = k_desc0 + static_cast<uint64_t>((ks * L::kKVStage) >> 4);
-        for (int t = 0; t < 2; ++t) {
-          if (s > 0) {
-            // PV of the previous step range by range, each as soon as its P is stored, while
-            // the softmax still works on the later keys.
-            if (t == 0 && !mbar_wait(bar_vfull + ((s - 1) % VS), ((s - 1) / VS) & 1, abort_flag,
-                                     p.status, DETAIL_WAIT_V_FULL)) {
+        if (ok) {
+          const int sl = nsteps - 1;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (t == 0 && !mbar_wait(bar_vfull + (sl % VS), (sl / VS) & 1, abort_flag, p.status,
+                                     DETAIL_WAIT_V_FULL)) {
               ok = false;
               break;
             }
             for (int q = 0; q < L::kParts && ok; ++q) {
               const bool last = q + 1 == L::kParts;
-              ok = mbar_wait(last ? bar_pfull + t : bar_ppart + 3 * t + q, (s - 1) & 1,
-                             abort_flag, p.status, last ? DETAIL_WAIT_P_FULL : DETAIL_WAIT_P_PART);
+              ok = mbar_wait(last ? bar_pfull + t : bar_ppart + 3 * t + q, sl & 1, abort_flag,
+                             p.status, last ? DETAIL_WAIT_P_FULL : DETAIL_WAIT_P_PART);
               if (!ok) break;
               tc_fence_after();
-              issue_pv(t, s - 1, q);
+              issue_pv(t, sl, q);
             }
-            if (!ok) break;
-            if (t == 1) mma_commit(bar_vempty + ((s - 1) % VS));
           }
-          const uint64_t qd = q_desc0 + static_cast<uint64_t>((t * L::kQTile) >> 4);
-          const uint32_t s_tmem = tmem + t * 128;
-          // K (= head dim) advances 32 bytes per MMA inside each 128-byte swizzle chunk.
-#pragma unroll
-          for (int kk = 0; kk < L::kRowBytes / 32; ++kk) {
-            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
-            const uint64_t adesc = qd + off;
-            const uint64_t bdesc = kd + off;
-            if constexpr (FP8)
-              mma_f8_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
-            else
-              mma_f16_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar_sfull + t);
+          if (ok) mma_commit(bar_ofull);
         }
-        if (!ok) break;
-        mma_commit(bar_kempty + ks);
+        // Whatever happened, let every issued MMA finish before TMEM is released.
+        mma_commit(bar_drain);
+        mbar_wait_drain(bar_drain, 0, p.status, DETAIL_WAIT_O_FULL);
       }
-      if (ok) {
-        const int sl = nsteps - 1;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (t == 0 && !mbar_wait(bar_vfull + (sl % VS), (sl / VS) & 1, abort_flag, p.status,
-                                   DETAIL_WAIT_V_FULL)) {
-            ok = false;
-            break;
-          }
-          for (int q = 0; q < L::kParts && ok; ++q) {
-            const bool last = q + 1 == L::kParts;
-            ok = mbar_wait(last ? bar_pfull + t : bar_ppart + 3 * t + q, sl & 1, abort_flag,
-                           p.status, last ? DETAIL_WAIT_P_FULL : DETAIL_WAIT_P_PART);
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv(t, sl, q);
-          }
-        }
-        if (ok) mma_commit(bar_ofull);
-      }
-      // Whatever happened, let every issued MMA finish before TMEM is released.
-      mma_commit(bar_drain);
-      mbar_wait_drain(bar_drain, 0, p.status, DETAIL_WAIT_O_FULL);
     }
   } else {
+    warpgroup_reg_inc<fwd::kRegsSoftmax>();
     // ------------------------------------------------------------ softmax warps
     const int t = warp >> 2;           // Q tile
     const int wq = warp & 3;           // TMEM lane quarter
@@ -705,6 +719,17 @@ size_t fwd_scratch_bytes(const AttnDims& a) {
   return 2 * counts + static_cast<size_t>(ctas) * a.n_kb * 4;
 }
 
+// The register split between warpgroups assumes the kernel is launched at exactly
+// fwd::kRegsLaunch registers a thread; with fewer, the softmax warpgroups' increase could
+// never be satisfied, so such a build is refused before any launch.
+template <typename Kernel>
+static cudaError_t check_fwd_registers(Kernel kernel) {
+  cudaFuncAttributes attr;
+  const cudaError_t e = cudaFuncGetAttributes(&attr, kernel);
+  if (e != cudaSuccess) return e;
+  return attr.numRegs == fwd::kRegsLaunch ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
 template <int D, bool FP8, bool VARLEN>
 static cudaError_t launch_fwd(const AttnDims& a, int rows_per_head, const void* q, const void* k,
                               const void* v, const FwdParams& prm, long long ctas,
@@ -719,6 +744,8 @@ static cudaError_t launch_fwd(const AttnDims& a, int rows_per_head, const void* 
   e = encode_tmap_3d(&tk, k, dt, eb, D, rows_per_head, bh, ce, 64);
   if (e != cudaSuccess) return e;
   e = encode_tmap_3d(&tv, v, dt, eb, D, rows_per_head, bh, ce, 64);
+  if (e != cudaSuccess) return e;
+  e = check_fwd_registers(bsattn_fwd_kernel<D, FP8, VARLEN>);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bsattn_fwd_kernel<D, FP8, VARLEN>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
@@ -780,7 +807,9 @@ template <int D>
 static cudaError_t launch_fwd_raster(const AttnDims& a, const void* q, const void* k,
                                      const void* v, FwdParams prm, cudaStream_t stream) {
   using L = FwdSmem<D, false>;
-  cudaError_t e = cudaFuncSetAttribute(bsattn_fwd_kernel<D, false, false, true>,
+  cudaError_t e = check_fwd_registers(bsattn_fwd_kernel<D, false, false, true>);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bsattn_fwd_kernel<D, false, false, true>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   const long long per_batch = static_cast<long long>(a.g.S) * a.heads * D;  // elements

@@ -313,6 +313,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 16; ++i) v[16 + i] = __uint_as_float(r[i]);
 }
 
+// Register budget moves between warpgroups: all four warps of a warpgroup execute the same
+// instruction.  An increase waits until decreases elsewhere in the CTA have freed enough of
+// the registers the CTA was launched with, so the shares must add up to the launch total.
+template <int N>
+__device__ __forceinline__ void warpgroup_reg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void warpgroup_reg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
