@@ -11,16 +11,25 @@
 // Since P is already normalised, O needs no rescaling and no final division.
 //
 // Layout and roles follow the block-sparse forward (attn_fwd.cu): 256 query slots per CTA
-// in two M=128 tiles, 320 threads (warps 0-7 row owners, warp 8 TMA, warp 9 MMA), TMEM
+// in two M=128 tiles, 384 threads (warps 0-7 row owners, warp 8 TMA, warp 9 MMA, warps
+// 10-11 completing the producer warpgroup, which hands registers to the row owners), TMEM
 // S0 S1 O0 O1.  In pass 1 the MMA of S_t(s+1) waits until the rows of S_t(s) have been
-// read (S_free); in pass 2 the order is PV_t(s-1), S_t(s) as in the forward.
+// read (S_free); in pass 2 the order is PV_t(s-1), S_t(s) as in the forward, the PV in two
+// halves: the first kv block's keys as soon as their P is stored (P_part).
 #include "bsa_kernels.cuh"
 
 namespace bsa {
 
 namespace calib {
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kRowsPerCta = 256;
+// Launched at 168 registers a thread (three warps per sub-partition); the producer
+// warpgroup gives some back: 2*128*kRegsRows + 128*kRegsProducer <= 384*168.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsRows = 184;
+constexpr int kRegsProducer = 136;
+static_assert(2 * 128 * kRegsRows + 128 * kRegsProducer <= kThreads * kRegsLaunch,
+              "register shares must fit the launch total");
 }  // namespace calib
 
 struct CalibParams {
@@ -44,7 +53,7 @@ struct CalibSmem {
   static constexpr int kVOff = kKOff + kKStages * kKVStage;
   static constexpr int kRedOff = kVOff + kVStages * kKVStage;  // float [2 parity][2 tile][4 warp][2 blk]
   static constexpr int kBarOff = kRedOff + 2 * 2 * 4 * 2 * 4;
-  static constexpr int kBytes = kBarOff + 256;
+  static constexpr int kBytes = kBarOff + 512;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
@@ -66,7 +75,8 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
   uint64_t* bar_sfull = bar_vempty + VS;  // [2]
   uint64_t* bar_sfree = bar_sfull + 2;    // [2] pass 1: rows of S_t read
   uint64_t* bar_pfull = bar_sfree + 2;    // [2] pass 2: P_t stored
-  uint64_t* bar_ofull = bar_pfull + 2;
+  uint64_t* bar_ppart = bar_pfull + 2;    // [2] pass 2: P_t of the step's first kv block stored
+  uint64_t* bar_ofull = bar_ppart + 2;
   uint64_t* bar_drain = bar_ofull + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -96,6 +106,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
       mbar_init(bar_sfull + t, 1);
       mbar_init(bar_sfree + t, 128);
       mbar_init(bar_pfull + t, 128);
+      mbar_init(bar_ppart + t, 128);
     }
     mbar_init(bar_ofull, 1);
     mbar_init(bar_drain, 1);
@@ -108,137 +119,137 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      prefetch_tensormap(&tm_q);
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
-      mbar_arrive_expect_tx(bar_q, 2 * L::kQTile);
-      for (int t = 0; t < 2; ++t)
-        for (int ch = 0; ch < L::kChunks; ++ch)
-          tma_load_3d(smem + L::kQOff + t * L::kQTile + ch * (128 * 128), &tm_q, bar_q, ch * 64,
-                      row0 + t * 128, bh);
-      for (int s = 0; s < nsteps; ++s) {
-        const int st = s >= npass ? s - npass : s;
-        const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
-        const int ks = s % KS;
-        if (s >= KS && !mbar_wait(bar_kempty + ks, ((s / KS) - 1) & 1, abort_flag, p.status,
-                                  DETAIL_WAIT_K_EMPTY))
-          break;
-        mbar_arrive_expect_tx(bar_kfull + ks, nb * 64 * D * 2);
-        uint8_t* kst = smem + L::kKOff + ks * L::kKVStage;
-        for (int ch = 0; ch < L::kChunks; ++ch) {
-          tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * 64, 2 * st * 64, bh);
-          if (nb == 2)
-            tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * 64,
-                        (2 * st + 1) * 64, bh);
-        }
-        if (s < npass) continue;  // V is needed in pass 2 only
-        const int u = s - npass;
-        const int vs = u % VS;
-        if (u >= VS && !mbar_wait(bar_vempty + vs, ((u / VS) - 1) & 1, abort_flag, p.status,
-                                  DETAIL_WAIT_V_EMPTY))
-          break;
-        mbar_arrive_expect_tx(bar_vfull + vs, nb * 64 * D * 2);
-        uint8_t* vst = smem + L::kVOff + vs * L::kKVStage;
-        for (int ch = 0; ch < L::kChunks; ++ch) {
-          tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * 64, 2 * st * 64, bh);
-          if (nb == 2)
-            tma_load_3d(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch * 64,
-                        (2 * st + 1) * 64, bh);
+  if (warp >= 8) {
+    warpgroup_reg_dec<calib::kRegsProducer>();
+    if (warp == 8) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        mbar_arrive_expect_tx(bar_q, 2 * L::kQTile);
+        for (int t = 0; t < 2; ++t)
+          for (int ch = 0; ch < L::kChunks; ++ch)
+            tma_load_3d(smem + L::kQOff + t * L::kQTile + ch * (128 * 128), &tm_q, bar_q, ch * 64,
+                        row0 + t * 128, bh);
+        for (int s = 0; s < nsteps; ++s) {
+          const int st = s >= npass ? s - npass : s;
+          const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+          const int ks = s % KS;
+          if (s >= KS && !mbar_wait(bar_kempty + ks, ((s / KS) - 1) & 1, abort_flag, p.status,
+                                    DETAIL_WAIT_K_EMPTY))
+            break;
+          mbar_arrive_expect_tx(bar_kfull + ks, nb * 64 * D * 2);
+          uint8_t* kst = smem + L::kKOff + ks * L::kKVStage;
+          for (int ch = 0; ch < L::kChunks; ++ch) {
+            tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * 64, 2 * st * 64, bh);
+            if (nb == 2)
+              tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * 64,
+                          (2 * st + 1) * 64, bh);
+          }
+          if (s < npass) continue;  // V is needed in pass 2 only
+          const int u = s - npass;
+          const int vs = u % VS;
+          if (u >= VS && !mbar_wait(bar_vempty + vs, ((u / VS) - 1) & 1, abort_flag, p.status,
+                                    DETAIL_WAIT_V_EMPTY))
+            break;
+          mbar_arrive_expect_tx(bar_vfull + vs, nb * 64 * D * 2);
+          uint8_t* vst = smem + L::kVOff + vs * L::kKVStage;
+          for (int ch = 0; ch < L::kChunks; ++ch) {
+            tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * 64, 2 * st * 64, bh);
+            if (nb == 2)
+              tma_load_3d(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch * 64,
+                          (2 * st + 1) * 64, bh);
+          }
         }
       }
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint64_t q_desc0 = make_sdesc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
-      const uint64_t k_desc0 = make_sdesc_sw128(smem_u32(smem + L::kKOff), 16, 1024);
-      const uint64_t v_desc0 = make_sdesc_sw128(smem_u32(smem + L::kVOff), 128 * 128, 1024);
-      const uint32_t idesc_pv = make_idesc(1u, 1u, 128u, static_cast<uint32_t>(D));
-      bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, DETAIL_WAIT_Q);
-      auto issue_pv = [&](int t, int u) {
-        // O_t (+)= P_t V over the keys of pass-2 step u (64 or 128 keys, 16 per MMA).
-        const int nbp = (2 * u + 1 < a.n_kb) ? 2 : 1;
-        const uint64_t vd = v_desc0 + static_cast<uint64_t>(((u % VS) * L::kKVStage) >> 4);
-        const uint32_t p_tmem = tmem + t * 128;
-        const uint32_t o_tmem = tmem + 256 + t * D;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          if (kk >= nbp * 4) break;
-          mma_f16_ts(o_tmem, p_tmem + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4),
-                     idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
-        }
-      };
-      for (int s = 0; s < nsteps && ok; ++s) {
-        const int st = s >= npass ? s - npass : s;
-        const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
-        const int ks = s % KS;
-        const uint32_t idesc_qk = make_idesc(1u, 0u, 128u, static_cast<uint32_t>(nb * 64));
-        if (!mbar_wait(bar_kfull + ks, (s / KS) & 1, abort_flag, p.status, DETAIL_WAIT_K_FULL)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint64_t kd = k_desc0 + static_cast<uint64_t>((ks * L::kKVStage) >> 4);
-        for (int t = 0; t < 2; ++t) {
-          if (s >= 1 && s <= npass) {
-            // S_t is free once its rows of the previous step were read (pass 1 and the
-            // first step of pass 2)
-            if (!mbar_wait(bar_sfree + t, (s - 1) & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL)) {
-              ok = false;
-              break;
-            }
-          } else if (s > npass) {
-            const int u = s - 1 - npass;  // pass-2 step whose P is consumed now
-            if (!mbar_wait(bar_pfull + t, u & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL)) {
-              ok = false;
-              break;
-            }
-            if (t == 0 && !mbar_wait(bar_vfull + (u % VS), (u / VS) & 1, abort_flag, p.status,
-                                     DETAIL_WAIT_V_FULL)) {
-              ok = false;
-              break;
+    } else if (warp == 9) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint64_t q_desc0 = make_sdesc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
+        const uint64_t k_desc0 = make_sdesc_sw128(smem_u32(smem + L::kKOff), 16, 1024);
+        const uint64_t v_desc0 = make_sdesc_sw128(smem_u32(smem + L::kVOff), 128 * 128, 1024);
+        const uint32_t idesc_pv = make_idesc(1u, 1u, 128u, static_cast<uint32_t>(D));
+        bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, DETAIL_WAIT_Q);
+        auto issue_pv = [&](int t, int u, int half) {
+          // O_t (+)= P_t V over the keys of pass-2 step u's first (half 0) or second (half 1)
+          // kv block, 16 keys per MMA.
+          const int nbp = (2 * u + 1 < a.n_kb) ? 2 : 1;
+          const uint64_t vd = v_desc0 + static_cast<uint64_t>(((u % VS) * L::kKVStage) >> 4);
+          const uint32_t p_tmem = tmem + t * 128;
+          const uint32_t o_tmem = tmem + 256 + t * D;
+          if (half >= nbp) return;
+  #pragma unroll
+          for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
+            mma_f16_ts(o_tmem, p_tmem + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4),
+                       idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
+        };
+        // PV of pass-2 step u for tile t: the first block's keys at P_part, the rest at P_full.
+        auto pv_step = [&](int t, int u) -> bool {
+          if (!mbar_wait(bar_ppart + t, u & 1, abort_flag, p.status, DETAIL_WAIT_P_PART))
+            return false;
+          if (t == 0 && !mbar_wait(bar_vfull + (u % VS), (u / VS) & 1, abort_flag, p.status,
+                                   DETAIL_WAIT_V_FULL))
+            return false;
+          tc_fence_after();
+          issue_pv(t, u, 0);
+          if (!mbar_wait(bar_pfull + t, u & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL))
+            return false;
+          tc_fence_after();
+          issue_pv(t, u, 1);
+          return true;
+        };
+        for (int s = 0; s < nsteps && ok; ++s) {
+          const int st = s >= npass ? s - npass : s;
+          const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+          const int ks = s % KS;
+          const uint32_t idesc_qk = make_idesc(1u, 0u, 128u, static_cast<uint32_t>(nb * 64));
+          if (!mbar_wait(bar_kfull + ks, (s / KS) & 1, abort_flag, p.status, DETAIL_WAIT_K_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t kd = k_desc0 + static_cast<uint64_t>((ks * L::kKVStage) >> 4);
+          for (int t = 0; t < 2; ++t) {
+            if (s >= 1 && s <= npass) {
+              // S_t is free once its rows of the previous step were read (pass 1 and the
+              // first step of pass 2)
+              if (!mbar_wait(bar_sfree + t, (s - 1) & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL)) {
+                ok = false;
+                break;
+              }
+            } else if (s > npass) {
+              const int u = s - 1 - npass;  // pass-2 step whose P is consumed now
+              if (!pv_step(t, u)) {
+                ok = false;
+                break;
+              }
+              if (t == 1) mma_commit(bar_vempty + (u % VS));
             }
             tc_fence_after();
-            issue_pv(t, u);
-            if (t == 1) mma_commit(bar_vempty + (u % VS));
+            const uint64_t qd = q_desc0 + static_cast<uint64_t>((t * L::kQTile) >> 4);
+            const uint32_t s_tmem = tmem + t * 128;
+  #pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
+              mma_f16_ss(s_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar_sfull + t);
           }
-          tc_fence_after();
-          const uint64_t qd = q_desc0 + static_cast<uint64_t>((t * L::kQTile) >> 4);
-          const uint32_t s_tmem = tmem + t * 128;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4);
-            mma_f16_ss(s_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar_sfull + t);
+          if (!ok) break;
+          mma_commit(bar_kempty + ks);
         }
-        if (!ok) break;
-        mma_commit(bar_kempty + ks);
-      }
-      if (ok) {
-        const int u = npass - 1;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (!mbar_wait(bar_pfull + t, u & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL)) {
-            ok = false;
-            break;
-          }
-          if (t == 0 && !mbar_wait(bar_vfull + (u % VS), (u / VS) & 1, abort_flag, p.status,
-                                   DETAIL_WAIT_V_FULL)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_pv(t, u);
+        if (ok) {
+          const int u = npass - 1;
+          for (int t = 0; t < 2 && ok; ++t) ok = pv_step(t, u);
+          if (ok) mma_commit(bar_ofull);
         }
-        if (ok) mma_commit(bar_ofull);
+        mma_commit(bar_drain);
+        mbar_wait_drain(bar_drain, 0, p.status, DETAIL_WAIT_O_FULL);
       }
-      mma_commit(bar_drain);
-      mbar_wait_drain(bar_drain, 0, p.status, DETAIL_WAIT_O_FULL);
     }
   } else {
+    warpgroup_reg_inc<calib::kRegsRows>();
     // ------------------------------------------------------------ row owners
     const int t = warp >> 2;
     const int wq = warp & 3;
@@ -332,6 +343,11 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
               pk[i] = pack_bf16x2(p0, p1);
             }
             BSA_TMEM_ST_X16(s_addr + 16 * ch, pk);
+            if (ch == 1) {  // the first kv block's P: its half of PV may start
+              tmem_st_wait();
+              tc_fence_before();
+              mbar_arrive(bar_ppart + t);
+            }
           }
           if (q_valid) {
             rs[0] = acc[0][0] + acc[0][1];
@@ -416,6 +432,11 @@ static cudaError_t launch_calib(const AttnDims& a, const void* q, const void* k,
   if (e != cudaSuccess) return e;
   e = encode_tmap_3d(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, a.g.Np, bh, 64, 64);
   if (e != cudaSuccess) return e;
+  // the register split between warpgroups needs the kernel launched at exactly kRegsLaunch
+  cudaFuncAttributes attr;
+  e = cudaFuncGetAttributes(&attr, calib_dense_mass_kernel<D>);
+  if (e != cudaSuccess) return e;
+  if (attr.numRegs != calib::kRegsLaunch) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(calib_dense_mass_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            L::kAlloc);
   if (e != cudaSuccess) return e;
