@@ -26,7 +26,7 @@ inline FastDiv make_fastdiv(int d) {
   return f;
 }
 
-__device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
+__host__ __device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
   return static_cast<int>((static_cast<unsigned long long>(static_cast<unsigned>(n)) * f.m) >>
                           f.shift);
 }
