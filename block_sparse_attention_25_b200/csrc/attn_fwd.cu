@@ -871,13 +871,16 @@ cudaError_t launch_bsattn_fwd_raster(const AttnDims& a, const void* q, const voi
 // and attends to the key clusters listed in CSR row bh * n_qc + c.
 
 // Per (bh, query cluster): the runs of <= 64 keys covering its selected key clusters, in
-// list order.  One CTA per CSR row; validates the row like bsattn_schedule_kernel.
+// list order.  One CTA per CSR row; validates the row like bsattn_schedule_kernel.  Selected
+// key clusters whose slot ranges touch (consecutive clusters of the cluster order, empty
+// ones between them included) form one span, cut into 64-key runs from its start, so only
+// a span's last run is partial: the keys attended are the same, with fewer masked columns.
 __global__ void __launch_bounds__(256) cluster_schedule_kernel(
     int n_rows, int n_kc, int max_ent, int S, const int32_t* __restrict__ row_ptr,
     const int32_t* __restrict__ col_idx, const int32_t* __restrict__ k_starts,
     const int32_t* __restrict__ k_counts, int32_t* __restrict__ ent_counts,
     uint32_t* __restrict__ entries, uint32_t* status) {
-  __shared__ int warp_tot[8];
+  __shared__ int st_sm[256], cn_sm[256];
   const int r = blockIdx.x;
   const int bh = r / n_rows;  // n_rows = query clusters per head
   const int tid = threadIdx.x;
@@ -890,16 +893,20 @@ __global__ void __launch_bounds__(256) cluster_schedule_kernel(
     return;
   }
   uint32_t* out = entries + static_cast<long long>(r) * max_ent;
-  int base = 0;
+  // walk state (thread 0): current span [span_s, span_e), next run start nb, runs written
+  int span_e = -1, nb = 0, pos = 0;
+  auto emit = [&](int start, int len) {
+    if (pos < max_ent) out[pos] = (static_cast<uint32_t>(start) << 7) | static_cast<uint32_t>(len);
+    ++pos;
+  };
   for (int e0 = beg; e0 < end; e0 += 256) {
     const int e = e0 + tid;
-    int kc = -1, nrun = 0, start = 0, cnt = 0;
+    int start = 0, cnt = 0;
     if (e < end) {
-      kc = col_idx[e];
+      const int kc = col_idx[e];
       if (kc < 0 || kc >= n_kc) {
         record_status(status, FLAG_DEVICE_INPUT, DETAIL_CSR_RANGE, static_cast<uint32_t>(r),
                       static_cast<uint32_t>(e));
-        kc = -1;
       } else {
         if (e > beg && col_idx[e - 1] >= kc)
           record_status(status, FLAG_DEVICE_INPUT, DETAIL_CSR_ORDER, static_cast<uint32_t>(r),
@@ -909,41 +916,36 @@ __global__ void __launch_bounds__(256) cluster_schedule_kernel(
         if (start < 0 || cnt < 0 || start > S - cnt) {  // runs must lie inside the head
           record_status(status, FLAG_DEVICE_INPUT, DETAIL_CLUSTER_RANGE, static_cast<uint32_t>(r),
                         static_cast<uint32_t>(e));
+          start = 0;
           cnt = 0;
         }
-        nrun = cnt > 0 ? (cnt + 63) >> 6 : 0;
       }
     }
-    // exclusive scan of the run counts over the 256 entries of this chunk
-    int incl = nrun;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane_id() >= static_cast<uint32_t>(o)) incl += y;
-    }
-    if (lane_id() == 31) warp_tot[tid >> 5] = incl;
+    st_sm[tid] = start;
+    cn_sm[tid] = cnt;
     __syncthreads();
-    int before = 0, tot = 0;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      if (w < (tid >> 5)) before += warp_tot[w];
-      tot += warp_tot[w];
+    if (tid == 0) {
+      const int n = min(256, end - e0);
+      for (int i = 0; i < n; ++i) {
+        const int a0 = st_sm[i], c0 = cn_sm[i];
+        if (c0 == 0) continue;
+        if (a0 != span_e) {  // a new span: the previous one's partial run first
+          if (span_e >= 0 && nb < span_e) emit(nb, span_e - nb);
+          nb = a0;
+        }
+        span_e = a0 + c0;
+        for (; nb + 64 <= span_e; nb += 64) emit(nb, 64);
+      }
     }
-    const int pos = base + before + incl - nrun;
-    for (int u = 0; u < nrun; ++u) {
-      const int len = min(64, cnt - 64 * u);
-      if (pos + u < max_ent)
-        out[pos + u] = (static_cast<uint32_t>(start + 64 * u) << 7) | static_cast<uint32_t>(len);
-    }
-    base += tot;
     __syncthreads();
   }
   if (tid == 0) {
-    if (base > max_ent) {
+    if (span_e >= 0 && nb < span_e) emit(nb, span_e - nb);
+    if (pos > max_ent) {
       record_status(status, FLAG_CAPACITY, DETAIL_COL_CAPACITY, static_cast<uint32_t>(r), 0u);
-      base = max_ent;
+      pos = max_ent;
     }
-    ent_counts[r] = base;
+    ent_counts[r] = pos;
   }
 }
 
