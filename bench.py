@@ -488,7 +488,7 @@ def run_e2e(args, bsa, s, draws, n_reuse, row_ptr, col_idx, flops_call, dev, str
 
     run(1)
     torch.cuda.synchronize()
-    steps = max(1, min(args.steps, 2))
+    steps = max(1, min(args.steps, 3))
     barrier(pg)
     torch.cuda.synchronize()
     counts["h2d"] = counts["d2h"] = 0
