@@ -125,6 +125,23 @@ def test_rejections_before_launch(B):
     bad[10] = ctypes.c_void_p(0x10002)                                       # lse not 4-byte aligned
     assert L.bsa_fwd(_c(B), 0, *bad, big, n) == 1
     assert L.bsa_fwd(_c(B, T=30), 0, *args, big, n) == 1                     # T > Tp
+    # the raster-layout forward: q, k, v, row_ptr, col_idx, scale, out, lse, ws
+    rargs = [FAKE, FAKE, FAKE, FAKE, FAKE, 0.088, FAKE, n, FAKE]
+    assert L.bsa_fwd_raster(_c(B), *rargs, 16, n) == 3                      # short workspace
+    bad = list(rargs)
+    bad[4] = n                                                               # col_idx missing
+    assert L.bsa_fwd_raster(_c(B), *bad, big, n) == 1
+    bad = list(rargs)
+    bad[6] = MISALIGNED                                                      # misaligned out
+    assert L.bsa_fwd_raster(_c(B), *bad, big, n) == 1
+    bad = list(rargs)
+    bad[7] = ctypes.c_void_p(0x10002)                                        # lse not 4-byte aligned
+    assert L.bsa_fwd_raster(_c(B), *bad, big, n) == 1
+    bad = list(rargs)
+    bad[5] = -1.0                                                            # bad scale
+    assert L.bsa_fwd_raster(_c(B), *bad, big, n) == 1
+    assert L.bsa_fwd_raster(_c(B, T=30), *rargs, big, n) == 1                # T > Tp
+    assert L.bsa_fwd_raster(_c(B, head_dim=96), *rargs, big, n) == 2         # unsupported D
     P = B.bsattn._Pattern
     assert L.bsa_pattern_csr(_c(B), None, FAKE, FAKE, 10, FAKE, big, n) == 1
     assert L.bsa_pattern_csr(_c(B), ctypes.byref(P(64)), FAKE, FAKE, 10, FAKE, big, n) == 1
