@@ -13,6 +13,8 @@
 //                        CTA, 4 x 4 per thread; writes the log2-domain logits into the
 //                        output tensor.
 //   pooled_softmax_kernel one warp per row: weighted softmax in place.
+#include <algorithm>
+
 #include "bsa_kernels.cuh"
 
 namespace bsa {
@@ -162,35 +164,86 @@ __global__ void __launch_bounds__(256) pooled_logits_kernel(const float* __restr
 }
 
 // In place: row of log2 logits -> n_j 2^(s_j - max) / sum.  Rows of query blocks without
-// valid queries become zero.
+// valid queries become zero.  A warp per row, looping over rows; rows of up to
+// 32 * kSmPerLane kv blocks stay in registers (one read, one write) with the weights n_j
+// from a per-CTA table; longer rows take three passes over memory.  Both give the same
+// per-lane order of operations, hence the same results.
+constexpr int kSmPerLane = 72;
 __global__ void __launch_bounds__(256) pooled_softmax_kernel(AttnDims a, long long rows,
                                                              float* __restrict__ m) {
-  const long long r = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  if (r >= rows) return;
+  __shared__ float wt[32 * kSmPerLane];
+  const bool in_regs = a.n_kb <= 32 * kSmPerLane;
+  if (in_regs) {
+    for (int j = threadIdx.x; j < a.n_kb; j += blockDim.x)
+      wt[j] = static_cast<float>(tile_valid_count(a.g, j));
+    __syncthreads();
+  }
   const int lane = threadIdx.x & 31;
-  const int i = static_cast<int>(r % a.n_qb);
   const int per = a.q_block / 64;
-  int nq = 0;
-  for (int u = i * per; u < (i + 1) * per; ++u) nq += tile_valid_count(a.g, u);
-  float* row = m + r * a.n_kb;
-  float mx = -INFINITY;
-  for (int j = lane; j < a.n_kb; j += 32) mx = fmaxf(mx, row[j]);
+  const int nu = (a.n_kb + 31) >> 5;
+  for (long long r = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5); r < rows;
+       r += static_cast<long long>(gridDim.x) * 8) {
+    const int i = static_cast<int>(r % a.n_qb);
+    int nq = 0;
+    for (int u = i * per; u < (i + 1) * per; ++u) nq += tile_valid_count(a.g, u);
+    float* row = m + r * a.n_kb;
+    if (in_regs) {
+      float v[kSmPerLane];
+      float mx = -INFINITY;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (nq == 0 || mx == -INFINITY) {  // no valid query, or no valid key in the head
-    for (int j = lane; j < a.n_kb; j += 32) row[j] = 0.f;
-    return;
-  }
-  float sum = 0.f;
-  for (int j = lane; j < a.n_kb; j += 32) {
-    const float w = static_cast<float>(tile_valid_count(a.g, j)) * exp2f(row[j] - mx);
-    row[j] = w;
-    sum += w;
-  }
+      for (int u = 0; u < kSmPerLane; ++u) {
+        const int j = lane + 32 * u;
+        v[u] = (u < nu && j < a.n_kb) ? row[j] : -INFINITY;
+        mx = fmaxf(mx, v[u]);
+      }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  const float inv = 1.f / sum;
-  for (int j = lane; j < a.n_kb; j += 32) row[j] *= inv;
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (nq == 0 || mx == -INFINITY) {  // no valid query, or no valid key in the head
+#pragma unroll
+        for (int u = 0; u < kSmPerLane; ++u) {
+          const int j = lane + 32 * u;
+          if (u < nu && j < a.n_kb) row[j] = 0.f;
+        }
+        continue;
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int u = 0; u < kSmPerLane; ++u) {
+        const int j = lane + 32 * u;
+        if (u < nu && j < a.n_kb) {
+          v[u] = wt[j] * exp2f(v[u] - mx);
+          sum += v[u];
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      const float inv = 1.f / sum;
+#pragma unroll
+      for (int u = 0; u < kSmPerLane; ++u) {
+        const int j = lane + 32 * u;
+        if (u < nu && j < a.n_kb) row[j] = v[u] * inv;
+      }
+    } else {
+      float mx = -INFINITY;
+      for (int j = lane; j < a.n_kb; j += 32) mx = fmaxf(mx, row[j]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (nq == 0 || mx == -INFINITY) {
+        for (int j = lane; j < a.n_kb; j += 32) row[j] = 0.f;
+        continue;
+      }
+      float sum = 0.f;
+      for (int j = lane; j < a.n_kb; j += 32) {
+        const float w = static_cast<float>(tile_valid_count(a.g, j)) * exp2f(row[j] - mx);
+        row[j] = w;
+        sum += w;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      const float inv = 1.f / sum;
+      for (int j = lane; j < a.n_kb; j += 32) row[j] *= inv;
+    }
+  }
 }
 
 size_t pooled_scratch_bytes(const AttnDims& a) {
@@ -209,7 +262,8 @@ cudaError_t launch_pooled_mass(const AttnDims& a, const void* q, const void* k, 
   const unsigned logit_ctas = static_cast<unsigned>(1LL * a.batch * a.heads *
                                                     ((a.n_qb + kLgTile - 1) / kLgTile) *
                                                     ((a.n_kb + kLgTile - 1) / kLgTile));
-  const unsigned sm_ctas = static_cast<unsigned>((rows + 7) / 8);
+  // a warp per row, CTAs looping over rows: the weight table is built once per CTA
+  const unsigned sm_ctas = static_cast<unsigned>(std::min<long long>((rows + 7) / 8, 148LL * 8));
   const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
   const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
   if (a.head_dim == 128) {
