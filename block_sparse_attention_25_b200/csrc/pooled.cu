@@ -59,12 +59,13 @@ __global__ void __launch_bounds__(256) pool_tiles_kernel(const __nv_bfloat16* __
 
 // Logits in log2 units: scale * log2(e) * qbar_i . kbar_j, -inf for tiles without valid keys
 // (the softmax kernel adds log2(n_j)).  A register-tiled product per (bh): a CTA of 256
-// threads computes a 64 x 64 tile of (query block, kv block) logits, 4 x 4 per thread; the
-// head dimension is staged 16 at a time in shared memory as [d][block] so each thread
-// reads its four qbar and four kbar values with two 16-byte loads.  qbar and kbar are formed
-// while staging: sums of the block's tiles times 1 / valid count (0 for an empty block).
-// Every logit sums over d in order 0..D-1 (deterministic).
-constexpr int kLgTile = 64;
+// threads computes a 128 x 128 tile of (query block, kv block) logits, 8 x 8 per thread
+// (rows 4ty..4ty+3 and 64+4ty.., columns likewise, so each 16-byte shared load of a warp is
+// conflict-free); the head dimension is staged 16 at a time in shared memory as
+// [d][block].  qbar and kbar are formed while staging: sums of the block's tiles times
+// 1 / valid count (0 for an empty block).  Every logit sums over d in order 0..D-1
+// (deterministic).
+constexpr int kLgTile = 128;
 constexpr int kLgK = 16;
 
 template <int D>
@@ -92,23 +93,25 @@ __global__ void __launch_bounds__(256) pooled_logits_kernel(const float* __restr
     if (i < a.n_qb)
       for (int u = i * per; u < (i + 1) * per; ++u) cnt += tile_valid_count(a.g, u);
     s_qinv[tid] = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
-  } else if (tid < 2 * kLgTile) {
+  } else {
     const int j = j0 + tid - kLgTile;
     const int cnt = j < a.n_kb ? tile_valid_count(a.g, j) : 0;
     s_kinv[tid - kLgTile] = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
   }
-  const int ty = tid >> 4, tx = tid & 15;  // rows 4ty.., cols 4tx..
-  float acc[4][4];
+  const int ty = tid >> 4, tx = tid & 15;
+  float acc[8][8];
 #pragma unroll
-  for (int r = 0; r < 4; ++r)
+  for (int r = 0; r < 8; ++r)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
   for (int d0 = 0; d0 < D; d0 += kLgK) {
     __syncthreads();
-    // stage 64 blocks x 16 dims of qbar and kbar, transposed to [d][block]: one 16-byte
-    // load of four consecutive dims per thread and matrix (64 x 16 = 256 x 4)
-    {
-      const int blk = tid >> 2, dq = (tid & 3) * 4;
+    // stage 128 blocks x 16 dims of qbar and kbar, transposed to [d][block]: two 16-byte
+    // loads of four consecutive dims per thread and matrix (128 x 16 = 2 x 256 x 4)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int f = tid + 256 * h;
+      const int blk = f >> 2, dq = (f & 3) * 4;
       const int i = i0 + blk, j = j0 + blk;
       float4 qv = make_float4(0.f, 0.f, 0.f, 0.f), kv = qv;
       if (i < a.n_qb) {
@@ -119,13 +122,13 @@ __global__ void __launch_bounds__(256) pooled_logits_kernel(const float* __restr
           qv.z += t.z;
           qv.w += t.w;
         }
-        const float f = s_qinv[blk];
-        qv = make_float4(qv.x * f, qv.y * f, qv.z * f, qv.w * f);
+        const float fq = s_qinv[blk];
+        qv = make_float4(qv.x * fq, qv.y * fq, qv.z * fq, qv.w * fq);
       }
       if (j < a.n_kb) {
         const float4 t = *reinterpret_cast<const float4*>(ksum + (tbase + j) * D + d0 + dq);
-        const float f = s_kinv[blk];
-        kv = make_float4(t.x * f, t.y * f, t.z * f, t.w * f);
+        const float fk = s_kinv[blk];
+        kv = make_float4(t.x * fk, t.y * fk, t.z * fk, t.w * fk);
       }
       sa[dq + 0][blk] = qv.x;
       sa[dq + 1][blk] = qv.y;
@@ -139,26 +142,39 @@ __global__ void __launch_bounds__(256) pooled_logits_kernel(const float* __restr
     __syncthreads();
 #pragma unroll
     for (int d = 0; d < kLgK; ++d) {
-      const float4 av = *reinterpret_cast<const float4*>(&sa[d][4 * ty]);
-      const float4 bv = *reinterpret_cast<const float4*>(&sb[d][4 * tx]);
-      const float ar[4] = {av.x, av.y, av.z, av.w};
-      const float br[4] = {bv.x, bv.y, bv.z, bv.w};
+      const float4 a0 = *reinterpret_cast<const float4*>(&sa[d][4 * ty]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&sa[d][64 + 4 * ty]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&sb[d][4 * tx]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&sb[d][64 + 4 * tx]);
+      const float ar[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float br[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int r = 0; r < 8; ++r)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(ar[r], br[c], acc[r][c]);
+        for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(ar[r], br[c], acc[r][c]);
     }
   }
+  const bool vec = (a.n_kb & 3) == 0;  // rows start 16-byte aligned
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int i = i0 + 4 * ty + r;
+  for (int r = 0; r < 8; ++r) {
+    const int i = i0 + (r < 4 ? 4 * ty + r : 64 + 4 * ty + r - 4);
     if (i >= a.n_qb) continue;
+    float* orow = out + (static_cast<long long>(bh) * a.n_qb + i) * a.n_kb;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int j = j0 + 4 * tx + c;
-      if (j < a.n_kb)
-        out[(static_cast<long long>(bh) * a.n_qb + i) * a.n_kb + j] =
-            s_kinv[4 * tx + c] > 0.f ? acc[r][c] * scale_log2 : -INFINITY;
+    for (int g = 0; g < 2; ++g) {
+      const int cl = 64 * g + 4 * tx;  // first of four columns inside the tile
+      const int j = j0 + cl;
+      float v[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        v[c] = s_kinv[cl + c] > 0.f ? acc[r][4 * g + c] * scale_log2 : -INFINITY;
+      if (vec && j + 3 < a.n_kb) {
+        *reinterpret_cast<float4*>(orow + j) = make_float4(v[0], v[1], v[2], v[3]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (j + c < a.n_kb) orow[j + c] = v[c];
+      }
     }
   }
 }
