@@ -9,18 +9,22 @@
 //
 // One CTA owns 256 query slots (two M=128 tiles) and walks every kv block twice, two
 // blocks (N = 128 keys) per step:
-//   pass 1: S = Q K^T on the tensor cores, online row max and sum -> exact log-sum-exp;
-//   pass 2: S again, p = exp2(S*c - lse2), per-block row sums, then a sum over the rows
-//           of each query block (warp shuffles + shared memory, fixed order, so the result
-//           is deterministic).
+//   pass 1: S = Q K^T on the tensor cores and the row max only (no exponentials);
+//   pass 2: S again, e[r,j] = sum over the keys of block j of exp2(S*c - max_r) -- every
+//           exponential of the calibration computed once -- written to this SM's slice of
+//           the workspace, and the row sums l_r = sum_j e[r,j];
+//   end:    mass[i,j] = (1 / valid queries of i) * sum over the rows r of query block i of
+//           e[r,j] / l_r, in a fixed order (deterministic).
+// The scratch slice is chosen by the SM the CTA runs on: the CTA's shared memory admits one
+// CTA per SM, so no two live CTAs share a slice.
 // Warp roles (576 threads): warps 0-7 and 10-17 own the rows, two threads per row: warps
 // 0-3 / 4-7 take the first kv block of each step of tile 0 / 1, warps 10-13 / 14-17 the
 // second (a warp reads the TMEM lane quarter of its sub-partition, warp % 4); warp 8 is
 // the TMA producer (K only), warp 9 the MMA issuer and TMEM owner.  Each thread keeps its
-// own running (max, sum) over its kv blocks; the two halves of a row are combined once,
-// at the end of pass 1.  Four row warps per sub-partition (instead of two) keep the
-// exponential unit fed.  TMEM holds two S buffers per tile (4 x 128 columns), so the
-// tensor core computes step s+1 while step s is reduced.
+// own running max and sum over its kv blocks; the two halves of a row are combined at the
+// end of each pass.  Four row warps per sub-partition keep the exponential unit fed.  TMEM
+// holds two S buffers per tile (4 x 128 columns), so the tensor core computes step s+1
+// while step s is reduced.
 #include "bsa_kernels.cuh"
 
 namespace bsa {
@@ -31,12 +35,16 @@ constexpr int kRowsPerCta = 256;
 // 18 warps: 5 share sub-partitions 0 and 1, whose 16K-register files then allow 96
 // registers per thread.
 constexpr int kMaxRegs = 96;
+// Scratch slices (one per SM id): comfortably above the SM ids of sm_100 parts; a CTA on an
+// SM id beyond it records a device flag and writes no masses.
+constexpr int kSlots = 192;
 }  // namespace mass
 
 struct MassParams {
   AttnDims a;
   float* mass;
   uint32_t* status;
+  float* scratch;  // [kSlots][n_kb][256] unnormalised row-block sums
   float scale_log2;
 };
 
@@ -48,8 +56,8 @@ struct MassSmem {
   static constexpr int kKStages = (D == 128) ? 4 : 6;
   static constexpr int kQOff = 0;
   static constexpr int kKOff = 2 * kQTile;
-  static constexpr int kRedOff = kKOff + kKStages * kKStage;   // float [2 parity][2 tile][4 warp][2 half]
-  static constexpr int kXchOff = kRedOff + 2 * 2 * 4 * 2 * 4;   // float [2 tile][2 half][128 row][2]
+  static constexpr int kRedOff = kKOff + kKStages * kKStage;   // float [256] 1 / row sum
+  static constexpr int kXchOff = kRedOff + 256 * 4;             // float [2 tile][2 half][128 row][2]
   static constexpr int kBarOff = kXchOff + 2 * 2 * 128 * 2 * 4;
   static constexpr int kBytes = kBarOff + 512;
   static constexpr int kAlloc = kBytes + 1024;
@@ -74,7 +82,7 @@ __global__ void __maxnreg__(mass::kMaxRegs)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* nvalid_sm = reinterpret_cast<int*>(tmem_slot + 2);  // [2 half][2 tile][4 warp]
-  float* red = reinterpret_cast<float*>(smem + L::kRedOff);
+  float* inv_l = reinterpret_cast<float*>(smem + L::kRedOff);
   float* xch = reinterpret_cast<float*>(smem + L::kXchOff);
 
   const AttnDims& a = p.a;
@@ -181,20 +189,19 @@ __global__ void __maxnreg__(mass::kMaxRegs)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float c = p.scale_log2;
     const int gbar = 1 + 2 * t + h;  // named barrier of the 4 warps of (tile, half)
-    // valid queries per warp, then per query block
+    // valid queries per warp (for the per-query-block means at the end)
     const int wcount = __popc(__ballot_sync(0xffffffffu, q_valid));
     if (lane == 0) nvalid_sm[(h * 2 + t) * 4 + wq] = wcount;
     named_bar_sync(gbar, 128);
-    const int warps_per_qb = a.q_block / 32;  // 2 or 4
-    const int qb_first_warp = (wq / warps_per_qb) * warps_per_qb;
-    int nvq = 0;
-    for (int i = 0; i < warps_per_qb; ++i) nvq += nvalid_sm[(h * 2 + t) * 4 + qb_first_warp + i];
-    const int qb_global = (row0 + t * 128 + qb_first_warp * 32) / a.q_block;
-    const bool writer = (wq == qb_first_warp) && lane == 0 && qb_global < a.n_qb;
-    float* mass_row = p.mass + (static_cast<long long>(bh) * a.n_qb + qb_global) * a.n_kb;
-    const float inv_nvq = nvq > 0 ? 1.f / static_cast<float>(nvq) : 0.f;
+    // this SM's scratch slice: [n_kb][256] row-block sums
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    const bool have_slice = smid < static_cast<uint32_t>(mass::kSlots);
+    if (!have_slice && h == 0 && local == 0)
+      record_status(p.status, FLAG_DEVICE_INPUT, DETAIL_MASS_SLICE, static_cast<uint32_t>(cta), smid);
+    float* sc = p.scratch + static_cast<size_t>(have_slice ? smid : 0u) * 256 * a.n_kb;
 
-    float m_run = -INFINITY, l_run = 0.f, lse2 = 0.f;
+    float m_run = -INFINITY, l_run = 0.f, m_row = -INFINITY;
     bool ok = true;
     // tile coordinates of this half's kv block 2*st + h, advanced incrementally (no
     // division inside the loop: integer division shares the pipe of the exponentials)
@@ -209,19 +216,10 @@ __global__ void __maxnreg__(mass::kMaxRegs)
       if (s == npass) {
         tw = th = tt = 0;
         tile_advance(a.g, h, tw, th, tt);
-        // Both halves' (max, sum) of the row -> the row's exact log-sum-exp (log2 units),
-        // combined in the same order by both threads.
-        float* x = xch + ((t * 2 + h) * 128 + row) * 2;
-        x[0] = m_run;
-        x[1] = l_run;
+        // both halves' maxima -> the row max (log2 units)
+        xch[((t * 2 + h) * 128 + row) * 2] = m_run;
         named_bar_sync(5 + t, 256);
-        const float* y0 = xch + ((t * 2 + 0) * 128 + row) * 2;
-        const float* y1 = xch + ((t * 2 + 1) * 128 + row) * 2;
-        const float m = fmaxf(y0[0], y1[0]);
-        const float l = (m == -INFINITY)
-                            ? 0.f
-                            : y0[1] * fast_exp2(y0[0] - m) + y1[1] * fast_exp2(y1[0] - m);
-        lse2 = (l > 0.f) ? m + log2f(l) : INFINITY;
+        m_row = fmaxf(xch[((t * 2 + 0) * 128 + row) * 2], xch[((t * 2 + 1) * 128 + row) * 2]);
       }
       // A warp that gives up keeps stepping (without touching TMEM) so that every warp of
       // the group passes the same named barriers.
@@ -230,7 +228,6 @@ __global__ void __maxnreg__(mass::kMaxRegs)
                     : false;
       got = __all_sync(0xffffffffu, got);
       ok = got;
-      float rs = 0.f;
       if (got) {
         float sv[64];
         tc_fence_after();
@@ -258,36 +255,61 @@ __global__ void __maxnreg__(mass::kMaxRegs)
             for (int i = 8; i < 64; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
             const float mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-            const float m_new = fmaxf(m_run, mrow * c);
-            if (m_new != -INFINITY) {
-              float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            m_run = fmaxf(m_run, mrow * c);  // c > 0, so -inf stays -inf
+          } else {
+            float e = 0.f;
+            if (m_row != -INFINITY) {
+              float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-              for (int i = 0; i < 64; ++i) ls[i & 3] += fast_exp2(fmaf(sv[i], c, -m_new));
-              l_run = l_run * fast_exp2(m_run - m_new) + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-              m_run = m_new;
+              for (int i = 0; i < 64; ++i) acc[i & 3] += fast_exp2(fmaf(sv[i], c, -m_row));
+              e = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             }
-          } else if (q_valid) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int i = 0; i < 64; ++i) acc[i & 3] += fast_exp2(fmaf(sv[i], c, -lse2));
-            rs = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            l_run += e;
+            if (have_slice) sc[static_cast<size_t>(2 * st + h) * 256 + local] = e;
           }
         }
       }
       tile_advance(a.g, 2, tw, th, tt);
-      if (pass2) {
-        // Sum the per-row block masses over the rows of each query block: warp shuffles,
-        // then the 2 or 4 warps of the block through shared memory in a fixed order.
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
-        float* rbuf = red + ((s & 1) * 2 + t) * 8;
-        if (lane == 0) rbuf[wq * 2 + h] = rs;
-        named_bar_sync(gbar, 128);
-        if (writer && mine) {
-          float tot = 0.f;
-          for (int i = 0; i < warps_per_qb; ++i) tot += rbuf[(qb_first_warp + i) * 2 + h];
-          mass_row[2 * st + h] = tot * inv_nvq;
+    }
+
+    // ------------------------------------------------------------ masses
+    // Row sum = the halves' partial sums (first half + second, in both threads); then
+    // mass[i, j] = (1 / valid queries of i) * sum_r e[r, j] / l_r over the rows of query
+    // block i, in row order, by all 512 row threads over the CTA's (query block, kv block)
+    // outputs.
+    xch[((t * 2 + h) * 128 + row) * 2 + 1] = l_run;
+    named_bar_sync(5 + t, 256);
+    if (h == 0) {
+      const float l = xch[((t * 2 + 0) * 128 + row) * 2 + 1] + xch[((t * 2 + 1) * 128 + row) * 2 + 1];
+      inv_l[local] = (q_valid && ok && l > 0.f) ? 1.f / l : 0.f;
+    }
+    named_bar_sync(7, 512);  // every row's block sums and 1 / l_r are written
+    if (have_slice) {
+      const int rt = (h ? warp - 10 : warp) * 32 + lane + 256 * h;  // 0 .. 511
+      const int warps_per_qb = a.q_block / 32;  // 2 or 4
+      const int nq_cta = mass::kRowsPerCta / a.q_block;
+      const int qb0 = row0 / a.q_block;
+      for (int o = rt; o < nq_cta * a.n_kb; o += 512) {
+        const int qi = o / a.n_kb;
+        const int j = o - qi * a.n_kb;
+        const int qb = qb0 + qi;
+        if (qb >= a.n_qb) continue;
+        int nvq = 0;
+        for (int w = 0; w < warps_per_qb; ++w) {
+          const int r0 = qi * a.q_block + 32 * w;  // first row of the warp's 32 in the CTA
+          nvq += nvalid_sm[(r0 >> 7) * 4 + ((r0 & 127) >> 5)];
         }
+        const float* col = sc + static_cast<size_t>(j) * 256 + qi * a.q_block;
+        float tot = 0.f;
+        for (int r = 0; r < a.q_block; r += 4) {
+          const float4 ev = *reinterpret_cast<const float4*>(col + r);
+          tot += ev.x * inv_l[qi * a.q_block + r];
+          tot += ev.y * inv_l[qi * a.q_block + r + 1];
+          tot += ev.z * inv_l[qi * a.q_block + r + 2];
+          tot += ev.w * inv_l[qi * a.q_block + r + 3];
+        }
+        p.mass[(static_cast<long long>(bh) * a.n_qb + qb) * a.n_kb + j] =
+            nvq > 0 ? tot / static_cast<float>(nvq) : 0.f;
       }
     }
   }
@@ -301,9 +323,9 @@ __global__ void __maxnreg__(mass::kMaxRegs)
   }
 }
 
+// Scratch after the status header: kSlots slices of n_kb x 256 fp32 row-block sums.
 size_t mass_scratch_bytes(const AttnDims& a) {
-  (void)a;
-  return 0;
+  return static_cast<size_t>(mass::kSlots) * 256 * static_cast<size_t>(a.n_kb) * sizeof(float);
 }
 
 template <int D>
@@ -332,6 +354,7 @@ cudaError_t launch_block_mass(const AttnDims& a, const void* q, const void* k, f
   prm.a = a;
   prm.mass = mass_out;
   prm.status = static_cast<uint32_t*>(ws);
+  prm.scratch = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kStatusBytes);
   prm.scale_log2 = softmax_scale * 1.4426950408889634f;
   if (a.head_dim == 128) return launch_mass<128>(a, q, k, prm, ctas, stream);
   return launch_mass<64>(a, q, k, prm, ctas, stream);

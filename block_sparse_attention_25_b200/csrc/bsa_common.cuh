@@ -37,6 +37,7 @@ enum : uint32_t {
   DETAIL_CSR_ORDER = 0x202,
   DETAIL_CSR_ROWPTR = 0x203,
   DETAIL_CLUSTER_RANGE = 0x204,
+  DETAIL_MASS_SLICE = 0x205,
   DETAIL_COL_CAPACITY = 0x300,
 };
 

@@ -141,7 +141,10 @@ BSA_API bsa_status bsa_tile_permute_quant_e4m3(const bsa_shape* shape, const voi
  * zero pad slots.  mass: fp32 [B,Hh,Np/q_block,Np/64]; mass[b,h,i,j] is the mean over
  * the valid queries of block i of the softmax(softmax_scale * q.k) probability on the
  * valid keys of block j (pad keys excluded).  Rows of a block with no valid query are
- * zero.  Two dense passes on tcgen05 tensor cores (log-sum-exp, then mass). */
+ * zero.  Two dense passes on tcgen05 tensor cores: the row maxima, then every probability
+ * once (unnormalised block sums per row, kept in the workspace, normalised by the row
+ * sums at the end).  Workspace: bsa_workspace_bytes(shape, BSA_OP_BLOCK_MASS) -- the
+ * status header plus 192 slices of 256 x Np/64 fp32, one per SM id. */
 BSA_API bsa_status bsa_block_mass(const bsa_shape* shape, const void* q, const void* k,
                           float softmax_scale, float* mass, void* ws, size_t ws_bytes,
                           bsa_stream_t stream);
