@@ -35,16 +35,13 @@ constexpr int kRowsPerCta = 256;
 // 18 warps: 5 share sub-partitions 0 and 1, whose 16K-register files then allow 96
 // registers per thread.
 constexpr int kMaxRegs = 96;
-// Scratch slices (one per SM id): comfortably above the SM ids of sm_100 parts; a CTA on an
-// SM id beyond it records a device flag and writes no masses.
-constexpr int kSlots = 192;
 }  // namespace mass
 
 struct MassParams {
   AttnDims a;
   float* mass;
   uint32_t* status;
-  float* scratch;  // [kSlots][n_kb][256] unnormalised row-block sums
+  float* scratch;  // [kMassSlots][n_kb][256] unnormalised row-block sums
   float scale_log2;
 };
 
@@ -196,7 +193,7 @@ __global__ void __maxnreg__(mass::kMaxRegs)
     // this SM's scratch slice: [n_kb][256] row-block sums
     uint32_t smid;
     asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-    const bool have_slice = smid < static_cast<uint32_t>(mass::kSlots);
+    const bool have_slice = smid < static_cast<uint32_t>(kMassSlots);
     if (!have_slice && h == 0 && local == 0)
       record_status(p.status, FLAG_DEVICE_INPUT, DETAIL_MASS_SLICE, static_cast<uint32_t>(cta), smid);
     float* sc = p.scratch + static_cast<size_t>(have_slice ? smid : 0u) * 256 * a.n_kb;
@@ -323,9 +320,9 @@ __global__ void __maxnreg__(mass::kMaxRegs)
   }
 }
 
-// Scratch after the status header: kSlots slices of n_kb x 256 fp32 row-block sums.
+// Scratch after the status header: kMassSlots slices of n_kb x 256 fp32 row-block sums.
 size_t mass_scratch_bytes(const AttnDims& a) {
-  return static_cast<size_t>(mass::kSlots) * 256 * static_cast<size_t>(a.n_kb) * sizeof(float);
+  return static_cast<size_t>(kMassSlots) * 256 * static_cast<size_t>(a.n_kb) * sizeof(float);
 }
 
 template <int D>

@@ -188,6 +188,10 @@ cudaError_t launch_bsattn_fwd(const AttnDims& a, int fp8, const void* q, const v
                               void* ws, cudaStream_t stream);
 
 // Dense calibration pass.
+// Per-SM scratch of the calibration kernels: kMassSlots slices (one per SM id, comfortably
+// above the SM ids of sm_100 parts) of 256 rows x n_kb fp32 row-block sums.  A CTA on an SM
+// id beyond them records DETAIL_MASS_SLICE and writes no masses.
+constexpr int kMassSlots = 192;
 size_t mass_scratch_bytes(const AttnDims& a);
 cudaError_t launch_block_mass(const AttnDims& a, const void* q, const void* k, float softmax_scale,
                               float* mass, void* ws, cudaStream_t stream);

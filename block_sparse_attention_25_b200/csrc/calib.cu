@@ -5,10 +5,12 @@
 // Abstract: the calibration step runs dense attention and measures the exact block masses
 // on it.  Computing them separately costs two QK^T passes for the masses plus a QK^T and a
 // PV pass for the output; here
-//   pass 1: S = Q K^T over every kv block -> exact row log-sum-exp (online max and sum);
-//   pass 2: S again, P = exp2(S*c - lse2) -- the exact softmax probabilities, <= 1 -- used
-//           both for the per-block mass sums and, stored to TMEM as bf16, for O += P V.
-// Since P is already normalised, O needs no rescaling and no final division.
+//   pass 1: S = Q K^T over every kv block -> the exact row max (no exponentials);
+//   pass 2: S again, P = exp2(S*c - max_r) <= 1, every probability computed once: stored to
+//           TMEM as bf16 for O += P V (no rescaling: the reference max is final), summed per
+//           kv block into this SM's workspace slice, and into the row sum l_r;
+//   end:    O / l_r, and mass[i,j] = (1 / valid queries of i) * sum over the rows of query
+//           block i of e[r,j] / l_r in a fixed order, as in bsa_block_mass.
 //
 // Layout and roles follow the block-sparse forward (attn_fwd.cu): 256 query slots per CTA
 // in two M=128 tiles, 384 threads (warps 0-7 row owners, warp 8 TMA, warp 9 MMA, warps
@@ -38,6 +40,7 @@ struct CalibParams {
   float* lse;
   float* mass;
   uint32_t* status;
+  float* scratch;  // [kMassSlots][n_kb][256] unnormalised row-block sums
   float scale_log2;
 };
 
@@ -51,8 +54,8 @@ struct CalibSmem {
   static constexpr int kQOff = 0;
   static constexpr int kKOff = 2 * kQTile;
   static constexpr int kVOff = kKOff + kKStages * kKVStage;
-  static constexpr int kRedOff = kVOff + kVStages * kKVStage;  // float [2 parity][2 tile][4 warp][2 blk]
-  static constexpr int kBarOff = kRedOff + 2 * 2 * 4 * 2 * 4;
+  static constexpr int kRedOff = kVOff + kVStages * kKVStage;  // float [256] 1 / row sum
+  static constexpr int kBarOff = kRedOff + 256 * 4;
   static constexpr int kBytes = kBarOff + 512;
   static constexpr int kAlloc = kBytes + 1024;
 };
@@ -81,7 +84,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* nvalid_sm = reinterpret_cast<int*>(tmem_slot + 2);  // [2 tile][4 warp]
-  float* red = reinterpret_cast<float*>(smem + L::kRedOff);
+  float* inv_l_sm = reinterpret_cast<float*>(smem + L::kRedOff);
 
   const AttnDims& a = p.a;
   const int warp = threadIdx.x >> 5;
@@ -254,7 +257,8 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
     const int t = warp >> 2;
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
-    const int slot = row0 + t * 128 + row;
+    const int local = t * 128 + row;
+    const int slot = row0 + local;
     const bool in_range = slot < a.g.Np;
     const bool q_valid = in_range && slot_valid(a.g, slot);
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
@@ -264,29 +268,26 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
     const int wcount = __popc(__ballot_sync(0xffffffffu, q_valid));
     if (lane == 0) nvalid_sm[t * 4 + wq] = wcount;
     named_bar_sync(1 + t, 128);
-    const int warps_per_qb = a.q_block / 32;  // 2 or 4
-    const int qb_first_warp = (wq / warps_per_qb) * warps_per_qb;
-    int nvq = 0;
-    for (int i = 0; i < warps_per_qb; ++i) nvq += nvalid_sm[t * 4 + qb_first_warp + i];
-    const int qb_global = (row0 + t * 128 + qb_first_warp * 32) / a.q_block;
-    const bool writer = (wq == qb_first_warp) && lane < 2 && qb_global < a.n_qb;
-    float* mass_row = p.mass + (static_cast<long long>(bh) * a.n_qb + qb_global) * a.n_kb;
-    const float inv_nvq = nvq > 0 ? 1.f / static_cast<float>(nvq) : 0.f;
+    // this SM's workspace slice: [n_kb][256] row-block sums
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    const bool have_slice = smid < static_cast<uint32_t>(kMassSlots);
+    if (!have_slice && local == 0)
+      record_status(p.status, FLAG_DEVICE_INPUT, DETAIL_MASS_SLICE, static_cast<uint32_t>(cta), smid);
+    float* sc = p.scratch + static_cast<size_t>(have_slice ? smid : 0u) * 256 * a.n_kb;
 
-    float m_run = -INFINITY, l_run = 0.f, lse2 = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int s = 0; s < nsteps; ++s) {
       const int st = s >= npass ? s - npass : s;
       const bool pass2 = s >= npass;
       const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
-      if (s == npass) lse2 = (l_run > 0.f) ? m_run + log2f(l_run) : INFINITY;
-      // A warp that gives up keeps stepping (without touching TMEM) so that every warp of
-      // the group passes the same named barriers.
+      // A warp that gives up keeps stepping (without touching TMEM) so that the row warps
+      // all reach the barrier before the masses.
       bool got = ok ? mbar_wait(bar_sfull + t, s & 1, abort_flag, p.status, DETAIL_WAIT_S_FULL)
                     : false;
       got = __all_sync(0xffffffffu, got);
       ok = got;
-      float rs[2] = {0.f, 0.f};
       if (got) {
         tc_fence_after();
         float sv[128];
@@ -320,16 +321,11 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
           for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
           const float mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                    fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-          const float m_new = fmaxf(m_run, mrow * c);
-          if (m_new != -INFINITY) {
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int i = 0; i < 128; ++i) ls[i & 3] += fast_exp2(fmaf(sv[i], c, -m_new));
-            l_run = l_run * fast_exp2(m_run - m_new) + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-            m_run = m_new;
-          }
+          m_run = fmaxf(m_run, mrow * c);  // c > 0, so -inf stays -inf
         } else {
-          // exact probabilities; pad query rows contribute nothing to the masses
+          // probabilities against the final row max (<= 1); a row with no valid key has
+          // m_run = -inf and every probability 0
+          const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
           float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
@@ -337,8 +333,8 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float p0 = fast_exp2(fmaf(sv[32 * ch + 2 * i], c, -lse2));
-              const float p1 = fast_exp2(fmaf(sv[32 * ch + 2 * i + 1], c, -lse2));
+              const float p0 = fast_exp2(fmaf(sv[32 * ch + 2 * i], c, -m_use));
+              const float p1 = fast_exp2(fmaf(sv[32 * ch + 2 * i + 1], c, -m_use));
               acc[ch >> 1][i & 1] += p0 + p1;
               pk[i] = pack_bf16x2(p0, p1);
             }
@@ -349,30 +345,16 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
               mbar_arrive(bar_ppart + t);
             }
           }
-          if (q_valid) {
-            rs[0] = acc[0][0] + acc[0][1];
-            rs[1] = acc[1][0] + acc[1][1];
+          const float e0 = acc[0][0] + acc[0][1];
+          const float e1 = acc[1][0] + acc[1][1];
+          l_run += e0 + e1;
+          if (have_slice) {
+            sc[static_cast<size_t>(j0) * 256 + local] = e0;
+            if (nb == 2) sc[static_cast<size_t>(j0 + 1) * 256 + local] = e1;
           }
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(bar_pfull + t);
-        }
-      }
-      if (pass2) {
-        // per-(query block, kv block) sums: warp shuffles, then the 2 or 4 warps of the
-        // query block through shared memory in a fixed order (deterministic)
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          rs[0] += __shfl_xor_sync(0xffffffffu, rs[0], o);
-          rs[1] += __shfl_xor_sync(0xffffffffu, rs[1], o);
-        }
-        float* rbuf = red + ((s & 1) * 2 + t) * 8;
-        if (lane < 2) rbuf[wq * 2 + lane] = lane == 0 ? rs[0] : rs[1];
-        named_bar_sync(1 + t, 128);
-        if (writer && (lane < nb)) {
-          float tot = 0.f;
-          for (int i = 0; i < warps_per_qb; ++i) tot += rbuf[(qb_first_warp + i) * 2 + lane];
-          mass_row[2 * st + lane] = tot * inv_nvq;
         }
       }
     }
@@ -384,7 +366,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
                           mbar_wait(bar_ofull, 0, abort_flag, p.status, DETAIL_WAIT_O_FULL));
       tc_fence_after();
     }
-    const float omul = (q_valid && l_run > 0.f) ? 1.f : 0.f;
+    const float inv_l = (q_valid && l_run > 0.f) ? 1.f / l_run : 0.f;
     __nv_bfloat16* orow = p.out + (static_cast<long long>(bh) * a.g.Np + slot) * D;
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
@@ -400,7 +382,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
         uint4 w[4];
         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) wp[i] = pack_bf16x2(ov[2 * i] * omul, ov[2 * i + 1] * omul);
+        for (int i = 0; i < 16; ++i) wp[i] = pack_bf16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l);
         uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
         for (int i = 0; i < 4; ++i) dst[i] = w[i];
@@ -408,7 +390,41 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
     }
     if (p.lse != nullptr && in_range)
       p.lse[static_cast<long long>(bh) * a.g.Np + slot] =
-          (q_valid && l_run > 0.f) ? lse2 * 0.6931471805599453f : -INFINITY;
+          (q_valid && l_run > 0.f) ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+
+    // ------------------------------------------------------------ masses
+    // mass[i, j] = (1 / valid queries of i) * sum_r e[r, j] / l_r over the rows of query
+    // block i, in row order, by the 256 row threads over the CTA's outputs.
+    inv_l_sm[local] = (q_valid && ok && l_run > 0.f) ? 1.f / l_run : 0.f;
+    named_bar_sync(7, 256);  // every row's block sums and 1 / l_r are written
+    if (have_slice) {
+      const int rt = warp * 32 + lane;  // 0 .. 255
+      const int warps_per_qb = a.q_block / 32;  // 2 or 4
+      const int nq_cta = calib::kRowsPerCta / a.q_block;
+      const int qb0 = row0 / a.q_block;
+      for (int o = rt; o < nq_cta * a.n_kb; o += 256) {
+        const int qi = o / a.n_kb;
+        const int j = o - qi * a.n_kb;
+        const int qb = qb0 + qi;
+        if (qb >= a.n_qb) continue;
+        int nvq = 0;
+        for (int w = 0; w < warps_per_qb; ++w) {
+          const int r0 = qi * a.q_block + 32 * w;  // first row of the warp's 32 in the CTA
+          nvq += nvalid_sm[(r0 >> 7) * 4 + ((r0 & 127) >> 5)];
+        }
+        const float* col = sc + static_cast<size_t>(j) * 256 + qi * a.q_block;
+        float tot = 0.f;
+        for (int r = 0; r < a.q_block; r += 4) {
+          const float4 ev = *reinterpret_cast<const float4*>(col + r);
+          tot += ev.x * inv_l_sm[qi * a.q_block + r];
+          tot += ev.y * inv_l_sm[qi * a.q_block + r + 1];
+          tot += ev.z * inv_l_sm[qi * a.q_block + r + 2];
+          tot += ev.w * inv_l_sm[qi * a.q_block + r + 3];
+        }
+        p.mass[(static_cast<long long>(bh) * a.n_qb + qb) * a.n_kb + j] =
+            nvq > 0 ? tot / static_cast<float>(nvq) : 0.f;
+      }
+    }
   }
 
   __syncwarp();
@@ -456,6 +472,7 @@ cudaError_t launch_calib_dense_mass(const AttnDims& a, const void* q, const void
   prm.lse = lse;
   prm.mass = mass;
   prm.status = static_cast<uint32_t*>(ws);
+  prm.scratch = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kStatusBytes);
   prm.scale_log2 = softmax_scale * 1.4426950408889634f;
   if (a.head_dim == 128) return launch_calib<128>(a, q, k, v, prm, ctas, stream);
   return launch_calib<64>(a, q, k, v, prm, ctas, stream);
