@@ -17,7 +17,8 @@
  * Conventions shared by every call
  *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The library
  *     allocates no memory and keeps no global state; scratch space is the caller's
- *     workspace (`ws`), sized by bsa_workspace_bytes().
+ *     workspace (`ws`), sized by bsa_workspace_bytes().  A workspace serves one call at a
+ *     time: calls that may overlap (other streams) need workspaces of their own.
  *   - Every call is asynchronous and ordered on `stream` (NULL = legacy default
  *     stream).  A call returns after launching; results are ready when the stream is.
  *   - Arguments are checked on the host before anything is launched.  A bad argument
