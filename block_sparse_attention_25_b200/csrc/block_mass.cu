@@ -338,6 +338,12 @@ static cudaError_t launch_mass(const AttnDims& a, const void* q, const void* k,
   e = cudaFuncSetAttribute(block_mass_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            L::kAlloc);
   if (e != cudaSuccess) return e;
+  // the workspace slices are per SM id: at most one CTA of this kernel may live on an SM
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, block_mass_kernel<D>, mass::kThreads,
+                                                    L::kAlloc);
+  if (e != cudaSuccess) return e;
+  if (per_sm != 1) return cudaErrorInvalidConfiguration;
   block_mass_kernel<D><<<static_cast<unsigned>(ctas), mass::kThreads, L::kAlloc, stream>>>(tq, tk,
                                                                                           prm);
   return cudaGetLastError();

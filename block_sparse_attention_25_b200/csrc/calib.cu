@@ -456,6 +456,12 @@ static cudaError_t launch_calib(const AttnDims& a, const void* q, const void* k,
   e = cudaFuncSetAttribute(calib_dense_mass_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            L::kAlloc);
   if (e != cudaSuccess) return e;
+  // the workspace slices are per SM id: at most one CTA of this kernel may live on an SM
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, calib_dense_mass_kernel<D>,
+                                                    calib::kThreads, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  if (per_sm != 1) return cudaErrorInvalidConfiguration;
   calib_dense_mass_kernel<D><<<static_cast<unsigned>(ctas), calib::kThreads, L::kAlloc, stream>>>(
       tq, tk, tv, prm);
   return cudaGetLastError();
