@@ -7,24 +7,27 @@
 // mass[b,h,i,j] = mean over the valid queries q of block i of
 //                 sum over the valid keys k of block j of softmax_k(scale * q.k).
 //
-// One CTA owns 256 query slots (two M=128 tiles) and walks every kv block twice, two
-// blocks (N = 128 keys) per step:
-//   pass 1: S = Q K^T on the tensor cores and the row max only (no exponentials);
-//   pass 2: S again, e[r,j] = sum over the keys of block j of exp2(S*c - max_r) -- every
-//           exponential of the calibration computed once -- written to this SM's slice of
-//           the workspace, and the row sums l_r = sum_j e[r,j];
-//   end:    mass[i,j] = (1 / valid queries of i) * sum over the rows r of query block i of
-//           e[r,j] / l_r, in a fixed order (deterministic).
+// One CTA owns 256 query slots (two M=128 tiles) and walks every kv block once, two blocks
+// (N = 128 keys) per step: S = Q K^T on the tensor cores, then per row and kv block j
+//   e[r,j] = sum over the keys of block j of exp2(S*c - m_r),
+// with m_r a lazy reference max: it is raised only when a block's max exceeds it by more
+// than kRescaleLog2 (every exponential then stays <= 2^kRescaleLog2, far from overflow).
+// On such a raise -- rare: only a row whose early blocks are far below its later ones --
+// the row's sum and the block sums it has already written are multiplied by
+// exp2(m_old - m_new) in place.  Every exponential of the calibration is computed once.
+// e[r,j] goes to this SM's slice of the workspace; at the end of the CTA
+//   mass[i,j] = (1 / valid queries of i) * sum over the rows r of query block i of
+//               e[r,j] * exp2(m_r,half(j) - m_r) / l_r,
+// in a fixed order (deterministic), where the two threads of a row (one per column half)
+// each kept their own reference max m_r,half and sum.
 // The scratch slice is chosen by the SM the CTA runs on: the CTA's shared memory admits one
 // CTA per SM, so no two live CTAs share a slice.
 // Warp roles (576 threads): warps 0-7 and 10-17 own the rows, two threads per row: warps
 // 0-3 / 4-7 take the first kv block of each step of tile 0 / 1, warps 10-13 / 14-17 the
 // second (a warp reads the TMEM lane quarter of its sub-partition, warp % 4); warp 8 is
-// the TMA producer (K only), warp 9 the MMA issuer and TMEM owner.  Each thread keeps its
-// own running max and sum over its kv blocks; the two halves of a row are combined at the
-// end of each pass.  Four row warps per sub-partition keep the exponential unit fed.  TMEM
-// holds two S buffers per tile (4 x 128 columns), so the tensor core computes step s+1
-// while step s is reduced.
+// the TMA producer (K only), warp 9 the MMA issuer and TMEM owner.  Four row warps per
+// sub-partition keep the exponential unit fed.  TMEM holds two S buffers per tile
+// (4 x 128 columns), so the tensor core computes step s+1 while step s is reduced.
 #include "bsa_kernels.cuh"
 
 namespace bsa {
@@ -35,6 +38,9 @@ constexpr int kRowsPerCta = 256;
 // 18 warps: 5 share sub-partitions 0 and 1, whose 16K-register files then allow 96
 // registers per thread.
 constexpr int kMaxRegs = 96;
+// Lazy reference max (log2 units): exponentials stay <= 2^64 and a row's sum below
+// 2^64 * keys, so fp32 cannot overflow for any sequence length the ABI admits.
+constexpr float kRescaleLog2 = 64.0f;
 }  // namespace mass
 
 struct MassParams {
@@ -53,8 +59,8 @@ struct MassSmem {
   static constexpr int kKStages = (D == 128) ? 4 : 6;
   static constexpr int kQOff = 0;
   static constexpr int kKOff = 2 * kQTile;
-  static constexpr int kRedOff = kKOff + kKStages * kKStage;   // float [256] 1 / row sum
-  static constexpr int kXchOff = kRedOff + 256 * 4;             // float [2 tile][2 half][128 row][2]
+  static constexpr int kRedOff = kKOff + kKStages * kKStage;   // float [2 half][256] row weights
+  static constexpr int kXchOff = kRedOff + 2 * 256 * 4;         // float [2 tile][2 half][128 row][2]
   static constexpr int kBarOff = kXchOff + 2 * 2 * 128 * 2 * 4;
   static constexpr int kBytes = kBarOff + 512;
   static constexpr int kAlloc = kBytes + 1024;
@@ -79,7 +85,7 @@ __global__ void __maxnreg__(mass::kMaxRegs)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* nvalid_sm = reinterpret_cast<int*>(tmem_slot + 2);  // [2 half][2 tile][4 warp]
-  float* inv_l = reinterpret_cast<float*>(smem + L::kRedOff);
+  float* row_w = reinterpret_cast<float*>(smem + L::kRedOff);  // [half][row] weight of e
   float* xch = reinterpret_cast<float*>(smem + L::kXchOff);
 
   const AttnDims& a = p.a;
@@ -88,8 +94,7 @@ __global__ void __maxnreg__(mass::kMaxRegs)
   const int cta = blockIdx.x;
   const int bh = cta / a.n_cta_per_head;
   const int row0 = (cta - bh * a.n_cta_per_head) * mass::kRowsPerCta;
-  const int npass = (a.n_kb + 1) >> 1;  // steps per pass
-  const int nsteps = 2 * npass;
+  const int nsteps = (a.n_kb + 1) >> 1;  // two kv blocks per step
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -121,8 +126,7 @@ __global__ void __maxnreg__(mass::kMaxRegs)
           tma_load_3d(smem + L::kQOff + t * L::kQTile + ch * (128 * 128), &tm_q, bar_q, ch * 64,
                       row0 + t * 128, bh);
       for (int s = 0; s < nsteps; ++s) {
-        const int st = s >= npass ? s - npass : s;
-        const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+        const int nb = (2 * s + 1 < a.n_kb) ? 2 : 1;
         const int ks = s % KS;
         if (s >= KS && !mbar_wait(bar_kempty + ks, ((s / KS) - 1) & 1, abort_flag, p.status,
                                   DETAIL_WAIT_K_EMPTY))
@@ -130,10 +134,10 @@ __global__ void __maxnreg__(mass::kMaxRegs)
         mbar_arrive_expect_tx(bar_kfull + ks, nb * 64 * D * 2);
         uint8_t* kst = smem + L::kKOff + ks * L::kKStage;
         for (int ch = 0; ch < L::kChunks; ++ch) {
-          tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * 64, 2 * st * 64, bh);
+          tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * 64, 2 * s * 64, bh);
           if (nb == 2)
             tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * 64,
-                        (2 * st + 1) * 64, bh);
+                        (2 * s + 1) * 64, bh);
         }
       }
     }
@@ -143,8 +147,7 @@ __global__ void __maxnreg__(mass::kMaxRegs)
       const uint32_t k_base = smem_u32(smem + L::kKOff);
       bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, DETAIL_WAIT_Q);
       for (int s = 0; s < nsteps && ok; ++s) {
-        const int st = s >= npass ? s - npass : s;
-        const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+        const int nb = (2 * s + 1 < a.n_kb) ? 2 : 1;
         const int ks = s % KS;
         const int buf = s & 1;
         const uint32_t idesc = make_idesc(1u, 0u, 128u, static_cast<uint32_t>(nb * 64));
@@ -198,26 +201,16 @@ __global__ void __maxnreg__(mass::kMaxRegs)
       record_status(p.status, FLAG_DEVICE_INPUT, DETAIL_MASS_SLICE, static_cast<uint32_t>(cta), smid);
     float* sc = p.scratch + static_cast<size_t>(have_slice ? smid : 0u) * 256 * a.n_kb;
 
-    float m_run = -INFINITY, l_run = 0.f, m_row = -INFINITY;
+    float m_ref = -INFINITY, l_run = 0.f;  // this half's reference max (log2 units) and sum
     bool ok = true;
-    // tile coordinates of this half's kv block 2*st + h, advanced incrementally (no
+    // tile coordinates of this half's kv block 2*s + h, advanced incrementally (no
     // division inside the loop: integer division shares the pipe of the exponentials)
     int tw = 0, th = 0, tt = 0;
     tile_advance(a.g, h, tw, th, tt);
     for (int s = 0; s < nsteps; ++s) {
-      const bool pass2 = s >= npass;
-      const int st = pass2 ? s - npass : s;
-      const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+      const int nb = (2 * s + 1 < a.n_kb) ? 2 : 1;
       const bool mine = h < nb;  // this half has a kv block in this step
       const int buf = s & 1;
-      if (s == npass) {
-        tw = th = tt = 0;
-        tile_advance(a.g, h, tw, th, tt);
-        // both halves' maxima -> the row max (log2 units)
-        xch[((t * 2 + h) * 128 + row) * 2] = m_run;
-        named_bar_sync(5 + t, 256);
-        m_row = fmaxf(xch[((t * 2 + 0) * 128 + row) * 2], xch[((t * 2 + 1) * 128 + row) * 2]);
-      }
       // A warp that gives up keeps stepping (without touching TMEM) so that every warp of
       // the group passes the same named barriers.
       bool got = ok ? mbar_wait(bar_sfull + 2 * t + buf, (s >> 1) & 1, abort_flag, p.status,
@@ -244,41 +237,56 @@ __global__ void __maxnreg__(mass::kMaxRegs)
 #pragma unroll
             for (int i = 0; i < 64; ++i) sv[i] = ((mw[i >> 5] >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
           }
-          if (!pass2) {
-            float mx[8];
+          float mx[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+          for (int i = 0; i < 8; ++i) mx[i] = sv[i];
 #pragma unroll
-            for (int i = 8; i < 64; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
-            const float mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-            m_run = fmaxf(m_run, mrow * c);  // c > 0, so -inf stays -inf
-          } else {
-            float e = 0.f;
-            if (m_row != -INFINITY) {
-              float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-              for (int i = 0; i < 64; ++i) acc[i & 3] += fast_exp2(fmaf(sv[i], c, -m_row));
-              e = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+          for (int i = 8; i < 64; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
+          const float mb = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                           c;  // c > 0, so -inf stays -inf
+          if (mb > m_ref + mass::kRescaleLog2) {
+            // Raise the reference (the first block always does).  Sums formed against the
+            // old one are scaled to the new; nothing was formed while it was -inf.
+            if (m_ref != -INFINITY) {
+              const float f = fast_exp2(m_ref - mb);
+              l_run *= f;
+              if (have_slice)
+                for (int j = h; j < 2 * s; j += 2) sc[static_cast<size_t>(j) * 256 + local] *= f;
             }
-            l_run += e;
-            if (have_slice) sc[static_cast<size_t>(2 * st + h) * 256 + local] = e;
+            m_ref = mb;
           }
+          float e = 0.f;
+          if (m_ref != -INFINITY) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 64; ++i) acc[i & 3] += fast_exp2(fmaf(sv[i], c, -m_ref));
+            e = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+          }
+          l_run += e;
+          if (have_slice) sc[static_cast<size_t>(2 * s + h) * 256 + local] = e;
         }
       }
       tile_advance(a.g, 2, tw, th, tt);
     }
 
     // ------------------------------------------------------------ masses
-    // Row sum = the halves' partial sums (first half + second, in both threads); then
-    // mass[i, j] = (1 / valid queries of i) * sum_r e[r, j] / l_r over the rows of query
-    // block i, in row order, by all 512 row threads over the CTA's (query block, kv block)
-    // outputs.
+    // The halves' (reference max, sum) pairs -> the row's max m and sum l; half h's block
+    // sums are weighted by exp2(m_h - m) / l.  Then mass[i, j] = (1 / valid queries of i) *
+    // sum_r e[r, j] * weight_r,half(j) over the rows of query block i, in row order, by all
+    // 512 row threads over the CTA's (query block, kv block) outputs.
+    xch[((t * 2 + h) * 128 + row) * 2] = m_ref;
     xch[((t * 2 + h) * 128 + row) * 2 + 1] = l_run;
     named_bar_sync(5 + t, 256);
-    if (h == 0) {
-      const float l = xch[((t * 2 + 0) * 128 + row) * 2 + 1] + xch[((t * 2 + 1) * 128 + row) * 2 + 1];
-      inv_l[local] = (q_valid && ok && l > 0.f) ? 1.f / l : 0.f;
+    {
+      const float m0 = xch[((t * 2 + 0) * 128 + row) * 2];
+      const float m1 = xch[((t * 2 + 1) * 128 + row) * 2];
+      const float mr = fmaxf(m0, m1);
+      const float f0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - mr);
+      const float f1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - mr);
+      const float l = xch[((t * 2 + 0) * 128 + row) * 2 + 1] * f0 +
+                      xch[((t * 2 + 1) * 128 + row) * 2 + 1] * f1;
+      row_w[h * 256 + local] = (q_valid && ok && l > 0.f) ? (h ? f1 : f0) / l : 0.f;
     }
     named_bar_sync(7, 512);  // every row's block sums and 1 / l_r are written
     if (have_slice) {
@@ -297,13 +305,14 @@ __global__ void __maxnreg__(mass::kMaxRegs)
           nvq += nvalid_sm[(r0 >> 7) * 4 + ((r0 & 127) >> 5)];
         }
         const float* col = sc + static_cast<size_t>(j) * 256 + qi * a.q_block;
+        const float* w = row_w + (j & 1) * 256 + qi * a.q_block;  // block j is half j & 1's
         float tot = 0.f;
         for (int r = 0; r < a.q_block; r += 4) {
           const float4 ev = *reinterpret_cast<const float4*>(col + r);
-          tot += ev.x * inv_l[qi * a.q_block + r];
-          tot += ev.y * inv_l[qi * a.q_block + r + 1];
-          tot += ev.z * inv_l[qi * a.q_block + r + 2];
-          tot += ev.w * inv_l[qi * a.q_block + r + 3];
+          tot += ev.x * w[r];
+          tot += ev.y * w[r + 1];
+          tot += ev.z * w[r + 2];
+          tot += ev.w * w[r + 3];
         }
         p.mass[(static_cast<long long>(bh) * a.n_qb + qb) * a.n_kb + j] =
             nvq > 0 ? tot / static_cast<float>(nvq) : 0.f;

@@ -96,14 +96,14 @@ def main(argv=None):
 
     mass = torch.empty((s.batch, Hh, s.n_qb, nkb), dtype=torch.float32, device=dev)
     ws_m = B.new_workspace(s, B.OP_BLOCK_MASS, dev)
-    dense_qk = 2.0 * 2 * Np * s.Np * D * Hh  # two QK^T passes over all slot pairs
+    qk_pass = 2.0 * Np * s.Np * D * Hh  # one QK^T over all slot pairs
     line("block_mass", _time(lambda: B.block_mass(qt, kt, s, out=mass, ws=ws_m), args.iters),
-         dense_qk, "TFLOP/s", "tensor", pk["bf16"])
+         qk_pass, "TFLOP/s", "tensor", pk["bf16"])
     out_t = torch.empty_like(qt)
     mass2 = torch.empty_like(mass)
     line("dense_fwd_mass",
          _time(lambda: B.dense_fwd_mass(qt, kt, vt, s, out=out_t, mass=mass2, ws=ws_m), args.iters),
-         1.5 * dense_qk, "TFLOP/s", "tensor", pk["bf16"])
+         3 * qk_pass, "TFLOP/s", "tensor", pk["bf16"])  # QK^T twice (row max, then P), PV once
 
     ws_t = B.new_workspace(s, B.OP_TOPP_SELECT, dev)
     row_ptr = torch.empty(R + 1, dtype=torch.int32, device=dev)

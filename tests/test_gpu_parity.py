@@ -92,6 +92,52 @@ def test_block_mass_parity(B, wl, sharp):
     assert np.all(got[ref == 0] == 0)
 
 
+@pytest.mark.parametrize("wl", [WLS[0], WLS[1], WLS[3]], ids=[IDS[0], IDS[1], IDS[3]])
+@pytest.mark.parametrize("ramp", ["ascending", "descending", "odd_blocks"])
+def test_block_mass_wide_logit_range(B, wl, ramp):
+    """Keys scaled per kv block so that a row's logits span far more than 64 log2 units:
+    ascending, each row's first blocks lie far below its later ones, so the kernel raises
+    its reference max and rescales the block sums already written; descending, later
+    blocks underflow against the first; odd_blocks, the two column halves of a row end
+    with reference maxima far apart, so the final merge weights one half by a tiny factor."""
+    g = Hp.grid_of(wl)
+    s = _shape(B, wl)
+    q, k, _ = Hp.draw(wl, value_scale=1.0, sharp=1.0)
+    qt64 = Hp.oracle_tiled(q, g)
+    kt64 = Hp.oracle_tiled(k, g)
+    n_kb = g.Np // 64
+    j = np.arange(n_kb)
+    if ramp == "ascending":     # each half's first block far below the rest
+        r = np.where(j < 2, 0.02, 1.0)
+    elif ramp == "descending":
+        r = 1.0 - 0.98 * j / (n_kb - 1)
+    else:
+        r = np.where(j % 2 == 1, 1.0, 0.02)
+    kt_bf = torch.from_numpy(kt64 * np.repeat(r, 64)[None, None, :, None]).to(torch.bfloat16)
+    kt64 = kt_bf.double().numpy()
+    valid = O.valid_slots(g)
+    z = np.einsum("bhqd,bhkd->bhqk", qt64, kt64)
+    z[..., ~valid] = -np.inf
+    # softmax scale putting the median valid row's max logit at 85 log2 units
+    scale = 85.0 * math.log(2.0) / float(np.median(z[:, :, valid].max(-1)))
+    # the data does what the docstring says: the spread of a row's block maxima, log2 units
+    bmax = (z * (scale / math.log(2.0))).reshape(*z.shape[:3], n_kb, 64).max(-1)[:, :, valid]
+    if ramp == "ascending":
+        assert np.median(bmax[..., 0::2].max(-1) - bmax[..., 0]) > 64.0
+    if ramp == "odd_blocks":
+        assert np.median(bmax[..., 1::2].max(-1) - bmax[..., 0::2].max(-1)) > 64.0
+    ws = B.new_workspace(s, B.OP_BLOCK_MASS)
+    m = B.block_mass(B.tile_permute(q.cuda(), s), kt_bf.cuda(), s, softmax_scale=scale, ws=ws)
+    assert B.device_status(ws) == 0
+    ref = O.block_mass(qt64, kt64, g, wl.q_block, 64, scale)
+    got = m.cpu().double().numpy()
+    err = np.abs(got - ref)
+    assert err.max() <= Hp.MASS_ABS, err.max()
+    nz = ref > 1e-6
+    assert (err[nz] / ref[nz]).max() < 1e-3
+    assert np.all(got[ref == 0] == 0)
+
+
 # ------------------------------------------------------------------ top-p selection
 def _topp_check(B, s, mass_np32, tau):
     mass = torch.from_numpy(np.ascontiguousarray(mass_np32)).cuda()
