@@ -3,21 +3,21 @@
 //
 // "LoSA: Near-Lossless Sparse Attention for Training-Free Video Diffusion Acceleration",
 // Abstract: the calibration step runs dense attention and measures the exact block masses
-// on it.  Computing them separately costs two QK^T passes for the masses plus a QK^T and a
-// PV pass for the output; here
-//   pass 1: S = Q K^T over every kv block -> the exact row max (no exponentials);
-//   pass 2: S again, P = exp2(S*c - max_r) <= 1, every probability computed once: stored to
-//           TMEM as bf16 for O += P V (no rescaling: the reference max is final), summed per
-//           kv block into this SM's workspace slice, and into the row sum l_r;
-//   end:    O / l_r, and mass[i,j] = (1 / valid queries of i) * sum over the rows of query
-//           block i of e[r,j] / l_r in a fixed order, as in bsa_block_mass.
+// on it.  Computing them separately costs a QK^T pass for the masses plus a QK^T and a PV
+// pass for the output; here one walk over the kv blocks does both:
+//   S = Q K^T, P = exp2(S*c - m_r) with m_r a lazy reference max (raised only when a step's
+//   max exceeds it by more than kRescaleLog2), every probability computed once: stored to
+//   TMEM as bf16 for O += P V, summed per kv block into this SM's workspace slice, and into
+//   the row sum l_r.  When m_r is raised -- rare -- the row's O, its sum and the block sums
+//   it has already written are multiplied by exp2(m_old - m_new);
+//   end: O / l_r, and mass[i,j] = (1 / valid queries of i) * sum over the rows of query
+//   block i of e[r,j] / l_r in a fixed order, as in bsa_block_mass.
 //
-// Layout and roles follow the block-sparse forward (attn_fwd.cu): 256 query slots per CTA
-// in two M=128 tiles, 384 threads (warps 0-7 row owners, warp 8 TMA, warp 9 MMA, warps
-// 10-11 completing the producer warpgroup, which hands registers to the row owners), TMEM
-// S0 S1 O0 O1.  In pass 1 the MMA of S_t(s+1) waits until the rows of S_t(s) have been
-// read (S_free); in pass 2 the order is PV_t(s-1), S_t(s) as in the forward, the PV in two
-// halves: the first kv block's keys as soon as their P is stored (P_part).
+// Layout, roles and pipeline follow the block-sparse forward (attn_fwd.cu): 256 query
+// slots per CTA in two M=128 tiles, 384 threads (warps 0-7 row owners, warp 8 TMA, warp 9
+// MMA, warps 10-11 completing the producer warpgroup, which hands registers to the row
+// owners), TMEM S0 S1 O0 O1 with P stored over S; the MMA order is PV_t(s-1), S_t(s), the
+// PV in two halves: the first kv block's keys as soon as their P is stored (P_part).
 #include "bsa_kernels.cuh"
 
 namespace bsa {
@@ -32,6 +32,8 @@ constexpr int kRegsRows = 184;
 constexpr int kRegsProducer = 136;
 static_assert(2 * 128 * kRegsRows + 128 * kRegsProducer <= kThreads * kRegsLaunch,
               "register shares must fit the launch total");
+// Lazy reference max (log2 units): P <= 2^16, so O = sum P V stays far inside fp32 range.
+constexpr float kRescaleLog2 = 16.0f;
 }  // namespace calib
 
 struct CalibParams {
@@ -76,9 +78,8 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
   uint64_t* bar_vfull = bar_kempty + KS;
   uint64_t* bar_vempty = bar_vfull + VS;
   uint64_t* bar_sfull = bar_vempty + VS;  // [2]
-  uint64_t* bar_sfree = bar_sfull + 2;    // [2] pass 1: rows of S_t read
-  uint64_t* bar_pfull = bar_sfree + 2;    // [2] pass 2: P_t stored
-  uint64_t* bar_ppart = bar_pfull + 2;    // [2] pass 2: P_t of the step's first kv block stored
+  uint64_t* bar_pfull = bar_sfull + 2;    // [2] P_t stored
+  uint64_t* bar_ppart = bar_pfull + 2;    // [2] P_t of the step's first kv block stored
   uint64_t* bar_ofull = bar_ppart + 2;
   uint64_t* bar_drain = bar_ofull + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
@@ -92,8 +93,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
   const int cta = blockIdx.x;
   const int bh = cta / a.n_cta_per_head;
   const int row0 = (cta - bh * a.n_cta_per_head) * calib::kRowsPerCta;
-  const int npass = (a.n_kb + 1) >> 1;  // steps per pass
-  const int nsteps = 2 * npass;
+  const int nsteps = (a.n_kb + 1) >> 1;  // two kv blocks per step
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -107,7 +107,6 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_sfull + t, 1);
-      mbar_init(bar_sfree + t, 128);
       mbar_init(bar_pfull + t, 128);
       mbar_init(bar_ppart + t, 128);
     }
@@ -136,8 +135,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
             tma_load_3d(smem + L::kQOff + t * L::kQTile + ch * (128 * 128), &tm_q, bar_q, ch * 64,
                         row0 + t * 128, bh);
         for (int s = 0; s < nsteps; ++s) {
-          const int st = s >= npass ? s - npass : s;
-          const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+          const int nb = (2 * s + 1 < a.n_kb) ? 2 : 1;
           const int ks = s % KS;
           if (s >= KS && !mbar_wait(bar_kempty + ks, ((s / KS) - 1) & 1, abort_flag, p.status,
                                     DETAIL_WAIT_K_EMPTY))
@@ -145,24 +143,22 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
           mbar_arrive_expect_tx(bar_kfull + ks, nb * 64 * D * 2);
           uint8_t* kst = smem + L::kKOff + ks * L::kKVStage;
           for (int ch = 0; ch < L::kChunks; ++ch) {
-            tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * 64, 2 * st * 64, bh);
+            tma_load_3d(kst + ch * (128 * 128), &tm_k, bar_kfull + ks, ch * 64, 2 * s * 64, bh);
             if (nb == 2)
               tma_load_3d(kst + ch * (128 * 128) + 64 * 128, &tm_k, bar_kfull + ks, ch * 64,
-                          (2 * st + 1) * 64, bh);
+                          (2 * s + 1) * 64, bh);
           }
-          if (s < npass) continue;  // V is needed in pass 2 only
-          const int u = s - npass;
-          const int vs = u % VS;
-          if (u >= VS && !mbar_wait(bar_vempty + vs, ((u / VS) - 1) & 1, abort_flag, p.status,
+          const int vs = s % VS;
+          if (s >= VS && !mbar_wait(bar_vempty + vs, ((s / VS) - 1) & 1, abort_flag, p.status,
                                     DETAIL_WAIT_V_EMPTY))
             break;
           mbar_arrive_expect_tx(bar_vfull + vs, nb * 64 * D * 2);
           uint8_t* vst = smem + L::kVOff + vs * L::kKVStage;
           for (int ch = 0; ch < L::kChunks; ++ch) {
-            tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * 64, 2 * st * 64, bh);
+            tma_load_3d(vst + ch * (128 * 128), &tm_v, bar_vfull + vs, ch * 64, 2 * s * 64, bh);
             if (nb == 2)
               tma_load_3d(vst + ch * (128 * 128) + 64 * 128, &tm_v, bar_vfull + vs, ch * 64,
-                          (2 * st + 1) * 64, bh);
+                          (2 * s + 1) * 64, bh);
           }
         }
       }
@@ -175,8 +171,8 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
         const uint32_t idesc_pv = make_idesc(1u, 1u, 128u, static_cast<uint32_t>(D));
         bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, DETAIL_WAIT_Q);
         auto issue_pv = [&](int t, int u, int half) {
-          // O_t (+)= P_t V over the keys of pass-2 step u's first (half 0) or second (half 1)
-          // kv block, 16 keys per MMA.
+          // O_t (+)= P_t V over the keys of step u's first (half 0) or second (half 1) kv
+          // block, 16 keys per MMA.
           const int nbp = (2 * u + 1 < a.n_kb) ? 2 : 1;
           const uint64_t vd = v_desc0 + static_cast<uint64_t>(((u % VS) * L::kKVStage) >> 4);
           const uint32_t p_tmem = tmem + t * 128;
@@ -187,7 +183,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
             mma_f16_ts(o_tmem, p_tmem + kk * 8, vd + static_cast<uint64_t>((kk * 2048) >> 4),
                        idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
         };
-        // PV of pass-2 step u for tile t: the first block's keys at P_part, the rest at P_full.
+        // PV of step u for tile t: the first block's keys at P_part, the rest at P_full.
         auto pv_step = [&](int t, int u) -> bool {
           if (!mbar_wait(bar_ppart + t, u & 1, abort_flag, p.status, DETAIL_WAIT_P_PART))
             return false;
@@ -203,8 +199,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
           return true;
         };
         for (int s = 0; s < nsteps && ok; ++s) {
-          const int st = s >= npass ? s - npass : s;
-          const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+          const int nb = (2 * s + 1 < a.n_kb) ? 2 : 1;
           const int ks = s % KS;
           const uint32_t idesc_qk = make_idesc(1u, 0u, 128u, static_cast<uint32_t>(nb * 64));
           if (!mbar_wait(bar_kfull + ks, (s / KS) & 1, abort_flag, p.status, DETAIL_WAIT_K_FULL)) {
@@ -214,20 +209,14 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
           tc_fence_after();
           const uint64_t kd = k_desc0 + static_cast<uint64_t>((ks * L::kKVStage) >> 4);
           for (int t = 0; t < 2; ++t) {
-            if (s >= 1 && s <= npass) {
-              // S_t is free once its rows of the previous step were read (pass 1 and the
-              // first step of pass 2)
-              if (!mbar_wait(bar_sfree + t, (s - 1) & 1, abort_flag, p.status, DETAIL_WAIT_P_FULL)) {
+            if (s > 0) {
+              // the previous step's PV; it also frees S_t (P is stored over it), and S_t(s)
+              // issued after it completes after it
+              if (!pv_step(t, s - 1)) {
                 ok = false;
                 break;
               }
-            } else if (s > npass) {
-              const int u = s - 1 - npass;  // pass-2 step whose P is consumed now
-              if (!pv_step(t, u)) {
-                ok = false;
-                break;
-              }
-              if (t == 1) mma_commit(bar_vempty + (u % VS));
+              if (t == 1) mma_commit(bar_vempty + ((s - 1) % VS));
             }
             tc_fence_after();
             const uint64_t qd = q_desc0 + static_cast<uint64_t>((t * L::kQTile) >> 4);
@@ -243,7 +232,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
           mma_commit(bar_kempty + ks);
         }
         if (ok) {
-          const int u = npass - 1;
+          const int u = nsteps - 1;
           for (int t = 0; t < 2 && ok; ++t) ok = pv_step(t, u);
           if (ok) mma_commit(bar_ofull);
         }
@@ -276,91 +265,109 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
       record_status(p.status, FLAG_DEVICE_INPUT, DETAIL_MASS_SLICE, static_cast<uint32_t>(cta), smid);
     float* sc = p.scratch + static_cast<size_t>(have_slice ? smid : 0u) * 256 * a.n_kb;
 
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_ref = -INFINITY, l_run = 0.f;  // reference max (log2 units) and sum against it
     bool ok = true;
     for (int s = 0; s < nsteps; ++s) {
-      const int st = s >= npass ? s - npass : s;
-      const bool pass2 = s >= npass;
-      const int nb = (2 * st + 1 < a.n_kb) ? 2 : 1;
+      const int nb = (2 * s + 1 < a.n_kb) ? 2 : 1;
       // A warp that gives up keeps stepping (without touching TMEM) so that the row warps
       // all reach the barrier before the masses.
       bool got = ok ? mbar_wait(bar_sfull + t, s & 1, abort_flag, p.status, DETAIL_WAIT_S_FULL)
                     : false;
       got = __all_sync(0xffffffffu, got);
       ok = got;
-      if (got) {
-        tc_fence_after();
-        float sv[128];
-        tmem_ld32(s_addr + 0, sv + 0);
-        tmem_ld32(s_addr + 32, sv + 32);
-        if (nb == 2) {
-          tmem_ld32(s_addr + 64, sv + 64);
-          tmem_ld32(s_addr + 96, sv + 96);
+      if (!got) continue;
+      tc_fence_after();
+      float sv[128];
+      tmem_ld32(s_addr + 0, sv + 0);
+      tmem_ld32(s_addr + 32, sv + 32);
+      if (nb == 2) {
+        tmem_ld32(s_addr + 64, sv + 64);
+        tmem_ld32(s_addr + 96, sv + 96);
+      }
+      tmem_ld_wait();
+      // pad keys and the absent half of a 1-block step -> -inf
+      const int j0 = 2 * s;
+      const uint64_t mk0 = tile_has_pad(a.g, j0) ? tile_valid_mask(a.g, j0) : ~0ull;
+      const uint64_t mk1 =
+          nb == 2 ? (tile_has_pad(a.g, j0 + 1) ? tile_valid_mask(a.g, j0 + 1) : ~0ull) : 0ull;
+      if ((mk0 & mk1) != ~0ull) {
+        const uint32_t mw[4] = {static_cast<uint32_t>(mk0), static_cast<uint32_t>(mk0 >> 32),
+                                static_cast<uint32_t>(mk1), static_cast<uint32_t>(mk1 >> 32)};
+#pragma unroll
+        for (int i = 0; i < 128; ++i) sv[i] = ((mw[i >> 5] >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
+      }
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+#pragma unroll
+      for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
+      const float m_new = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                          c;  // c > 0, so -inf stays -inf
+      float factor = 1.f;
+      bool resc = false;
+      if (m_new > m_ref + calib::kRescaleLog2) {  // the first step with a valid key always
+        if (m_ref != -INFINITY) {
+          factor = fast_exp2(m_ref - m_new);
+          resc = true;
         }
-        tmem_ld_wait();
-        if (!pass2) {
-          tc_fence_before();
-          mbar_arrive(bar_sfree + t);
+        m_ref = m_new;
+      }
+      // P = exp2(S*c - m) stored over S_t as bf16 pairs; the first kv block's P releases
+      // its half of PV unless this warp must first rescale its rows of O (then both halves
+      // are released at the end).  A row with no valid key so far has every P = 0.
+      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      const bool warp_resc = __any_sync(0xffffffffu, resc);
+      float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        if (ch >= 2 && nb == 1) break;
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(fmaf(sv[32 * ch + 2 * i], c, -m_use));
+          const float p1 = fast_exp2(fmaf(sv[32 * ch + 2 * i + 1], c, -m_use));
+          acc[ch >> 1][i & 1] += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
         }
-        // pad keys and the absent half of a 1-block step -> -inf
-        const int j0 = 2 * st;
-        const uint64_t mk0 = tile_has_pad(a.g, j0) ? tile_valid_mask(a.g, j0) : ~0ull;
-        const uint64_t mk1 =
-            nb == 2 ? (tile_has_pad(a.g, j0 + 1) ? tile_valid_mask(a.g, j0 + 1) : ~0ull) : 0ull;
-        if ((mk0 & mk1) != ~0ull) {
-          const uint32_t mw[4] = {static_cast<uint32_t>(mk0), static_cast<uint32_t>(mk0 >> 32),
-                                  static_cast<uint32_t>(mk1), static_cast<uint32_t>(mk1 >> 32)};
-#pragma unroll
-          for (int i = 0; i < 128; ++i) sv[i] = ((mw[i >> 5] >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
-        }
-        if (!pass2) {
-          float mx[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) mx[i] = sv[i];
-#pragma unroll
-          for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
-          const float mrow = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-          m_run = fmaxf(m_run, mrow * c);  // c > 0, so -inf stays -inf
-        } else {
-          // probabilities against the final row max (<= 1); a row with no valid key has
-          // m_run = -inf and every probability 0
-          const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-          float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            if (ch >= 2 && nb == 1) break;
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float p0 = fast_exp2(fmaf(sv[32 * ch + 2 * i], c, -m_use));
-              const float p1 = fast_exp2(fmaf(sv[32 * ch + 2 * i + 1], c, -m_use));
-              acc[ch >> 1][i & 1] += p0 + p1;
-              pk[i] = pack_bf16x2(p0, p1);
-            }
-            BSA_TMEM_ST_X16(s_addr + 16 * ch, pk);
-            if (ch == 1) {  // the first kv block's P: its half of PV may start
-              tmem_st_wait();
-              tc_fence_before();
-              mbar_arrive(bar_ppart + t);
-            }
-          }
-          const float e0 = acc[0][0] + acc[0][1];
-          const float e1 = acc[1][0] + acc[1][1];
-          l_run += e0 + e1;
-          if (have_slice) {
-            sc[static_cast<size_t>(j0) * 256 + local] = e0;
-            if (nb == 2) sc[static_cast<size_t>(j0 + 1) * 256 + local] = e1;
-          }
+        BSA_TMEM_ST_X16(s_addr + 16 * ch, pk);
+        if (ch == 1 && !warp_resc) {  // the first kv block's P: its half of PV may start
           tmem_st_wait();
           tc_fence_before();
-          mbar_arrive(bar_pfull + t);
+          mbar_arrive(bar_ppart + t);
         }
       }
+      const float e0 = acc[0][0] + acc[0][1];
+      const float e1 = acc[1][0] + acc[1][1];
+      l_run = fmaf(l_run, factor, e0 + e1);
+      if (have_slice) {
+        if (resc)  // the block sums formed against the old reference
+          for (int j = 0; j < j0; ++j) sc[static_cast<size_t>(j) * 256 + local] *= factor;
+        sc[static_cast<size_t>(j0) * 256 + local] = e0;
+        if (nb == 2) sc[static_cast<size_t>(j0 + 1) * 256 + local] = e1;
+      }
+      if (warp_resc) {
+        // O_t is quiescent: the PV of the previous step completed before S_full fired.
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float ov[32];
+          tmem_ld32(o_addr + c0, ov);
+          tmem_ld_wait();
+          uint32_t r[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(ov[i] * factor);
+          BSA_TMEM_ST_X16(o_addr + c0, r);
+          BSA_TMEM_ST_X16(o_addr + c0 + 16, (r + 16));
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      if (warp_resc) mbar_arrive(bar_ppart + t);
+      mbar_arrive(bar_pfull + t);
     }
 
     // ------------------------------------------------------------ epilogue
-    bool have_o = ok && npass > 0;
+    bool have_o = ok && nsteps > 0;
     if (have_o) {
       have_o = __all_sync(0xffffffffu,
                           mbar_wait(bar_ofull, 0, abort_flag, p.status, DETAIL_WAIT_O_FULL));
@@ -390,7 +397,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
     }
     if (p.lse != nullptr && in_range)
       p.lse[static_cast<long long>(bh) * a.g.Np + slot] =
-          (q_valid && l_run > 0.f) ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+          (q_valid && l_run > 0.f) ? (m_ref + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
 
     // ------------------------------------------------------------ masses
     // mass[i, j] = (1 / valid queries of i) * sum_r e[r, j] / l_r over the rows of query

@@ -74,3 +74,35 @@ def csr_to_device(rp, ci, device):
 
 def scale_of(wl) -> float:
     return 1.0 / math.sqrt(wl.head_dim)
+
+
+def wide_range_keys(wl, q, k, ramp, target_log2=85.0):
+    """Keys scaled per kv block so that a row's logits span far more than 64 log2 units.
+
+    ramp "ascending": each column half's first block (kv blocks 0 and 1) at 2% of the rest;
+    "descending": a linear ramp from 1 down to 0.02; "odd_blocks": even blocks at 2% of the
+    odd ones.  The softmax scale puts the median valid row's max logit at target_log2.
+    Returns (tile-major bf16 keys on the CPU, the same as float64, the scale, each valid
+    row's block maxima [B, Hh, valid rows, n_kb] in log2 units)."""
+    g = grid_of(wl)
+    qt64 = oracle_tiled(q, g)
+    kt64 = oracle_tiled(k, g)
+    n_kb = g.Np // 64
+    j = np.arange(n_kb)
+    if ramp == "ascending":
+        r = np.where(j < 2, 0.02, 1.0)
+    elif ramp == "descending":
+        r = 1.0 - 0.98 * j / (n_kb - 1)
+    elif ramp == "odd_blocks":
+        r = np.where(j % 2 == 1, 1.0, 0.02)
+    else:
+        raise ValueError(ramp)
+    kt_bf = torch.from_numpy(kt64 * np.repeat(r, 64)[None, None, :, None]).to(torch.bfloat16)
+    kt64 = kt_bf.double().numpy()
+    valid = O.valid_slots(g)
+    z = np.einsum("bhqd,bhkd->bhqk", qt64, kt64)
+    z[..., ~valid] = -np.inf
+    scale = target_log2 * math.log(2.0) / float(np.median(z[:, :, valid].max(-1)))
+    bmax = (z * (scale / math.log(2.0))).reshape(*z.shape[:3], n_kb, 64).max(-1)[:, :, valid]
+    return kt_bf, kt64, scale, bmax
+

@@ -1,5 +1,5 @@
 """GPU parity of the fused calibration call: dense attention output and block masses in one
-pass pair, against the oracle's dense attention (every block kept) and its block masses."""
+pass, against the oracle's dense attention (every block kept) and its block masses."""
 import numpy as np
 import pytest
 
@@ -39,6 +39,41 @@ def test_dense_fwd_mass_parity(B, wl, sharp):
     rp = np.arange(R + 1) * n_kb
     ci = np.tile(np.arange(n_kb), R)
     o_ref, lse_ref = O.masked_attention(qo, ko, vo, g, wl.q_block, 64, rp, ci, Hp.scale_of(wl))
+    e = Hp.attn_errors(out.cpu().double().numpy(), o_ref)
+    assert e["max_abs"] <= Hp.ATTN_MAX_ABS and e["mean_abs"] <= Hp.ATTN_MEAN_ABS, e
+    zero = ~np.isfinite(lse_ref)
+    lg = lse.cpu().double().numpy()
+    assert np.all(np.isneginf(lg[zero]))
+    assert np.abs(lg[~zero] - lse_ref[~zero]).max() <= 1e-3
+
+
+@pytest.mark.parametrize("wl", [WLS[0], WLS[1], WLS[3]], ids=[WLS[i].name for i in (0, 1, 3)])
+@pytest.mark.parametrize("ramp", ["ascending", "descending", "odd_blocks"])
+def test_dense_fwd_mass_wide_logit_range(B, wl, ramp):
+    """Keys scaled per kv block so that rows raise their reference max mid-walk (ascending:
+    the output, the row sum and the block sums already written are rescaled), underflow
+    against the first blocks (descending), or alternate between tiny and large blocks."""
+    g = Hp.grid_of(wl)
+    s = B.Shape.of(wl)
+    q, k, v = Hp.draw(wl, value_scale=1.0, sharp=1.0)
+    kt_bf, ko, scale, bmax = Hp.wide_range_keys(wl, q, k, ramp)
+    if ramp == "ascending":  # most rows raise their reference after the first step
+        assert np.median(bmax[..., 2:].max(-1) - bmax[..., :2].max(-1)) > 16.0
+    qt, vt = (B.tile_permute(x.cuda(), s) for x in (q, v))
+    ws = B.new_workspace(s, B.OP_BLOCK_MASS)
+    out, mass, lse = B.dense_fwd_mass(qt, kt_bf.cuda(), vt, s, softmax_scale=scale,
+                                      want_lse=True, ws=ws)
+    assert B.device_status(ws) == 0, B.device_status_words(ws)
+    qo, vo = (Hp.oracle_tiled(x, g) for x in (q, v))
+    m_ref = O.block_mass(qo, ko, g, wl.q_block, 64, scale)
+    got_m = mass.cpu().double().numpy()
+    assert np.abs(got_m - m_ref).max() <= Hp.MASS_ABS
+    assert np.all(got_m[m_ref == 0] == 0)
+    n_qb, n_kb = wl.Np // wl.q_block, wl.Np // 64
+    R = wl.batch * wl.heads * n_qb
+    rp = np.arange(R + 1) * n_kb
+    ci = np.tile(np.arange(n_kb), R)
+    o_ref, lse_ref = O.masked_attention(qo, ko, vo, g, wl.q_block, 64, rp, ci, scale)
     e = Hp.attn_errors(out.cpu().double().numpy(), o_ref)
     assert e["max_abs"] <= Hp.ATTN_MAX_ABS and e["mean_abs"] <= Hp.ATTN_MEAN_ABS, e
     zero = ~np.isfinite(lse_ref)

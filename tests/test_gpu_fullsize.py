@@ -161,6 +161,44 @@ def test_fwd_full_size_sampled_rows(B, full):
     assert errs.max() <= 2e-2 * refmax
 
 
+def test_dense_fwd_mass_full_size(B, full):
+    """The fused calibration at full size: its masses equal bsa_block_mass's within fp32
+    rounding, and sampled output rows and log-sum-exps match the oracle's dense rows."""
+    wl, s, _, (qt, kt, vt) = full
+    g = Hp.grid_of(wl)
+    ws = B.new_workspace(s, B.OP_BLOCK_MASS)
+    out, mass, lse = B.dense_fwd_mass(qt, kt, vt, s, want_lse=True, ws=ws)
+    assert B.device_status(ws) == 0, B.device_status_words(ws)
+    m2 = B.block_mass(qt, kt, s, ws=ws)
+    assert B.device_status(ws) == 0
+    assert float((mass - m2).abs().max()) <= 1e-6
+    del m2
+    rng = np.random.default_rng(3)
+    scale = Hp.scale_of(wl)
+    all_blocks = np.arange(s.n_kb, dtype=np.int64)
+    errs, refmax = [], 0.0
+    for h in np.unique(rng.integers(0, s.heads, 3)):
+        qh, kh, vh = (x[0:1, h:h + 1].cpu().double().numpy() for x in (qt, kt, vt))
+        for p in rng.integers(0, s.Np, 96).tolist() + [0, s.Np - 1]:
+            rp1 = np.zeros(s.n_qb + 1, dtype=np.int64)
+            rp1[p // wl.q_block + 1:] = s.n_kb  # one dense row: every block kept
+            o_ref, l_ref = O.masked_attention_query(qh, kh, vh, g, 0, 0, int(p), wl.q_block, 64,
+                                                    rp1, all_blocks, scale)
+            got = out[0, h, p].double().cpu().numpy()
+            errs.append(np.abs(got - o_ref).max())
+            refmax = max(refmax, np.abs(o_ref).max())
+            lg = float(lse[0, h, p])
+            if math.isinf(l_ref):
+                assert math.isinf(lg) and lg < 0 and np.all(got == 0)
+            else:
+                assert abs(lg - l_ref) <= 1e-3
+    errs = np.array(errs)
+    assert errs.max() <= Hp.ATTN_MAX_ABS and errs.mean() <= Hp.ATTN_MEAN_ABS
+    assert errs.max() <= 2e-2 * refmax
+    del out, mass, lse
+    torch.cuda.empty_cache()
+
+
 def test_fwd_raster_full_size_matches_permuted_path(B, full):
     """The fused raster forward at full size, in the bench's launch configuration:
     bit-identical to the tile-major forward permuted back (whose rows the oracle checks)."""

@@ -104,24 +104,8 @@ def test_block_mass_wide_logit_range(B, wl, ramp):
     s = _shape(B, wl)
     q, k, _ = Hp.draw(wl, value_scale=1.0, sharp=1.0)
     qt64 = Hp.oracle_tiled(q, g)
-    kt64 = Hp.oracle_tiled(k, g)
-    n_kb = g.Np // 64
-    j = np.arange(n_kb)
-    if ramp == "ascending":     # each half's first block far below the rest
-        r = np.where(j < 2, 0.02, 1.0)
-    elif ramp == "descending":
-        r = 1.0 - 0.98 * j / (n_kb - 1)
-    else:
-        r = np.where(j % 2 == 1, 1.0, 0.02)
-    kt_bf = torch.from_numpy(kt64 * np.repeat(r, 64)[None, None, :, None]).to(torch.bfloat16)
-    kt64 = kt_bf.double().numpy()
-    valid = O.valid_slots(g)
-    z = np.einsum("bhqd,bhkd->bhqk", qt64, kt64)
-    z[..., ~valid] = -np.inf
-    # softmax scale putting the median valid row's max logit at 85 log2 units
-    scale = 85.0 * math.log(2.0) / float(np.median(z[:, :, valid].max(-1)))
+    kt_bf, kt64, scale, bmax = Hp.wide_range_keys(wl, q, k, ramp)
     # the data does what the docstring says: the spread of a row's block maxima, log2 units
-    bmax = (z * (scale / math.log(2.0))).reshape(*z.shape[:3], n_kb, 64).max(-1)[:, :, valid]
     if ramp == "ascending":
         assert np.median(bmax[..., 0::2].max(-1) - bmax[..., 0]) > 64.0
     if ramp == "odd_blocks":
