@@ -142,9 +142,9 @@ BSA_API bsa_status bsa_tile_permute_quant_e4m3(const bsa_shape* shape, const voi
  * zero pad slots.  mass: fp32 [B,Hh,Np/q_block,Np/64]; mass[b,h,i,j] is the mean over
  * the valid queries of block i of the softmax(softmax_scale * q.k) probability on the
  * valid keys of block j (pad keys excluded).  Rows of a block with no valid query are
- * zero.  Two dense passes on tcgen05 tensor cores: the row maxima, then every probability
- * once (unnormalised block sums per row, kept in the workspace, normalised by the row
- * sums at the end).  Workspace: bsa_workspace_bytes(shape, BSA_OP_BLOCK_MASS) -- the
+ * zero.  One dense pass on tcgen05 tensor cores: every probability computed once against a
+ * lazily raised reference max, unnormalised block sums per row kept in the workspace and
+ * normalised by the row sums at the end.  Workspace: bsa_workspace_bytes(shape, BSA_OP_BLOCK_MASS) -- the
  * status header plus 192 slices of 256 x Np/64 fp32, one per SM id. */
 BSA_API bsa_status bsa_block_mass(const bsa_shape* shape, const void* q, const void* k,
                           float softmax_scale, float* mass, void* ws, size_t ws_bytes,
@@ -152,8 +152,8 @@ BSA_API bsa_status bsa_block_mass(const bsa_shape* shape, const void* q, const v
 
 /* Fused calibration step: the dense attention output and the exact block masses in one
  * call ("LoSA", Abstract: the calibration step is a dense attention step on which the
- * block masses are measured).  Pass 1 computes each query row's exact log-sum-exp; pass 2
- * forms the exact probabilities once and uses them for both the masses (as
+ * block masses are measured).  One dense pass: each probability is formed once (against a
+ * lazily raised reference max, O rescaled when it moves) and used for both the masses (as
  * bsa_block_mass) and out = P V.  q, k, v: tile-major bf16 [B,Hh,Np,D].  out: bf16
  * tile-major (pad query slots zero); lse (nullable): fp32 [B,Hh,Np] natural log; mass:
  * fp32 [B,Hh,Np/q_block,Np/64].  Workspace as for BSA_OP_BLOCK_MASS. */
