@@ -97,8 +97,14 @@ def main(argv=None):
     mass = torch.empty((s.batch, Hh, s.n_qb, nkb), dtype=torch.float32, device=dev)
     ws_m = B.new_workspace(s, B.OP_BLOCK_MASS, dev)
     qk_pass = 2.0 * Np * s.Np * D * Hh  # one QK^T over all slot pairs
-    line("block_mass", _time(lambda: B.block_mass(qt, kt, s, out=mass, ws=ws_m), args.iters),
-         qk_pass, "TFLOP/s", "tensor", pk["bf16"])
+    # The exponential unit binds the calibration: one ex2 per (query slot, key slot) pair of
+    # every 256-row tile, against 16 ex2 per clock per SM on 148 SMs at the 1965 MHz maximum.
+    n_ex2 = float(s.batch) * Hh * (-(-s.Np // 256) * 256) * s.Np
+    ex2_peak = 16.0 * 148 * 1.965e9
+    ms_m = _time(lambda: B.block_mass(qt, kt, s, out=mass, ws=ws_m), args.iters)
+    line("block_mass", ms_m, qk_pass, "TFLOP/s", "tensor", pk["bf16"],
+         {"ex2_per_s": n_ex2 / (ms_m * 1e-3), "ex2_peak_per_s": ex2_peak,
+          "ex2_frac": round(n_ex2 / (ms_m * 1e-3) / ex2_peak, 4)})
     out_t = torch.empty_like(qt)
     mass2 = torch.empty_like(mass)
     line("dense_fwd_mass",
