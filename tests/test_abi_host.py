@@ -106,6 +106,19 @@ def test_rejections_before_launch(B):
     assert L.bsa_block_mass(_c(B), FAKE, FAKE, 0.088, FAKE, FAKE, 0, n) == 3     # no workspace
     assert L.bsa_block_mass(_c(B), FAKE, FAKE, -1.0, FAKE, FAKE, big, n) == 1    # bad scale
     assert L.bsa_block_mass(_c(B, q_block=96), FAKE, FAKE, 0.088, FAKE, FAKE, big, n) == 2
+    # the calibration kernels scale the row max by softmax_scale: it must be finite and > 0
+    for sc in (0.0, -1.0, float("nan"), float("inf")):
+        assert L.bsa_block_mass(_c(B), FAKE, FAKE, sc, FAKE, FAKE, big, n) == 1
+        assert L.bsa_dense_fwd_mass(_c(B), FAKE, FAKE, FAKE, sc, FAKE, n, FAKE, FAKE, big, n) == 1
+    dfm = [FAKE, FAKE, FAKE, 0.088, FAKE, n, FAKE, FAKE]  # q, k, v, scale, out, lse, mass, ws
+    assert L.bsa_dense_fwd_mass(_c(B), *dfm, 16, n) == 3                          # short workspace
+    bad = list(dfm)
+    bad[2] = n                                                                    # v missing
+    assert L.bsa_dense_fwd_mass(_c(B), *bad, big, n) == 1
+    bad = list(dfm)
+    bad[5] = ctypes.c_void_p(0x10002)                                             # lse misaligned
+    assert L.bsa_dense_fwd_mass(_c(B), *bad, big, n) == 1
+    assert L.bsa_dense_fwd_mass(_c(B, head_dim=96), *dfm, big, n) == 2
     assert L.bsa_topp_select(_c(B), FAKE, 1.5, FAKE, FAKE, 10, FAKE, big, n) == 1
     assert L.bsa_topp_select(_c(B), FAKE, 0.0, FAKE, FAKE, 10, FAKE, big, n) == 1
     assert L.bsa_topp_select(_c(B), FAKE, float("nan"), FAKE, FAKE, 10, FAKE, big, n) == 1
