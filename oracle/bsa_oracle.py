@@ -460,19 +460,32 @@ def pooled_block_mass(qt, kt, g: Grid, q_block: int, kv_block: int, scale: float
 #     given initial centroids for a fixed number of rounds; a round assigns every token to
 #     the nearest centroid (squared Euclidean distance, ties to the lowest index) and then
 #     replaces each centroid by the mean of its tokens (an empty cluster keeps its centroid);
-#   * the assignment is an integer decided by floating point, so it is taken in float32 as
-#     argmin_c (|c|^2 - 2 x.c), the kernel's precision; the means are float64 here;
+#   * the assignment is the definition itself: squared Euclidean distance sum_d (x_d - c_d)^2
+#     in float64, first minimum (lowest index) on ties; the means are float64 too.  A
+#     device computing the distance in lower precision may pick another centroid only
+#     where two distances agree to that precision: tests compare labels where the oracle's
+#     minimum is unique at the device's precision and check the others for validity;
 #   * cluster order: clusters by index, tokens of one cluster in their raster order;
 #   * cluster-level estimate as in R8 with clusters for tiles: weights n_j exp(s qc_i . kc_j)
 #     over the key clusters, normalised per query cluster (qc, kc the final centroids);
 #   * the selection is R3 applied to those rows; a query token attends to every key of the
 #     key clusters selected for its cluster, softmax renormalised over them (R4).
+def kmeans_distances(x, centroids) -> np.ndarray:
+    """Squared Euclidean distance [N, C] of every row of x to every centroid, float64,
+    summed over the coordinates as written in the definition."""
+    x = np.asarray(x, dtype=np.float64)
+    c = np.asarray(centroids, dtype=np.float64)
+    d = np.empty((x.shape[0], c.shape[0]))
+    for j in range(c.shape[0]):
+        diff = x - c[j][None, :]
+        d[:, j] = (diff * diff).sum(axis=1)
+    return d
+
+
 def kmeans_assign(x, centroids) -> np.ndarray:
-    """Nearest centroid of every row of x, decided in float32 (reading R10)."""
-    x32 = np.asarray(x, dtype=np.float32)
-    c32 = np.asarray(centroids, dtype=np.float32)
-    d = (c32 * c32).sum(axis=1, dtype=np.float32)[None, :] - np.float32(2.0) * (x32 @ c32.T)
-    return np.argmin(d, axis=1).astype(np.int64)  # first minimum: the lowest index
+    """Nearest centroid of every row of x (reading R10): the first minimum of the float64
+    squared distances, i.e. the lowest index among equidistant centroids."""
+    return np.argmin(kmeans_distances(x, centroids), axis=1).astype(np.int64)
 
 
 def kmeans_lloyd(x, init, rounds: int):

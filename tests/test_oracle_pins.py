@@ -570,6 +570,20 @@ def test_kmeans_ties_go_to_lowest_index():
     assert O.kmeans_assign(x, c).tolist() == [0, 0]
 
 
+def test_kmeans_distance_is_the_definition_far_from_the_origin():
+    # 1e4 from the origin, centroids 1.5 and 1.0 away: the expanded |c|^2 - 2 x.c form in
+    # float32 rounds both to the same value (ulp 8 at 1e8); the squared difference does not
+    x = np.array([[1.0e4, 0.0]])
+    c = np.array([[1.0e4 - 1.5, 0.0], [1.0e4 + 1.0, 0.0]])
+    np.testing.assert_allclose(O.kmeans_distances(x, c), [[2.25, 1.0]], rtol=0, atol=1e-9)
+    assert O.kmeans_assign(x, c).tolist() == [1]
+    # brute force on random data, one distance at a time
+    rng = np.random.default_rng(9)
+    xs, cs = rng.standard_normal((20, 5)), rng.standard_normal((4, 5))
+    brute = [[sum((xs[i, d] - cs[j, d]) ** 2 for d in range(5)) for j in range(4)] for i in range(20)]
+    np.testing.assert_allclose(O.kmeans_distances(xs, cs), brute, rtol=1e-14, atol=0)
+
+
 def test_cluster_layout_is_stable_counting_sort():
     rng = np.random.default_rng(5)
     labels = rng.integers(0, 7, size=300)
