@@ -14,6 +14,17 @@ ATTN_MAX_ABS = 2e-2
 ATTN_MEAN_ABS = 2e-3
 MASS_ABS = 1e-4
 FP8_MAX_ABS = 6e-2
+# Error relative to the largest reference output.  bf16: P and O are rounded to 8
+# significant bits (half-ulp 2^-9) -- 2e-2 leaves room for the sums of many such
+# roundings.  e4m3: P is rounded to 4 significant bits before PV, a relative step of at
+# most 2^-4 per probability; its contribution to an output element is bounded by 2^-4 of
+# the probability-weighted |v| of the row, and the test inputs keep the largest output of
+# a case within a small factor of that, so the bound is 2^-4 of the largest output.
+ATTN_REL_TO_MAX = 2e-2
+FP8_REL_TO_MAX = 2.0 ** -4
+# A comparison is only meaningful where the reference output is well above the absolute
+# tolerance: an all-zero output must fail it.
+SIGNAL_FACTOR = 10.0
 
 
 def grid_of(wl) -> O.Grid:
@@ -57,6 +68,31 @@ def attn_errors(got: np.ndarray, ref: np.ndarray):
     return dict(max_abs=float(err.max()), mean_abs=float(err.mean()),
                 max_rel_to_max=float(err.max() / scale),
                 rms_rel=float(np.sqrt((err ** 2).mean()) / max(np.sqrt((ref ** 2).mean()), 1e-30)))
+
+
+def assert_attn_close(got: np.ndarray, ref: np.ndarray, fp8: bool = False,
+                      signal_guard: bool = True) -> dict:
+    """Element-wise check of an attention output against the oracle's.
+
+    bf16: max abs <= ATTN_MAX_ABS, mean abs <= ATTN_MEAN_ABS, max |err| / max |ref| <=
+    ATTN_REL_TO_MAX.  e4m3: max abs <= FP8_MAX_ABS and max |err| / max |ref| <=
+    FP8_REL_TO_MAX.  With signal_guard the reference's largest output must be at least
+    SIGNAL_FACTOR x the absolute bound, so that the absolute bound alone already rejects an
+    all-zero output.  The relative bound rejects it in any case (its ratio is 1)."""
+    e = attn_errors(got, ref)
+    refmax = float(np.abs(ref).max()) if ref.size else 0.0
+    e["ref_max"] = refmax
+    abs_tol = FP8_MAX_ABS if fp8 else ATTN_MAX_ABS
+    if signal_guard:
+        assert refmax >= SIGNAL_FACTOR * abs_tol, ("reference output too small to test", e)
+    assert refmax > 0.0, ("all-zero reference", e)
+    assert e["max_abs"] <= abs_tol, e
+    if fp8:
+        assert e["max_rel_to_max"] <= FP8_REL_TO_MAX, e
+    else:
+        assert e["mean_abs"] <= ATTN_MEAN_ABS, e
+        assert e["max_rel_to_max"] <= ATTN_REL_TO_MAX, e
+    return e
 
 
 def csr_from_oracle(mass64: np.ndarray, tau: float):

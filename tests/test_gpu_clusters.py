@@ -2,9 +2,10 @@
 scatter, cluster-level estimate, row top-p, attention in cluster order) against the oracle.
 
 Integer work (layouts, permutations, selections) is compared bit for bit.  k-means labels
-are integers decided by float32 distances; on separated blobs they are unique and compared
-exactly, on general data the GPU's choice is checked to be a nearest centroid within the
-float32 rounding of the distance.  No oracle input comes from the GPU: both sides start
+are integers decided by distances the kernel forms in float32 precision; the oracle takes the
+definition in float64.  On separated blobs the nearest centroid is unique and the labels are
+compared exactly; on general data they are compared wherever the oracle's minimum wins by
+more than float32 rounding, and elsewhere checked to be a nearest centroid within it.  No oracle input comes from the GPU: both sides start
 from the same seeded draws.
 """
 import math
@@ -65,13 +66,18 @@ def test_kmeans_general_data_is_nearest_within_rounding(B):
     for h in range(Hh):
         X = xf[h].double().numpy()
         C0 = init[0, h].double().numpy()
-        d = (C0 * C0).sum(1)[None, :] - 2.0 * X @ C0.T      # float64 distances
+        d = O.kmeans_distances(X, C0)                       # the definition, float64
         lab = labels[0, h].cpu().numpy().astype(np.int64)
-        chosen = d[np.arange(S), lab]
-        scale = np.abs(X).max() * np.abs(C0).max() * D
-        assert np.all(chosen <= d.min(axis=1) + 2e-5 * scale)
         ref = O.kmeans_assign(X, C0)
-        assert (lab == ref).mean() > 0.999
+        # the kernel decides in float32 precision: the labels must be the oracle's wherever
+        # the oracle's nearest centroid wins by more than that rounding, and elsewhere a
+        # centroid whose distance is within it of the minimum
+        tol = 2e-5 * np.abs(X).max() * np.abs(C0).max() * D
+        srt = np.sort(d, axis=1)
+        unique = srt[:, 1] - srt[:, 0] > tol
+        assert unique.mean() > 0.99
+        assert np.array_equal(lab[unique], ref[unique])
+        assert np.all(d[np.arange(S), lab] <= srt[:, 0] + tol)
         n = np.bincount(lab, minlength=C)
         assert np.array_equal(counts[0, h].cpu().numpy(), n)
         means = np.stack([X[lab == j].mean(0) if n[j] else C0[j] for j in range(C)])
@@ -153,12 +159,13 @@ def test_topp_select_rows_bit_exact(B, cols):
     assert np.array_equal(ci[:n].cpu().numpy(), ref_ci)
 
 
-def _cluster_case(B, Bt, Hh, S, D, Cq, Ck, seed, keep_prob, sharp):
+def _cluster_case(B, Bt, Hh, S, D, Cq, Ck, seed, keep_prob, sharp, v_scale=0.25):
     cs = B.ClusterShape(Bt, Hh, D, S, Cq, Ck)
     g = torch.Generator().manual_seed(seed)
     q, k, v = (torch.randn((Bt, Hh, S, D), generator=g) for _ in range(3))
-    # |v| ~ 0.25 keeps outputs at the scale the bf16 bar (max abs 2e-2) is set for
-    q, k, v = q * sharp, k * sharp, v * 0.25
+    # |v| ~ 0.25 keeps sharp-attention outputs near 1; near-uniform attention averages V
+    # down, so those cases take |v| ~ 1.5 to keep the largest output above 10x the bound
+    q, k, v = q * sharp, k * sharp, v * v_scale
     q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))     # already in cluster order
     lq = synth.draw_cluster_labels(Bt, Hh, S, Cq, seed=seed + 1, empty=(1,))
     lk = synth.draw_cluster_labels(Bt, Hh, S, Ck, seed=seed + 2, empty=(2,))
@@ -172,10 +179,11 @@ def _cluster_case(B, Bt, Hh, S, D, Cq, Ck, seed, keep_prob, sharp):
 
 
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("keep_prob,sharp", [(1.0, 1.0), (0.3, 3.0), (0.05, 3.0)])
-def test_cluster_fwd_parity(B, D, keep_prob, sharp):
+@pytest.mark.parametrize("keep_prob,sharp,v_scale", [(1.0, 1.0, 1.5), (0.3, 3.0, 0.25), (0.05, 3.0, 0.25)])
+def test_cluster_fwd_parity(B, D, keep_prob, sharp, v_scale):
     Bt, Hh, S, Cq, Ck = 2, 2, 1500, 9, 23
-    cs, q, k, v, qs, qn, ks, kn, rp, ci = _cluster_case(B, Bt, Hh, S, D, Cq, Ck, 40 + D, keep_prob, sharp)
+    cs, q, k, v, qs, qn, ks, kn, rp, ci = _cluster_case(B, Bt, Hh, S, D, Cq, Ck, 40 + D, keep_prob,
+                                                        sharp, v_scale)
     dev = lambda t: t.cuda()
     ws = B.new_cluster_fwd_workspace(cs)
     out, lse = B.cluster_fwd(dev(q), dev(k), dev(v), cs, dev(qs), dev(qn), dev(ks), dev(kn),
@@ -190,8 +198,7 @@ def test_cluster_fwd_parity(B, D, keep_prob, sharp):
             ref = O.cluster_attention(q[b, h].double().numpy(), k[b, h].double().numpy(),
                                       v[b, h].double().numpy(), qs[b, h].numpy(), qn[b, h].numpy(),
                                       ks[b, h].numpy(), kn[b, h].numpy(), rows, cols, scale)
-            e = Hp.attn_errors(_np(out[b, h]), ref)
-            assert e["max_abs"] <= Hp.ATTN_MAX_ABS and e["mean_abs"] <= Hp.ATTN_MEAN_ABS, e
+            e = Hp.assert_attn_close(_np(out[b, h]), ref)
             # rows of cluster 0 (no kept key cluster) are zero with lse -inf
             z = slice(int(qs[b, h, 0]), int(qs[b, h, 0] + qn[b, h, 0]))
             if b == 0 and h == 0:
@@ -254,8 +261,7 @@ def test_semantic_pipeline_on_blobs_matches_oracle(B):
         ref = np.empty_like(ref_p)
         ref[Tq] = ref_p
         rows = np.isin(Lq, np.flatnonzero(same))
-        e = Hp.attn_errors(out[0, :, h].cpu().double().numpy()[rows], ref[rows])
-        assert e["max_abs"] <= Hp.ATTN_MAX_ABS and e["mean_abs"] <= Hp.ATTN_MEAN_ABS, e
+        e = Hp.assert_attn_close(out[0, :, h].cpu().double().numpy()[rows], ref[rows], signal_guard=False)
 
 
 # ------------------------------------------------------------------ full size (720p tokens)
@@ -268,7 +274,9 @@ def test_cluster_path_full_size_sampled_rows(B):
     S, Hh, D = FULL_WL.T * FULL_WL.H * FULL_WL.W, FULL_WL.heads, 128
     Cq, Ck = 64, 256
     cs = B.ClusterShape(1, Hh, D, S, Cq, Ck)
-    q, k, v = synth.draw_qkv(FULL_WL, device="cuda")            # raster bf16
+    # raster bf16 at unit value scale with sharp logits: with the recipe's literal 1/sqrt(128)
+    # scale the outputs are ~1e-4 and an absolute bound of 2e-2 would test nothing
+    q, k, v = synth.draw_qkv(FULL_WL.scaled(value_scale=1.0), device="cuda", sharpness=8.0)
     lq = synth.draw_cluster_labels(1, Hh, S, Cq, seed=101, empty=(5,))
     lk = synth.draw_cluster_labels(1, Hh, S, Ck, seed=102, empty=(7,))
     nq, sq, tq, _ = B.cluster_layout(lq.cuda(), cs, Cq)
@@ -281,7 +289,7 @@ def test_cluster_path_full_size_sampled_rows(B):
     assert B.device_status(ws) == 0
     scale = 1.0 / math.sqrt(D)
     g = torch.Generator().manual_seed(104)
-    errs = []
+    gots, refs = [], []
     for h in (0, Hh // 2, Hh - 1):
         st_q, tos_q, _ = O.cluster_layout(lq[0, h].numpy(), Cq)
         st_k, tos_k, _ = O.cluster_layout(lk[0, h].numpy(), Ck)
@@ -300,10 +308,9 @@ def test_cluster_path_full_size_sampled_rows(B):
         Xv = v[0, :, h].float().cpu().double().numpy()[tos_k]
         ref = O.cluster_attention(Xq, Xk, Xv, st_q, cq_, st_k, ck_, rows, cols, scale,
                                   rows=slots[toks])
-        got = back[0, torch.from_numpy(toks), h].float().cpu().double().numpy()
-        errs.append(Hp.attn_errors(got, ref[slots[toks]]))
-    for e in errs:
-        assert e["max_abs"] <= Hp.ATTN_MAX_ABS and e["mean_abs"] <= Hp.ATTN_MEAN_ABS, e
+        gots.append(back[0, torch.from_numpy(toks), h].float().cpu().double().numpy())
+        refs.append(ref[slots[toks]])
+    Hp.assert_attn_close(np.concatenate(gots), np.concatenate(refs))
 
 
 def test_kmeans_full_size_properties(B):
@@ -383,5 +390,4 @@ def test_cluster_fwd_edge_shapes(B, S):
     ref = O.cluster_attention(q[0, 0].double().numpy(), k[0, 0].double().numpy(), v[0, 0].double().numpy(),
                               qs[0, 0].numpy(), qn[0, 0].numpy(), ks[0, 0].numpy(), kn[0, 0].numpy(),
                               rp.numpy(), ci.numpy(), 1.0 / math.sqrt(D))
-    e = Hp.attn_errors(_np(out[0, 0]), ref)
-    assert e["max_abs"] <= Hp.ATTN_MAX_ABS and e["mean_abs"] <= Hp.ATTN_MEAN_ABS, e
+    e = Hp.assert_attn_close(_np(out[0, 0]), ref, signal_guard=False)
