@@ -153,6 +153,7 @@ def lib() -> ctypes.CDLL:
         "bsa_cluster_fwd": (I, [CSP, P, P, P, P, P, P, P, P, P, F, P, P, P, S, P]),
         "bsa_selftest_wait": (I, [P, S, L64, P]),
         "bsa_fwd_raster": (I, [SP, P, P, P, P, P, F, P, P, P, S, P]),
+        "bsa_kernel_binary_version": (I, [ctypes.POINTER(ctypes.c_int32)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -170,7 +171,7 @@ EXPORTED_SYMBOLS = ("bsa_workspace_bytes", "bsa_clear_status", "bsa_device_statu
                     "bsa_cluster_fwd_workspace_bytes", "bsa_topp_rows_workspace_bytes",
                     "bsa_kmeans", "bsa_cluster_layout", "bsa_cluster_permute", "bsa_cluster_mass",
                     "bsa_topp_select_rows", "bsa_cluster_fwd", "bsa_selftest_wait",
-                    "bsa_fwd_raster")
+                    "bsa_fwd_raster", "bsa_kernel_binary_version")
 
 
 def _check(status: int, what: str):

@@ -8,6 +8,7 @@ is newer than the library (or when force=True).
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -54,8 +55,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         return LIB_PATH
     objdir = os.path.join(PKG_DIR, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
-    for src in sources():
+
+    def compile_one(src):
         obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
         cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
         if ptxas_info:
@@ -67,7 +68,11 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
             raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
         if ptxas_info or verbose:
             sys.stderr.write(r.stderr)
-        objs.append(obj)
+        return obj
+
+    # one nvcc per translation unit, run side by side
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        objs = list(ex.map(compile_one, sources()))
     tmp = LIB_PATH + ".tmp"
     cmd = [_nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp, *objs,
            "-lcudart"]

@@ -94,6 +94,8 @@ using bsa::ClusterDims;
 namespace {
 
 // Host-side shape checks shared by every entry point.
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
 bsa_status check_shape(const bsa_shape* s, bool attention) {
   if (s == nullptr) return BSA_ERR_INVALID_ARG;
   if (s->batch < 1 || s->heads < 1 || s->head_dim < 1) return BSA_ERR_INVALID_ARG;
@@ -176,6 +178,15 @@ size_t workspace_bytes(const bsa_shape* s, int op) {
 extern "C" {
 
 const char* bsa_version(void) { return "bsattn 0.1 sm_100a"; }
+
+bsa_status bsa_kernel_binary_version(int32_t* version) {
+  if (version == nullptr) return BSA_ERR_INVALID_ARG;
+  int v = 0;
+  const cudaError_t e = bsa::kernel_binary_version(&v);
+  if (e != cudaSuccess) return from_cuda(e);
+  *version = v;
+  return BSA_OK;
+}
 
 const char* bsa_status_string(bsa_status st) {
   switch (st) {
@@ -297,7 +308,7 @@ bsa_status bsa_topp_select(const bsa_shape* shape, const float* mass, float thre
   bsa_status st = check_shape(shape, true);
   if (st != BSA_OK) return st;
   if (mass == nullptr || row_ptr == nullptr || ws == nullptr || !bsa::aligned16(ws) ||
-      (reinterpret_cast<uintptr_t>(mass) & 3u))
+      (reinterpret_cast<uintptr_t>(mass) & 3u) || !aligned4(row_ptr) || !aligned4(col_idx))
     return BSA_ERR_INVALID_ARG;
   if (col_capacity < 0 || (col_capacity > 0 && col_idx == nullptr)) return BSA_ERR_INVALID_ARG;
   if (!(threshold > 0.f && threshold <= 1.f)) return BSA_ERR_INVALID_ARG;
@@ -313,7 +324,8 @@ bsa_status bsa_pattern_csr(const bsa_shape* shape, const bsa_pattern* pattern, i
                            bsa_stream_t stream) {
   bsa_status st = check_shape(shape, true);
   if (st != BSA_OK) return st;
-  if (pattern == nullptr || row_ptr == nullptr || ws == nullptr || !bsa::aligned16(ws))
+  if (pattern == nullptr || row_ptr == nullptr || ws == nullptr || !bsa::aligned16(ws) ||
+      !aligned4(row_ptr) || !aligned4(col_idx))
     return BSA_ERR_INVALID_ARG;
   if (col_capacity < 0 || (col_capacity > 0 && col_idx == nullptr)) return BSA_ERR_INVALID_ARG;
   const uint32_t all = BSA_PAT_DIAGONAL | BSA_PAT_MULTI_DIAGONAL | BSA_PAT_VERTICAL_STRIPE |
@@ -346,7 +358,7 @@ bsa_status bsa_topp_select_noalloc(const bsa_shape* shape, const float* mass, fl
   bsa_status st = check_shape(shape, true);
   if (st != BSA_OK) return st;
   if (mass == nullptr || row_ptr == nullptr || (reinterpret_cast<uintptr_t>(mass) & 3u) ||
-      (status != nullptr && (reinterpret_cast<uintptr_t>(status) & 3u)))
+      !aligned4(row_ptr) || !aligned4(col_idx) || (status != nullptr && (reinterpret_cast<uintptr_t>(status) & 3u)))
     return BSA_ERR_INVALID_ARG;
   if (col_capacity < 0 || (col_capacity > 0 && col_idx == nullptr)) return BSA_ERR_INVALID_ARG;
   if (!(threshold > 0.f && threshold <= 1.f)) return BSA_ERR_INVALID_ARG;
@@ -370,7 +382,8 @@ bsa_status bsa_fwd(const bsa_shape* shape, bsa_dtype dtype, const void* q, const
       out == nullptr || ws == nullptr)
     return BSA_ERR_INVALID_ARG;
   if (!bsa::aligned16(q) || !bsa::aligned16(k) || !bsa::aligned16(v) || !bsa::aligned16(out) ||
-      !bsa::aligned16(ws) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+      !bsa::aligned16(ws) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+      !aligned4(row_ptr) || !aligned4(col_idx))
     return BSA_ERR_INVALID_ARG;
   if (dtype == BSA_E4M3) {
     if (q_scales == nullptr || k_scales == nullptr || v_scales == nullptr) return BSA_ERR_INVALID_ARG;
@@ -395,8 +408,6 @@ bsa_status bsa_fwd(const bsa_shape* shape, bsa_dtype dtype, const void* q, const
 
 // ---------------------------------------------------------------- semantic clusters
 namespace {
-
-bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 bsa_status check_cluster_shape(const bsa_cluster_shape* s) {
   if (s == nullptr) return BSA_ERR_INVALID_ARG;

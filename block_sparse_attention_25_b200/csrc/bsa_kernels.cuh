@@ -249,6 +249,7 @@ cudaError_t launch_bsattn_fwd_raster(const AttnDims& a, const void* q, const voi
 
 // Failure-detection self-test (bounded wait on a barrier nothing completes).
 cudaError_t launch_selftest_wait(void* ws, uint64_t limit_ns, cudaStream_t stream);
+cudaError_t kernel_binary_version(int* version);
 
 // Encode a rank-3 bf16/e4m3 tensor map over [bh][Np][D] with a (box_d x box_rows x 1) box
 // and 128-byte swizzle.

@@ -37,4 +37,13 @@ cudaError_t launch_selftest_wait(void* ws, uint64_t limit_ns, cudaStream_t strea
   return cudaGetLastError();
 }
 
+// The compute capability the library's device code was built for (major * 10 + minor), as
+// the runtime reports it for a kernel of this library: 100 for sm_100a.
+cudaError_t kernel_binary_version(int* version) {
+  cudaFuncAttributes attr;
+  const cudaError_t e = cudaFuncGetAttributes(&attr, selftest_wait_kernel);
+  if (e == cudaSuccess) *version = attr.binaryVersion;
+  return e;
+}
+
 }  // namespace bsa

@@ -340,25 +340,69 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
 // cudaGetSymbolAddress below.
 static __device__ __align__(256) uint8_t g_topp_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kMaxDevices] = {nullptr};
+// The array's device address belongs to the CUDA context the module was loaded into: another
+// context on the same device (a driver-API context of the caller's own) sees the array at
+// another address, and a device reset unloads the module, so an address found before the
+// reset may no longer belong to the library.  The address is therefore cached per context,
+// keyed by the context's unique ID (cuCtxGetId: never reused within a process, unlike the
+// context handle), so the first call in every context -- a new one after a device reset
+// included -- looks it up with that context current.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of the scratch array for the current device, looked up once per device
-// (with that device current) and cached.
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<Fn>(p);
+  return nullptr;
+}
+
+constexpr int kMaxContexts = 64;
+std::mutex g_noalloc_mu;
+unsigned long long g_noalloc_ctx_id[kMaxContexts] = {0};
+void* g_noalloc_addr[kMaxContexts] = {nullptr};
+int g_noalloc_n = 0;     // entries in use
+int g_noalloc_next = 0;  // entry replaced next once all are in use
+
+// Device address of the scratch array in the current context.
 cudaError_t noalloc_scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+  static CtxGetCurrentFn get_ctx = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    get_ctx = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  });
+  if (get_ctx == nullptr || get_id == nullptr) return cudaErrorInitializationError;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  if (ctx == nullptr) {
+    // No context current on this thread yet: the runtime's lookup makes the current
+    // device's primary context current.
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_topp_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_noalloc_addr[dev] = p;
+    const cudaError_t e0 = cudaGetSymbolAddress(&p, g_topp_noalloc_scratch);
+    if (e0 != cudaSuccess) return e0;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorDeviceUninitialized;
   }
-  *out = g_noalloc_addr[dev];
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  cudaError_t e = cudaSuccess;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  for (int i = 0; i < g_noalloc_n; ++i)
+    if (g_noalloc_ctx_id[i] == id) {
+      *out = g_noalloc_addr[i];
+      return cudaSuccess;
+    }
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_topp_noalloc_scratch);
+  if (e != cudaSuccess) return e;
+  int slot = g_noalloc_n < kMaxContexts ? g_noalloc_n++ : g_noalloc_next++ % kMaxContexts;
+  g_noalloc_ctx_id[slot] = id;
+  g_noalloc_addr[slot] = p;
+  *out = p;
   return cudaSuccess;
 }
 

@@ -16,7 +16,8 @@
  *
  * Conventions shared by every call
  *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The library
- *     allocates no memory and keeps no global state; scratch space is the caller's
+ *     allocates no memory and keeps no global state (the one exception is the fixed
+ *     scratch array of bsa_topp_select_noalloc, below); scratch space is the caller's
  *     workspace (`ws`), sized by bsa_workspace_bytes().  A workspace serves one call at a
  *     time: calls that may overlap (other streams) need workspaces of their own.
  *   - Every call is asynchronous and ordered on `stream` (NULL = legacy default
@@ -121,6 +122,11 @@ BSA_API bsa_status bsa_device_status_words(const void* ws, uint32_t out_words[4]
 
 BSA_API const char* bsa_status_string(bsa_status status);
 
+/* The compute capability the library's kernels were compiled for, as the CUDA runtime
+ * reports it for a kernel of the loaded library (cudaFuncGetAttributes binaryVersion:
+ * major*10 + minor, 100 for sm_100a).  Needs a CUDA device; BSA_ERR_CUDA otherwise. */
+BSA_API bsa_status bsa_kernel_binary_version(int32_t* version);
+
 /* 3D tile permutation ("FPSAttention", Abstract, innovation 1: unified 3D tile-wise
  * granularity).  inverse = 0: raster src [B,S,Hh,D] -> tile-major dst [B,Hh,Np,D],
  * pad slots written as zero.  inverse = 1: tile-major src -> raster dst, pad slots
@@ -203,9 +209,12 @@ BSA_API bsa_status bsa_topp_select(const bsa_shape* shape, const float* mass, fl
  *   - Size limit: R*4 rounded up to 256 bytes, plus R*ceil((Np/64)/32)*4 bytes, must fit in
  *     16 MiB (R = B*Hh*Np/q_block); larger problems return BSA_ERR_CAPACITY and launch
  *     nothing.  The 720p 40-head shape needs 10.6 MB.
- *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
- *     with that device current) and caches it; make that first call before any stream
- *     capture.
+ *   - Set-up: the array's device address depends on the CUDA context (each context that
+ *     loads the library has its own copy, and a device reset reloads it elsewhere), so the
+ *     first call in each context -- the device's primary context, a driver-API context of
+ *     the caller's own, or the new context after a device reset -- looks the address up
+ *     (cudaGetSymbolAddress, with that context current) and caches it under the context's
+ *     unique ID.  Make that first call before any stream capture.
  *   - Every call shares the one array and leaves its contents behind; each call rewrites
  *     all of the scratch it reads, so nothing needs clearing, but calls that overlap on the
  *     GPU (different streams, or several host threads) race on it and must be serialised
