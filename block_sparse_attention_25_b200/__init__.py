@@ -10,7 +10,7 @@ from .bsattn import (  # noqa: F401
     topp_select_noalloc, PAT_DIAGONAL, PAT_MULTI_DIAGONAL, PAT_VERTICAL_STRIPE, PAT_SURROUNDING,
     PAT_CRISS_CROSS, ClusterShape, kmeans, cluster_layout, cluster_permute, cluster_mass,
     topp_select_rows, cluster_fwd, new_cluster_workspace, new_cluster_fwd_workspace,
-    bsattn_fwd_raster,
+    bsattn_fwd_raster, save_lists, load_lists,
 )
 
 __all__ = [
@@ -18,5 +18,6 @@ __all__ = [
     "device_status", "device_status_words", "lib", "new_workspace", "tile_permute",
     "tile_permute_quant_e4m3", "topp_select", "workspace_bytes", "pattern_csr",
     "topp_select_noalloc", "ClusterShape", "kmeans", "cluster_layout", "cluster_permute",
-    "cluster_mass", "topp_select_rows", "cluster_fwd", "bsattn_fwd_raster",
+    "cluster_mass", "topp_select_rows", "cluster_fwd", "bsattn_fwd_raster", "save_lists",
+    "load_lists",
 ]

@@ -24,7 +24,8 @@ LIB_PATH = os.path.join(_PKG_DIR, "libbsattn.so")
 
 BSA_OK = 0
 STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "capacity too small",
-                4: "CUDA error", 5: "device wait timed out", 6: "device-side input check failed"}
+                4: "CUDA error", 5: "device wait timed out", 6: "device-side input check failed",
+                7: "list file missing, unreadable or corrupt"}
 BSA_BF16, BSA_FP32, BSA_E4M3 = 0, 1, 2
 OP_BLOCK_MASS, OP_TOPP_SELECT, OP_FWD, OP_PATTERN, OP_POOLED_MASS = 0, 1, 2, 3, 4
 PAT_DIAGONAL, PAT_MULTI_DIAGONAL, PAT_VERTICAL_STRIPE, PAT_SURROUNDING, PAT_CRISS_CROSS = 1, 2, 4, 8, 16
@@ -154,6 +155,10 @@ def lib() -> ctypes.CDLL:
         "bsa_selftest_wait": (I, [P, S, L64, P]),
         "bsa_fwd_raster": (I, [SP, P, P, P, P, P, F, P, P, P, S, P]),
         "bsa_kernel_binary_version": (I, [ctypes.POINTER(ctypes.c_int32)]),
+        "bsa_lists_save": (I, [ctypes.c_char_p, SP, F, P, P]),
+        "bsa_lists_read_header": (I, [ctypes.c_char_p, SP, ctypes.POINTER(F),
+                                      ctypes.POINTER(L64)]),
+        "bsa_lists_load": (I, [ctypes.c_char_p, SP, ctypes.POINTER(F), P, P, L64]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -171,7 +176,8 @@ EXPORTED_SYMBOLS = ("bsa_workspace_bytes", "bsa_clear_status", "bsa_device_statu
                     "bsa_cluster_fwd_workspace_bytes", "bsa_topp_rows_workspace_bytes",
                     "bsa_kmeans", "bsa_cluster_layout", "bsa_cluster_permute", "bsa_cluster_mass",
                     "bsa_topp_select_rows", "bsa_cluster_fwd", "bsa_selftest_wait",
-                    "bsa_fwd_raster", "bsa_kernel_binary_version")
+                    "bsa_fwd_raster", "bsa_kernel_binary_version", "bsa_lists_save",
+                    "bsa_lists_read_header", "bsa_lists_load")
 
 
 def _check(status: int, what: str):
@@ -337,6 +343,33 @@ def topp_select(mass, shape: Shape, threshold: float = 0.99, col_capacity=None, 
                                  _ptr(row_ptr), _ptr(col_idx), cap, _ptr(ws), ws.numel(),
                                  _stream(stream)), "bsa_topp_select")
     return row_ptr, col_idx
+
+
+def save_lists(path, row_ptr, col_idx, shape: Shape, threshold: float):
+    """bsa_lists_save: write frozen lists (device or host int32 tensors) to `path`."""
+    rp = row_ptr.detach().to("cpu", torch.int32).contiguous()
+    if rp.numel() != shape.rows + 1:
+        raise ValueError(f"row_ptr: expected {shape.rows + 1} entries, got {rp.numel()}")
+    nnz = int(rp[-1])
+    ci = col_idx.detach()[:nnz].to("cpu", torch.int32).contiguous()
+    _check(lib().bsa_lists_save(os.fsencode(path), ctypes.byref(shape.c()), float(threshold),
+                                _ptr(rp), _ptr(ci) if nnz else None), "bsa_lists_save")
+
+
+def load_lists(path, shape: Shape, device="cuda"):
+    """bsa_lists_load: (row_ptr, col_idx, threshold) from a list file written for `shape`;
+    row_ptr and col_idx land on `device` (col_idx holds exactly nnz entries, at least one)."""
+    L = lib()
+    stored = _Shape()
+    tau = ctypes.c_float(0.0)
+    nnz = ctypes.c_int64(0)
+    _check(L.bsa_lists_read_header(os.fsencode(path), ctypes.byref(stored), ctypes.byref(tau),
+                                   ctypes.byref(nnz)), "bsa_lists_read_header")
+    rp = torch.empty(shape.rows + 1, dtype=torch.int32)
+    ci = torch.zeros(max(nnz.value, 1), dtype=torch.int32)
+    _check(L.bsa_lists_load(os.fsencode(path), ctypes.byref(shape.c()), ctypes.byref(tau),
+                            _ptr(rp), _ptr(ci), nnz.value), "bsa_lists_load")
+    return rp.to(device), ci.to(device), float(tau.value)
 
 
 def topp_select_noalloc(mass, shape: Shape, threshold: float = 0.99, row_ptr=None, col_idx=None,

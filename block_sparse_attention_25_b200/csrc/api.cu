@@ -118,6 +118,14 @@ bsa_status check_shape(const bsa_shape* s, bool attention) {
   return BSA_OK;
 }
 
+}  // namespace
+
+namespace bsa {
+bsa_status check_attention_shape(const bsa_shape* s) { return check_shape(s, true); }
+}  // namespace bsa
+
+namespace {
+
 GridDims make_grid(const bsa_shape* s) {
   GridDims g;
   g.T = s->T;
@@ -197,6 +205,7 @@ const char* bsa_status_string(bsa_status st) {
     case BSA_ERR_CUDA: return "CUDA error";
     case BSA_ERR_TIMEOUT: return "device wait timed out";
     case BSA_ERR_DEVICE_INPUT: return "device-side input check failed";
+    case BSA_ERR_IO: return "list file missing, unreadable or corrupt";
   }
   return "unknown status";
 }

@@ -64,7 +64,8 @@ typedef enum {
   BSA_ERR_CAPACITY = 3,      /* workspace or col_idx capacity too small */
   BSA_ERR_CUDA = 4,          /* a CUDA runtime / driver call failed */
   BSA_ERR_TIMEOUT = 5,       /* a device pipeline wait hit its time limit and gave up */
-  BSA_ERR_DEVICE_INPUT = 6   /* device data failed a check (CSR order/range, mass values) */
+  BSA_ERR_DEVICE_INPUT = 6,  /* device data failed a check (CSR order/range, mass values) */
+  BSA_ERR_IO = 7             /* a list file is missing, unwritable, truncated or corrupt */
 } bsa_status;
 
 typedef enum { BSA_BF16 = 0, BSA_FP32 = 1, BSA_E4M3 = 2 } bsa_dtype;
@@ -225,6 +226,30 @@ BSA_API bsa_status bsa_topp_select_noalloc(const bsa_shape* shape, const float* 
                                            float threshold, int32_t* row_ptr, int32_t* col_idx,
                                            int64_t col_capacity, uint32_t* status,
                                            bsa_stream_t stream);
+
+/* Frozen lists on disk ("LoSA", Abstract: the block indices selected at the calibration
+ * step are frozen and reused for all remaining steps -- they are the method's only state,
+ * so a run can resume after the calibration with the very same lists).  HOST pointers,
+ * owned by the caller; these calls touch no device memory and launch nothing.
+ * File: magic "BSALISTS", version 1, the bsa_shape, the threshold (float32, kept for the
+ * record), R and nnz (int64), row_ptr int32 [R+1], col_idx int32 [nnz], then a 64-bit
+ * FNV-1a hash of everything before it; little-endian.
+ *   bsa_lists_save: row_ptr [R+1] and col_idx [row_ptr[R]] as a selection produces them
+ *     (row_ptr[0] = 0, non-decreasing, each row's indices strictly ascending in
+ *     [0, Np/64)), else BSA_ERR_INVALID_ARG; written to `path`.tmp and renamed, so `path`
+ *     never holds half a file; BSA_ERR_IO if it cannot be written.
+ *   bsa_lists_read_header: the stored shape, threshold and nnz (any output may be NULL),
+ *     so the caller can size col_idx.
+ *   bsa_lists_load: `shape` must equal the stored one (else BSA_ERR_INVALID_ARG) and
+ *     col_capacity >= nnz (else BSA_ERR_CAPACITY); a missing, truncated, altered (hash) or
+ *     malformed file returns BSA_ERR_IO.  The caller's buffers are written only on
+ *     BSA_OK. */
+BSA_API bsa_status bsa_lists_save(const char* path, const bsa_shape* shape, float threshold,
+                                  const int32_t* row_ptr, const int32_t* col_idx);
+BSA_API bsa_status bsa_lists_read_header(const char* path, bsa_shape* shape, float* threshold,
+                                         int64_t* nnz);
+BSA_API bsa_status bsa_lists_load(const char* path, const bsa_shape* shape, float* threshold,
+                                  int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity);
 
 /* Static structured kv-block lists ("Sparse-vDiT", Abstract: diagonal, multi-diagonal and
  * vertical-stripe attention structures; "GRAT", Abstract: key regions restricted to

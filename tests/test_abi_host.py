@@ -259,7 +259,7 @@ def test_selftest_rejections_before_launch(B):
 
 def test_status_strings(B):
     L = B.lib()
-    for code in range(7):
+    for code in range(8):
         assert L.bsa_status_string(code)
     assert b"sm_100a" in L.bsa_version()
 

@@ -396,3 +396,23 @@ def test_fwd_fp8_rescale_path(B):
     rp = np.arange(R + 1) * n_kb
     ci = np.tile(np.arange(n_kb), R)
     _fp8_compare(B, wl, q2, k2, v, rp, ci)
+
+
+# ------------------------------------------------------------------ frozen lists on disk
+def test_forward_on_reloaded_lists_is_bit_identical(B, tmp_path):
+    """Calibrate, select, save the lists, load them back: the forward over the loaded lists
+    equals the forward over the selection's own lists bit for bit."""
+    wl = WLS[0]
+    s = _shape(B, wl)
+    q, k, v = Hp.draw(wl, value_scale=1.0, sharp=6.0)
+    qt, kt, vt = (B.tile_permute(x.cuda(), s) for x in (q, k, v))
+    rp, ci = B.topp_select(B.block_mass(qt, kt, s), s, 0.95)
+    path = tmp_path / "frozen.bin"
+    B.save_lists(path, rp, ci, s, 0.95)
+    rp2, ci2, tau = B.load_lists(path, s)
+    assert np.float32(tau) == np.float32(0.95)
+    n = int(rp[-1])
+    assert torch.equal(rp2, rp) and torch.equal(ci2[:n], ci[:n])
+    out = B.bsattn_fwd(qt, kt, vt, rp, ci, s)
+    out2 = B.bsattn_fwd(qt, kt, vt, rp2, ci2, s)
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))

@@ -1,0 +1,95 @@
+"""Frozen lists on disk (bsa_lists_save / bsa_lists_read_header / bsa_lists_load): host
+calls only, no GPU.  The lists are the method's only state between the calibration and
+the later steps ("LoSA", Abstract: the selected block indices are frozen and reused), so a
+saved file must give back exactly the lists that went in, and a damaged one must be
+refused rather than read."""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_25_b200 import synth
+
+WL = synth.Workload("lists-6x10x11-h3", 2, 3, 128, 6, 10, 11, 8, 12, 12, 64, 64)
+
+
+@pytest.fixture(scope="module")
+def B():
+    from block_sparse_attention_25_b200 import build
+    build.build()
+    import block_sparse_attention_25_b200 as b
+    return b
+
+
+def _lists(B, keep=0.4, seed=5):
+    s = B.Shape.of(WL)
+    rp, ci = synth.draw_keep_csr(s.rows, s.n_kb, keep, seed=seed, empty_rows=(0, 7))
+    return s, rp, ci
+
+
+def test_round_trip_is_exact(B, tmp_path):
+    s, rp, ci = _lists(B)
+    path = tmp_path / "lists.bin"
+    B.save_lists(path, rp, ci, s, 0.99)
+    rp2, ci2, tau = B.load_lists(path, s, device="cpu")
+    assert torch.equal(rp2, rp) and torch.equal(ci2[:int(rp[-1])], ci)
+    assert np.float32(tau) == np.float32(0.99)
+    # a capacity-sized col_idx (as the selection returns it) saves the same file
+    big = torch.full((s.rows * s.n_kb,), -1, dtype=torch.int32)
+    big[:ci.numel()] = ci
+    p2 = tmp_path / "lists2.bin"
+    B.save_lists(p2, rp, big, s, 0.99)
+    assert p2.read_bytes() == path.read_bytes()
+
+
+def test_empty_lists_round_trip(B, tmp_path):
+    s = B.Shape.of(WL)
+    rp = torch.zeros(s.rows + 1, dtype=torch.int32)
+    path = tmp_path / "empty.bin"
+    B.save_lists(path, rp, torch.zeros(0, dtype=torch.int32), s, 0.5)
+    rp2, ci2, _ = B.load_lists(path, s, device="cpu")
+    assert torch.equal(rp2, rp) and ci2.numel() == 1
+
+
+def test_damaged_files_are_refused(B, tmp_path):
+    s, rp, ci = _lists(B)
+    path = tmp_path / "lists.bin"
+    B.save_lists(path, rp, ci, s, 0.99)
+    good = path.read_bytes()
+
+    def refused(data, status=7):
+        bad = tmp_path / "bad.bin"
+        bad.write_bytes(data)
+        with pytest.raises(B.BsaError) as e:
+            B.load_lists(bad, s, device="cpu")
+        assert e.value.status == status
+
+    refused(good[:-1])                                   # truncated hash
+    refused(good[:200])                                  # truncated payload
+    refused(good + b"\0")                                # trailing bytes
+    refused(b"X" + good[1:])                             # magic
+    flip = bytearray(good)
+    flip[100] ^= 1                                       # one bit of row_ptr: hash mismatch
+    refused(bytes(flip))
+    with pytest.raises(B.BsaError) as e:                 # missing file
+        B.load_lists(tmp_path / "nope.bin", s, device="cpu")
+    assert e.value.status == 7
+    other = B.Shape.of(WL.scaled(heads=2))               # lists of another shape
+    with pytest.raises(B.BsaError) as e:
+        B.load_lists(path, other, device="cpu")
+    assert e.value.status in (1, 7)
+
+
+def test_malformed_lists_are_not_saved(B, tmp_path):
+    s, rp, ci = _lists(B)
+    bad = ci.clone()
+    r = int(torch.nonzero(rp[1:] - rp[:-1] >= 2)[0])    # a row with two entries
+    b = int(rp[r])
+    bad[b], bad[b + 1] = bad[b + 1].item(), bad[b].item()   # not ascending
+    with pytest.raises(B.BsaError) as e:
+        B.save_lists(tmp_path / "x.bin", rp, bad, s, 0.99)
+    assert e.value.status == 1
+    out = ci.clone()
+    out[0] = s.n_kb                                      # out of range
+    with pytest.raises(B.BsaError):
+        B.save_lists(tmp_path / "x.bin", rp, out, s, 0.99)
+    assert not (tmp_path / "x.bin").exists() and not (tmp_path / "x.bin.tmp").exists()
