@@ -1,6 +1,7 @@
 """Benchmark: retained-mass block-sparse attention on B200, one JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+                    [--split problems|heads]
 
 A step is one calibrate-then-reuse cycle of the 720p workload (the default config,
 Wan-14B-like: B=1, 40 heads, D=128, 21x45x80 tokens padded to 24x48x80, 64-token blocks):
@@ -11,15 +12,22 @@ Wan-14B-like: B=1, 40 heads, D=128, 21x45x80 tokens padded to 24x48x80, 64-token
                  tile_permute_quant_e4m3 x3 -> bsattn_fwd -> inverse)
 on seeded synthetic inputs already resident in HBM (Q/K/V of 774 MB each, far above L2).
 
-value  = executed attention TFLOP/s of the whole step: FLOPs of the kept blocks of the 10
-         reuse calls (4 * 64 * 64 * D per kept (query block, kv block) pair) divided by
-         the device time of the whole cycle, max over ranks.
+value  = executed attention TFLOP/s of the whole step (a step rate): FLOPs of the kept
+         blocks of the 10 reuse calls (4 * 64 * 64 * D per kept (query block, kv block)
+         pair) divided by the device time of the whole cycle, calibration included, max
+         over ranks.
 fwd    = the same FLOPs over the forward launches alone (CUDA events on the launch
          stream) -> roofline of the dominant kernel.
 e2e    = the same metric through the public API with inputs copied from pinned host
          memory and outputs copied back inside the timed region.
 --impl reference times the CPU oracle (the only other implementation of the method) on
 a bounded sample of the same workload.
+
+With N > 1 ranks (one per GPU) the path needs no exchange step: --split problems (the
+default) gives every rank an independent problem of the workload's size (weak scaling);
+--split heads gives rank r the heads [r*Hh/N, (r+1)*Hh/N) of one problem (strong scaling;
+Hh must divide by N).  The process group carries only the timing barrier and the
+max-over-ranks reduction.
 """
 from __future__ import annotations
 
@@ -39,7 +47,7 @@ CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.a
                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3)
@@ -55,7 +63,10 @@ def parse_args():
     ap.add_argument("--cpu-sample-rows", type=int, default=256)
     ap.add_argument("--clock-log", default=None,
                     help="CSV of the nvidia-smi clock samples ({rank} is replaced); default /tmp")
-    return ap.parse_args()
+    ap.add_argument("--split", default="problems", choices=["problems", "heads"],
+                    help="N > 1: an independent problem per rank, or the heads of one problem "
+                         "divided over the ranks")
+    return ap.parse_args(argv)
 
 
 def peaks():
@@ -65,6 +76,18 @@ def peaks():
         return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
                     source="measured")
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16 tensor peak (NVIDIA's figure without 2:4 sparsity)
+
+
+def head_range(rank: int, world: int, heads: int):
+    """Heads [h0, h1) of one problem owned by `rank` when the heads are split over `world`
+    ranks (equal shares; the head count must divide by the rank count)."""
+    if heads % world:
+        raise ValueError(f"{heads} heads do not divide over {world} ranks")
+    n = heads // world
+    return rank * n, (rank + 1) * n
 
 
 def measured_traffic(fp8: bool, raster: bool):
@@ -142,14 +165,22 @@ class ClockSampler:
 
 
 def dist_setup(args):
+    """One process per GPU: NCCL when CUDA is available (the device of LOCAL_RANK), gloo on
+    a host without GPUs (the CPU tests)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     pg = None
     if world > 1:
         import datetime
+        import torch
         import torch.distributed as dist
-        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=600))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=300))
         pg = dist
     return world, rank, local, pg
 
@@ -158,8 +189,19 @@ def max_over_ranks(x: float, pg) -> float:
     if pg is None:
         return x
     import torch
-    t = torch.tensor([x], dtype=torch.float64)
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, pg) -> float:
+    if pg is None:
+        return x
+    import torch
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.SUM)
     return float(t.item())
 
 
@@ -178,17 +220,31 @@ def run_ours(args, world, rank, local, pg):
     build.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    wl = synth.WORKLOADS[args.config]
-    n_reuse = args.reuse if args.reuse is not None else max(wl.redraws, 1)
+    wl_full = synth.WORKLOADS[args.config]
+    n_reuse = args.reuse if args.reuse is not None else max(wl_full.redraws, 1)
+    heads = args.split == "heads" and world > 1
+    if heads:
+        # rank's share of one problem: its heads of the same draws
+        h0, h1 = head_range(rank, world, wl_full.heads)
+        wl = wl_full.scaled(heads=h1 - h0)
+        draw_wl = wl_full
+
+        def mine(qkv):
+            return tuple(x[:, :, h0:h1].contiguous() for x in qkv)
+    else:
+        wl = wl_full
+        draw_wl = wl_full.scaled(seed=wl_full.seed + 7919 * rank)  # independent problem per rank
+
+        def mine(qkv):
+            return qkv
     s = bsa.Shape.of(wl)
     fp8 = wl.fp8
     raster = not fp8 and args.layout == "raster"
-    seed_wl = wl.scaled(seed=wl.seed + 7919 * rank)  # independent problem per rank
 
     # ---- inputs resident in HBM: the calibration draw and n_reuse correlated re-draws
-    draws = [synth.draw_qkv(seed_wl, device=dev)]
+    draws = [mine(synth.draw_qkv(draw_wl, device=dev))]
     for r in range(1, n_reuse + 1):
-        draws.append(synth.redraw_qkv(seed_wl, r, device=dev))
+        draws.append(mine(synth.redraw_qkv(draw_wl, r, device=dev)))
     torch.cuda.synchronize()
 
     tiled = (s.batch, s.heads, s.Np, s.head_dim)
@@ -267,6 +323,8 @@ def run_ours(args, world, rank, local, pg):
             raise RuntimeError(f"device status {st} after warm-up: {bsa.device_status_words(w)}")
 
     # executed FLOPs of one reuse call: kept pairs * 4 * q_block * 64 * D
+    from block_sparse_attention_25_b200.microbench import schedule_work
+    work = schedule_work(row_ptr, col_idx, s)
     nnz = int(row_ptr[-1].item())
     kept_frac = nnz / float(s.rows * s.n_kb)
     flops_call = 4.0 * nnz * s.q_block * 64 * s.head_dim
@@ -299,7 +357,8 @@ def run_ours(args, world, rank, local, pg):
             raise RuntimeError(f"device status {st} after timing: {bsa.device_status_words(w)}")
 
     ms_step = elapsed_ms / args.steps
-    total_flops = flops_call * n_reuse * args.steps * world
+    # every rank's executed FLOPs (a rank's problem, or its share of one problem's heads)
+    total_flops = sum_over_ranks(flops_call * n_reuse * args.steps, pg)
     value = total_flops / (elapsed_ms * 1e-3) / 1e12
     fwd_avg_ms = sum(fwd_ms) / len(fwd_ms)
     fwd_tflops = flops_call / (fwd_avg_ms * 1e-3) / 1e12
@@ -316,13 +375,13 @@ def run_ours(args, world, rank, local, pg):
     result = {
         "metric": "bsattn_fwd ms/call & executed TFLOPS at 99% retained mass, % of bf16 peak",
         "value": round(value, 2),
-        "unit": "TFLOP/s (executed, kept blocks)",
+        "unit": "TFLOP/s (executed, kept blocks; step rate: calibration + 10 reuse calls)",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms_step, 3),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if heads else "weak",
         "vs_baseline": None,
         "dtype": "e4m3" if fp8 else "bf16",
         "data": "synthetic (seeded 3D random-Fourier-feature Q/K/V + noise, correlated re-draws)",
@@ -338,11 +397,20 @@ def run_ours(args, world, rank, local, pg):
             "bsattn_fwd_ms_per_call": round(fwd_avg_ms, 3),
             "bsattn_fwd_tflops": round(fwd_tflops, 2),
             "bsattn_fwd_pct_of_peak": round(100.0 * fwd_tflops / peak, 2),
+            "bsattn_fwd_pct_of_peak_note": "of the sustained measured peak (" + peak_note + ")",
+            "bsattn_fwd_pct_of_burst_peak": round(
+                100.0 * fwd_tflops / (pk["bf16"] * (2.0 if fp8 else 1.0)), 2),
+            "bsattn_fwd_pct_of_nominal_peak": round(
+                100.0 * fwd_tflops / (NOMINAL_BF16_TFLOPS * (2.0 if fp8 else 1.0)), 2),
+            "pairs_kept": work["kept_pairs"],
+            "pairs_computed": work["computed_pairs"],
+            "computed_over_kept": work["computed_over_kept"],
             "dense_equivalent_tflops": round(dense_flops_call / (fwd_avg_ms * 1e-3) / 1e12, 2),
             "calibration_ms": round(cal_ms, 3),
             "executed_tflop_per_call": round(flops_call / 1e12, 3),
             "l2": "inputs larger than L2 (774 MB per tensor); no flush needed",
-            "parallelism": f"independent problem per GPU x{world}",
+            "parallelism": (f"heads of one problem split over {world} GPUs ({wl.heads} each)"
+                            if heads else f"independent problem per GPU x{world}"),
         },
         "roofline": {
             "bound": "tensor", "achieved": round(fwd_tflops, 2), "peak": peak, "unit": "TFLOP/s",
@@ -501,7 +569,7 @@ def run_e2e(args, bsa, s, draws, n_reuse, row_ptr, col_idx, flops_call, dev, str
     b.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b), pg)
-    val = flops_call * n_reuse * steps * world / (ms * 1e-3) / 1e12
+    val = sum_over_ranks(flops_call * n_reuse * steps, pg) / (ms * 1e-3) / 1e12
     return {"value": round(val, 2), "unit": "TFLOP/s (executed, kept blocks)",
             "h2d_bytes_per_step": counts["h2d"] // steps, "d2h_bytes_per_step": counts["d2h"] // steps,
             "steps": steps, "ms_per_step": round(ms / steps, 3),

@@ -15,13 +15,13 @@
 // On such a raise -- rare: only a row whose early blocks are far below its later ones --
 // the row's sum and the block sums it has already written are multiplied by
 // exp2(m_old - m_new) in place.  Every exponential of the calibration is computed once.
-// e[r,j] goes to this SM's slice of the workspace; at the end of the CTA
+// e[r,j] goes to the CTA's slice of the workspace; at the end of the CTA
 //   mass[i,j] = (1 / valid queries of i) * sum over the rows r of query block i of
 //               e[r,j] * exp2(m_r,half(j) - m_r) / l_r,
 // in a fixed order (deterministic), where the two threads of a row (one per column half)
 // each kept their own reference max m_r,half and sum.
-// The scratch slice is chosen by the SM the CTA runs on: the CTA's shared memory admits one
-// CTA per SM, so no two live CTAs share a slice.
+// The slice is claimed from a pool when the CTA starts and given back when it ends, so no
+// two live CTAs ever write the same slice, wherever and whenever they run.
 // Warp roles (576 threads): warps 0-7 and 10-17 own the rows, two threads per row: warps
 // 0-3 / 4-7 take the first kv block of each step of tile 0 / 1, warps 10-13 / 14-17 the
 // second (a warp reads the TMEM lane quarter of its sub-partition, warp % 4); warp 8 is
@@ -48,6 +48,7 @@ struct MassParams {
   float* mass;
   uint32_t* status;
   float* scratch;  // [kMassSlots][n_kb][256] unnormalised row-block sums
+  uint32_t* pool;  // kMassSlots bits: slices held by live CTAs
   float scale_log2;
 };
 
@@ -85,6 +86,7 @@ __global__ void __maxnreg__(mass::kMaxRegs)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* nvalid_sm = reinterpret_cast<int*>(tmem_slot + 2);  // [2 half][2 tile][4 warp]
+  int* slice_sm = reinterpret_cast<int*>(tmem_slot + 20);  // this CTA's scratch slice
   float* row_w = reinterpret_cast<float*>(smem + L::kRedOff);  // [half][row] weight of e
   float* xch = reinterpret_cast<float*>(smem + L::kXchOff);
 
@@ -108,6 +110,7 @@ __global__ void __maxnreg__(mass::kMaxRegs)
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
+    *slice_sm = claim_mass_slice(p.pool, p.status);
     fence_mbar_init();
   }
   if (warp == 9) tmem_alloc(tmem_slot, 512);
@@ -193,13 +196,11 @@ __global__ void __maxnreg__(mass::kMaxRegs)
     const int wcount = __popc(__ballot_sync(0xffffffffu, q_valid));
     if (lane == 0) nvalid_sm[(h * 2 + t) * 4 + wq] = wcount;
     named_bar_sync(gbar, 128);
-    // this SM's scratch slice: [n_kb][256] row-block sums
-    uint32_t smid;
-    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-    const bool have_slice = smid < static_cast<uint32_t>(kMassSlots);
-    if (!have_slice && h == 0 && local == 0)
-      record_status(p.status, FLAG_DEVICE_INPUT, DETAIL_MASS_SLICE, static_cast<uint32_t>(cta), smid);
-    float* sc = p.scratch + static_cast<size_t>(have_slice ? smid : 0u) * 256 * a.n_kb;
+    // this CTA's scratch slice: [n_kb][256] row-block sums (none: the claim timed out, no
+    // masses are written and the status header says so)
+    const int slice = *slice_sm;
+    const bool have_slice = slice >= 0;
+    float* sc = p.scratch + static_cast<size_t>(have_slice ? slice : 0) * 256 * a.n_kb;
 
     float m_ref = -INFINITY, l_run = 0.f;  // this half's reference max (log2 units) and sum
     bool ok = true;
@@ -327,11 +328,14 @@ __global__ void __maxnreg__(mass::kMaxRegs)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (threadIdx.x == 0) release_mass_slice(p.pool, *slice_sm);
 }
 
-// Scratch after the status header: kMassSlots slices of n_kb x 256 fp32 row-block sums.
+// Scratch after the status header: the slice pool's bitmap, then kMassSlots slices of
+// n_kb x 256 fp32 row-block sums.
 size_t mass_scratch_bytes(const AttnDims& a) {
-  return static_cast<size_t>(kMassSlots) * 256 * static_cast<size_t>(a.n_kb) * sizeof(float);
+  return kMassPoolBytes +
+         static_cast<size_t>(kMassSlots) * 256 * static_cast<size_t>(a.n_kb) * sizeof(float);
 }
 
 template <int D>
@@ -347,12 +351,15 @@ static cudaError_t launch_mass(const AttnDims& a, const void* q, const void* k,
   e = cudaFuncSetAttribute(block_mass_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            L::kAlloc);
   if (e != cudaSuccess) return e;
-  // the workspace slices are per SM id: at most one CTA of this kernel may live on an SM
+  // one CTA per SM, so the live CTAs (at most the SM count) never exhaust the kMassSlots
+  // slices and no claim waits
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, block_mass_kernel<D>, mass::kThreads,
                                                     L::kAlloc);
   if (e != cudaSuccess) return e;
   if (per_sm != 1) return cudaErrorInvalidConfiguration;
+  e = cudaMemsetAsync(prm.pool, 0, kMassPoolBytes, stream);
+  if (e != cudaSuccess) return e;
   block_mass_kernel<D><<<static_cast<unsigned>(ctas), mass::kThreads, L::kAlloc, stream>>>(tq, tk,
                                                                                           prm);
   return cudaGetLastError();
@@ -366,7 +373,8 @@ cudaError_t launch_block_mass(const AttnDims& a, const void* q, const void* k, f
   prm.a = a;
   prm.mass = mass_out;
   prm.status = static_cast<uint32_t*>(ws);
-  prm.scratch = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+  prm.pool = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+  prm.scratch = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kStatusBytes + kMassPoolBytes);
   prm.scale_log2 = softmax_scale * 1.4426950408889634f;
   if (a.head_dim == 128) return launch_mass<128>(a, q, k, prm, ctas, stream);
   return launch_mass<64>(a, q, k, prm, ctas, stream);

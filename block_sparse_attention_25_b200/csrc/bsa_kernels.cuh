@@ -181,6 +181,12 @@ cudaError_t launch_topp_select_noalloc(const float* mass, long long rows, int n_
 
 // Block-sparse forward.  Scratch after the status header: per-CTA schedule.
 size_t fwd_scratch_bytes(const AttnDims& a);
+// The bf16 D = 128 tile-major forward on CTA pairs (attn_fwd_pair.cu), over the schedule
+// of bsattn_schedule_kernel: `groups` lists of 256 query slots each.
+cudaError_t launch_bsattn_fwd_pair(const AttnDims& a, const void* q, const void* k, const void* v,
+                                   const int32_t* counts, const uint32_t* entries,
+                                   float softmax_scale, void* out, float* lse, uint32_t* status,
+                                   long long groups, cudaStream_t stream);
 cudaError_t launch_bsattn_fwd(const AttnDims& a, int fp8, const void* q, const void* k,
                               const void* v, const float* q_scales, const float* k_scales,
                               const float* v_scales, const int32_t* row_ptr,
@@ -188,11 +194,48 @@ cudaError_t launch_bsattn_fwd(const AttnDims& a, int fp8, const void* q, const v
                               void* ws, cudaStream_t stream);
 
 // Dense calibration pass.
-// Per-SM scratch of the calibration kernels: kMassSlots slices (one per SM id, comfortably
-// above the SM ids of sm_100 parts) of 256 rows x n_kb fp32 row-block sums.  A CTA on an SM
-// id beyond them records DETAIL_MASS_SLICE and writes no masses.
+// Scratch of the calibration kernels: kMassSlots slices of 256 rows x n_kb fp32 row-block
+// sums after a 256-byte pool bitmap (one bit per slice, cleared by the launcher).  A CTA
+// claims a free slice when it starts and frees it when it ends, so live CTAs never share a
+// slice; with one CTA per SM (their shared memory admits no second) and more slices than
+// SMs, a claim always finds a free slice.
 constexpr int kMassSlots = 192;
+constexpr size_t kMassPoolBytes = 256;
+
+// Claim a free slice (bit of `pool`), or -1 after kWaitLimitNs without one (TIMEOUT recorded).
+__device__ __forceinline__ int claim_mass_slice(uint32_t* pool, uint32_t* status) {
+  constexpr int kWords = kMassSlots / 32;
+  const int w0 = static_cast<int>(blockIdx.x % kWords);
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    for (int i = 0; i < kWords; ++i) {
+      const int w = (w0 + i) % kWords;
+      uint32_t v = *reinterpret_cast<volatile uint32_t*>(pool + w);
+      while (v != 0xffffffffu) {
+        const int b = __ffs(~v) - 1;
+        const uint32_t old = atomicOr(pool + w, 1u << b);
+        if (!(old & (1u << b))) {
+          __threadfence();  // the previous holder's accesses come before ours
+          return w * 32 + b;
+        }
+        v = old | (1u << b);
+      }
+    }
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_status(status, FLAG_TIMEOUT, DETAIL_MASS_SLICE, blockIdx.x, 0u);
+      return -1;
+    }
+  }
+}
+
+__device__ __forceinline__ void release_mass_slice(uint32_t* pool, int slice) {
+  if (slice < 0) return;
+  __threadfence();  // this CTA's accesses to the slice come before the next holder's
+  atomicAnd(pool + (slice >> 5), ~(1u << (slice & 31)));
+}
+
 size_t mass_scratch_bytes(const AttnDims& a);
+cudaError_t mass_grid(const AttnDims& a, int* grid);
 cudaError_t launch_block_mass(const AttnDims& a, const void* q, const void* k, float softmax_scale,
                               float* mass, void* ws, cudaStream_t stream);
 

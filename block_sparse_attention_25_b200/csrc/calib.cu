@@ -7,7 +7,7 @@
 // pass for the output; here one walk over the kv blocks does both:
 //   S = Q K^T, P = exp2(S*c - m_r) with m_r a lazy reference max (raised only when a step's
 //   max exceeds it by more than kRescaleLog2), every probability computed once: stored to
-//   TMEM as bf16 for O += P V, summed per kv block into this SM's workspace slice, and into
+//   TMEM as bf16 for O += P V, summed per kv block into the CTA's workspace slice, and into
 //   the row sum l_r.  When m_r is raised -- rare -- the row's O, its sum and the block sums
 //   it has already written are multiplied by exp2(m_old - m_new);
 //   end: O / l_r, and mass[i,j] = (1 / valid queries of i) * sum over the rows of query
@@ -43,6 +43,7 @@ struct CalibParams {
   float* mass;
   uint32_t* status;
   float* scratch;  // [kMassSlots][n_kb][256] unnormalised row-block sums
+  uint32_t* pool;  // kMassSlots bits: slices held by live CTAs
   float scale_log2;
 };
 
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* nvalid_sm = reinterpret_cast<int*>(tmem_slot + 2);  // [2 tile][4 warp]
+  int* slice_sm = reinterpret_cast<int*>(tmem_slot + 12);  // this CTA's scratch slice
   float* inv_l_sm = reinterpret_cast<float*>(smem + L::kRedOff);
 
   const AttnDims& a = p.a;
@@ -113,6 +115,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
     mbar_init(bar_ofull, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
+    *slice_sm = claim_mass_slice(p.pool, p.status);
     fence_mbar_init();
   }
   if (warp == 9) tmem_alloc(tmem_slot, 512);
@@ -257,13 +260,11 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
     const int wcount = __popc(__ballot_sync(0xffffffffu, q_valid));
     if (lane == 0) nvalid_sm[t * 4 + wq] = wcount;
     named_bar_sync(1 + t, 128);
-    // this SM's workspace slice: [n_kb][256] row-block sums
-    uint32_t smid;
-    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-    const bool have_slice = smid < static_cast<uint32_t>(kMassSlots);
-    if (!have_slice && local == 0)
-      record_status(p.status, FLAG_DEVICE_INPUT, DETAIL_MASS_SLICE, static_cast<uint32_t>(cta), smid);
-    float* sc = p.scratch + static_cast<size_t>(have_slice ? smid : 0u) * 256 * a.n_kb;
+    // this CTA's scratch slice: [n_kb][256] row-block sums (none: the claim timed out, no
+    // masses are written and the status header says so)
+    const int slice = *slice_sm;
+    const bool have_slice = slice >= 0;
+    float* sc = p.scratch + static_cast<size_t>(have_slice ? slice : 0) * 256 * a.n_kb;
 
     float m_ref = -INFINITY, l_run = 0.f;  // reference max (log2 units) and sum against it
     bool ok = true;
@@ -441,6 +442,7 @@ __global__ void __launch_bounds__(calib::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (threadIdx.x == 0) release_mass_slice(p.pool, *slice_sm);
 }
 
 template <int D>
@@ -463,12 +465,15 @@ static cudaError_t launch_calib(const AttnDims& a, const void* q, const void* k,
   e = cudaFuncSetAttribute(calib_dense_mass_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            L::kAlloc);
   if (e != cudaSuccess) return e;
-  // the workspace slices are per SM id: at most one CTA of this kernel may live on an SM
+  // one CTA per SM, so the live CTAs (at most the SM count) never exhaust the kMassSlots
+  // slices and no claim waits
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, calib_dense_mass_kernel<D>,
                                                     calib::kThreads, L::kAlloc);
   if (e != cudaSuccess) return e;
   if (per_sm != 1) return cudaErrorInvalidConfiguration;
+  e = cudaMemsetAsync(prm.pool, 0, kMassPoolBytes, stream);
+  if (e != cudaSuccess) return e;
   calib_dense_mass_kernel<D><<<static_cast<unsigned>(ctas), calib::kThreads, L::kAlloc, stream>>>(
       tq, tk, tv, prm);
   return cudaGetLastError();
@@ -485,7 +490,8 @@ cudaError_t launch_calib_dense_mass(const AttnDims& a, const void* q, const void
   prm.lse = lse;
   prm.mass = mass;
   prm.status = static_cast<uint32_t*>(ws);
-  prm.scratch = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+  prm.pool = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+  prm.scratch = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kStatusBytes + kMassPoolBytes);
   prm.scale_log2 = softmax_scale * 1.4426950408889634f;
   if (a.head_dim == 128) return launch_calib<128>(a, q, k, v, prm, ctas, stream);
   return launch_calib<64>(a, q, k, v, prm, ctas, stream);

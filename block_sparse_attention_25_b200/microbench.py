@@ -48,6 +48,50 @@ def _time(fn, iters: int) -> float:
     return sorted(ms)[len(ms) // 2]
 
 
+def schedule_work(row_ptr: torch.Tensor, col_idx: torch.Tensor, s) -> dict:
+    """The attention work the forward's schedule performs for given lists, in (64-key kv
+    block x query block) pair units: `kept` = the lists' entries; `computed` = what the
+    kernel multiplies -- a CTA owns 256 query slots in two 128-row tiles and walks the union
+    of its query blocks' lists two kv blocks per step, ordered by which tiles need a block
+    (both, tile 0 only, tile 1 only); a tile skips the steps none of its query blocks keeps,
+    and computes every block of the steps it takes part in; `cta_union` = the work of
+    walking the whole union with both tiles (the schedule without per-tile skipping)."""
+    dev = row_ptr.device
+    R, n_kb, n_qb = s.rows, s.n_kb, s.n_qb
+    nq = 256 // s.q_block                      # query blocks per CTA
+    tq = nq // 2                               # per tile
+    rp = row_ptr.long()
+    nnz = int(rp[-1])
+    rows = torch.repeat_interleave(torch.arange(R, device=dev), rp[1:] - rp[:-1])
+    keep = torch.zeros(R, n_kb, dtype=torch.bool, device=dev)
+    keep[rows, col_idx[:nnz].long()] = True
+    bh = s.batch * s.heads
+    n_cta = -(-n_qb // nq)
+    kp = torch.zeros(bh, n_cta * nq, n_kb, dtype=torch.bool, device=dev)
+    kp[:, :n_qb] = keep.view(bh, n_qb, n_kb)
+    kp = kp.view(bh, n_cta, nq, n_kb)
+    need0, need1 = kp[:, :, :tq].any(2), kp[:, :, tq:].any(2)
+    nb = (need0 & need1).sum(-1)
+    n0 = (need0 & ~need1).sum(-1)
+    n1 = (~need0 & need1).sum(-1)
+    N = nb + n0 + n1
+    s_end = (N + 1) // 2
+
+    def blocks(x, y):  # kv blocks in steps [x, y): two per step, one in an odd union's last
+        n = (y - x).clamp(min=0)
+        return 2 * n - ((N % 2 == 1) & (y == s_end) & (n > 0)).long()
+    b0 = blocks(torch.zeros_like(N), (nb + n0 + 1) // 2)
+    a_end, b_start = (nb + 1) // 2, (nb + n0) // 2
+    b1 = torch.where(n1 == 0, blocks(torch.zeros_like(N), a_end),
+                     torch.where(b_start <= a_end, blocks(torch.zeros_like(N), s_end),
+                                 blocks(torch.zeros_like(N), a_end) + blocks(b_start, s_end)))
+    computed = int((b0 + b1).sum()) * tq
+    union = int(N.sum()) * nq
+    return {"kept_pairs": nnz, "computed_pairs": computed, "cta_union_pairs": union,
+            "computed_over_kept": round(computed / max(nnz, 1), 4),
+            "cta_union_over_kept": round(union / max(nnz, 1), 4)}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--config", default="wan14b_720p")
@@ -56,12 +100,18 @@ def main(argv=None):
     ap.add_argument("--q-clusters", type=int, default=64, help="k-means clusters of the queries")
     ap.add_argument("--k-clusters", type=int, default=256, help="k-means clusters of the keys")
     ap.add_argument("--rounds", type=int, default=10, help="k-means rounds")
-    ap.add_argument("--only", choices=["all", "tiles", "semantic"], default="all",
-                    help="the 3D-tile path, the semantic-aware permutation path, or both")
+    ap.add_argument("--only", choices=["all", "tiles", "semantic", "fwd", "calib"], default="all",
+                    help="the 3D-tile path, the semantic-aware permutation path, or both; fwd: "
+                         "only the calibration's lists and the forward calls; calib: only "
+                         "block_mass and dense_fwd_mass (small profiling cases)")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the workload's head count (profiling on a smaller case)")
     args = ap.parse_args(argv)
     build.build()
     dev = torch.device("cuda")
     wl = synth.WORKLOADS[args.config]
+    if args.heads is not None:
+        wl = wl.scaled(heads=args.heads, name=f"{wl.name}-h{args.heads}")
     s = B.Shape.of(wl)
     pk = _peaks()
     q, k, v = synth.draw_qkv(wl, device=dev)
@@ -82,6 +132,8 @@ def main(argv=None):
         semantic(args, wl, q, k, v, line, pk)
         return
     qt, kt, vt = (B.tile_permute(x, s) for x in (q, k, v))
+    if args.only in ("fwd", "calib"):
+        return focused(args, wl, s, q, k, v, qt, kt, vt, line, pk)
     out_r = torch.empty_like(q)
     line("tile_permute", _time(lambda: B.tile_permute(q, s, out=qt), args.iters),
          S * Hh * D * e + Np * Hh * D * e, "GB/s", "hbm", pk["hbm"])
@@ -141,9 +193,10 @@ def main(argv=None):
     ws_f = B.new_workspace(s, B.OP_FWD, dev)
     out_t = torch.empty_like(qt)
     fl = 4.0 * nnz * s.q_block * 64 * D
+    work = schedule_work(row_ptr, col_idx, s)
     line("bsattn_fwd", _time(lambda: B.bsattn_fwd(qt, kt, vt, row_ptr, col_idx, s, out=out_t, ws=ws_f),
                              args.iters), fl, "TFLOP/s", "tensor", pk["bf16"],
-         {"kept_fraction": round(nnz / (R * nkb), 5)})
+         {"kept_fraction": round(nnz / (R * nkb), 5), **work})
     # the permutation fused into the forward: raster in, raster out
     out_r = torch.empty_like(q)
     line("bsattn_fwd_raster",
@@ -176,7 +229,7 @@ def main(argv=None):
     pfl = 4.0 * pnnz * s.q_block * 64 * D
     line("bsattn_fwd_pattern", _time(lambda: B.bsattn_fwd(qt, kt, vt, prp, pci, s, out=out_t, ws=ws_f),
                                      args.iters), pfl, "TFLOP/s", "tensor", pk["bf16"],
-         {"kept_fraction": round(pnnz / (R * nkb), 5)})
+         {"kept_fraction": round(pnnz / (R * nkb), 5), **schedule_work(prp, pci, s)})
     for w in (ws_m, ws_t, ws_p, ws_pt, ws_f):
         st = B.device_status(w)
         if st != 0:
@@ -185,6 +238,47 @@ def main(argv=None):
     torch.cuda.empty_cache()
     if args.only == "all":
         semantic(args, wl, q, k, v, line, pk)
+
+
+def focused(args, wl, s, q, k, v, qt, kt, vt, line, pk):
+    """--only fwd: the calibration's lists (untimed), then the tile-major forward (bf16 and,
+    for D = 128, e4m3); --only calib: block_mass and dense_fwd_mass.  Small launch counts
+    for profiler captures."""
+    dev = qt.device
+    D, Hh, R, nkb = s.head_dim, s.heads, s.rows, s.n_kb
+    ws_m = B.new_workspace(s, B.OP_BLOCK_MASS, dev)
+    mass = B.block_mass(qt, kt, s, ws=ws_m)
+    if args.only == "calib":
+        qk_pass = 2.0 * s.batch * s.Np * s.Np * D * Hh
+        line("block_mass", _time(lambda: B.block_mass(qt, kt, s, out=mass, ws=ws_m), args.iters),
+             qk_pass, "TFLOP/s", "tensor", pk["bf16"])
+        out_t, m2 = torch.empty_like(qt), torch.empty_like(mass)
+        line("dense_fwd_mass",
+             _time(lambda: B.dense_fwd_mass(qt, kt, vt, s, out=out_t, mass=m2, ws=ws_m), args.iters),
+             2 * qk_pass, "TFLOP/s", "tensor", pk["bf16"])
+    else:
+        rp, ci = B.topp_select(mass, s, args.tau)
+        nnz = int(rp[-1])
+        fl = 4.0 * nnz * s.q_block * 64 * D
+        ws_f = B.new_workspace(s, B.OP_FWD, dev)
+        out_t = torch.empty_like(qt)
+        line("bsattn_fwd", _time(lambda: B.bsattn_fwd(qt, kt, vt, rp, ci, s, out=out_t, ws=ws_f),
+                                 args.iters), fl, "TFLOP/s", "tensor", pk["bf16"],
+             {"kept_fraction": round(nnz / (R * nkb), 5), **schedule_work(rp, ci, s)})
+        if D == 128:
+            q8 = [torch.empty(qt.shape, dtype=torch.uint8, device=dev) for _ in range(3)]
+            sc = [torch.empty((s.batch, Hh, s.Np // 64), dtype=torch.float32, device=dev)
+                  for _ in range(3)]
+            for x, o, c in zip((q, k, v), q8, sc):
+                B.tile_permute_quant_e4m3(x, s, out=o, scales=c)
+            line("bsattn_fwd_e4m3",
+                 _time(lambda: B.bsattn_fwd(q8[0], q8[1], q8[2], rp, ci, s, scales=sc, out=out_t,
+                                            ws=ws_f), args.iters),
+                 fl, "TFLOP/s", "tensor", 2 * pk["bf16"], {"kept_fraction": round(nnz / (R * nkb), 5)})
+        ws_m = ws_f
+    st = B.device_status(ws_m)
+    if st != 0:
+        raise RuntimeError(f"device status {st}: {B.device_status_words(ws_m)}")
 
 
 def semantic(args, wl, q, k, v, line, pk):

@@ -16,6 +16,13 @@ Recipe (a reading of the workload descriptions; the pages fix no data):
 * A re-draw r of a workload (the later denoising steps of the calibrate-then-reuse
   cycle) is X_r = rho * X + sqrt(1 - rho^2) * X'_r with rho = 0.95, where X'_r is an
   independent draw of the same recipe from the stream seed 1000 * seed + r.
+* The "local" generator (an auxiliary workload, not one of the five): Q and K are
+  LOCAL_GAIN * (RFF + LOCAL_NOISE * N(0, 1)) with the per-head frequency drawn from
+  U(LOCAL_FREQ) -- smooth features with little noise, so attention concentrates on a
+  spatial neighbourhood spanning several tiles and the retained-mass lists are really
+  sparse (about 60% of the kv blocks kept at 0.99, between ~45% and ~85% per head); V
+  follows the standard recipe.  With the standard recipe the N(0, 1) term dominates q.k
+  and every block's mass is close to uniform, whatever the scale.
 
 The draws use torch's seeded generator on the requested device (MT19937 on the CPU,
 Philox on CUDA), so the same seed gives different numbers on different devices;
@@ -62,6 +69,7 @@ class Workload:
     taus: tuple = (0.99,)
     redraws: int = 0
     fp8: bool = False
+    generator: str = "rff"           # "rff" (the recipe above) or "local"
     extra: dict = field(default_factory=dict, compare=False, hash=False)
 
     @property
@@ -94,6 +102,11 @@ class Workload:
 
 _INV_SQRT128 = 1.0 / math.sqrt(128.0)
 
+# The "local" generator of Q and K (see the module docstring).
+LOCAL_FREQ = (0.05, 0.3)
+LOCAL_NOISE = 0.1
+LOCAL_GAIN = 10.0
+
 # The five workloads: a tiny case the oracle finishes in seconds, then three
 # video-DiT-shaped long sequences and the FP8 variant of the 720p one.
 WORKLOADS = {
@@ -107,6 +120,10 @@ WORKLOADS = {
                              128, 64, seed=3, value_scale=_INV_SQRT128, taus=(0.90, 0.95, 0.99)),
     "wan14b_720p_fp8": Workload("wan14b-720p-fp8-e4m3", 1, 40, 128, 21, 45, 80, 24, 48, 80,
                                 64, 64, seed=2, value_scale=_INV_SQRT128, fp8=True),
+    # auxiliary: the 720p shape with spatially local attention (about 60% kept at 0.99)
+    "wan14b_720p_local": Workload("wan14b-720p-local-21x45x80-h40-d128", 1, 40, 128, 21, 45, 80,
+                                  24, 48, 80, 64, 64, seed=2, value_scale=1.0,
+                                  generator="local"),
 }
 
 
@@ -142,10 +159,12 @@ def _draw_fp32(wl: Workload, seed: int, device, sharpness: float = 1.0):
     pos = _positions(wl, device)
     out = []
     maps = []
-    for _ in range(2):  # map 0 shared by Q and K, map 1 for V
+    local = wl.generator == "local"
+    for m in range(2):  # map 0 shared by Q and K, map 1 for V
         omega = torch.randn(3, D, generator=g, device=device)
         phase = torch.rand(D, generator=g, device=device) * (2.0 * math.pi)
-        freq = 0.5 + 3.5 * torch.rand(Hh, generator=g, device=device)
+        lo, hi = LOCAL_FREQ if (local and m == 0) else (0.5, 4.0)
+        freq = lo + (hi - lo) * torch.rand(Hh, generator=g, device=device)
         maps.append((omega, phase, freq))
     for which in ("q", "k", "v"):
         omega, phase, freq = maps[1 if which == "v" else 0]
@@ -153,8 +172,11 @@ def _draw_fp32(wl: Workload, seed: int, device, sharpness: float = 1.0):
         for _b in range(wl.batch):
             rff = _rff(pos, omega, phase, freq)
             noise = torch.randn(rff.shape, generator=g, device=device)
-            xs.append(0.7 * rff + 0.3 * noise)
-        x = torch.stack(xs, 0) * wl.value_scale
+            if local and which != "v":
+                xs.append(LOCAL_GAIN * (rff + LOCAL_NOISE * noise))
+            else:
+                xs.append((0.7 * rff + 0.3 * noise) * wl.value_scale)
+        x = torch.stack(xs, 0)
         if which != "v" and sharpness != 1.0:
             x = x * sharpness
         out.append(x)

@@ -96,3 +96,46 @@ def test_dense_fwd_mass_matches_separate_calls(B):
     ci = torch.arange(n_kb, dtype=torch.int32).repeat(R).cuda()
     o2 = B.bsattn_fwd(qt, kt, vt, rp, ci, s)
     assert float((out.float() - o2.float()).abs().max()) <= 1e-2
+
+
+# More than twice as many CTAs (head, 256 query slots) as the GPU has SMs, so the
+# calibration kernels' workspace slices are claimed, given back and claimed again by later
+# CTAs; ragged pads keep partial last CTAs in every head.
+MANY = [
+    Hp.synth.Workload("many-heads-6x10x11-h64-d128-bq64", 1, 64, 128, 6, 10, 11, 8, 12, 12, 64, 64,
+                      seed=21),
+    Hp.synth.Workload("many-heads-5x7x9-b2-h80-d64-bq128", 2, 80, 64, 5, 7, 9, 8, 8, 12, 128, 64,
+                      seed=22),
+]
+
+
+@pytest.mark.parametrize("wl", MANY, ids=[w.name for w in MANY])
+def test_calibration_reuses_workspace_slices(B, wl):
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    items = wl.batch * wl.heads * ((wl.Np + 255) // 256)
+    assert items > 2 * sms
+    g = Hp.grid_of(wl)
+    s = B.Shape.of(wl)
+    q, k, v = Hp.draw(wl, value_scale=1.0, sharp=4.0)
+    qt, kt, vt = (B.tile_permute(x.cuda(), s) for x in (q, k, v))
+    qo, ko, vo = (Hp.oracle_tiled(x, g) for x in (q, k, v))
+    m_ref = O.block_mass(qo, ko, g, wl.q_block, 64, Hp.scale_of(wl))
+    ws = B.new_workspace(s, B.OP_BLOCK_MASS)
+    m = B.block_mass(qt, kt, s, ws=ws)
+    assert B.device_status(ws) == 0, B.device_status_words(ws)
+    got = m.cpu().double().numpy()
+    assert np.abs(got - m_ref).max() <= Hp.MASS_ABS
+    nz = m_ref > 1e-6
+    assert (np.abs(got - m_ref)[nz] / m_ref[nz]).max() < 1e-3
+    assert np.all(got[m_ref == 0] == 0)
+    out, mass, lse = B.dense_fwd_mass(qt, kt, vt, s, want_lse=True, ws=ws)
+    assert B.device_status(ws) == 0, B.device_status_words(ws)
+    assert float((mass - m).abs().max()) <= 1e-6
+    n_qb, n_kb = wl.Np // wl.q_block, wl.Np // 64
+    R = wl.batch * wl.heads * n_qb
+    o_ref, lse_ref = O.masked_attention(qo, ko, vo, g, wl.q_block, 64, np.arange(R + 1) * n_kb,
+                                        np.tile(np.arange(n_kb), R), Hp.scale_of(wl))
+    Hp.assert_attn_close(out.cpu().double().numpy(), o_ref, signal_guard=False)
+    fin = np.isfinite(lse_ref)
+    assert np.abs(lse.cpu().double().numpy()[fin] - lse_ref[fin]).max() <= 1e-3

@@ -1,8 +1,9 @@
 """The bench's multi-GPU plumbing on CPU: two gloo ranks, no GPU.
 
-The path shards with no exchange step (each GPU runs an independent problem), so the
-process group only carries the start/stop barrier and the max-over-ranks reduction of
-the timed region.  These tests run that plumbing as two processes on the host.
+The path shards with no exchange step -- each GPU runs an independent problem, or owns a
+share of one problem's heads -- so the process group only carries the start/stop barrier,
+the max-over-ranks reduction of the timed region and the sum of the ranks' executed work.
+These tests run that plumbing as two processes on the host.
 """
 import os
 import socket
@@ -36,6 +37,13 @@ def _worker(rank, world, port, out):
     wl = synth.WORKLOADS["tiny"]
     q, _, _ = synth.draw_qkv(wl.scaled(seed=wl.seed + 7919 * rank))
     out[world + rank] = float(q.double().sum())
+    # --split heads: every rank draws the one problem and keeps its heads; the shares
+    # cover the heads once, and the executed work adds up over the ranks
+    h0, h1 = bench.head_range(rank, world, wl.heads)
+    qf, _, _ = synth.draw_qkv(wl)
+    mine = qf[:, :, h0:h1].contiguous()
+    out[2 * world + rank] = float(mine.double().sum())
+    out[3 * world + rank] = bench.sum_over_ranks(float(h1 - h0), pg)
     bench.barrier(pg)
     pg.destroy_process_group()
 
@@ -43,7 +51,7 @@ def _worker(rank, world, port, out):
 def test_two_gloo_ranks_reduce_max_and_draw_independent_problems():
     world = 2
     ctx = mp.get_context("spawn")
-    out = ctx.Array("d", 2 * world)
+    out = ctx.Array("d", 4 * world)
     port = _free_port()
     procs = [ctx.Process(target=_worker, args=(r, world, port, out)) for r in range(world)]
     for p in procs:
@@ -53,6 +61,26 @@ def test_two_gloo_ranks_reduce_max_and_draw_independent_problems():
         assert p.exitcode == 0
     assert list(out[:world]) == [1.5 + world - 1] * world
     assert out[world] != out[world + 1]
+    # the head shares of one problem add up to the whole problem
+    from block_sparse_attention_25_b200 import synth
+    wl = synth.WORKLOADS["tiny"]
+    qf, _, _ = synth.draw_qkv(wl)
+    assert abs(out[2 * world] + out[2 * world + 1] - float(qf.double().sum())) < 1e-9
+    assert list(out[3 * world:]) == [float(wl.heads)] * world
+
+
+def test_head_ranges_partition_the_heads():
+    sys.path.insert(0, ROOT)
+    import bench
+    for heads, world in ((40, 1), (40, 2), (40, 4), (40, 8), (24, 8), (12, 4)):
+        seen = []
+        for r in range(world):
+            h0, h1 = bench.head_range(r, world, heads)
+            assert h1 - h0 == heads // world
+            seen += list(range(h0, h1))
+        assert seen == list(range(heads))
+    with pytest.raises(ValueError):
+        bench.head_range(0, 3, 40)
 
 
 def test_single_rank_needs_no_process_group(monkeypatch):
