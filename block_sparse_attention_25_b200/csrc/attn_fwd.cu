@@ -794,9 +794,7 @@ cudaError_t launch_bsattn_fwd(const AttnDims& a, int fp8, const void* q, const v
   prm.raster_b = 0;
   prm.cta_offset = 0;
   if (fp8) return launch_fwd<128, true, false>(a, a.g.Np, q, k, v, prm, ctas, stream);
-  if (a.head_dim == 128)  // one 128-row tile per SM of a CTA pair
-    return launch_bsattn_fwd_pair(a, q, k, v, counts, entries, softmax_scale, out, lse, status,
-                                  ctas, stream);
+  if (a.head_dim == 128) return launch_fwd<128, false, false>(a, a.g.Np, q, k, v, prm, ctas, stream);
   return launch_fwd<64, false, false>(a, a.g.Np, q, k, v, prm, ctas, stream);
 }
 

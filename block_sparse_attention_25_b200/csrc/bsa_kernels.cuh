@@ -181,12 +181,7 @@ cudaError_t launch_topp_select_noalloc(const float* mass, long long rows, int n_
 
 // Block-sparse forward.  Scratch after the status header: per-CTA schedule.
 size_t fwd_scratch_bytes(const AttnDims& a);
-// The bf16 D = 128 tile-major forward on CTA pairs (attn_fwd_pair.cu), over the schedule
-// of bsattn_schedule_kernel: `groups` lists of 256 query slots each.
-cudaError_t launch_bsattn_fwd_pair(const AttnDims& a, const void* q, const void* k, const void* v,
-                                   const int32_t* counts, const uint32_t* entries,
-                                   float softmax_scale, void* out, float* lse, uint32_t* status,
-                                   long long groups, cudaStream_t stream);
+
 cudaError_t launch_bsattn_fwd(const AttnDims& a, int fp8, const void* q, const void* k,
                               const void* v, const float* q_scales, const float* k_scales,
                               const float* v_scales, const int32_t* row_ptr,
@@ -298,6 +293,7 @@ cudaError_t kernel_binary_version(int* version);
 // and 128-byte swizzle.
 cudaError_t encode_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                            int elem_bytes, int D, int Np, int bh, int box_d, int box_rows);
+
 // Same with explicit extents (innermost first), byte strides of dims 1 and 2, and box.
 cudaError_t encode_tmap_3d_strided(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                                    const unsigned long long dims[3],
