@@ -51,15 +51,13 @@ def _time(fn, iters: int) -> float:
 def schedule_work(row_ptr: torch.Tensor, col_idx: torch.Tensor, s) -> dict:
     """The attention work the forward's schedule performs for given lists, in (64-key kv
     block x query block) pair units: `kept` = the lists' entries; `computed` = what the
-    kernel multiplies -- a CTA owns 256 query slots in two 128-row tiles and walks the union
-    of its query blocks' lists two kv blocks per step, ordered by which tiles need a block
-    (both, tile 0 only, tile 1 only); a tile skips the steps none of its query blocks keeps,
-    and computes every block of the steps it takes part in; `cta_union` = the work of
-    walking the whole union with both tiles (the schedule without per-tile skipping)."""
+    kernel multiplies -- a CTA owns 256 query slots (2 or 4 query blocks in two 128-row
+    tiles) and walks the ascending union of its query blocks' lists with both tiles, masking
+    for each query block the kv blocks it did not keep, so every query block of the CTA
+    pays for every kv block of the union."""
     dev = row_ptr.device
     R, n_kb, n_qb = s.rows, s.n_kb, s.n_qb
     nq = 256 // s.q_block                      # query blocks per CTA
-    tq = nq // 2                               # per tile
     rp = row_ptr.long()
     nnz = int(rp[-1])
     rows = torch.repeat_interleave(torch.arange(R, device=dev), rp[1:] - rp[:-1])
@@ -69,27 +67,10 @@ def schedule_work(row_ptr: torch.Tensor, col_idx: torch.Tensor, s) -> dict:
     n_cta = -(-n_qb // nq)
     kp = torch.zeros(bh, n_cta * nq, n_kb, dtype=torch.bool, device=dev)
     kp[:, :n_qb] = keep.view(bh, n_qb, n_kb)
-    kp = kp.view(bh, n_cta, nq, n_kb)
-    need0, need1 = kp[:, :, :tq].any(2), kp[:, :, tq:].any(2)
-    nb = (need0 & need1).sum(-1)
-    n0 = (need0 & ~need1).sum(-1)
-    n1 = (~need0 & need1).sum(-1)
-    N = nb + n0 + n1
-    s_end = (N + 1) // 2
-
-    def blocks(x, y):  # kv blocks in steps [x, y): two per step, one in an odd union's last
-        n = (y - x).clamp(min=0)
-        return 2 * n - ((N % 2 == 1) & (y == s_end) & (n > 0)).long()
-    b0 = blocks(torch.zeros_like(N), (nb + n0 + 1) // 2)
-    a_end, b_start = (nb + 1) // 2, (nb + n0) // 2
-    b1 = torch.where(n1 == 0, blocks(torch.zeros_like(N), a_end),
-                     torch.where(b_start <= a_end, blocks(torch.zeros_like(N), s_end),
-                                 blocks(torch.zeros_like(N), a_end) + blocks(b_start, s_end)))
-    computed = int((b0 + b1).sum()) * tq
-    union = int(N.sum()) * nq
-    return {"kept_pairs": nnz, "computed_pairs": computed, "cta_union_pairs": union,
-            "computed_over_kept": round(computed / max(nnz, 1), 4),
-            "cta_union_over_kept": round(union / max(nnz, 1), 4)}
+    union = kp.view(bh, n_cta, nq, n_kb).any(2).sum(-1)   # kv blocks each CTA walks
+    computed = int(union.sum()) * nq
+    return {"kept_pairs": nnz, "computed_pairs": computed,
+            "computed_over_kept": round(computed / max(nnz, 1), 4)}
 
 
 def main(argv=None):
