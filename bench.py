@@ -91,11 +91,10 @@ def head_range(rank: int, world: int, heads: int):
 
 
 def measured_traffic(fp8: bool, raster: bool):
-    """DRAM bytes per forward launch from the committed full-size ncu capture of the variant
-    the bench times, or None when the kernel sources have changed since it was taken (or for
-    a variant not captured)."""
-    if fp8:
-        return None
+    """DRAM bytes per forward launch of the variant the bench times, from the committed ncu
+    summary (bf16: the recorded full-size capture; e4m3: the 8-head capture scaled to 40
+    heads; raster: the recorded full-size capture), or None when the kernel sources have
+    changed since it was taken."""
     import hashlib
     import re
     name = "bsattn_fwd_raster_wan14b_720p_dram.md" if raster else "bsattn_fwd_wan14b_720p_dram.md"
@@ -103,7 +102,8 @@ def measured_traffic(fp8: bool, raster: bool):
     if not os.path.exists(path):
         return None
     text = open(path).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
+    key = "traffic_bytes_per_launch_e4m3" if fp8 else "traffic_bytes_per_launch"
+    m = re.search(key + r":\s*(\d+)", text)
     if not m:
         return None
     csrc = os.path.join(ROOT, "block_sparse_attention_25_b200", "csrc")
@@ -375,7 +375,7 @@ def run_ours(args, world, rank, local, pg):
     result = {
         "metric": "bsattn_fwd ms/call & executed TFLOPS at 99% retained mass, % of bf16 peak",
         "value": round(value, 2),
-        "unit": "TFLOP/s (executed, kept blocks; step rate: calibration + 10 reuse calls)",
+        "unit": f"TFLOP/s (executed, kept blocks; step rate: calibration + {n_reuse} reuse calls)",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
@@ -416,8 +416,11 @@ def run_ours(args, world, rank, local, pg):
             "bound": "tensor", "achieved": round(fwd_tflops, 2), "peak": peak, "unit": "TFLOP/s",
             "frac": round(fwd_tflops / peak, 4),
             "traffic": (measured_traffic(fp8, raster)
-                        if wl.name == synth.WORKLOADS["wan14b_720p"].name else None),
-            "traffic_unit": "bytes per launch (dram read + write, one full-size ncu capture)",
+                        if wl.name in (synth.WORKLOADS["wan14b_720p"].name,
+                                       synth.WORKLOADS["wan14b_720p_fp8"].name) else None),
+            "traffic_unit": ("bytes per launch (dram read + write; an 8-head ncu capture x 5)"
+                             if fp8 else
+                             "bytes per launch (dram read + write, one full-size ncu capture)"),
             "kernel": (f"bsattn_fwd_kernel<{s.head_dim},false,false,true> (raster layout)" if raster
                        else f"bsattn_fwd_kernel<{s.head_dim},{'true' if fp8 else 'false'},false,false>"),
             "peak_source": peak_note,
@@ -594,7 +597,7 @@ def oracle_sample(wl, n_rows: int, seed: int = 0):
     q, k, v = synth.draw_qkv(small, device="cpu")
     qt, kt, vt = (O.permute_forward(x.to(torch.float64).numpy(), g) for x in (q, k, v))
     n_qb, n_kb = wl.Np // wl.q_block, wl.Np // 64
-    rp, ci = synth.draw_keep_csr(heads * n_qb, n_kb, 0.957, seed=seed)
+    rp, ci = synth.draw_keep_csr(heads * n_qb, n_kb, wl.nominal_kept, seed=seed)
     rp, ci = rp.numpy(), ci.numpy()
     valid = O.valid_slots(g)
     rng = np.random.default_rng(seed)
@@ -612,7 +615,7 @@ def oracle_sample(wl, n_rows: int, seed: int = 0):
             flops += 4.0 * wl.head_dim * nk
         dt = time.perf_counter() - t
     desc = (f"oracle masked attention (numpy fp64, 1 thread) on {n_rows} sampled query rows of "
-            f"{wl.name} with a seeded CSR at 0.957 kept; TFLOP/s = executed FLOPs of those rows / time")
+            f"{wl.name} with a seeded CSR at {wl.nominal_kept} kept; TFLOP/s = executed FLOPs of those rows / time")
     return flops, dt, desc
 
 
