@@ -7,9 +7,9 @@
 //
 // Per row the masses become integers q = rint(m * 2^40) and the target is
 // ceil(tau * sum q) (one fp64 multiply).  The shortest prefix of the (q desc, index asc)
-// order that reaches the target is found without sorting: an exact radix select over the
-// row's value range (256 bins per level, per-bin sums in shared memory) finds the value t*
-// of the last kept element and the sum A of everything above it; all blocks with q > t*
+// order that reaches the target is found without sorting: an exact quickselect over the
+// row's values (64-bit integer sums reduced over a warp) finds the value t* of the last
+// kept element and the sum A of everything above it; all blocks with q > t*
 // are kept, plus the ceil((target - A) / t*) lowest-index blocks with q == t*.  Integer
 // arithmetic makes the result independent of reduction order, so it is bit-identical to
 // a sequential sort-and-scan.
@@ -25,39 +25,32 @@ namespace bsa {
 
 
 // One warp per row, kSelWarps rows per CTA, warp-synchronous (no CTA barriers).
-// Shared memory per warp: the row's fixed-point masses (n_kb uint64) and a 256-bin
-// histogram (counts and remainder sums, 32-bit).
+// Shared memory per warp: the row's fixed-point masses (n_kb uint64) and the candidate
+// list (n_kb uint32 row indices).
 constexpr int kSelWarps = 4;
+constexpr int kBatch = 8;  // elements per lane loaded back to back in each pass over a row
 
 __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
-__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long n = __shfl_xor_sync(0xffffffffu, v, o);
-    v = n > v ? n : v;
-  }
-  return v;
-}
-__device__ __forceinline__ unsigned long long warp_min_u64(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long n = __shfl_xor_sync(0xffffffffu, v, o);
-    v = n < v ? n : v;
-  }
-  return v;
+// Per row: the masses become integers in shared memory, then a quickselect finds the value
+// t* of the last kept element and the sum A of everything above it.  Each round takes a
+// pivot p (median of three candidates), sums the candidates above p and counts those equal
+// to it (exact 64-bit integer sums, reduced over the warp), and either stops (t* = p), or
+// keeps only the candidates above p, or adds everything >= p to A and keeps only those
+// below p.  Every round removes the pivot's value from the candidates, so the loop ends;
+// the candidate list (row indices) is compacted in place, so the work is about four passes
+// over the row whatever its value range.  The final pass walks the row 32 blocks at a time,
+// so a ballot of the keep decisions is one bitmap word, in index order (ties go to the
+// lower index).
+__device__ __forceinline__ unsigned long long median3(unsigned long long a, unsigned long long b,
+                                                      unsigned long long c) {
+  const unsigned long long lo = a < b ? a : b, hi = a < b ? b : a;
+  return c < lo ? lo : (c > hi ? hi : c);
 }
 
-// Radix select over the row's own value range: each level splits the candidate range
-// [lo, hi] into 256 bins of width 2^shift (relative to lo, so similar masses still spread
-// over many bins), sums the masses per bin, and keeps the bin where the running sum from
-// the top crosses the target.  Each lane scans 8 consecutive bins; a warp scan of the
-// lane totals finds the crossing.  The final pass walks the row 32 blocks at a time, so
-// a ballot of the keep decisions is one bitmap word, in index order (ties go to the lower
-// index).
 __global__ void __launch_bounds__(32 * kSelWarps) topp_select_rows_kernel(
     const float* __restrict__ mass, long long rows, int n_kb, double tau,
     int32_t* __restrict__ counts, uint32_t* __restrict__ bitmaps, int words, uint32_t* status) {
@@ -66,127 +59,144 @@ __global__ void __launch_bounds__(32 * kSelWarps) topp_select_rows_kernel(
   const int lane = threadIdx.x & 31;
   const long long r = static_cast<long long>(blockIdx.x) * kSelWarps + warp;
   if (r >= rows) return;
-  unsigned long long* qrow = sel_smem + static_cast<size_t>(warp) * (n_kb + 512);
-  unsigned long long* hist = qrow + n_kb;  // 4 KB: 256 counts + 3 x 256 remainder sums
+  unsigned long long* qrow = sel_smem + static_cast<size_t>(warp) * (n_kb + (n_kb + 1) / 2);
+  uint32_t* cand = reinterpret_cast<uint32_t*>(qrow + n_kb);  // candidate row indices
   const float* row = mass + r * n_kb;
+  const unsigned lt_mask = (1u << lane) - 1u;
 
-  // fixed-point masses into shared memory; sum, max, min
-  unsigned long long sum = 0, mx = 0, mn = ~0ull;
+  // fixed-point masses into shared memory, and their sum.  Each lane issues kBatch loads
+  // before using any of them, so a row costs a few memory round trips, not n_kb / 32.
+  unsigned long long sum = 0;
   bool bad = false;
-  for (int j = lane; j < n_kb; j += 32) {
-    const float m = row[j];
-    unsigned long long q = 0;
-    // valid: finite and 0 <= m <= 4096 (NaN fails both comparisons)
-    if (m >= 0.f && m <= 4096.f)
-      q = static_cast<unsigned long long>(__double2ll_rn(static_cast<double>(m) * 1099511627776.0));
-    else
-      bad = true;
-    qrow[j] = q;
-    sum += q;
-    mx = q > mx ? q : mx;
-    mn = q < mn ? q : mn;
+  for (int j0 = 0; j0 < n_kb; j0 += 32 * kBatch) {
+    float m[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int j = j0 + 32 * u + lane;
+      m[u] = j < n_kb ? __ldcs(row + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int j = j0 + 32 * u + lane;
+      if (j < n_kb) {
+        unsigned long long q = 0;
+        // valid: finite and 0 <= m <= 4096 (NaN fails both comparisons)
+        if (m[u] >= 0.f && m[u] <= 4096.f)
+          q = static_cast<unsigned long long>(
+              __double2ll_rn(static_cast<double>(m[u]) * 1099511627776.0));
+        else
+          bad = true;
+        qrow[j] = q;
+        sum += q;
+      }
+    }
   }
   if (bad) record_status(status, FLAG_DEVICE_INPUT, DETAIL_MASS_VALUE, static_cast<uint32_t>(r), 0u);
   sum = warp_sum_u64(sum);
-  unsigned long long hi = warp_max_u64(mx);
-  unsigned long long lo = warp_min_u64(mn);
   const unsigned long long target =
       static_cast<unsigned long long>(ceil(__dmul_rn(tau, static_cast<double>(sum))));
   __syncwarp();
 
-  // Invariant: elements above hi are all kept, their sum is A < target, and the value of
-  // the last kept element lies in [lo, hi].
-  // Bin sums use only native 32-bit shared atomics: inside a level every candidate is
-  // q = lo + (d << shift) + rem with rem < 2^shift, so a bin's exact sum is
-  // count * (lo + (d << shift)) + sum(rem), and sum(rem) is kept as up to three 32-bit
-  // sums of 16-bit pieces of rem (each at most 4096 * 2^16).
-  unsigned long long A = 0;
-  uint32_t* hcnt = reinterpret_cast<uint32_t*>(hist);   // [256]
-  uint32_t* hrem = hcnt + 256;                          // [3][256]
-  while (target > 0 && hi > lo) {
-    const unsigned long long span = hi - lo;
-    const int nbits = 64 - __clzll(static_cast<long long>(span));
-    const int shift = nbits > 8 ? nbits - 8 : 0;
-    const int pieces = (shift + 15) >> 4;  // 16-bit pieces of rem (<= 3: shift <= 45)
+  // Invariant: every element outside the candidates is either above them (kept; its sum is
+  // in A < target) or below them (dropped), and the last kept element is a candidate.  The
+  // host admits 0 < tau <= 1, so target <= sum and the invariant holds from the start.
+  unsigned long long A = 0, tstar = 0;
+  if (target > 0) {
+    int nc = n_kb;
+    bool all = true;  // the candidates are still the whole row (cand not yet written)
+    unsigned long long p = median3(qrow[0], qrow[n_kb >> 1], qrow[n_kb - 1]);
+    while (true) {
+      // sum of the candidates above p and the count of those equal to it
+      unsigned long long sgt = 0;
+      uint32_t ceq = 0;
+      for (int j0 = 0; j0 < nc; j0 += 32 * kBatch) {
+        unsigned long long qv[kBatch];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      hcnt[lane * 8 + i] = 0u;
-      hrem[lane * 8 + i] = 0u;
-      hrem[256 + lane * 8 + i] = 0u;
-      hrem[512 + lane * 8 + i] = 0u;
-    }
-    __syncwarp();
-    for (int j = lane; j < n_kb; j += 32) {
-      const unsigned long long q = qrow[j];
-      if (q >= lo && q <= hi) {
-        const unsigned long long x = q - lo;
-        const int d = static_cast<int>(x >> shift);
-        const unsigned long long rem = x & ((1ull << shift) - 1ull);
-        atomicAdd(&hcnt[d], 1u);
-        for (int k = 0; k < pieces; ++k)
-          atomicAdd(&hrem[256 * k + d], static_cast<uint32_t>((rem >> (16 * k)) & 0xFFFFull));
+        for (int u = 0; u < kBatch; ++u) {
+          const int j = j0 + 32 * u + lane;
+          qv[u] = j < nc ? qrow[all ? j : static_cast<int>(cand[j])] : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const int j = j0 + 32 * u + lane;
+          if (j < nc) {
+            if (qv[u] > p) sgt += qv[u];
+            else if (qv[u] == p) ++ceq;
+          }
+        }
       }
+      sgt = warp_sum_u64(sgt);
+      const unsigned long long neq = static_cast<unsigned long long>(__reduce_add_sync(0xffffffffu, ceq));
+      bool above;
+      if (A + sgt >= target) {
+        above = true;                  // the crossing lies above p
+      } else if (A + sgt + neq * p >= target) {
+        A += sgt;                      // the crossing is one of the elements equal to p
+        tstar = p;
+        break;
+      } else {
+        A += sgt + neq * p;            // everything >= p is kept
+        above = false;
+      }
+      // compact the candidates on the kept side of p, in place: a batch is read into
+      // registers before any of it is written, and writes land below the batch's end
+      int kept_nc = 0;
+      for (int j0 = 0; j0 < nc; j0 += 32 * kBatch) {
+        uint32_t idx[kBatch];
+        bool sel[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const int j = j0 + 32 * u + lane;
+          idx[u] = j < nc ? (all ? static_cast<uint32_t>(j) : cand[j]) : 0u;
+          const unsigned long long q = j < nc ? qrow[idx[u]] : 0ull;
+          sel[u] = j < nc && (above ? q > p : q < p);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const unsigned bal = __ballot_sync(0xffffffffu, sel[u]);
+          if (sel[u]) cand[kept_nc + __popc(bal & lt_mask)] = idx[u];
+          kept_nc += __popc(bal);
+        }
+        __syncwarp();
+      }
+      nc = kept_nc;
+      all = false;
+      if (nc == 0) {  // unreachable while the invariant holds; ends the loop regardless
+        tstar = p;
+        break;
+      }
+      p = median3(qrow[cand[0]], qrow[cand[nc >> 1]], qrow[cand[nc - 1]]);
     }
-    __syncwarp();
-    // lane l owns bins 255-8l .. 248-8l (descending); inclusive sums from the top
-    unsigned long long b[8];
-    unsigned long long run = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int d = 255 - 8 * lane - i;
-      const unsigned long long cnt = hcnt[d];
-      unsigned long long bs = cnt * (lo + (static_cast<unsigned long long>(d) << shift));
-      bs += static_cast<unsigned long long>(hrem[d]);
-      bs += static_cast<unsigned long long>(hrem[256 + d]) << 16;
-      bs += static_cast<unsigned long long>(hrem[512 + d]) << 32;
-      run += bs;
-      b[i] = run;
-    }
-    unsigned long long before = run;  // exclusive warp scan of lane totals
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned long long n = __shfl_up_sync(0xffffffffu, before, o);
-      if (lane >= o) before += n;
-    }
-    before -= run;
-    int first = 8;
-#pragma unroll
-    for (int i = 7; i >= 0; --i)
-      if (A + before + b[i] >= target) first = i;
-    const unsigned bal = __ballot_sync(0xffffffffu, first < 8);
-    const int src = __ffs(bal) - 1;  // the crossing exists (see the invariant)
-    unsigned long long above = before;  // sum of the bins strictly above the crossing bin
-#pragma unroll
-    for (int i = 1; i < 8; ++i)
-      if (first == i) above = before + b[i - 1];
-    const int dbin = 255 - 8 * lane - first;
-    above = __shfl_sync(0xffffffffu, above, src);
-    const int d_src = __shfl_sync(0xffffffffu, dbin, src);
-    A += above;
-    const unsigned long long nlo = lo + (static_cast<unsigned long long>(d_src) << shift);
-    const unsigned long long nhi = nlo + ((1ull << shift) - 1ull);
-    lo = nlo;
-    hi = nhi < hi ? nhi : hi;
-    __syncwarp();
   }
-  const unsigned long long tstar = lo;
 
   // Keep q > t*, and the c lowest-index blocks with q == t*.
   const unsigned long long c = target > 0 ? (target - A + tstar - 1) / tstar : 0ull;
   unsigned long long ties_before = 0;
   unsigned long long kept = 0;
   uint32_t* out_bits = bitmaps + r * words;
-  for (int j0 = 0; j0 < n_kb; j0 += 32) {
-    const int j = j0 + lane;
-    const unsigned long long q = j < n_kb ? qrow[j] : 0ull;
-    const bool is_tie = target > 0 && j < n_kb && q == tstar;
-    const unsigned tb = __ballot_sync(0xffffffffu, is_tie);
-    const unsigned long long rank = ties_before + __popc(tb & ((1u << lane) - 1u));
-    const bool keep = target > 0 && j < n_kb && (q > tstar || (is_tie && rank < c));
-    const unsigned kb = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0) out_bits[j0 >> 5] = kb;
-    ties_before += __popc(tb);
-    kept += __popc(kb);
+  for (int j1 = 0; j1 < n_kb; j1 += 32 * kBatch) {
+    unsigned long long qv[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int j = j1 + 32 * u + lane;
+      qv[u] = j < n_kb ? qrow[j] : 0ull;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int j0 = j1 + 32 * u;
+      if (j0 >= n_kb) break;  // warp-uniform
+      const int j = j0 + lane;
+      const unsigned long long q = qv[u];
+      const bool is_tie = target > 0 && j < n_kb && q == tstar;
+      const unsigned tb = __ballot_sync(0xffffffffu, is_tie);
+      const unsigned long long rank = ties_before + __popc(tb & lt_mask);
+      const bool keep = target > 0 && j < n_kb && (q > tstar || (is_tie && rank < c));
+      const unsigned kb = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0) out_bits[j0 >> 5] = kb;
+      ties_before += __popc(tb);
+      kept += __popc(kb);
+    }
   }
   if (lane == 0) counts[r] = static_cast<int32_t>(kept);
 }
@@ -270,7 +280,7 @@ __global__ void __launch_bounds__(256) topp_fill_kernel(const uint32_t* __restri
 static cudaError_t launch_select_rows(const float* mass, long long rows, int n_kb, float threshold,
                                       int32_t* counts, uint32_t* bitmaps, int words,
                                       uint32_t* status, cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(kSelWarps) * (n_kb + 512) * sizeof(unsigned long long);
+  const size_t smem = static_cast<size_t>(kSelWarps) * (n_kb + (n_kb + 1) / 2) * sizeof(unsigned long long);
   cudaError_t e = cudaFuncSetAttribute(topp_select_rows_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));

@@ -167,6 +167,55 @@ def test_topp_bit_exact_on_oracle_masses(B, wl):
         _topp_check(B, s, ref, tau)
 
 
+def _structured_rows(n_rows, n, seed):
+    """Rows whose shapes stress a pivoting selector: sorted either way, geometric (values
+    over many orders of magnitude), two levels, one non-zero, dyadic values whose running
+    sums hit the target exactly, and shuffled distinct values."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    for i in range(n_rows):
+        kind = i % 8
+        if kind == 0:
+            r = np.arange(1, n + 1, dtype=np.float64)
+        elif kind == 1:
+            r = np.arange(n, 0, -1, dtype=np.float64)
+        elif kind == 2:
+            r = 2.0 ** -np.minimum(np.arange(n), 60)
+        elif kind == 3:
+            r = np.where(rng.random(n) < 0.5, 1.0, 3.0)
+        elif kind == 4:
+            r = np.zeros(n)
+            r[rng.integers(0, n)] = 1.0
+        elif kind == 5:
+            r = 2.0 ** -rng.integers(1, 12, n).astype(np.float64)
+        elif kind == 6:
+            r = rng.permutation(n).astype(np.float64) + 1.0
+        else:
+            r = 2.0 ** -np.minimum(np.arange(n), 60)[::-1]
+        rows.append(r / r.sum())
+    return np.asarray(rows, dtype=np.float32)
+
+
+@pytest.mark.parametrize("tau", [0.5, 0.9, 0.99, 1.0])
+def test_topp_bit_exact_structured_rows(B, tau):
+    wl = WLS[0]
+    s = _shape(B, wl)
+    m = _structured_rows(s.rows, s.n_kb, seed=21)
+    _topp_check(B, s, m.reshape(s.batch, s.heads, s.n_qb, s.n_kb), tau)
+
+
+@pytest.mark.parametrize("cols", [1, 2, 3, 31, 33, 257])
+def test_topp_rows_bit_exact_short_and_odd_rows(B, cols):
+    m = np.concatenate([_structured_rows(16, cols, seed=cols),
+                        synth.draw_mass_rows(16, cols, seed=cols, kind="ties").numpy()])
+    for tau in (0.5, 0.99, 1.0):
+        rp, ci = B.topp_select_rows(torch.from_numpy(m).cuda(), tau)
+        rp_ref, ci_ref = O.topp_select(m, tau)
+        rp_got = rp.cpu().numpy().astype(np.int64)
+        assert np.array_equal(rp_got, rp_ref)
+        assert np.array_equal(ci[:int(rp_got[-1])].cpu().numpy().astype(np.int64), ci_ref)
+
+
 def test_topp_capacity_overflow_is_reported(B):
     wl = WLS[0]
     s = _shape(B, wl)
