@@ -7,11 +7,17 @@
 //   M_est[i, j] = n_j exp(scale qbar_i . kbar_j) / sum_j' n_j' exp(scale qbar_i . kbar_j').
 // The result feeds bsa_topp_select like the exact masses do.
 //
-// Kernels (fp32 CUDA-core math: the estimate is ~Np^2/4096 * D multiply-adds per head):
-//   pool_tiles_kernel   one warp per (bh, tile): sums of the valid rows of Q and K.
-//   pooled_logits_kernel a register-tiled qbar . kbar product per (bh): 64 x 64 logits per
-//                        CTA, 4 x 4 per thread; writes the log2-domain logits into the
-//                        output tensor.
+// Kernels:
+//   pool_tiles_kernel    one warp per (bh, tile): sums of the valid rows of Q and K.
+//   pooled_split_kernel  qbar_i and kbar_j (sums times 1 / valid count, fp32), each cut
+//                        into three bf16 parts hi + mid + lo (the fp32 value to ~2^-24),
+//                        laid out as rows of six D-wide segments so that one bf16 product
+//                        of a q row and a k row sums the six terms
+//                        hi.hi + hi.mid + mid.hi + hi.lo + lo.hi + mid.mid.
+//   pooled_logits_tc_kernel  that product on the tensor cores: a 128 x 128 tile of
+//                        (query block, kv block) logits per CTA, K = 6 D, TMA-fed
+//                        128-byte-swizzled stages, fp32 accumulator in TMEM; writes the
+//                        log2-domain logits (-inf for tiles without valid keys).
 //   pooled_softmax_kernel one warp per row: weighted softmax in place.
 #include <algorithm>
 
@@ -57,125 +63,177 @@ __global__ void __launch_bounds__(256) pool_tiles_kernel(const __nv_bfloat16* __
   }
 }
 
+// qbar / kbar rows, split for the tensor cores: row r of qs is query block i of head bh
+// (r = bh * n_qb + i), row r of ks kv block j (r = bh * n_kb + j); each row holds six
+// D-wide bf16 segments, q: [hi, hi, mid, hi, lo, mid], k: [hi, mid, hi, lo, hi, mid].  A
+// block without valid rows is all zeros.  One thread per (row, dim).
+template <int D>
+__global__ void __launch_bounds__(256) pooled_split_kernel(const float* __restrict__ qsum,
+                                                           const float* __restrict__ ksum,
+                                                           AttnDims a,
+                                                           __nv_bfloat16* __restrict__ qs,
+                                                           __nv_bfloat16* __restrict__ ks) {
+  const long long bhn = static_cast<long long>(a.batch) * a.heads;
+  const long long nq = bhn * a.n_qb, nk = bhn * a.n_kb;
+  const long long idx = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  const long long row = idx / D;
+  const int d = static_cast<int>(idx - row * D);
+  if (row >= nq + nk) return;
+  float x;
+  __nv_bfloat16* dst;
+  const bool isq = row < nq;
+  if (isq) {
+    const long long bh = row / a.n_qb;
+    const int i = static_cast<int>(row - bh * a.n_qb);
+    const int per = a.q_block / 64;  // tiles per query block
+    float acc = 0.f;
+    int cnt = 0;
+    for (int u = i * per; u < (i + 1) * per; ++u) {
+      acc += qsum[(bh * a.n_kb + u) * D + d];
+      cnt += tile_valid_count(a.g, u);
+    }
+    x = cnt > 0 ? acc * (1.f / static_cast<float>(cnt)) : 0.f;
+    dst = qs + row * (6 * D);
+  } else {
+    const long long rk = row - nq;
+    const long long bh = rk / a.n_kb;
+    const int j = static_cast<int>(rk - bh * a.n_kb);
+    const int cnt = tile_valid_count(a.g, j);
+    x = cnt > 0 ? ksum[(bh * a.n_kb + j) * D + d] * (1.f / static_cast<float>(cnt)) : 0.f;
+    dst = ks + rk * (6 * D);
+  }
+  const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(hi);  // exact
+  const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+  const __nv_bfloat16 seg[6] = {hi, isq ? hi : mid, isq ? mid : hi, isq ? hi : lo,
+                                isq ? lo : hi, mid};
+#pragma unroll
+  for (int t = 0; t < 6; ++t) dst[t * D + d] = seg[t];
+}
+
 // Logits in log2 units: scale * log2(e) * qbar_i . kbar_j, -inf for tiles without valid keys
-// (the softmax kernel adds log2(n_j)).  A register-tiled product per (bh): a CTA of 256
-// threads computes a 128 x 128 tile of (query block, kv block) logits, 8 x 8 per thread
-// (rows 4ty..4ty+3 and 64+4ty.., columns likewise, so each 16-byte shared load of a warp is
-// conflict-free); the head dimension is staged 16 at a time in shared memory as
-// [d][block].  qbar and kbar are formed while staging: sums of the block's tiles times
-// 1 / valid count (0 for an empty block).  Every logit sums over d in order 0..D-1
-// (deterministic).
-constexpr int kLgTile = 128;
-constexpr int kLgK = 16;
+// (the softmax kernel adds log2(n_j)).  One CTA of 128 threads per 128 x 128 tile: thread 0
+// of warp 0 issues the TMA loads of 64-column (128-byte) chunks of the split rows into a
+// kPlStages-deep ring, thread 0 of warp 1 the MMAs (M = N = 128, K = 16 each) into one
+// fp32 TMEM accumulator, and all four warps read it back (a thread per query block).
+constexpr int kPlStages = 3;
+constexpr int kPlStage = 2 * 128 * 128;  // A and B chunks of one stage, bytes
+constexpr int kPlAlloc = kPlStages * kPlStage + 1024 + 1024;
 
 template <int D>
-__global__ void __launch_bounds__(256) pooled_logits_kernel(const float* __restrict__ qsum,
-                                                            const float* __restrict__ ksum,
-                                                            AttnDims a, float scale_log2,
-                                                            float* __restrict__ out) {
-  __shared__ __align__(16) float sa[kLgK][kLgTile];
-  __shared__ __align__(16) float sb[kLgK][kLgTile];
-  __shared__ float s_qinv[kLgTile];
-  __shared__ float s_kinv[kLgTile];
-  const int ti = (a.n_qb + kLgTile - 1) / kLgTile;
-  const int tj = (a.n_kb + kLgTile - 1) / kLgTile;
+__global__ void __launch_bounds__(128) pooled_logits_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+    AttnDims a, float scale_log2, float* __restrict__ out, uint32_t* status) {
+  constexpr int KC = 6 * D / 64;  // 128-byte chunks along the product's K
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPlStages * kPlStage);
+  uint64_t* bar_full = bars;
+  uint64_t* bar_empty = bars + kPlStages;
+  uint64_t* bar_acc = bars + 2 * kPlStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_acc + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* jvalid = const_cast<int*>(abort_flag) + 1;  // [128]
+
+  const int ti = (a.n_qb + 127) / 128;
+  const int tj = (a.n_kb + 127) / 128;
   const int per_bh = ti * tj;
   const int bh = blockIdx.x / per_bh;
   const int rem = blockIdx.x - bh * per_bh;
-  const int i0 = (rem / tj) * kLgTile;
-  const int j0 = (rem % tj) * kLgTile;
-  const int tid = threadIdx.x;
-  const int per = a.q_block / 64;  // tiles per query block
-  const long long tbase = static_cast<long long>(bh) * a.n_kb;
-  if (tid < kLgTile) {
-    const int i = i0 + tid;
-    int cnt = 0;
-    if (i < a.n_qb)
-      for (int u = i * per; u < (i + 1) * per; ++u) cnt += tile_valid_count(a.g, u);
-    s_qinv[tid] = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
-  } else {
-    const int j = j0 + tid - kLgTile;
-    const int cnt = j < a.n_kb ? tile_valid_count(a.g, j) : 0;
-    s_kinv[tid - kLgTile] = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
-  }
-  const int ty = tid >> 4, tx = tid & 15;
-  float acc[8][8];
-#pragma unroll
-  for (int r = 0; r < 8; ++r)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
-  for (int d0 = 0; d0 < D; d0 += kLgK) {
-    __syncthreads();
-    // stage 128 blocks x 16 dims of qbar and kbar, transposed to [d][block]: two 16-byte
-    // loads of four consecutive dims per thread and matrix (128 x 16 = 2 x 256 x 4)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int f = tid + 256 * h;
-      const int blk = f >> 2, dq = (f & 3) * 4;
-      const int i = i0 + blk, j = j0 + blk;
-      float4 qv = make_float4(0.f, 0.f, 0.f, 0.f), kv = qv;
-      if (i < a.n_qb) {
-        for (int u = i * per; u < (i + 1) * per; ++u) {
-          const float4 t = *reinterpret_cast<const float4*>(qsum + (tbase + u) * D + d0 + dq);
-          qv.x += t.x;
-          qv.y += t.y;
-          qv.z += t.z;
-          qv.w += t.w;
-        }
-        const float fq = s_qinv[blk];
-        qv = make_float4(qv.x * fq, qv.y * fq, qv.z * fq, qv.w * fq);
-      }
-      if (j < a.n_kb) {
-        const float4 t = *reinterpret_cast<const float4*>(ksum + (tbase + j) * D + d0 + dq);
-        const float fk = s_kinv[blk];
-        kv = make_float4(t.x * fk, t.y * fk, t.z * fk, t.w * fk);
-      }
-      sa[dq + 0][blk] = qv.x;
-      sa[dq + 1][blk] = qv.y;
-      sa[dq + 2][blk] = qv.z;
-      sa[dq + 3][blk] = qv.w;
-      sb[dq + 0][blk] = kv.x;
-      sb[dq + 1][blk] = kv.y;
-      sb[dq + 2][blk] = kv.z;
-      sb[dq + 3][blk] = kv.w;
+  const int i0 = (rem / tj) * 128;
+  const int j0 = (rem % tj) * 128;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kPlStages; ++st) {
+      mbar_init(bar_full + st, 1);
+      mbar_init(bar_empty + st, 1);
     }
-    __syncthreads();
-#pragma unroll
-    for (int d = 0; d < kLgK; ++d) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&sa[d][4 * ty]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&sa[d][64 + 4 * ty]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&sb[d][4 * tx]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&sb[d][64 + 4 * tx]);
-      const float ar[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float br[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(ar[r], br[c], acc[r][c]);
-    }
+    mbar_init(bar_acc, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
+  {
+    const int j = j0 + threadIdx.x;
+    jvalid[threadIdx.x] = (j < a.n_kb && tile_valid_count(a.g, j) > 0) ? 1 : 0;
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    prefetch_tensormap(&tm_a);
+    prefetch_tensormap(&tm_b);
+    for (int kc = 0; kc < KC; ++kc) {
+      const int st = kc % kPlStages;
+      if (kc >= kPlStages && !mbar_wait(bar_empty + st, ((kc / kPlStages) - 1) & 1, abort_flag,
+                                        status, DETAIL_WAIT_K_EMPTY))
+        break;
+      uint8_t* sa = smem + st * kPlStage;
+      mbar_arrive_expect_tx(bar_full + st, kPlStage);
+      tma_load_3d(sa, &tm_a, bar_full + st, kc * 64, i0, bh);
+      tma_load_3d(sa + 128 * 128, &tm_b, bar_full + st, kc * 64, j0, bh);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = make_idesc(1u, 0u, 128u, 128u);
+    for (int kc = 0; kc < KC; ++kc) {
+      const int st = kc % kPlStages;
+      if (!mbar_wait(bar_full + st, (kc / kPlStages) & 1, abort_flag, status, DETAIL_WAIT_K_FULL))
+        break;
+      tc_fence_after();
+      const uint32_t sa = smem_u32(smem + st * kPlStage);
+      const uint64_t ad = make_sdesc_sw128(sa, 16, 1024);
+      const uint64_t bd = make_sdesc_sw128(sa + 128 * 128, 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_f16_ss(tmem, ad + static_cast<uint64_t>((kk * 32) >> 4),
+                   bd + static_cast<uint64_t>((kk * 32) >> 4), idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(bar_empty + st);
+    }
+    // Whatever happened, every issued MMA completes before the accumulator is read or
+    // the tensor memory released.
+    mma_commit(bar_acc);
+    mbar_wait_drain(bar_acc, 0, status, DETAIL_WAIT_O_FULL);
+  }
+  __syncwarp();
+  // ------------------------------------------------------------ epilogue
+  const bool got = __all_sync(0xffffffffu,
+                              mbar_wait(bar_acc, 0, abort_flag, status, DETAIL_WAIT_O_FULL));
+  tc_fence_after();
+  const int i = i0 + warp * 32 + lane;
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  float* orow = out + (static_cast<long long>(bh) * a.n_qb + i) * a.n_kb;
   const bool vec = (a.n_kb & 3) == 0;  // rows start 16-byte aligned
+#pragma unroll 1
+  for (int c0 = 0; c0 < 128; c0 += 32) {
+    float v[32];
+    tmem_ld32(lane_base + c0, v);
+    tmem_ld_wait();
+    if (!got || i >= a.n_qb) continue;
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const int i = i0 + (r < 4 ? 4 * ty + r : 64 + 4 * ty + r - 4);
-    if (i >= a.n_qb) continue;
-    float* orow = out + (static_cast<long long>(bh) * a.n_qb + i) * a.n_kb;
+    for (int c = 0; c < 32; ++c) v[c] = jvalid[c0 + c] ? v[c] * scale_log2 : -INFINITY;
+    const int j = j0 + c0;
+    if (vec && j + 31 < a.n_kb) {
 #pragma unroll
-    for (int g = 0; g < 2; ++g) {
-      const int cl = 64 * g + 4 * tx;  // first of four columns inside the tile
-      const int j = j0 + cl;
-      float v[4];
+      for (int c = 0; c < 32; c += 4)
+        *reinterpret_cast<float4*>(orow + j + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+    } else {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        v[c] = s_kinv[cl + c] > 0.f ? acc[r][4 * g + c] * scale_log2 : -INFINITY;
-      if (vec && j + 3 < a.n_kb) {
-        *reinterpret_cast<float4*>(orow + j) = make_float4(v[0], v[1], v[2], v[3]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (j + c < a.n_kb) orow[j + c] = v[c];
-      }
+      for (int c = 0; c < 32; ++c)
+        if (j + c < a.n_kb) orow[j + c] = v[c];
     }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
   }
 }
 
@@ -262,8 +320,37 @@ __global__ void __launch_bounds__(256) pooled_softmax_kernel(AttnDims a, long lo
   }
 }
 
+// Scratch after the status header: per-tile sums qsum, ksum fp32 [bh][n_kb][D], then the
+// split rows qs bf16 [bh][n_qb][6D] and ks bf16 [bh][n_kb][6D] (16-byte aligned rows).
 size_t pooled_scratch_bytes(const AttnDims& a) {
-  return 2 * static_cast<size_t>(a.batch) * a.heads * a.n_kb * a.head_dim * sizeof(float);
+  const size_t bhn = static_cast<size_t>(a.batch) * a.heads;
+  return 2 * bhn * a.n_kb * a.head_dim * sizeof(float) +
+         bhn * (static_cast<size_t>(a.n_qb) + a.n_kb) * 6 * a.head_dim * sizeof(__nv_bfloat16);
+}
+
+template <int D>
+static cudaError_t launch_pooled_logits(const AttnDims& a, const float* qsum, const float* ksum,
+                                        __nv_bfloat16* qs, __nv_bfloat16* ks, float sl2,
+                                        float* mass, uint32_t* status, cudaStream_t stream) {
+  const long long bhn = 1LL * a.batch * a.heads;
+  const long long rows = bhn * (a.n_qb + a.n_kb);
+  pooled_split_kernel<D><<<static_cast<unsigned>((rows * D + 255) / 256), 256, 0, stream>>>(
+      qsum, ksum, a, qs, ks);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap ta, tb;
+  e = encode_tmap_3d(&ta, qs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 6 * D, a.n_qb,
+                     static_cast<int>(bhn), 64, 128);
+  if (e != cudaSuccess) return e;
+  e = encode_tmap_3d(&tb, ks, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 6 * D, a.n_kb,
+                     static_cast<int>(bhn), 64, 128);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(pooled_logits_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kPlAlloc);
+  if (e != cudaSuccess) return e;
+  const unsigned ctas = static_cast<unsigned>(bhn * ((a.n_qb + 127) / 128) * ((a.n_kb + 127) / 128));
+  pooled_logits_tc_kernel<D><<<ctas, 128, kPlAlloc, stream>>>(ta, tb, a, sl2, mass, status);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_pooled_mass(const AttnDims& a, const void* q, const void* k, float softmax_scale,
@@ -271,25 +358,25 @@ cudaError_t launch_pooled_mass(const AttnDims& a, const void* q, const void* k, 
   const long long tiles = 1LL * a.batch * a.heads * a.n_kb;
   const long long rows = 1LL * a.batch * a.heads * a.n_qb;
   if (tiles == 0) return cudaSuccess;
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   float* qsum = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kStatusBytes);
   float* ksum = qsum + tiles * a.head_dim;
+  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(ksum + tiles * a.head_dim);
+  __nv_bfloat16* ks = qs + rows * 6 * a.head_dim;
   const float sl2 = softmax_scale * 1.4426950408889634f;
   const unsigned pool_ctas = static_cast<unsigned>((tiles + 7) / 8);
-  const unsigned logit_ctas = static_cast<unsigned>(1LL * a.batch * a.heads *
-                                                    ((a.n_qb + kLgTile - 1) / kLgTile) *
-                                                    ((a.n_kb + kLgTile - 1) / kLgTile));
   // a warp per row, CTAs looping over rows: the weight table is built once per CTA
   const unsigned sm_ctas = static_cast<unsigned>(std::min<long long>((rows + 7) / 8, 148LL * 8));
   const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
   const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
+  cudaError_t e;
   if (a.head_dim == 128) {
     pool_tiles_kernel<128><<<pool_ctas, 256, 0, stream>>>(qb, kb, a.g, tiles, qsum, ksum);
-    pooled_logits_kernel<128><<<logit_ctas, 256, 0, stream>>>(qsum, ksum, a, sl2, mass);
+    e = launch_pooled_logits<128>(a, qsum, ksum, qs, ks, sl2, mass, status, stream);
   } else {
     pool_tiles_kernel<64><<<pool_ctas, 256, 0, stream>>>(qb, kb, a.g, tiles, qsum, ksum);
-    pooled_logits_kernel<64><<<logit_ctas, 256, 0, stream>>>(qsum, ksum, a, sl2, mass);
+    e = launch_pooled_logits<64>(a, qsum, ksum, qs, ks, sl2, mass, status, stream);
   }
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   pooled_softmax_kernel<<<sm_ctas, 256, 0, stream>>>(a, rows, mass);
   return cudaGetLastError();
