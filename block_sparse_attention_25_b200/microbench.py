@@ -81,10 +81,12 @@ def main(argv=None):
     ap.add_argument("--q-clusters", type=int, default=64, help="k-means clusters of the queries")
     ap.add_argument("--k-clusters", type=int, default=256, help="k-means clusters of the keys")
     ap.add_argument("--rounds", type=int, default=10, help="k-means rounds")
-    ap.add_argument("--only", choices=["all", "tiles", "semantic", "fwd", "calib"], default="all",
+    ap.add_argument("--only", choices=["all", "tiles", "semantic", "fwd", "calib", "select"],
+                    default="all",
                     help="the 3D-tile path, the semantic-aware permutation path, or both; fwd: "
                          "only the calibration's lists and the forward calls; calib: only "
-                         "block_mass and dense_fwd_mass (small profiling cases)")
+                         "block_mass and dense_fwd_mass; select: only topp_select on the "
+                         "calibration's masses (small profiling cases)")
     ap.add_argument("--heads", type=int, default=None,
                     help="override the workload's head count (profiling on a smaller case)")
     args = ap.parse_args(argv)
@@ -113,7 +115,7 @@ def main(argv=None):
         semantic(args, wl, q, k, v, line, pk)
         return
     qt, kt, vt = (B.tile_permute(x, s) for x in (q, k, v))
-    if args.only in ("fwd", "calib"):
+    if args.only in ("fwd", "calib", "select"):
         return focused(args, wl, s, q, k, v, qt, kt, vt, line, pk)
     out_r = torch.empty_like(q)
     line("tile_permute", _time(lambda: B.tile_permute(q, s, out=qt), args.iters),
@@ -223,13 +225,23 @@ def main(argv=None):
 
 def focused(args, wl, s, q, k, v, qt, kt, vt, line, pk):
     """--only fwd: the calibration's lists (untimed), then the tile-major forward (bf16 and,
-    for D = 128, e4m3); --only calib: block_mass and dense_fwd_mass.  Small launch counts
-    for profiler captures."""
+    for D = 128, e4m3); --only calib: block_mass and dense_fwd_mass; --only select:
+    topp_select on the calibration's masses.  Small launch counts for profiler captures."""
     dev = qt.device
     D, Hh, R, nkb = s.head_dim, s.heads, s.rows, s.n_kb
     ws_m = B.new_workspace(s, B.OP_BLOCK_MASS, dev)
     mass = B.block_mass(qt, kt, s, ws=ws_m)
-    if args.only == "calib":
+    if args.only == "select":
+        ws_t = B.new_workspace(s, B.OP_TOPP_SELECT, dev)
+        rp = torch.empty(R + 1, dtype=torch.int32, device=dev)
+        ci = torch.empty(R * nkb, dtype=torch.int32, device=dev)
+        ms = _time(lambda: B.topp_select(mass, s, args.tau, ws=ws_t, row_ptr=rp, col_idx=ci),
+                   args.iters)
+        nnz = int(rp[-1])
+        line("topp_select", ms, 4 * R * nkb + 4 * (R + 1 + nnz), "GB/s", "hbm", pk["hbm"],
+             {"kept_fraction": round(nnz / (R * nkb), 5)})
+        ws_m = ws_t
+    elif args.only == "calib":
         qk_pass = 2.0 * s.batch * s.Np * s.Np * D * Hh
         line("block_mass", _time(lambda: B.block_mass(qt, kt, s, out=mass, ws=ws_m), args.iters),
              qk_pass, "TFLOP/s", "tensor", pk["bf16"])
