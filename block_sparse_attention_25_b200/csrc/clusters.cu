@@ -21,7 +21,8 @@
 //                          (deterministic); empty clusters keep theirs.
 //   cluster_gather/scatter row copies between raster [B, S, Hh, D] and cluster order
 //                          [B, Hh, S, D].
-//   cluster_mass_kernel    one CTA per (bh, query cluster): weighted softmax over key clusters.
+//   cluster_mass_kernel    one CTA per (bh, 8 query clusters): logits with each key centroid row
+//                          read once per group, then a weighted softmax per row.
 #include "bsa_kernels.cuh"
 
 namespace bsa {
@@ -450,57 +451,79 @@ __global__ void __launch_bounds__(256) cluster_permute_kernel(ClusterDims cd, in
 }
 
 // Cluster-level estimate: M[i][j] = n_j exp(s qc_i . kc_j) / sum_j' n_j' exp(s qc_i . kc_j').
-// One CTA of 256 threads per (bh, query cluster); logits in shared memory (<= 1024).
+// One CTA of 8 warps per (bh, group of kMassGroup query clusters).  Logits: warp w takes key
+// clusters w, w + 8, ...; its lanes read a key centroid row once, coalesced, and form its
+// dot products with every query centroid of the group (lanes over d, a fixed xor-shuffle
+// tree), so each key row is read once per group instead of once per query cluster.  Then
+// warp q normalises row q of the group (weighted softmax over the key clusters).
+constexpr int kMassGroup = 8;
+constexpr int kMassMaxKc = 1024;
+constexpr int kMassMaxD = 128;
+
 __global__ void __launch_bounds__(256) cluster_mass_kernel(int heads, int D, int n_qc, int n_kc,
                                                            const float* __restrict__ qc,
                                                            const int32_t* __restrict__ q_counts,
                                                            const float* __restrict__ kc,
                                                            const int32_t* __restrict__ k_counts,
                                                            float scale_log2, float* __restrict__ mass) {
-  __shared__ float sq[128];
-  __shared__ float lg[1024];
-  __shared__ float red[8];
-  const int bh = blockIdx.x / n_qc;
-  const int i = blockIdx.x - bh * n_qc;
+  __shared__ float sq[kMassGroup][kMassMaxD];
+  __shared__ float lg[kMassGroup][kMassMaxKc];
+  const int groups = (n_qc + kMassGroup - 1) / kMassGroup;
+  const int bh = blockIdx.x / groups;
+  const int i0 = (blockIdx.x - bh * groups) * kMassGroup;
+  const int ng = min(kMassGroup, n_qc - i0);  // query clusters in this group
   const int tid = threadIdx.x;
-  float* out = mass + static_cast<long long>(blockIdx.x) * n_kc;
-  if (q_counts[static_cast<long long>(bh) * n_qc + i] <= 0) {
-    for (int j = tid; j < n_kc; j += 256) out[j] = 0.f;
-    return;
+  const int warp = tid >> 5, lane = tid & 31;
+  const long long qrow0 = static_cast<long long>(bh) * n_qc + i0;
+  for (int e = tid; e < kMassGroup * D; e += 256) {
+    const int q = e / D, d = e - q * D;
+    sq[q][d] = q < ng ? qc[(qrow0 + q) * D + d] : 0.f;
   }
-  for (int d = tid; d < D; d += 256) sq[d] = qc[static_cast<long long>(blockIdx.x) * D + d];
   __syncthreads();
   const float* kb = kc + static_cast<long long>(bh) * n_kc * D;
   const int32_t* nk = k_counts + static_cast<long long>(bh) * n_kc;
-  float mx = -INFINITY;
-  for (int j = tid; j < n_kc; j += 256) {
-    float acc = 0.f;
-    for (int d = 0; d < D; ++d) acc = fmaf(sq[d], kb[static_cast<long long>(j) * D + d], acc);
-    const float l = nk[j] > 0 ? acc * scale_log2 : -INFINITY;
-    lg[j] = l;
-    mx = fmaxf(mx, l);
+  for (int j = warp; j < n_kc; j += 8) {
+    float acc[kMassGroup];
+#pragma unroll
+    for (int q = 0; q < kMassGroup; ++q) acc[q] = 0.f;
+    for (int d = lane; d < D; d += 32) {
+      const float kv = kb[static_cast<long long>(j) * D + d];
+#pragma unroll
+      for (int q = 0; q < kMassGroup; ++q) acc[q] = fmaf(sq[q][d], kv, acc[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < kMassGroup; ++q)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], o);
+    if (lane < kMassGroup) {
+      float v = acc[0];
+#pragma unroll
+      for (int q = 1; q < kMassGroup; ++q) v = lane == q ? acc[q] : v;
+      lg[lane][j] = nk[j] > 0 ? v * scale_log2 : -INFINITY;
+    }
   }
+  __syncthreads();
+  if (warp >= ng) return;
+  float* out = mass + (qrow0 + warp) * n_kc;
+  if (q_counts[qrow0 + warp] <= 0) {  // an empty query cluster: all-zero row
+    for (int j = lane; j < n_kc; j += 32) out[j] = 0.f;
+    return;
+  }
+  float* row = lg[warp];
+  float mx = -INFINITY;
+  for (int j = lane; j < n_kc; j += 32) mx = fmaxf(mx, row[j]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane_id() == 0) red[tid >> 5] = mx;
-  __syncthreads();
-  mx = red[0];
-#pragma unroll
-  for (int w = 1; w < 8; ++w) mx = fmaxf(mx, red[w]);
-  __syncthreads();
   float sum = 0.f;
-  for (int j = tid; j < n_kc; j += 256) {
-    const float w = mx == -INFINITY ? 0.f : static_cast<float>(max(nk[j], 0)) * exp2f(lg[j] - mx);
-    lg[j] = w;
+  for (int j = lane; j < n_kc; j += 32) {
+    const float w = mx == -INFINITY ? 0.f : static_cast<float>(max(nk[j], 0)) * exp2f(row[j] - mx);
+    row[j] = w;
     sum += w;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane_id() == 0) red[tid >> 5] = sum;
-  __syncthreads();
-  sum = ((red[0] + red[1]) + (red[2] + red[3])) + ((red[4] + red[5]) + (red[6] + red[7]));
   const float inv = sum > 0.f ? 1.f / sum : 0.f;
-  for (int j = tid; j < n_kc; j += 256) out[j] = lg[j] * inv;
+  for (int j = lane; j < n_kc; j += 32) out[j] = row[j] * inv;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -656,7 +679,9 @@ cudaError_t launch_cluster_mass(int batch, int heads, int head_dim, int n_qc, in
                                 cudaStream_t stream) {
   const long long rows = static_cast<long long>(batch) * heads * n_qc;
   if (rows == 0 || n_kc == 0) return cudaSuccess;
-  cluster_mass_kernel<<<static_cast<unsigned>(rows), 256, 0, stream>>>(
+  if (head_dim > kMassMaxD || n_kc > kMassMaxKc) return cudaErrorNotSupported;
+  const long long ctas = static_cast<long long>(batch) * heads * ((n_qc + kMassGroup - 1) / kMassGroup);
+  cluster_mass_kernel<<<static_cast<unsigned>(ctas), 256, 0, stream>>>(
       heads, head_dim, n_qc, n_kc, qc, q_counts, kc, k_counts, softmax_scale * 1.4426950408889634f,
       mass);
   return cudaGetLastError();

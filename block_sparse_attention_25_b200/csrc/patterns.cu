@@ -8,8 +8,10 @@
 // holds for one of them (union over kinds).  The lists are the same for every (batch,
 // head); each CSR row is still written out so the forward sees an ordinary CSR.
 //
-// One warp per CSR row: 32 kv blocks per ballot -> kept bitmap + count in the workspace;
-// then the selection's scan and compaction kernels turn the bitmaps into row_ptr/col_idx.
+// One warp per distinct CSR row (the n_qb rows of one (batch, head)): 32 kv blocks per
+// ballot -> kept bitmap + count in the workspace; a copy kernel repeats them for the other
+// (batch, head) pairs; then the selection's scan and compaction kernels turn the bitmaps
+// into row_ptr/col_idx.
 #include "bsa_kernels.cuh"
 
 namespace bsa {
@@ -62,6 +64,20 @@ __global__ void __launch_bounds__(256) pattern_rows_kernel(PatternParams pp, int
   if (lane == 0) counts[r] = kept;
 }
 
+// Rows [n_qb, rows): the counts and bitmap words of row r % n_qb.  One thread per word.
+__global__ void __launch_bounds__(256) pattern_repeat_kernel(long long rows, int n_qb, int words,
+                                                             int32_t* __restrict__ counts,
+                                                             uint32_t* __restrict__ bitmaps) {
+  const long long w = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  const long long total = (rows - n_qb) * words;
+  if (w >= total) return;
+  const long long r = n_qb + w / words;
+  const int k = static_cast<int>(w - (r - n_qb) * words);
+  const int src = static_cast<int>(r % n_qb);
+  bitmaps[r * words + k] = bitmaps[static_cast<long long>(src) * words + k];
+  if (k == 0) counts[r] = counts[src];
+}
+
 cudaError_t launch_pattern_csr(const AttnDims& a, const PatternParams& pp_in, int32_t* row_ptr,
                                int32_t* col_idx, long long col_capacity, void* ws,
                                cudaStream_t stream) {
@@ -75,10 +91,19 @@ cudaError_t launch_pattern_csr(const AttnDims& a, const PatternParams& pp_in, in
   int32_t* counts = reinterpret_cast<int32_t*>(base + kStatusBytes);
   uint32_t* bitmaps = reinterpret_cast<uint32_t*>(base + kStatusBytes + counts_bytes);
   if (rows == 0) return cudaMemsetAsync(row_ptr, 0, sizeof(int32_t), stream);
-  pattern_rows_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
-      pp, a.g.nth, a.g.ntw, a.q_block, a.n_qb, a.n_kb, rows, counts, bitmaps, words);
+  // the lists are the same for every (batch, head): evaluate the n_qb rows of the first
+  // one and repeat them
+  pattern_rows_kernel<<<static_cast<unsigned>((a.n_qb + 7) / 8), 256, 0, stream>>>(
+      pp, a.g.nth, a.g.ntw, a.q_block, a.n_qb, a.n_kb, a.n_qb, counts, bitmaps, words);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (rows > a.n_qb) {
+    const long long total = (rows - a.n_qb) * words;
+    pattern_repeat_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(
+        rows, a.n_qb, words, counts, bitmaps);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   return launch_bitmap_to_csr(counts, bitmaps, rows, words, row_ptr, col_idx, col_capacity,
                               status, stream);
 }
