@@ -16,8 +16,9 @@
 //                          chunk's first slot inside every cluster.
 //   layout_scatter_kernel  one warp per chunk walks its tokens in order: rank among equal
 //                          labels by __match_any_sync, so the order is stable.
-//   kmeans_update_kernel   centroid = sum of the cluster's tokens / size: 8 warps over fixed
-//                          segments of the cluster order, partial sums added in a fixed order
+//   kmeans_update_kernel   centroid = sum of the cluster's tokens / size: 8 warps (32 for
+//                          clusters of 1,024 tokens or more on average) over fixed segments
+//                          of the cluster order, partial sums added in a fixed order
 //                          (deterministic); empty clusters keep theirs.
 //   cluster_gather/scatter row copies between raster [B, S, Hh, D] and cluster order
 //                          [B, Hh, S, D].
@@ -282,12 +283,21 @@ __global__ void __launch_bounds__(1024) layout_scan_kernel(ClusterDims cd, int32
   const int c = threadIdx.x;
   const int nchunks = (cd.S + kLayoutChunk - 1) / kLayoutChunk;
   int32_t* hb = hist + static_cast<long long>(bh) * nchunks * cd.C;
+  // eight chunks' counts are loaded before any is written back, so a head's scan costs
+  // nchunks / 8 memory round trips rather than nchunks
+  constexpr int kU = 8;
   int run = 0;
   if (c < cd.C) {
-    for (int k = 0; k < nchunks; ++k) {
-      const int n = hb[static_cast<long long>(k) * cd.C + c];
-      hb[static_cast<long long>(k) * cd.C + c] = run;
-      run += n;
+    for (int k0 = 0; k0 < nchunks; k0 += kU) {
+      int n[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        n[u] = k0 + u < nchunks ? hb[static_cast<long long>(k0 + u) * cd.C + c] : 0;
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        if (k0 + u < nchunks) hb[static_cast<long long>(k0 + u) * cd.C + c] = run;
+        run += n[u];
+      }
     }
   }
   // exclusive scan of the cluster sizes over the CTA
@@ -305,7 +315,15 @@ __global__ void __launch_bounds__(1024) layout_scan_kernel(ClusterDims cd, int32
   if (c < cd.C) {
     counts[static_cast<long long>(bh) * cd.C + c] = run;
     starts[static_cast<long long>(bh) * cd.C + c] = start;
-    for (int k = 0; k < nchunks; ++k) hb[static_cast<long long>(k) * cd.C + c] += start;
+    for (int k0 = 0; k0 < nchunks; k0 += kU) {
+      int f[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        f[u] = k0 + u < nchunks ? hb[static_cast<long long>(k0 + u) * cd.C + c] : 0;
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        if (k0 + u < nchunks) hb[static_cast<long long>(k0 + u) * cd.C + c] = f[u] + start;
+    }
   }
 }
 
@@ -352,15 +370,15 @@ __global__ void __launch_bounds__(32 * kScatterWarps) layout_scatter_kernel(
 // warp w sums the w-th of 8 contiguous segments of the cluster's slots (lane l holds dims
 // D/32 * l ..), the 8 partial sums are added in warp order: a fixed summation order
 // (deterministic).  An empty cluster keeps its centroid.
-template <int D>
-__global__ void __launch_bounds__(256) kmeans_update_kernel(ClusterDims cd,
+template <int D, int W>
+__global__ void __launch_bounds__(32 * W) kmeans_update_kernel(ClusterDims cd,
                                                             const __nv_bfloat16* __restrict__ x,
                                                             const int32_t* __restrict__ token_of_slot,
                                                             const int32_t* __restrict__ starts,
                                                             const int32_t* __restrict__ counts,
                                                             float* __restrict__ cent) {
   constexpr int PER = D / 32;  // dims per lane: 4 (D = 128) or 2 (D = 64)
-  __shared__ float part[8][D];
+  __shared__ float part[W][D];
   const int bh = blockIdx.x / cd.C;
   const int c = blockIdx.x - bh * cd.C;
   const int b = bh / cd.heads, h = bh - b * cd.heads;
@@ -368,7 +386,7 @@ __global__ void __launch_bounds__(256) kmeans_update_kernel(ClusterDims cd,
   if (n <= 0) return;  // uniform over the CTA
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int st = starts[static_cast<long long>(bh) * cd.C + c];
-  const int seg = (n + 7) / 8;
+  const int seg = (n + W - 1) / W;
   const int lo = min(n, warp * seg), hi = min(n, lo + seg);
   const int32_t* tos = token_of_slot + static_cast<long long>(bh) * cd.S + st;
   const __nv_bfloat16* xb = x + static_cast<long long>(b) * cd.S * cd.heads * D + h * D + lane * PER;
@@ -414,7 +432,7 @@ __global__ void __launch_bounds__(256) kmeans_update_kernel(ClusterDims cd,
   if (threadIdx.x < D) {
     float sum = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) sum += part[w][threadIdx.x];
+    for (int w = 0; w < W; ++w) sum += part[w][threadIdx.x];
     cent[(static_cast<long long>(bh) * cd.C + c) * D + threadIdx.x] = __fdiv_rn(sum, static_cast<float>(n));
   }
 }
@@ -647,10 +665,19 @@ cudaError_t launch_kmeans(const ClusterDims& cd, const void* x, int rounds, floa
     if (e != cudaSuccess) return e;
     e = layout_into(cd, labels, counts, starts, tos, sot, hist, status, stream);
     if (e != cudaSuccess) return e;
-    if (cd.head_dim == 128)
-      kmeans_update_kernel<128><<<upd_ctas, 256, 0, stream>>>(cd, xb, tos, starts, counts, centroids);
-    else
-      kmeans_update_kernel<64><<<upd_ctas, 256, 0, stream>>>(cd, xb, tos, starts, counts, centroids);
+    // large clusters (1,024 tokens or more on average) get 32 warps, smaller ones 8
+    const bool wide = cd.S >= 1024LL * cd.C;
+    if (cd.head_dim == 128) {
+      if (wide)
+        kmeans_update_kernel<128, 32><<<upd_ctas, 1024, 0, stream>>>(cd, xb, tos, starts, counts, centroids);
+      else
+        kmeans_update_kernel<128, 8><<<upd_ctas, 256, 0, stream>>>(cd, xb, tos, starts, counts, centroids);
+    } else {
+      if (wide)
+        kmeans_update_kernel<64, 32><<<upd_ctas, 1024, 0, stream>>>(cd, xb, tos, starts, counts, centroids);
+      else
+        kmeans_update_kernel<64, 8><<<upd_ctas, 256, 0, stream>>>(cd, xb, tos, starts, counts, centroids);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
