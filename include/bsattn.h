@@ -152,7 +152,8 @@ BSA_API bsa_status bsa_tile_permute_quant_e4m3(const bsa_shape* shape, const voi
  * zero.  One dense pass on tcgen05 tensor cores: every probability computed once against a
  * lazily raised reference max, unnormalised block sums per row kept in the workspace and
  * normalised by the row sums at the end.  Workspace: bsa_workspace_bytes(shape, BSA_OP_BLOCK_MASS) -- the
- * status header plus 192 slices of 256 x Np/64 fp32, one per SM id. */
+ * status header, a 256-byte slice pool, and 192 slices of 256 x Np/64 fp32, each held by
+ * one live CTA at a time (claimed from the pool when the CTA starts, freed when it ends). */
 BSA_API bsa_status bsa_block_mass(const bsa_shape* shape, const void* q, const void* k,
                           float softmax_scale, float* mass, void* ws, size_t ws_bytes,
                           bsa_stream_t stream);
