@@ -701,6 +701,8 @@ def main():
         res = run_reference(args, world, rank, pg)
         if rank == 0:
             print(json.dumps(res), flush=True)
+        if pg is not None:
+            pg.destroy_process_group()
         return
     res = run_ours(args, world, rank, local, pg)
     if rank == 0:

@@ -91,3 +91,23 @@ def test_single_rank_needs_no_process_group(monkeypatch):
     w, r, local, pg = bench.dist_setup(None)
     assert (w, r, local, pg) == (1, 0, 0, None)
     assert bench.max_over_ranks(3.25, pg) == 3.25
+
+
+def test_reference_arm_under_torchrun_prints_one_line_from_rank_0(tmp_path):
+    """bench.py --impl reference launched as two gloo ranks: rank 0 times the oracle and
+    prints the JSON line, rank 1 exits without work, and both leave cleanly."""
+    import json
+    import subprocess
+    port = _free_port()
+    env = dict(os.environ, MASTER_ADDR="127.0.0.1")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+           "--steps", "1", "--warmup", "1", "--cpu-sample-rows", "2", "--config", "tiny"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
