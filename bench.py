@@ -11,6 +11,9 @@ Wan-14B-like: B=1, 40 heads, D=128, 21x45x80 tokens padded to 24x48x80, 64-token
                  forward's loads and stores; the e4m3 workload always takes
                  tile_permute_quant_e4m3 x3 -> bsattn_fwd -> inverse)
 on seeded synthetic inputs already resident in HBM (Q/K/V of 774 MB each, far above L2).
+--config wan14b_720p_local runs the same shape with spatially local attention (~66% of
+the block pairs kept at 0.99); --config wan14b_720p_fp8 the e4m3 operands; both also
+take 10 reuse calls per step (--reuse overrides).
 
 value  = executed attention TFLOP/s of the whole step (a step rate): FLOPs of the kept
          blocks of the 10 reuse calls (4 * 64 * 64 * D per kept (query block, kv block)
@@ -26,8 +29,8 @@ a bounded sample of the same workload.
 With N > 1 ranks (one per GPU) the path needs no exchange step: --split problems (the
 default) gives every rank an independent problem of the workload's size (weak scaling);
 --split heads gives rank r the heads [r*Hh/N, (r+1)*Hh/N) of one problem (strong scaling;
-Hh must divide by N).  The process group carries only the timing barrier and the
-max-over-ranks reduction.
+Hh must divide by N).  The process group carries only the timing barrier, the
+max-over-ranks reduction of the timed region and the sum of the ranks' executed work.
 """
 from __future__ import annotations
 
