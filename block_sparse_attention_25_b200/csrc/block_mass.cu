@@ -224,8 +224,7 @@ __global__ void __maxnreg__(mass::kMaxRegs)
         tc_fence_after();
         if (mine) {
           const uint32_t s_addr = lane_base + (2 * t + buf) * 128 + 64 * h;
-          tmem_ld32(s_addr + 0, sv + 0);
-          tmem_ld32(s_addr + 32, sv + 32);
+          tmem_ld64(s_addr, sv);  // one load instruction (107.7 vs 108.4 ms at 720p)
           tmem_ld_wait();
         }
         tc_fence_before();
