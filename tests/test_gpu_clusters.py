@@ -128,24 +128,32 @@ def test_cluster_permute_round_trip(B, D):
     assert torch.equal(z.cpu(), x)
 
 
-def test_cluster_mass_parity(B):
-    Bt, Hh, D, Cq, Ck = 1, 3, 128, 40, 70
-    cs = B.ClusterShape(Bt, Hh, D, 1000, Cq, Ck)
+@pytest.mark.parametrize("Bt,Hh,D,Cq,Ck", [(1, 3, 128, 40, 70), (2, 2, 64, 13, 1024),
+                                            (1, 1, 128, 1, 1), (1, 2, 128, 1024, 9)])
+def test_cluster_mass_parity(B, Bt, Hh, D, Cq, Ck):
+    """Query clusters in groups of eight with a ragged last group, up to the ABI's 1,024
+    clusters on either side, and single clusters."""
+    cs = B.ClusterShape(Bt, Hh, D, 4096, Cq, Ck)
     g = torch.Generator().manual_seed(8)
     qc = torch.randn((Bt, Hh, Cq, D), generator=g)
     kc = torch.randn((Bt, Hh, Ck, D), generator=g)
     qn = torch.randint(0, 50, (Bt, Hh, Cq), generator=g, dtype=torch.int32)
     kn = torch.randint(0, 50, (Bt, Hh, Ck), generator=g, dtype=torch.int32)
-    qn[0, 0, 3] = 0
-    kn[0, 1, :5] = 0
+    if Cq > 3:
+        qn[0, 0, 3] = 0
+    if Ck > 5 and Hh > 1:
+        kn[0, 1, :5] = 0
+    qn[..., 0] = qn[..., 0].clamp_min(1)   # at least one non-empty cluster on each side
+    kn[..., 0] = kn[..., 0].clamp_min(1)
     scale = 1.5 / math.sqrt(D)
     m = B.cluster_mass(cs, qc.cuda(), qn.cuda(), kc.cuda(), kn.cuda(), scale)
-    for h in range(Hh):
-        ref = O.cluster_mass(qc[0, h].double().numpy(), qn[0, h].numpy(), kc[0, h].double().numpy(),
-                             kn[0, h].numpy(), scale)
-        got = _np(m[0, h])
-        assert np.abs(got - ref).max() <= 1e-5
-        assert np.all(got[ref == 0] == 0)
+    for b in range(Bt):
+        for h in range(Hh):
+            ref = O.cluster_mass(qc[b, h].double().numpy(), qn[b, h].numpy(),
+                                 kc[b, h].double().numpy(), kn[b, h].numpy(), scale)
+            got = _np(m[b, h])
+            assert np.abs(got - ref).max() <= 1e-5
+            assert np.all(got[ref == 0] == 0)
 
 
 @pytest.mark.parametrize("cols", [1, 37, 256, 1440])
