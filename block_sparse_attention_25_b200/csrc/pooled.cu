@@ -66,50 +66,80 @@ __global__ void __launch_bounds__(256) pool_tiles_kernel(const __nv_bfloat16* __
 // qbar / kbar rows, split for the tensor cores: row r of qs is query block i of head bh
 // (r = bh * n_qb + i), row r of ks kv block j (r = bh * n_kb + j); each row holds six
 // D-wide bf16 segments, q: [hi, hi, mid, hi, lo, mid], k: [hi, mid, hi, lo, hi, mid].  A
-// block without valid rows is all zeros.  One thread per (row, dim).
+// block without valid rows is all zeros.  One thread per (row, 8 dims): two 16-byte loads
+// of the sums, six 16-byte stores.
 template <int D>
 __global__ void __launch_bounds__(256) pooled_split_kernel(const float* __restrict__ qsum,
                                                            const float* __restrict__ ksum,
                                                            AttnDims a,
                                                            __nv_bfloat16* __restrict__ qs,
                                                            __nv_bfloat16* __restrict__ ks) {
+  constexpr int G = D / 8;  // 8-dim groups per row
   const long long bhn = static_cast<long long>(a.batch) * a.heads;
   const long long nq = bhn * a.n_qb, nk = bhn * a.n_kb;
   const long long idx = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
-  const long long row = idx / D;
-  const int d = static_cast<int>(idx - row * D);
+  const long long row = idx / G;
+  const int d0 = static_cast<int>(idx - row * G) * 8;
   if (row >= nq + nk) return;
-  float x;
+  float x[8];
   __nv_bfloat16* dst;
   const bool isq = row < nq;
   if (isq) {
     const long long bh = row / a.n_qb;
     const int i = static_cast<int>(row - bh * a.n_qb);
     const int per = a.q_block / 64;  // tiles per query block
-    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = 0.f;
     int cnt = 0;
     for (int u = i * per; u < (i + 1) * per; ++u) {
-      acc += qsum[(bh * a.n_kb + u) * D + d];
+      const float4* src = reinterpret_cast<const float4*>(qsum + (bh * a.n_kb + u) * D + d0);
+      const float4 v0 = src[0], v1 = src[1];
+      x[0] += v0.x; x[1] += v0.y; x[2] += v0.z; x[3] += v0.w;
+      x[4] += v1.x; x[5] += v1.y; x[6] += v1.z; x[7] += v1.w;
       cnt += tile_valid_count(a.g, u);
     }
-    x = cnt > 0 ? acc * (1.f / static_cast<float>(cnt)) : 0.f;
-    dst = qs + row * (6 * D);
+    const float inv = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = cnt > 0 ? x[e] * inv : 0.f;
+    dst = qs + row * (6 * D) + d0;
   } else {
     const long long rk = row - nq;
     const long long bh = rk / a.n_kb;
     const int j = static_cast<int>(rk - bh * a.n_kb);
     const int cnt = tile_valid_count(a.g, j);
-    x = cnt > 0 ? ksum[(bh * a.n_kb + j) * D + d] * (1.f / static_cast<float>(cnt)) : 0.f;
-    dst = ks + rk * (6 * D);
-  }
-  const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-  const float r1 = x - __bfloat162float(hi);  // exact
-  const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-  const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-  const __nv_bfloat16 seg[6] = {hi, isq ? hi : mid, isq ? mid : hi, isq ? hi : lo,
-                                isq ? lo : hi, mid};
+    const float inv = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
+    const float4* src = reinterpret_cast<const float4*>(ksum + (bh * a.n_kb + j) * D + d0);
+    const float4 v0 = src[0], v1 = src[1];
+    const float t[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-  for (int t = 0; t < 6; ++t) dst[t * D + d] = seg[t];
+    for (int e = 0; e < 8; ++e) x[e] = cnt > 0 ? t[e] * inv : 0.f;
+    dst = ks + rk * (6 * D) + d0;
+  }
+  uint4 hi, mid, lo;
+  uint32_t* ph = reinterpret_cast<uint32_t*>(&hi);
+  uint32_t* pm = reinterpret_cast<uint32_t*>(&mid);
+  uint32_t* pl = reinterpret_cast<uint32_t*>(&lo);
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    float h2[2], m2[2], l2[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const __nv_bfloat16 hb = __float2bfloat16_rn(x[e + u]);
+      const float r1 = x[e + u] - __bfloat162float(hb);  // exact
+      const __nv_bfloat16 mb = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 lb = __float2bfloat16_rn(r1 - __bfloat162float(mb));
+      h2[u] = __bfloat162float(hb);
+      m2[u] = __bfloat162float(mb);
+      l2[u] = __bfloat162float(lb);
+    }
+    // the parts are bf16 values already, so packing them back is exact
+    ph[e / 2] = pack_bf16x2(h2[0], h2[1]);
+    pm[e / 2] = pack_bf16x2(m2[0], m2[1]);
+    pl[e / 2] = pack_bf16x2(l2[0], l2[1]);
+  }
+  const uint4 seg[6] = {hi, isq ? hi : mid, isq ? mid : hi, isq ? hi : lo, isq ? lo : hi, mid};
+#pragma unroll
+  for (int t = 0; t < 6; ++t) *reinterpret_cast<uint4*>(dst + t * D) = seg[t];
 }
 
 // Logits in log2 units: scale * log2(e) * qbar_i . kbar_j, -inf for tiles without valid keys
@@ -334,7 +364,7 @@ static cudaError_t launch_pooled_logits(const AttnDims& a, const float* qsum, co
                                         float* mass, uint32_t* status, cudaStream_t stream) {
   const long long bhn = 1LL * a.batch * a.heads;
   const long long rows = bhn * (a.n_qb + a.n_kb);
-  pooled_split_kernel<D><<<static_cast<unsigned>((rows * D + 255) / 256), 256, 0, stream>>>(
+  pooled_split_kernel<D><<<static_cast<unsigned>((rows * (D / 8) + 255) / 256), 256, 0, stream>>>(
       qsum, ksum, a, qs, ks);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
