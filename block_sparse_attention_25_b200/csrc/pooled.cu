@@ -8,7 +8,8 @@
 // The result feeds bsa_topp_select like the exact masses do.
 //
 // Kernels:
-//   pool_tiles_kernel    one warp per (bh, tile): sums of the valid rows of Q and K.
+//   pool_tiles_kernel    one warp per (bh, tile): sums of the valid rows of Q and K, 16-byte
+//                        loads with eight rows in flight per lane.
 //   pooled_split_kernel  qbar_i and kbar_j (sums times 1 / valid count, fp32), each cut
 //                        into three bf16 parts hi + mid + lo (the fp32 value to ~2^-24),
 //                        laid out as rows of six D-wide segments so that one bf16 product
@@ -30,36 +31,70 @@ __device__ __forceinline__ int tile_valid_count(const GridDims& g, int j) {
   return __popcll(tile_valid_mask(g, j));
 }
 
+// One warp per (bh, tile): sums of the tile's valid rows of Q and of K.  A lane reads 8
+// dims (16 bytes) of a row; the warp's lane groups (two for D = 128, four for D = 64) take
+// rows r = group (mod groups), each lane with eight rows' loads in flight before they are
+// added.  The groups' partial sums are combined at the end by a fixed xor tree, so the
+// result does not depend on timing.
 template <int D>
 __global__ void __launch_bounds__(256) pool_tiles_kernel(const __nv_bfloat16* __restrict__ q,
                                                          const __nv_bfloat16* __restrict__ k,
                                                          GridDims g, long long tiles,
                                                          float* __restrict__ qsum,
                                                          float* __restrict__ ksum) {
-  constexpr int PER = D / 32;  // dims per lane (4 or 2)
+  constexpr int LPR = D / 8;         // lanes per row (16 for D = 128, 8 for D = 64)
+  constexpr int RPI = 32 / LPR;      // rows per warp instruction (2 or 4)
+  constexpr int kU = 8;              // row loads in flight per lane
   const long long w = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (w >= tiles) return;
   const int lane = threadIdx.x & 31;
   const int ntiles = g.Np / 64;
   const int j = static_cast<int>(w % ntiles);
   const uint64_t vm = tile_valid_mask(g, j);
-  const __nv_bfloat16* qt = q + w * 64 * D + lane * PER;
-  const __nv_bfloat16* kt = k + w * 64 * D + lane * PER;
-  float aq[PER], ak[PER];
+  const int sub = lane / LPR;        // which of the instruction's rows
+  const int d0 = (lane % LPR) * 8;
+  const __nv_bfloat16* qt = q + w * 64 * D + d0;
+  const __nv_bfloat16* kt = k + w * 64 * D + d0;
+  float aq[8], ak[8];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) aq[e] = ak[e] = 0.f;
-  for (int r = 0; r < 64; ++r) {
-    if (!((vm >> r) & 1ull)) continue;
+  for (int e = 0; e < 8; ++e) aq[e] = ak[e] = 0.f;
+  for (int r0 = 0; r0 < 64; r0 += RPI * kU) {
+    uint4 vq[kU], vk[kU];
 #pragma unroll
-    for (int e = 0; e < PER; ++e) {
-      aq[e] += __bfloat162float(qt[r * D + e]);
-      ak[e] += __bfloat162float(kt[r * D + e]);
+    for (int u = 0; u < kU; ++u) {
+      const int r = r0 + u * RPI + sub;
+      const bool ok = r < 64 && ((vm >> r) & 1ull);
+      vq[u] = ok ? *reinterpret_cast<const uint4*>(qt + r * D) : make_uint4(0u, 0u, 0u, 0u);
+      vk[u] = ok ? *reinterpret_cast<const uint4*>(kt + r * D) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const uint32_t wq[4] = {vq[u].x, vq[u].y, vq[u].z, vq[u].w};
+      const uint32_t wk[4] = {vk[u].x, vk[u].y, vk[u].z, vk[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        aq[2 * e] += __uint_as_float(wq[e] << 16);
+        aq[2 * e + 1] += __uint_as_float(wq[e] & 0xFFFF0000u);
+        ak[2 * e] += __uint_as_float(wk[e] << 16);
+        ak[2 * e + 1] += __uint_as_float(wk[e] & 0xFFFF0000u);
+      }
     }
   }
+  // combine the row groups in a fixed order (xor tree over the lanes holding the same dims)
 #pragma unroll
-  for (int e = 0; e < PER; ++e) {
-    qsum[w * D + lane * PER + e] = aq[e];
-    ksum[w * D + lane * PER + e] = ak[e];
+  for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      aq[e] += __shfl_xor_sync(0xffffffffu, aq[e], o);
+      ak[e] += __shfl_xor_sync(0xffffffffu, ak[e], o);
+    }
+  if (sub == 0) {
+    float4* oq = reinterpret_cast<float4*>(qsum + w * D + d0);
+    float4* okk = reinterpret_cast<float4*>(ksum + w * D + d0);
+    oq[0] = make_float4(aq[0], aq[1], aq[2], aq[3]);
+    oq[1] = make_float4(aq[4], aq[5], aq[6], aq[7]);
+    okk[0] = make_float4(ak[0], ak[1], ak[2], ak[3]);
+    okk[1] = make_float4(ak[4], ak[5], ak[6], ak[7]);
   }
 }
 
