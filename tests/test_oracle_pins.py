@@ -69,6 +69,22 @@ def test_tile_grid_is_walked_w_fastest():
     src = O.tile_slot_source(g)
     # block 1 is the next tile along w, block 2 the next along h
     assert src[64] == 4 and src[128] == 4 * 8
+    # inside a tile, row-major over (dt, dh, dw): slot 1 is the next token along w, slot 4
+    # the next along h, slot 16 the next along t (token index (t * H + h) * W + w)
+    assert src[0] == 0 and src[1] == 1 and src[4] == 8 and src[16] == 64
+    assert src[63] == (3 * 8 + 3) * 8 + 3
+
+
+def _block_tile_coords(g):
+    """(tile t, tile h, tile w) of every block, read off the raster positions of the
+    tokens the permutation puts there (independent of any tile-index arithmetic)."""
+    src = O.tile_slot_source(g)
+    out = []
+    for blk in range(g.Np // 64):
+        toks = src[blk * 64:(blk + 1) * 64]
+        tok = int(toks[toks >= 0][0])
+        out.append((tok // (g.H * g.W) // 4, (tok // g.W) % g.H // 4, tok % g.W // 4))
+    return out
 
 
 # ------------------------------------------------------------------ block mass
@@ -253,6 +269,43 @@ def test_topp_hand_examples():
     # so 0.5 is just short of half the total
     m = np.array([0.05, 0.5, 0.15, 0.3], np.float32)
     assert O.topp_select_row(m, 0.5).tolist() == [1, 3]
+    # the kept mass must reach tau of the total, not just its integer part: masses 3, 2, 2
+    # units of 2^-40 and a threshold just above 3/7 need 3.00000x units, so block 0 alone
+    # (3 units) is not enough
+    m = np.array([3, 2, 2], np.float32) * np.float32(2.0 ** -40)
+    tau = np.nextafter(np.float32(3 / 7), np.float32(1))
+    assert float(tau) * 7 > 3
+    assert O.topp_select_row(m, tau).tolist() == [0, 1]
+    # the threshold is the float32 value: 0.9 as float32 is 0.899999976..., which the top
+    # block here holds exactly, so it is kept alone (a float64 0.9 would need both blocks)
+    t32 = np.float32(0.9)
+    m = np.array([t32, np.float32(1.0) - t32], np.float32)
+    assert float(m[0]) + float(m[1]) == 1.0 and float(t32) < 0.9
+    assert O.topp_select_row(m, 0.9).tolist() == [0]
+    assert O.topp_select_row(m, np.float32(0.9)).tolist() == [0]
+
+
+def test_fixed_point_masses_round_half_to_even():
+    """q = m * 2^40 rounded to the nearest integer, halves to even; values hand-computed
+    from float32 masses whose scaled value has a fractional part."""
+    u = 2.0 ** -40
+    m = np.array([0.25 * u, 0.5 * u, 0.75 * u, 1.5 * u, 2.5 * u, 3.0 * u, 1.0], np.float32)
+    assert O.fixed_point_masses(m).tolist() == [0, 0, 1, 2, 2, 3, 2 ** 40]
+
+
+def test_topp_target_is_the_exact_ceiling_where_the_product_is_exact():
+    """For totals below 2^29 the float32 threshold times the total is exact in float64, so
+    the target is the exact rational ceiling of tau * total."""
+    from fractions import Fraction
+    rng = np.random.default_rng(11)
+    for _ in range(2000):
+        total = int(rng.integers(0, 2 ** 29))
+        tau = np.float32(rng.uniform(0.0, 1.0))
+        exact = Fraction(float(tau)) * total
+        want = exact.numerator // exact.denominator + (exact.denominator != 1 and exact > 0)
+        assert O.topp_target(total, tau) == want
+    for total, tau, want in ((7, 0.5, 4), (8, 0.5, 4), (10, 1.0, 10), (0, 0.99, 0)):
+        assert O.topp_target(total, tau) == want
 
 
 def test_topp_rejects_bad_masses():
@@ -448,6 +501,28 @@ def test_pattern_surrounding_counts_closed_form():
     assert rows0 == [[u] for u in range(27)]
 
 
+def test_pattern_surrounding_asymmetric_radii_on_a_non_cubic_grid():
+    """Radii (0, 1, 2) on 2 x 3 x 4 tiles: the kept set is the box of tiles around the
+    query tile, with coordinates taken from the tokens' raster positions."""
+    g = O.Grid(7, 11, 14, 8, 12, 16)        # ragged in every axis
+    xyz = _block_tile_coords(g)
+    rows = _rows(*O.pattern_csr(g, 64, 1, 1, O.PAT_SURROUNDING, radius=(0, 1, 2)))
+    for u, r in enumerate(rows):
+        tu, hu, wu = xyz[u]
+        assert r == [v for v, (tv, hv, wv) in enumerate(xyz)
+                     if tv == tu and abs(hv - hu) <= 1 and abs(wv - wu) <= 2]
+    assert len(rows[xyz.index((0, 1, 1))]) == 3 * 4
+
+
+def test_pattern_criss_cross_sets_on_a_non_cubic_grid():
+    g = O.Grid(12, 12, 16, 12, 12, 16)      # 3 x 3 x 4 tiles
+    xyz = _block_tile_coords(g)
+    rows = _rows(*O.pattern_csr(g, 64, 1, 1, O.PAT_CRISS_CROSS))
+    for u, r in enumerate(rows):
+        assert r == [v for v, c in enumerate(xyz)
+                     if sum(int(a == b) for a, b in zip(c, xyz[u])) >= 2]
+
+
 def test_pattern_criss_cross_is_three_axis_lines():
     g = O.Grid(12, 12, 16, 12, 12, 16)      # 3 x 3 x 4 tiles
     rows = _rows(*O.pattern_csr(g, 64, 1, 1, O.PAT_CRISS_CROSS))
@@ -500,6 +575,18 @@ def test_pooled_estimate_rows_and_zero_scale():
     for i in range(g.Np // 64):
         if valid[i * 64:(i + 1) * 64].any():
             assert np.allclose(z[0, 0, i], nvk / nvk.sum(), atol=1e-14, rtol=0)
+    # a whole temporal layer of pad tiles: its query blocks get all-zero rows and its kv
+    # blocks zero mass in every row
+    g2 = O.Grid(4, 4, 9, 8, 4, 12)
+    q2, k2 = _qk(g2, heads=1, D=8, seed=12)
+    e2 = O.pooled_block_mass(q2, k2, g2, 64, 64, 0.4)
+    v2 = O.valid_slots(g2)
+    empty = [i for i in range(g2.Np // 64) if not v2[i * 64:(i + 1) * 64].any()]
+    assert empty == [3, 4, 5]
+    for i in empty:
+        assert np.all(e2[0, 0, i] == 0) and np.all(e2[0, 0, :, i] == 0)
+    for i in range(3):
+        assert np.allclose(e2[0, 0, i].sum(), 1.0, atol=1e-12, rtol=0)
 
 
 # ------------------------------------------------------------------ semantic clusters
