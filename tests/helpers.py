@@ -95,6 +95,27 @@ def assert_attn_close(got: np.ndarray, ref: np.ndarray, fp8: bool = False,
     return e
 
 
+LSE_ABS = 1e-3  # natural-log units; a dropped share p of a row's mass moves it by -log(1-p)
+
+
+def assert_fwd_close(got: np.ndarray, lse_got: np.ndarray, o_ref: np.ndarray,
+                     lse_ref: np.ndarray, fp8: bool = False):
+    """The forward's whole check against the oracle: outputs element-wise
+    (assert_attn_close; e4m3 with its signal guard), rows the oracle leaves empty exactly
+    zero with log-sum-exp -inf, and every other row's log-sum-exp within LSE_ABS."""
+    zero = ~np.isfinite(lse_ref)
+    if fp8:
+        e = assert_attn_close(got, o_ref, fp8=True)
+    else:
+        # every row empty: nothing to compare but the exact zeros below
+        e = None if zero.all() else assert_attn_close(got, o_ref, signal_guard=False)
+    assert np.all(got[zero] == 0)
+    assert np.all(np.isneginf(lse_got[zero]))
+    if (~zero).any():
+        assert np.abs(lse_got[~zero] - lse_ref[~zero]).max() <= LSE_ABS
+    return e
+
+
 def csr_from_oracle(mass64: np.ndarray, tau: float):
     rp, ci = O.topp_select(mass64.astype(np.float32).reshape(-1, mass64.shape[-1]), tau)
     return rp, ci

@@ -5,7 +5,11 @@ same helper is fed the oracle's outputs for inputs the GPU tests draw on the CPU
 all-zero and a perturbed stand-in for the device output: both must be rejected, while the
 oracle's output itself (and one rounded to bf16) passes.  For the e4m3 and cluster-order
 cases, whose tests also demand a reference output above 10x the absolute bound, the guard
-is checked to hold on the very inputs those tests use.
+is checked to hold on the very inputs those tests use.  The forward's whole check (outputs,
+empty rows, log-sum-exp) is also fed the oracle's answers to wrong computations that a
+kernel bug would produce -- a skipped kv block, a missing or doubled log2(e) factor, K or V
+of the neighbouring block, unmasked pad keys, rows stored one slot off -- and must reject
+every one.
 """
 import math
 
@@ -89,3 +93,83 @@ def test_cluster_cases_clear_the_signal_guard():
                                               rows, cols, 1.0 / math.sqrt(D))
                     assert np.abs(ref).max() >= Hp.SIGNAL_FACTOR * Hp.ATTN_MAX_ABS, (D, keep, b, h)
                     _rejects(np.zeros_like(ref), ref)
+
+
+# ------------------------------------------------------------------ plausible kernel bugs
+def _drop_one_block(rp, ci, which):
+    """CSR with the first (which=0) or last (which=-1) kept block of every row removed,
+    as a loop bound off by one would leave it."""
+    rows, out_rp = [], [0]
+    for r in range(len(rp) - 1):
+        blocks = list(ci[rp[r]:rp[r + 1]])
+        if blocks:
+            del blocks[which]
+        rows += blocks
+        out_rp.append(len(rows))
+    return np.array(out_rp, np.int64), np.array(rows, np.int64)
+
+
+def _attend_with_pad_keys(qt, kt, vt, g, q_block, rp, ci, scale):
+    """Attention whose kept blocks also admit their pad slots as keys (zero K and V), as a
+    kernel that forgot the key mask would compute it; pad query rows stay empty."""
+    B, Hh, Np, D = qt.shape
+    valid = O.valid_slots(g)
+    n_qb = Np // q_block
+    o = np.zeros((B, Hh, Np, D))
+    lse = np.full((B, Hh, Np), -math.inf)
+    for b in range(B):
+        for h in range(Hh):
+            for p in np.flatnonzero(valid):
+                r = (b * Hh + h) * n_qb + p // q_block
+                blocks = ci[rp[r]:rp[r + 1]]
+                if blocks.size == 0:
+                    continue
+                keys = (blocks[:, None] * 64 + np.arange(64)[None, :]).reshape(-1)
+                lg = scale * (kt[b, h, keys] @ qt[b, h, p])
+                mx = lg.max()
+                e = np.exp(lg - mx)
+                o[b, h, p] = (e / e.sum()) @ vt[b, h, keys]
+                lse[b, h, p] = mx + math.log(e.sum())
+    return o, lse
+
+
+@pytest.mark.parametrize("wl", WLS[:2], ids=[w.name for w in WLS[:2]])
+@pytest.mark.parametrize("sharp", [1.0, 6.0])
+def test_fwd_check_rejects_plausible_kernel_mistakes(wl, sharp):
+    """The GPU forward tests' whole check (helpers.assert_fwd_close) is fed the oracle's
+    answer to a wrong computation -- what a kernel with that bug would return -- and must
+    reject each one, while the right answer rounded to bf16 passes."""
+    g = Hp.grid_of(wl)
+    q, k, v = Hp.draw(wl, value_scale=1.0, sharp=sharp)
+    qt, kt, vt = (Hp.oracle_tiled(x, g) for x in (q, k, v))
+    scale = Hp.scale_of(wl)
+    mass = O.block_mass(qt, kt, g, wl.q_block, 64, scale)
+    rp, ci = Hp.csr_from_oracle(mass, 0.9)
+    o_ref, lse_ref = O.masked_attention(qt, kt, vt, g, wl.q_block, 64, rp, ci, scale)
+    Hp.assert_fwd_close(_bf16(o_ref), lse_ref, o_ref, lse_ref)
+
+    def attend(qx=qt, kx=kt, vx=vt, r=rp, c=ci, s=scale):
+        return O.masked_attention(qx, kx, vx, g, wl.q_block, 64, r, c, s)
+
+    roll = lambda x: np.roll(x, -64, axis=2)          # noqa: E731  block j reads block j+1
+    rp_last, ci_last = _drop_one_block(rp, ci, -1)
+    rp_first, ci_first = _drop_one_block(rp, ci, 0)
+    mistakes = {
+        "last kept block skipped": attend(r=rp_last, c=ci_last),
+        "first kept block skipped": attend(r=rp_first, c=ci_first),
+        "exp2 without the log2(e) factor": attend(s=scale * math.log(2.0)),
+        "log2(e) applied twice": attend(s=scale / math.log(2.0)),
+        "K of the next kv block": attend(kx=roll(kt)),
+        "V of the next kv block": attend(vx=roll(vt)),
+        "pad keys not masked": _attend_with_pad_keys(qt, kt, vt, g, wl.q_block, rp, ci, scale),
+    }
+    for name, (o_bad, lse_bad) in mistakes.items():
+        with pytest.raises(AssertionError):
+            Hp.assert_fwd_close(o_bad, lse_bad, o_ref, lse_ref)
+            raise RuntimeError(name)  # not reached when the check rejects
+    # output rows stored one slot off inside each query block
+    o_bad, lse_bad = o_ref.copy(), lse_ref.copy()
+    o_bad[:, :, 1:] = o_ref[:, :, :-1]
+    lse_bad[:, :, 1:] = lse_ref[:, :, :-1]
+    with pytest.raises(AssertionError):
+        Hp.assert_fwd_close(o_bad, lse_bad, o_ref, lse_ref)

@@ -240,16 +240,8 @@ def _fwd_compare(B, wl, q, k, v, rp, ci, want_lse=True):
     o_ref, lse_ref = O.masked_attention(Hp.oracle_tiled(q, g), Hp.oracle_tiled(k, g),
                                         Hp.oracle_tiled(v, g), g, wl.q_block, 64, rp, ci,
                                         Hp.scale_of(wl))
-    got = out.cpu().double().numpy()
-    zero = ~np.isfinite(lse_ref)
-    # every row empty: nothing to compare but the exact zeros below
-    e = None if zero.all() else Hp.assert_attn_close(got, o_ref, signal_guard=False)
-    assert np.all(got[zero] == 0)
-    lg = lse.cpu().double().numpy()
-    assert np.all(np.isneginf(lg[zero]))
-    if (~zero).any():
-        assert np.abs(lg[~zero] - lse_ref[~zero]).max() <= 1e-3
-    return e
+    return Hp.assert_fwd_close(out.cpu().double().numpy(), lse.cpu().double().numpy(),
+                               o_ref, lse_ref)
 
 
 @pytest.mark.parametrize("wl", WLS, ids=IDS)
@@ -399,14 +391,8 @@ def _fp8_compare(B, wl, q, k, v, rp, ci):
     assert B.device_status(ws) == 0, B.device_status_words(ws)
     o_ref, lse_ref = O.masked_attention(deq[0], deq[1], deq[2], g, wl.q_block, 64, rp, ci,
                                         Hp.scale_of(wl))
-    got = out.cpu().double().numpy()
-    e = Hp.assert_attn_close(got, o_ref, fp8=True)
-    zero = ~np.isfinite(lse_ref)
-    assert np.all(got[zero] == 0)
-    lg = lse.cpu().double().numpy()
-    if (~zero).any():
-        assert np.abs(lg[~zero] - lse_ref[~zero]).max() <= 1e-3
-    return e
+    return Hp.assert_fwd_close(out.cpu().double().numpy(), lse.cpu().double().numpy(),
+                               o_ref, lse_ref, fp8=True)
 
 
 @pytest.mark.parametrize("wl", FP8_WLS, ids=[w.name for w in FP8_WLS])
