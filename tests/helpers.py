@@ -95,6 +95,17 @@ def assert_attn_close(got: np.ndarray, ref: np.ndarray, fp8: bool = False,
     return e
 
 
+def assert_mass_close(got: np.ndarray, ref: np.ndarray):
+    """Block masses against the oracle's: abs error <= MASS_ABS everywhere, relative error
+    < 1e-3 wherever the reference exceeds 1e-6, and the structural zeros (pad-only kv
+    blocks, query blocks without valid queries) exactly zero."""
+    err = np.abs(got - ref)
+    assert err.max() <= MASS_ABS, err.max()
+    nz = ref > 1e-6
+    assert (err[nz] / ref[nz]).max() < 1e-3
+    assert np.all(got[ref == 0] == 0)
+
+
 LSE_ABS = 1e-3  # natural-log units; a dropped share p of a row's mass moves it by -log(1-p)
 
 

@@ -173,3 +173,52 @@ def test_fwd_check_rejects_plausible_kernel_mistakes(wl, sharp):
     lse_bad[:, :, 1:] = lse_ref[:, :, :-1]
     with pytest.raises(AssertionError):
         Hp.assert_fwd_close(o_bad, lse_bad, o_ref, lse_ref)
+
+
+def _mass_with_pad_keys(qt, kt, g, q_block, scale):
+    """Block masses whose softmax also admits the pad slots as keys (zero K), as a kernel
+    that forgot the key mask would compute them."""
+    B, Hh, Np, _ = qt.shape
+    valid = O.valid_slots(g)
+    n_qb, n_kb = Np // q_block, Np // 64
+    out = np.zeros((B, Hh, n_qb, n_kb))
+    for b in range(B):
+        for h in range(Hh):
+            for i in range(n_qb):
+                rows = np.arange(i * q_block, (i + 1) * q_block)
+                rows = rows[valid[rows]]
+                if rows.size == 0:
+                    continue
+                lg = scale * (qt[b, h, rows] @ kt[b, h].T)
+                p = np.exp(lg - lg.max(axis=1, keepdims=True))
+                p /= p.sum(axis=1, keepdims=True)
+                out[b, h, i] = p.sum(axis=0).reshape(n_kb, 64).sum(axis=1) / rows.size
+    return out
+
+
+@pytest.mark.parametrize("wl", WLS[:2], ids=[w.name for w in WLS[:2]])
+@pytest.mark.parametrize("sharp", [1.0, 6.0])
+def test_mass_check_rejects_plausible_kernel_mistakes(wl, sharp):
+    """The block-mass check of the GPU tests (helpers.assert_mass_close) rejects the masses
+    a kernel bug would produce, and accepts the right masses rounded to float32."""
+    g = Hp.grid_of(wl)
+    q, k, _ = Hp.draw(wl, value_scale=1.0, sharp=sharp)
+    qt, kt = Hp.oracle_tiled(q, g), Hp.oracle_tiled(k, g)
+    scale = Hp.scale_of(wl)
+    ref = O.block_mass(qt, kt, g, wl.q_block, 64, scale)
+    Hp.assert_mass_close(ref.astype(np.float32).astype(np.float64), ref)
+    valid = O.valid_slots(g).reshape(-1, wl.q_block)
+    share = (valid.sum(axis=1) / wl.q_block)[None, None, :, None]
+    mistakes = {
+        "exp2 without the log2(e) factor": O.block_mass(qt, kt, g, wl.q_block, 64,
+                                                        scale * math.log(2.0)),
+        "mass put in the next kv block": np.roll(ref, 1, axis=-1),
+        "mean over every row of the block, pads included": ref * share,
+        "pad keys not masked": _mass_with_pad_keys(qt, kt, g, wl.q_block, scale),
+        "rows of the neighbouring head": np.roll(ref, 1, axis=1),
+        "row of the next query block": np.roll(ref, -1, axis=2),
+    }
+    for name, bad in mistakes.items():
+        with pytest.raises(AssertionError):
+            Hp.assert_mass_close(bad, ref)
+            raise RuntimeError(name)  # not reached when the check rejects
