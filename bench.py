@@ -24,7 +24,11 @@ fwd    = the same FLOPs over the forward launches alone (CUDA events on the laun
 e2e    = the same metric through the public API with inputs copied from pinned host
          memory and outputs copied back inside the timed region.
 --impl reference times the CPU oracle (the only other implementation of the method) on
-a bounded sample of the same workload.
+a bounded sample of the same workload: the inputs are drawn once, each step times the
+oracle's masked attention on its own sampled query rows and CSR, and the rows per step are
+sized from a short probe so that all steps together take about REF_BUDGET_S seconds
+(16 to --cpu-sample-rows rows a step).  The main line's cpu_baseline times
+--cpu-sample-rows rows once.
 
 With N > 1 ranks (one per GPU) the path needs no exchange step: --split problems (the
 default) gives every rank an independent problem of the workload's size (weak scaling);
@@ -583,28 +587,44 @@ def run_e2e(args, bsa, s, draws, n_reuse, row_ptr, col_idx, flops_call, dev, str
 
 
 # ============================================================================ CPU oracle
-def oracle_sample(wl, n_rows: int, seed: int = 0):
-    """Time the oracle's masked attention on n_rows sampled query rows of the workload
-    (seeded synthetic inputs on the host, a seeded CSR at the workload's kept fraction).
-    Returns (executed FLOPs, seconds, description)."""
-    import numpy as np
+# Seconds of oracle work the reference arm's timed steps take together (about).
+REF_BUDGET_S = 120.0
+
+
+def oracle_inputs(wl):
+    """Seeded synthetic inputs of the workload for the oracle, drawn and permuted once on
+    the host: two heads of Q, K and V in tile-major float64 (the rows are sampled from
+    them; a head's cost per row does not depend on the head count)."""
     import torch
-    from threadpoolctl import threadpool_limits
 
     from block_sparse_attention_25_b200 import synth
     from oracle import bsa_oracle as O
 
     g = O.Grid(wl.T, wl.H, wl.W, wl.Tp, wl.Hp, wl.Wp)
     heads = 2
-    small = wl.scaled(heads=heads)
-    q, k, v = synth.draw_qkv(small, device="cpu")
+    q, k, v = synth.draw_qkv(wl.scaled(heads=heads), device="cpu")
     qt, kt, vt = (O.permute_forward(x.to(torch.float64).numpy(), g) for x in (q, k, v))
+    return dict(wl=wl, g=g, heads=heads, qkv=(qt, kt, vt))
+
+
+def oracle_rows(inp, n_rows: int, seed: int = 0):
+    """Time the oracle's masked attention on n_rows sampled query rows (a seeded CSR at the
+    workload's kept fraction).  Returns (executed FLOPs, seconds, description)."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    from block_sparse_attention_25_b200 import synth
+    from oracle import bsa_oracle as O
+
+    wl, g, heads = inp["wl"], inp["g"], inp["heads"]
+    qt, kt, vt = inp["qkv"]
     n_qb, n_kb = wl.Np // wl.q_block, wl.Np // 64
     rp, ci = synth.draw_keep_csr(heads * n_qb, n_kb, wl.nominal_kept, seed=seed)
     rp, ci = rp.numpy(), ci.numpy()
     valid = O.valid_slots(g)
     rng = np.random.default_rng(seed)
     cand = np.nonzero(valid)[0]
+    n_rows = min(n_rows, cand.size)
     rows = [(0, int(rng.integers(0, heads)), int(p)) for p in rng.choice(cand, n_rows, replace=False)]
     flops = 0.0
     with threadpool_limits(limits=1):
@@ -620,6 +640,11 @@ def oracle_sample(wl, n_rows: int, seed: int = 0):
     desc = (f"oracle masked attention (numpy fp64, 1 thread) on {n_rows} sampled query rows of "
             f"{wl.name} with a seeded CSR at {wl.nominal_kept} kept; TFLOP/s = executed FLOPs of those rows / time")
     return flops, dt, desc
+
+
+def oracle_sample(wl, n_rows: int, seed: int = 0):
+    """oracle_rows on freshly drawn inputs (the main line's CPU baseline)."""
+    return oracle_rows(oracle_inputs(wl), n_rows, seed)
 
 
 def oracle_units(wl, seed: int = 0):
@@ -669,12 +694,20 @@ def run_reference(args, world, rank, pg):
     wl = synth.WORKLOADS[args.config]
     if rank != 0:
         return None
+    # inputs drawn once; each step samples its own rows and CSR.  Rows per step: as many as
+    # fit REF_BUDGET_S over all steps at the rate of an 8-row probe (at least 16, at most
+    # --cpu-sample-rows), so the run stays within a few minutes for any --steps.
+    inp = oracle_inputs(wl)
     for _ in range(max(0, min(args.warmup, 1))):
-        oracle_sample(wl, 4)
+        oracle_rows(inp, 4, seed=100_000)
+    _, t_probe, _ = oracle_rows(inp, 8, seed=100_001)
+    per_row = max(t_probe / 8, 1e-6)
+    n_rows = int(min(args.cpu_sample_rows,
+                     max(16, REF_BUDGET_S / max(1, args.steps) / per_row)))
     tot_f = tot_t = 0.0
     desc = ""
     for i in range(args.steps):
-        f, t, desc = oracle_sample(wl, args.cpu_sample_rows, seed=i)
+        f, t, desc = oracle_rows(inp, n_rows, seed=i)
         tot_f += f
         tot_t += t
     val = tot_f / tot_t / 1e12
