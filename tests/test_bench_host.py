@@ -69,3 +69,39 @@ def test_traffic_is_reported_only_for_the_captured_sources(tmp_path, monkeypatch
         f.write("\n// edited\n")
     assert bench.measured_traffic(False, False) is None
     assert bench.measured_traffic(True, False) is None
+
+
+def test_reference_arm_sizes_its_rows_to_the_budget(monkeypatch):
+    """The reference arm draws its inputs once and takes between 16 and --cpu-sample-rows
+    rows a step, fewer when the steps would otherwise exceed the oracle budget."""
+    calls = []
+    real_rows = bench.oracle_rows
+
+    def counting_rows(inp, n_rows, seed=0):
+        calls.append(n_rows)
+        return real_rows(inp, n_rows, seed)
+
+    drawn = []
+    real_inputs = bench.oracle_inputs
+
+    def counting_inputs(wl):
+        drawn.append(wl.name)
+        return real_inputs(wl)
+
+    monkeypatch.setattr(bench, "oracle_rows", counting_rows)
+    monkeypatch.setattr(bench, "oracle_inputs", counting_inputs)
+    args = bench.parse_args(["--impl", "reference", "--config", "tiny", "--steps", "3",
+                             "--warmup", "3", "--cpu-sample-rows", "40"])
+    res = bench.run_reference(args, 1, 0, None)
+    assert len(drawn) == 1
+    step_rows = calls[2:]                       # after the warm-up and the 8-row probe
+    assert calls[:2] == [4, 8] and len(step_rows) == 3
+    assert all(r == 40 for r in step_rows)      # tiny rows are cheap: the cap applies
+    assert res["value"] > 0 and res["steps"] == 3 and "40 sampled query rows" in res["cpu_baseline"]["sample"]
+    # a budget far below one row's cost gives the floor of 16 rows a step
+    calls.clear()
+    monkeypatch.setattr(bench, "REF_BUDGET_S", 1e-9)
+    bench.run_reference(args, 1, 0, None)
+    assert calls[2:] == [16, 16, 16]
+    # ranks other than 0 do no work
+    assert bench.run_reference(args, 2, 1, None) is None
