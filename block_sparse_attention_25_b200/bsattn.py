@@ -194,12 +194,33 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _is_device(t) -> bool:
+    return t.is_cuda
+
+
 def _need(t, dtype, shape, name):
     if t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
     if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
-    if not t.is_cuda or not t.is_contiguous():
+    if not _is_device(t) or not t.is_contiguous():
+        raise ValueError(f"{name}: must be a contiguous CUDA tensor")
+
+
+def _dev(t, dtype, name, shape=None, min_numel=None):
+    """A buffer the library reads or writes through a raw pointer (an output, a workspace, a
+    list): of `dtype`, contiguous and on the GPU, and of `shape` or at least `min_numel`
+    elements when given -- so a host tensor or a short buffer is refused here instead of
+    reaching a kernel.  None passes (an optional output the caller did not ask for)."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name}: needs at least {min_numel} elements, has {t.numel()}")
+    if not _is_device(t) or not t.is_contiguous():
         raise ValueError(f"{name}: must be a contiguous CUDA tensor")
 
 
@@ -213,11 +234,13 @@ def new_workspace(shape: Shape, op: int, device="cuda") -> torch.Tensor:
     if n == 0:
         raise BsaError(1, "workspace size")
     ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _dev(ws, torch.uint8, "ws")
     _check(lib().bsa_clear_status(_ptr(ws), _stream()), "bsa_clear_status")
     return ws
 
 
 def clear_status(ws: torch.Tensor, stream=None):
+    _dev(ws, torch.uint8, "ws")
     _check(lib().bsa_clear_status(_ptr(ws), _stream(stream)), "bsa_clear_status")
 
 
@@ -258,6 +281,8 @@ def tile_permute_quant_e4m3(x: torch.Tensor, shape: Shape, out=None, scales=None
     if scales is None:
         scales = torch.empty((shape.batch, shape.heads, shape.Np // 64), dtype=torch.float32,
                              device=x.device)
+    _dev(out, torch.uint8, "dst", (shape.batch, shape.heads, shape.Np, shape.head_dim))
+    _dev(scales, torch.float32, "scales", (shape.batch, shape.heads, shape.Np // 64))
     _check(lib().bsa_tile_permute_quant_e4m3(ctypes.byref(shape.c()), _ptr(x), _ptr(out),
                                              _ptr(scales), _stream(stream)),
            "bsa_tile_permute_quant_e4m3")
@@ -278,6 +303,8 @@ def block_mass(q, k, shape: Shape, softmax_scale=None, out=None, ws=None, stream
                           device=q.device)
     if ws is None:
         ws = new_workspace(shape, OP_BLOCK_MASS, q.device)
+    _dev(out, torch.float32, "mass", (shape.batch, shape.heads, shape.n_qb, shape.n_kb))
+    _dev(ws, torch.uint8, "ws")
     scale = default_scale(shape) if softmax_scale is None else float(softmax_scale)
     _check(lib().bsa_block_mass(ctypes.byref(shape.c()), _ptr(q), _ptr(k), scale, _ptr(out),
                                 _ptr(ws), ws.numel(), _stream(stream)), "bsa_block_mass")
@@ -300,6 +327,10 @@ def dense_fwd_mass(q, k, v, shape: Shape, softmax_scale=None, want_lse=False, ou
         lse = torch.empty((shape.batch, shape.heads, shape.Np), dtype=torch.float32, device=q.device)
     if ws is None:
         ws = new_workspace(shape, OP_BLOCK_MASS, q.device)
+    _dev(out, torch.bfloat16, "out", tiled)
+    _dev(mass, torch.float32, "mass", (shape.batch, shape.heads, shape.n_qb, shape.n_kb))
+    _dev(lse, torch.float32, "lse", (shape.batch, shape.heads, shape.Np))
+    _dev(ws, torch.uint8, "ws")
     scale = default_scale(shape) if softmax_scale is None else float(softmax_scale)
     _check(lib().bsa_dense_fwd_mass(ctypes.byref(shape.c()), _ptr(q), _ptr(k), _ptr(v), scale,
                                     _ptr(out), _ptr(lse), _ptr(mass), _ptr(ws), ws.numel(),
@@ -317,6 +348,8 @@ def pooled_mass(q, k, shape: Shape, softmax_scale=None, out=None, ws=None, strea
                           device=q.device)
     if ws is None:
         ws = new_workspace(shape, OP_POOLED_MASS, q.device)
+    _dev(out, torch.float32, "mass_est", (shape.batch, shape.heads, shape.n_qb, shape.n_kb))
+    _dev(ws, torch.uint8, "ws")
     scale = default_scale(shape) if softmax_scale is None else float(softmax_scale)
     _check(lib().bsa_pooled_mass(ctypes.byref(shape.c()), _ptr(q), _ptr(k), scale, _ptr(out),
                                  _ptr(ws), ws.numel(), _stream(stream)), "bsa_pooled_mass")
@@ -339,6 +372,9 @@ def topp_select(mass, shape: Shape, threshold: float = 0.99, col_capacity=None, 
         col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=mass.device)
     if ws is None:
         ws = new_workspace(shape, OP_TOPP_SELECT, mass.device)
+    _dev(row_ptr, torch.int32, "row_ptr", (R + 1,))
+    _dev(col_idx, torch.int32, "col_idx", min_numel=cap)
+    _dev(ws, torch.uint8, "ws")
     _check(lib().bsa_topp_select(ctypes.byref(shape.c()), _ptr(mass), float(threshold),
                                  _ptr(row_ptr), _ptr(col_idx), cap, _ptr(ws), ws.numel(),
                                  _stream(stream)), "bsa_topp_select")
@@ -384,6 +420,12 @@ def topp_select_noalloc(mass, shape: Shape, threshold: float = 0.99, row_ptr=Non
         row_ptr = torch.empty(R + 1, dtype=torch.int32, device=mass.device)
     if col_idx is None:
         col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=mass.device)
+    _dev(row_ptr, torch.int32, "row_ptr", (R + 1,))
+    _dev(col_idx, torch.int32, "col_idx", min_numel=cap)
+    if status is not None:
+        _dev(status, status.dtype, "status", min_numel=4)
+        if status.dtype not in (torch.int32, torch.uint32):
+            raise TypeError("status: int32 or uint32")
     _check(lib().bsa_topp_select_noalloc(ctypes.byref(shape.c()), _ptr(mass), float(threshold),
                                          _ptr(row_ptr), _ptr(col_idx), cap, _ptr(status),
                                          _stream(stream)), "bsa_topp_select_noalloc")
@@ -402,6 +444,9 @@ def pattern_csr(shape: Shape, kinds: int, diag_width=0, multi_count=0, multi_per
         col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=device)
     if ws is None:
         ws = new_workspace(shape, OP_PATTERN, device)
+    _dev(row_ptr, torch.int32, "row_ptr", (R + 1,))
+    _dev(col_idx, torch.int32, "col_idx", min_numel=cap)
+    _dev(ws, torch.uint8, "ws")
     pat = _Pattern(int(kinds), diag_width, multi_count, multi_period, stripe_stride, stripe_offset,
                    *radius)
     _check(lib().bsa_pattern_csr(ctypes.byref(shape.c()), ctypes.byref(pat), _ptr(row_ptr),
@@ -418,14 +463,16 @@ def bsattn_fwd_raster(q, k, v, row_ptr, col_idx, shape: Shape, softmax_scale=Non
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, raster, n)
     _need(row_ptr, torch.int32, (shape.rows + 1,), "row_ptr")
-    if col_idx.dtype != torch.int32 or not col_idx.is_cuda:
-        raise TypeError("col_idx: int32 CUDA tensor")
+    _dev(col_idx, torch.int32, "col_idx")
     if out is None:
         out = torch.empty(raster, dtype=torch.bfloat16, device=q.device)
     if want_lse and lse is None:
         lse = torch.empty((shape.batch, shape.heads, shape.S), dtype=torch.float32, device=q.device)
     if ws is None:
         ws = new_workspace(shape, OP_FWD, q.device)
+    _dev(out, torch.bfloat16, "out", raster)
+    _dev(lse, torch.float32, "lse", (shape.batch, shape.heads, shape.S))
+    _dev(ws, torch.uint8, "ws")
     scale = default_scale(shape) if softmax_scale is None else float(softmax_scale)
     _check(lib().bsa_fwd_raster(ctypes.byref(shape.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr),
                                 _ptr(col_idx), scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
@@ -442,8 +489,7 @@ def bsattn_fwd(q, k, v, row_ptr, col_idx, shape: Shape, softmax_scale=None, scal
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.uint8 if fp8 else torch.bfloat16, tiled, n)
     _need(row_ptr, torch.int32, (shape.rows + 1,), "row_ptr")
-    if col_idx.dtype != torch.int32 or not col_idx.is_cuda:
-        raise TypeError("col_idx: int32 CUDA tensor")
+    _dev(col_idx, torch.int32, "col_idx")
     sq = sk = sv = None
     if fp8:
         if scales is None:
@@ -457,6 +503,9 @@ def bsattn_fwd(q, k, v, row_ptr, col_idx, shape: Shape, softmax_scale=None, scal
         lse = torch.empty((shape.batch, shape.heads, shape.Np), dtype=torch.float32, device=q.device)
     if ws is None:
         ws = new_workspace(shape, OP_FWD, q.device)
+    _dev(out, torch.bfloat16, "out", tiled)
+    _dev(lse, torch.float32, "lse", (shape.batch, shape.heads, shape.Np))
+    _dev(ws, torch.uint8, "ws")
     scale = default_scale(shape) if softmax_scale is None else float(softmax_scale)
     _check(lib().bsa_fwd(ctypes.byref(shape.c()), BSA_E4M3 if fp8 else BSA_BF16, _ptr(q), _ptr(k),
                          _ptr(v), _ptr(sq), _ptr(sk), _ptr(sv), _ptr(row_ptr), _ptr(col_idx), scale,
@@ -482,6 +531,9 @@ def kmeans(x, cs: ClusterShape, n_clusters: int, init, rounds: int, labels=None,
         counts = torch.empty((B, Hh, n_clusters), dtype=torch.int32, device=x.device)
     if ws is None:
         ws = new_cluster_workspace(cs, n_clusters, x.device)
+    _dev(labels, torch.int32, "labels", (B, Hh, S))
+    _dev(counts, torch.int32, "counts", (B, Hh, n_clusters))
+    _dev(ws, torch.uint8, "ws")
     _check(lib().bsa_kmeans(ctypes.byref(cs.c()), int(n_clusters), _ptr(x), int(rounds), _ptr(init),
                             _ptr(labels), _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)),
            "bsa_kmeans")
@@ -493,6 +545,7 @@ def new_cluster_workspace(cs: ClusterShape, n_clusters: int, device="cuda") -> t
     if n == 0:
         raise BsaError(1, "cluster workspace size")
     ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _dev(ws, torch.uint8, "ws")
     _check(lib().bsa_clear_status(_ptr(ws), _stream()), "bsa_clear_status")
     return ws
 
@@ -508,6 +561,7 @@ def cluster_layout(labels, cs: ClusterShape, n_clusters: int, ws=None, stream=No
     sot = torch.empty_like(tos)
     if ws is None:
         ws = new_cluster_workspace(cs, n_clusters, dev)
+    _dev(ws, torch.uint8, "ws")
     _check(lib().bsa_cluster_layout(ctypes.byref(cs.c()), int(n_clusters), _ptr(labels), _ptr(counts),
                                     _ptr(starts), _ptr(tos), _ptr(sot), _ptr(ws), ws.numel(),
                                     _stream(stream)), "bsa_cluster_layout")
@@ -522,6 +576,7 @@ def cluster_permute(x, cs: ClusterShape, token_of_slot, inverse: bool = False, o
     _i32(token_of_slot, (B, Hh, S), "token_of_slot")
     if out is None:
         out = torch.zeros(raster if inverse else perm, dtype=torch.bfloat16, device=x.device)
+    _dev(out, torch.bfloat16, "dst", raster if inverse else perm)
     _check(lib().bsa_cluster_permute(ctypes.byref(cs.c()), int(bool(inverse)), _ptr(token_of_slot),
                                      _ptr(x), _ptr(out), _stream(stream)), "bsa_cluster_permute")
     return out
@@ -537,6 +592,7 @@ def cluster_mass(cs: ClusterShape, q_centroids, q_counts, k_centroids, k_counts,
     _i32(k_counts, (B, Hh, Ck), "k_counts")
     if out is None:
         out = torch.empty((B, Hh, Cq, Ck), dtype=torch.float32, device=q_centroids.device)
+    _dev(out, torch.float32, "mass", (B, Hh, Cq, Ck))
     scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
     _check(lib().bsa_cluster_mass(ctypes.byref(cs.c()), _ptr(q_centroids), _ptr(q_counts),
                                   _ptr(k_centroids), _ptr(k_counts), scale, _ptr(out),
@@ -547,7 +603,7 @@ def cluster_mass(cs: ClusterShape, q_centroids, q_counts, k_centroids, k_counts,
 def topp_select_rows(mass, threshold: float = 0.99, col_capacity=None, ws=None, row_ptr=None,
                      col_idx=None, stream=None):
     """bsa_topp_select_rows on a [..., cols] fp32 tensor viewed as rows x cols."""
-    if mass.dtype != torch.float32 or not mass.is_cuda or not mass.is_contiguous():
+    if mass.dtype != torch.float32 or not _is_device(mass) or not mass.is_contiguous():
         raise TypeError("mass: contiguous float32 CUDA tensor")
     cols = int(mass.shape[-1])
     rows = mass.numel() // cols
@@ -561,7 +617,11 @@ def topp_select_rows(mass, threshold: float = 0.99, col_capacity=None, ws=None, 
         if n == 0:
             raise BsaError(2, "topp rows workspace size")
         ws = torch.empty(n, dtype=torch.uint8, device=mass.device)
+        _dev(ws, torch.uint8, "ws")
         _check(lib().bsa_clear_status(_ptr(ws), _stream()), "bsa_clear_status")
+    _dev(row_ptr, torch.int32, "row_ptr", (rows + 1,))
+    _dev(col_idx, torch.int32, "col_idx", min_numel=cap)
+    _dev(ws, torch.uint8, "ws")
     _check(lib().bsa_topp_select_rows(_ptr(mass), rows, cols, float(threshold), _ptr(row_ptr),
                                       _ptr(col_idx), cap, _ptr(ws), ws.numel(), _stream(stream)),
            "bsa_topp_select_rows")
@@ -573,6 +633,7 @@ def new_cluster_fwd_workspace(cs: ClusterShape, device="cuda") -> torch.Tensor:
     if n == 0:
         raise BsaError(1, "cluster fwd workspace size")
     ws = torch.empty(n, dtype=torch.uint8, device=device)
+    _dev(ws, torch.uint8, "ws")
     _check(lib().bsa_clear_status(_ptr(ws), _stream()), "bsa_clear_status")
     return ws
 
@@ -589,14 +650,16 @@ def cluster_fwd(q, k, v, cs: ClusterShape, q_starts, q_counts, k_starts, k_count
     _i32(k_starts, (B, Hh, Ck), "k_starts")
     _i32(k_counts, (B, Hh, Ck), "k_counts")
     _i32(row_ptr, (B * Hh * Cq + 1,), "row_ptr")
-    if col_idx.dtype != torch.int32 or not col_idx.is_cuda:
-        raise TypeError("col_idx: int32 CUDA tensor")
+    _dev(col_idx, torch.int32, "col_idx")
     if out is None:
         out = torch.empty((B, Hh, S, D), dtype=torch.bfloat16, device=q.device)
     if want_lse and lse is None:
         lse = torch.empty((B, Hh, S), dtype=torch.float32, device=q.device)
     if ws is None:
         ws = new_cluster_fwd_workspace(cs, q.device)
+    _dev(out, torch.bfloat16, "out", (B, Hh, S, D))
+    _dev(lse, torch.float32, "lse", (B, Hh, S))
+    _dev(ws, torch.uint8, "ws")
     scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
     _check(lib().bsa_cluster_fwd(ctypes.byref(cs.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(q_starts),
                                  _ptr(q_counts), _ptr(k_starts), _ptr(k_counts), _ptr(row_ptr),
@@ -609,6 +672,7 @@ def selftest_wait(ws, limit_ns: int = 20_000_000, stream=None):
     """bsa_selftest_wait: a bounded wait that must give up (see include/bsattn.h).
     Returns the status header words after the kernel: (flags, detail, ...) and the three
     result words (first wait completed, second wait completed, abort flag seen)."""
+    _dev(ws, torch.uint8, "ws")
     _check(lib().bsa_selftest_wait(_ptr(ws), ws.numel(), int(limit_ns), _stream(stream)),
            "bsa_selftest_wait")
     torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
