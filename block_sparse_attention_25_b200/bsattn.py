@@ -401,6 +401,11 @@ def load_lists(path, shape: Shape, device="cuda"):
     nnz = ctypes.c_int64(0)
     _check(L.bsa_lists_read_header(os.fsencode(path), ctypes.byref(stored), ctypes.byref(tau),
                                    ctypes.byref(nnz)), "bsa_lists_read_header")
+    # refuse a file for another shape before sizing any buffer from its header
+    if bytes(stored) != bytes(shape.c()):
+        raise BsaError(1, "bsa_lists_load: the file holds lists of another shape")
+    if not 0 <= nnz.value <= shape.rows * shape.n_kb:
+        raise BsaError(7, "bsa_lists_load: entry count out of range")
     rp = torch.empty(shape.rows + 1, dtype=torch.int32)
     ci = torch.zeros(max(nnz.value, 1), dtype=torch.int32)
     _check(L.bsa_lists_load(os.fsencode(path), ctypes.byref(shape.c()), ctypes.byref(tau),

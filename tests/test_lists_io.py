@@ -79,6 +79,37 @@ def test_damaged_files_are_refused(B, tmp_path):
     assert e.value.status in (1, 7)
 
 
+def test_a_header_for_another_shape_sizes_no_buffer(B, tmp_path, monkeypatch):
+    """A file whose (intact) header describes a much larger problem is refused by the shape
+    comparison before the binding sizes any buffer from the header's entry count."""
+    import ctypes
+    big = B.Shape.of(synth.WORKLOADS["wan14b_720p"])
+    rp = torch.arange(big.rows + 1, dtype=torch.int32) * big.n_kb   # every block kept
+    path = tmp_path / "big.bin"
+    # a header only: the payload is never reached
+    B.save_lists(path, torch.zeros(big.rows + 1, dtype=torch.int32),
+                 torch.zeros(0, dtype=torch.int32), big, 0.99)
+    data = bytearray(path.read_bytes()[:80])
+    data[72:80] = (int(rp[-1])).to_bytes(8, "little")                # 83 M entries claimed
+    path.write_bytes(bytes(data) + b"\0" * 16)
+    stored, tau, nnz = B.bsattn._Shape(), ctypes.c_float(), ctypes.c_int64()
+    assert B.lib().bsa_lists_read_header(str(path).encode(), ctypes.byref(stored),
+                                         ctypes.byref(tau), ctypes.byref(nnz)) == 0
+    assert nnz.value == big.rows * big.n_kb
+    sizes = []
+    real_zeros = torch.zeros
+
+    def counting_zeros(*a, **kw):
+        sizes.append(a)
+        return real_zeros(*a, **kw)
+
+    monkeypatch.setattr(torch, "zeros", counting_zeros)
+    s = B.Shape.of(WL)
+    with pytest.raises(B.BsaError) as e:
+        B.load_lists(path, s, device="cpu")
+    assert e.value.status == 1 and sizes == []
+
+
 def test_malformed_lists_are_not_saved(B, tmp_path):
     s, rp, ci = _lists(B)
     bad = ci.clone()
