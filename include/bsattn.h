@@ -36,6 +36,12 @@
  *   - Sizes: head_dim in {64, 128}; q_block in {64, 128}; kv_block = 64; Tp, Hp, Wp
  *     multiples of 4 covering T, H, W; B*Hh*Np*D < 2^31 elements per tensor is not
  *     required (64-bit offsets are used), but B*Hh*(Np/q_block) rows must fit int32.
+ *     Also Np = Tp*Hp*Wp < 2^30 and a multiple of q_block, at most 4096 kv blocks per head
+ *     (Np/64 <= 4096), and R*(Np/64) < 2^31 with R = B*Hh*(Np/q_block) (CSR offsets are
+ *     int32).  Inconsistent extents (a size below 1, a padded extent below its valid one
+ *     or not a multiple of 4, Np not a multiple of q_block) return BSA_ERR_INVALID_ARG;
+ *     a consistent shape beyond these limits returns BSA_ERR_UNSUPPORTED; either way
+ *     bsa_workspace_bytes gives 0.
  *   - Pointers to bf16 / fp32 / e4m3 tensors must be 16-byte aligned.
  */
 #ifndef BSATTN_H
