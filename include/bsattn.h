@@ -299,6 +299,10 @@ BSA_API bsa_status bsa_fwd(const bsa_shape* shape, bsa_dtype dtype,
  * raster order; per-head int32 arrays [B, Hh, S] or [B, Hh, C]; centroids fp32
  * [B, Hh, C, D].  All pointers are device pointers owned by the caller; tensors of bf16
  * rows must be 16-byte aligned, int32 and fp32 arrays 4-byte aligned. */
+/* Limits: batch, heads >= 1 (else BSA_ERR_INVALID_ARG, as for a size below 1); head_dim,
+ * n_tokens and the cluster counts as below, B*Hh*S*(D/8) < 2^31 and
+ * B*Hh*n_q_clusters*n_k_clusters < 2^31 (flat indices fit 31 bits), else
+ * BSA_ERR_UNSUPPORTED; the workspace-size calls give 0 for a shape outside them. */
 typedef struct {
   int32_t batch, heads;
   int32_t head_dim;                    /* 64 or 128 */

@@ -121,3 +121,37 @@ def test_status_codes_follow_the_documented_classes(B):
             assert st in (1, 2), (d, st)
         seen.add(st)
     assert seen == {1, 2, 3}
+
+
+def _cluster_valid(d):
+    if min(d["batch"], d["heads"], d["n_tokens"], d["n_q_clusters"], d["n_k_clusters"]) < 1:
+        return False
+    if d["head_dim"] not in (64, 128) or d["n_tokens"] > 2 ** 24:
+        return False
+    if d["n_q_clusters"] > 1024 or d["n_k_clusters"] > 1024:
+        return False
+    bh = d["batch"] * d["heads"]
+    return (bh * d["n_tokens"] * (d["head_dim"] // 8) < 2 ** 31
+            and bh * d["n_q_clusters"] * d["n_k_clusters"] < 2 ** 31)
+
+
+def test_cluster_workspace_sizes_follow_the_documented_limits(B):
+    rng = np.random.default_rng(79)
+    n_valid = n_bad = 0
+    for _ in range(3000):
+        d = dict(batch=int(rng.choice([0, 1, 1, 2, 4, 1 << 12])),
+                 heads=int(rng.choice([-1, 1, 2, 40, 1 << 10])),
+                 head_dim=int(rng.choice([32, 64, 64, 128, 128, 256])),
+                 n_tokens=int(rng.choice([0, 1, 300, 75600, 1 << 20, 1 << 24, (1 << 24) + 1])),
+                 n_q_clusters=int(rng.choice([0, 1, 64, 1024, 1025])),
+                 n_k_clusters=int(rng.choice([1, 256, 1024, 2048])))
+        cs = B.ClusterShape(**d)
+        got = B.lib().bsa_cluster_fwd_workspace_bytes(ctypes.byref(cs.c()))
+        km = B.lib().bsa_kmeans_workspace_bytes(ctypes.byref(cs.c()), int(d["n_q_clusters"]))
+        if _cluster_valid(d):
+            assert got >= 256 and km >= 256, d
+            n_valid += 1
+        else:
+            assert got == 0 and km == 0, d
+            n_bad += 1
+    assert n_valid > 100 and n_bad > 500
