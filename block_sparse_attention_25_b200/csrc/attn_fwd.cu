@@ -12,7 +12,7 @@
 //   kv blocks (N = 128 keys) per step; keys of a block that a query block did not keep
 //   are masked to -inf for that block's rows.
 //
-// Warp roles (320 threads)
+// Warp roles (384 threads; warps 10-11 only complete the producer warpgroup)
 //   warps 0-3  softmax for Q tile 0, one thread per query row (TMEM lanes 0..127)
 //   warps 4-7  softmax for Q tile 1
 //   warp 8     TMA producer: Q once, then K and V of every step into rings
